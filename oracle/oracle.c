@@ -1,0 +1,414 @@
+/*
+ * CPU ORACLE -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, single-threaded C restatement of what the expert-parallel
+ * dispatch path computes, written from the source pages' definitions.  Only the
+ * test suite, the package's smoke check and the benchmark's CPU-baseline leg
+ * may load it.  It shares no code, header, table or helper with the CUDA
+ * library; the two meet only in the seeded inputs of the workload module.
+ *
+ * Sources (cited by page title and section):
+ *  [GR] "MoonEP: πώς η εξισορρόπηση των AI experts αλλάζει την υποδομή των
+ *       MoE μοντέλων" (twodots.gr)
+ *  [FR] "Moonshot AI открыла код MoonEP — библиотеки для обучения MoE-модели
+ *       Kimi K3" (news.hamidun.com)
+ *  [ZH] the MoE Align & Sort report (新智元报道, los70adestajo.com page)
+ *  [JA] "Xiaohongshuと北京大学がUltraEPを発表、静的MoE負荷分散に挑戦" (remio.ai)
+ *
+ * Notation: R ranks, S tokens per rank, K experts per token, E experts,
+ * E_R = E/R experts homed per rank, T = R*S tokens, P = T*K routed pairs,
+ * flattened pair index p = t*K + k.  Rank r owns buffer rows [r*S*K, (r+1)*S*K).
+ *
+ * Floating point: the pages fix fp32 accumulation for combine and gradient
+ * reduction and bf16 rows, so those are done in fp32 here, one IEEE operation
+ * at a time (the file is compiled with -ffp-contract=off: no fused multiply-add).
+ * max_vio is computed in fp64.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- bf16 */
+
+static float bf16_to_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* round to nearest, ties to even; NaN stays NaN */
+static uint16_t f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x40u);
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------ 1. stats */
+/*
+ * [FR] "Pourquoi le parallélisme d'experts est-il nécessaire": the imbalance
+ * metric is max_vio = max_e(T_e / T̄) - 1, zero meaning perfect balance; [GR]
+ * "Γιατί τα Mixture-of-Experts δημιουργούν πρόβλημα κατανομής" says the same.
+ * T_e = number of routed (token, k) pairs whose expert is e.  T̄ is read as
+ * the mean of T_e over the E experts, P / E, the only choice for which a
+ * perfectly even routing gives 0.  max_e(T_e / (P/E)) - 1 is evaluated as
+ * (max_e T_e) * E / P - 1 in fp64 (the product is exact).
+ *
+ * Returns the number of ids outside [0, E); those pairs are not counted.
+ */
+int64_t oracle_route_stats(const int32_t* topk, int64_t T, int K, int E, int32_t* loads, double* max_vio) {
+  int64_t P = T * (int64_t)K, bad = 0;
+  for (int e = 0; e < E; ++e) loads[e] = 0;
+  for (int64_t p = 0; p < P; ++p) {
+    int32_t e = topk[p];
+    if (e < 0 || e >= E) {
+      ++bad;
+      continue;
+    }
+    loads[e] += 1;
+  }
+  int32_t mx = 0;
+  for (int e = 0; e < E; ++e)
+    if (loads[e] > mx) mx = loads[e];
+  *max_vio = (P > 0) ? ((double)mx * (double)E) / (double)P - 1.0 : 0.0;
+  return bad;
+}
+
+/* ------------------------------------------------------------- 2. plan */
+/*
+ * [GR] "Η βασική υπόσχεση του MoonEP: σταθερό φορτίο S × K" and [FR]
+ * "Comment fonctionne MoonEP": every rank must end up processing exactly S*K
+ * routed pairs, which the library reaches by planning a few temporary copies
+ * (replicas) of hot experts on other ranks, online, from the current router
+ * output.  [JA] "その仕組みは高速なエキスパート複製に依存する": the plan
+ * decides which hot experts get copies, where each copy runs and how many
+ * tokens each instance takes.  The pages do not print the rule; this library's
+ * deterministic reading is:
+ *   - home placement: expert e lives on rank floor(e / E_R) ([GR] "Το memory
+ *     contract...": rows 0..E-1 hold the ranks' own experts);
+ *   - rank load L_r = sum of T_e over its home experts; excess X_r = L_r - S*K
+ *     when positive, deficit D_r = S*K - L_r when positive;
+ *   - each overloaded rank (ascending r) cuts its excess into chunks taken from
+ *     its home experts in DESCENDING id: chunk = min(T_e, remaining excess),
+ *     empty chunks skipped, stop when the excess is used up;
+ *   - the chunk sequence is matched against the deficit sequence (underloaded
+ *     ranks in ascending r) by walking both in order: each step emits one
+ *     replica (expert of the current chunk, rank of the current deficit,
+ *     min(chunk left, deficit left)) and advances whichever is exhausted (both
+ *     when they end together) -- the sequential form of a merge of the two
+ *     prefix sums.  Emission order is the "match order".
+ *   - home_count[e] = T_e minus the pairs its replicas take.
+ *
+ * Returns n_rep (>= 0), or -1 when sum(loads) != R*S*K.
+ */
+int oracle_plan(const int32_t* loads, int R, int64_t S, int K, int E, int32_t* rep_expert, int32_t* rep_rank,
+                int32_t* rep_count, int32_t* home_count) {
+  int ER = E / R;
+  int64_t SK = S * (int64_t)K;
+  int64_t total = 0;
+  for (int e = 0; e < E; ++e) total += loads[e];
+  if (total != (int64_t)R * SK) return -1;
+
+  int64_t* L = (int64_t*)calloc((size_t)R, sizeof(int64_t));
+  for (int e = 0; e < E; ++e) L[e / ER] += loads[e];
+
+  /* supply: chunks (expert, size) */
+  int32_t* ch_e = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+  int64_t* ch_n = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+  int nch = 0;
+  for (int r = 0; r < R; ++r) {
+    int64_t rem = L[r] - SK;
+    if (rem <= 0) continue;
+    for (int e = (r + 1) * ER - 1; e >= r * ER && rem > 0; --e) {
+      int64_t take = loads[e] < rem ? loads[e] : rem;
+      if (take <= 0) continue;
+      ch_e[nch] = e;
+      ch_n[nch] = take;
+      ++nch;
+      rem -= take;
+    }
+  }
+  /* demand: underloaded ranks (rank, deficit) */
+  int32_t* dm_r = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+  int64_t* dm_n = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
+  int ndm = 0;
+  for (int r = 0; r < R; ++r) {
+    if (SK - L[r] > 0) {
+      dm_r[ndm] = r;
+      dm_n[ndm] = SK - L[r];
+      ++ndm;
+    }
+  }
+  /* two-pointer walk */
+  int nrep = 0, i = 0, j = 0;
+  int64_t left_c = nch ? ch_n[0] : 0, left_d = ndm ? dm_n[0] : 0;
+  while (i < nch && j < ndm) {
+    int64_t take = left_c < left_d ? left_c : left_d;
+    rep_expert[nrep] = ch_e[i];
+    rep_rank[nrep] = dm_r[j];
+    rep_count[nrep] = (int32_t)take;
+    ++nrep;
+    left_c -= take;
+    left_d -= take;
+    if (left_c == 0) {
+      ++i;
+      if (i < nch) left_c = ch_n[i];
+    }
+    if (left_d == 0) {
+      ++j;
+      if (j < ndm) left_d = dm_n[j];
+    }
+  }
+  for (int e = 0; e < E; ++e) home_count[e] = loads[e];
+  for (int m = 0; m < nrep; ++m) home_count[rep_expert[m]] -= rep_count[m];
+
+  free(L);
+  free(ch_e);
+  free(ch_n);
+  free(dm_r);
+  free(dm_n);
+  return nrep;
+}
+
+/* ----------------------------------------------------------- 3. layout */
+/*
+ * [GR] "Online planning, zero copy και στατικά σχήματα": tokens are written
+ * straight to their final positions, grouped by expert, in a static S*K buffer
+ * per rank.  [JA] "UltraEPのMoE負荷分散はルーティング後に対応する": the
+ * selected tokens are split between the original expert and its temporary
+ * replicas.  Reading used here:
+ *   - pairs of each expert are listed in ascending flattened index p (a stable
+ *     grouping by expert, ties in (source rank, token, k) order);
+ *   - the home copy takes the first home_count[e] pairs of e's list, then each
+ *     replica of e, in match order, takes the next rep_count[m];
+ *   - rank r's rows, from r*S*K on, hold its home experts in id order, then the
+ *     replicas it receives in match order.
+ * Global slot ids: e for the home copy of e, E + m for replica m.  slot_order
+ * lists slot ids in buffer order; cu_seqlens[i] is the first row of the i-th
+ * slot in that order, cu_seqlens[E + n_rep] = P.
+ * pos[p] = row of pair p, src[row] = p, pair_slot[p] = slot id of pair p.
+ * Pairs with an id outside [0, E) get pos = -1 and slot = -1.
+ * Returns 0, or -1 if a rank's rows do not come out to S*K.
+ */
+int oracle_layout(const int32_t* topk, int64_t T, int K, int E, int R, int64_t S, int n_rep,
+                  const int32_t* rep_expert, const int32_t* rep_rank, const int32_t* rep_count,
+                  const int32_t* home_count, int32_t* pos, int32_t* src, int32_t* pair_slot, int32_t* slot_order,
+                  int32_t* cu_seqlens) {
+  int64_t P = T * (int64_t)K, SK = S * (int64_t)K;
+  int ER = E / R;
+  /* per-expert lists in ascending p */
+  int64_t* start = (int64_t*)calloc((size_t)E + 1, sizeof(int64_t));
+  for (int64_t p = 0; p < P; ++p)
+    if (topk[p] >= 0 && topk[p] < E) start[topk[p] + 1] += 1;
+  for (int e = 0; e < E; ++e) start[e + 1] += start[e];
+  int64_t* fill = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+  for (int e = 0; e < E; ++e) fill[e] = start[e];
+  int32_t* list = (int32_t*)malloc(sizeof(int32_t) * (size_t)(P > 0 ? P : 1));
+  for (int64_t p = 0; p < P; ++p) {
+    pos[p] = -1;
+    pair_slot[p] = -1;
+    if (topk[p] >= 0 && topk[p] < E) list[fill[topk[p]]++] = (int32_t)p;
+  }
+  /* where each copy's range starts in its expert's list: the home copy at 0,
+   * replica m after the home copy and the earlier replicas of the same expert */
+  int64_t* next = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+  for (int e = 0; e < E; ++e) next[e] = home_count[e];
+  int64_t* rep_first = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_rep > 0 ? n_rep : 1));
+  for (int m = 0; m < n_rep; ++m) {
+    rep_first[m] = next[rep_expert[m]];
+    next[rep_expert[m]] += rep_count[m];
+  }
+  int rc = 0, nslot = 0;
+  for (int r = 0; r < R; ++r) {
+    int64_t row = (int64_t)r * SK;
+    for (int e = r * ER; e < (r + 1) * ER; ++e) {
+      slot_order[nslot] = e;
+      cu_seqlens[nslot] = (int32_t)row;
+      ++nslot;
+      for (int64_t i = 0; i < home_count[e]; ++i) {
+        int32_t p = list[start[e] + i];
+        pos[p] = (int32_t)row;
+        src[row] = p;
+        pair_slot[p] = e;
+        ++row;
+      }
+    }
+    for (int m = 0; m < n_rep; ++m) {
+      if (rep_rank[m] != r) continue;
+      int e = rep_expert[m];
+      slot_order[nslot] = E + m;
+      cu_seqlens[nslot] = (int32_t)row;
+      ++nslot;
+      for (int64_t i = 0; i < rep_count[m]; ++i) {
+        int32_t p = list[start[e] + rep_first[m] + i];
+        pos[p] = (int32_t)row;
+        src[row] = p;
+        pair_slot[p] = E + m;
+        ++row;
+      }
+    }
+    if (row != (int64_t)(r + 1) * SK) rc = -1;
+  }
+  cu_seqlens[nslot] = (int32_t)P;
+  free(start);
+  free(fill);
+  free(list);
+  free(next);
+  free(rep_first);
+  return rc;
+}
+
+/* ------------------------------------------------------- 4. align-sort */
+/*
+ * [ZH] MoE Align & Sort: sort the routed token ids by expert id and pad each
+ * expert's group to a multiple of the block size, so the grouped GEMM can take
+ * every block from a single expert; the result carries one expert id per block
+ * and the padded total.  Readings: the ids sorted are flattened pair indices p
+ * (consumers recover the token as p / K), stable in p; padding and the unused
+ * tail hold the sentinel P; unused expert_ids entries hold -1; an expert with no
+ * pairs gets no block.
+ *   c_e = #pairs of e;  pc_e = ceil(c_e / block_m) * block_m;
+ *   off_e = sum_{e' < e} pc_e';  num_tokens_post_pad = sum_e pc_e;
+ *   sorted_ids[off_e + i] = i-th pair of e in ascending p, i < c_e.
+ * Returns num_tokens_post_pad, or -1 if a capacity is too small.
+ */
+int64_t oracle_align_sort(const int32_t* topk, int64_t T, int K, int E, int block_m, int32_t* sorted_ids,
+                          int64_t sorted_cap, int32_t* expert_ids, int64_t expert_ids_cap) {
+  int64_t P = T * (int64_t)K;
+  int64_t* cnt = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+  for (int64_t p = 0; p < P; ++p)
+    if (topk[p] >= 0 && topk[p] < E) cnt[topk[p]] += 1;
+  int64_t* off = (int64_t*)malloc(sizeof(int64_t) * ((size_t)E + 1));
+  off[0] = 0;
+  for (int e = 0; e < E; ++e) {
+    int64_t padded = (cnt[e] + block_m - 1) / block_m * block_m;
+    off[e + 1] = off[e] + padded;
+  }
+  int64_t total = off[E];
+  if (total > sorted_cap || total / block_m > expert_ids_cap) {
+    free(cnt);
+    free(off);
+    return -1;
+  }
+  for (int64_t i = 0; i < sorted_cap; ++i) sorted_ids[i] = (int32_t)P;
+  for (int64_t b = 0; b < expert_ids_cap; ++b) expert_ids[b] = -1;
+  int64_t* fill = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+  for (int e = 0; e < E; ++e) fill[e] = off[e];
+  for (int64_t p = 0; p < P; ++p)
+    if (topk[p] >= 0 && topk[p] < E) sorted_ids[fill[topk[p]]++] = (int32_t)p;
+  for (int e = 0; e < E; ++e)
+    for (int64_t b = off[e] / block_m; b < off[e + 1] / block_m; ++b) expert_ids[b] = e;
+  free(cnt);
+  free(off);
+  free(fill);
+  return total;
+}
+
+/* --------------------------------------------------------- 5. dispatch */
+/*
+ * [GR] "Online planning, zero copy και στατικά σχήματα": each routed copy of a
+ * token's hidden row is written straight into its final row of the expert-
+ * grouped buffer.  buf[pos[p]] = x[p / K], bitwise, for every pair p with a
+ * valid pos.
+ */
+void oracle_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf) {
+  int64_t P = T * (int64_t)K;
+  for (int64_t p = 0; p < P; ++p) {
+    if (pos[p] < 0) continue;
+    memcpy(buf + (int64_t)pos[p] * H, x + (p / K) * H, (size_t)H * 2);
+  }
+}
+
+/* Stand-in for the expert computation (the grouped GEMM is outside the path):
+ * y[row] = bf16_rn(float(buf[row]) * s[e]) with e the logical expert of the row,
+ * found through src: e = topk[src[row]]. */
+void oracle_expert_standin(const uint16_t* buf, int64_t nrows, int64_t H, const int32_t* src, const int32_t* topk,
+                           const float* scale, uint16_t* y) {
+  for (int64_t row = 0; row < nrows; ++row) {
+    float s = scale[topk[src[row]]];
+    for (int64_t h = 0; h < H; ++h) {
+      float v = bf16_to_f32(buf[row * H + h]) * s;
+      y[row * H + h] = f32_to_bf16(v);
+    }
+  }
+}
+
+/* ---------------------------------------------------------- 6. combine */
+/*
+ * [GR] "Τι δείχνουν — και τι δεν αποδεικνύουν — τα benchmarks" names combine
+ * among the steps of the layer: the K expert outputs of each token are brought
+ * back and weighted by the gate.  out[t] = bf16_rn( sum_{k=0..K-1} w[t,k] *
+ * float(y[pos[t*K+k]]) ), accumulated in fp32 in k order from 0.0f, each
+ * product and each sum rounded separately, one final rounding to bf16.
+ * Pairs with pos < 0 contribute nothing.
+ */
+void oracle_combine(const uint16_t* y, const float* w, const int32_t* pos, int64_t T, int K, int64_t H,
+                    uint16_t* out) {
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t h = 0; h < H; ++h) {
+      float acc = 0.0f;
+      for (int k = 0; k < K; ++k) {
+        int32_t row = pos[t * K + k];
+        if (row < 0) continue;
+        float prod = w[t * K + k] * bf16_to_f32(y[(int64_t)row * H + h]);
+        acc = acc + prod;
+      }
+      out[t * H + h] = f32_to_bf16(acc);
+    }
+  }
+}
+
+/*
+ * Combine for the stand-in expert in closed form.  Because the stand-in's
+ * output row depends only on the token and the logical expert, combine's
+ * result does not depend on the plan or the layout:
+ *   out[t] = bf16_rn( sum_k w[t,k] * float(bf16_rn(float(x[t]) * s[e_k])) ).
+ * Rows of x, w and topk are given for nt selected tokens (row i = token i of
+ * the selection), so the check streams at any workload size.
+ */
+void oracle_combine_closed(const uint16_t* x_rows, const float* w_rows, const int32_t* topk_rows, int64_t nt,
+                           int K, int64_t H, const float* scale, uint16_t* out) {
+  for (int64_t i = 0; i < nt; ++i) {
+    for (int64_t h = 0; h < H; ++h) {
+      float xv = bf16_to_f32(x_rows[i * H + h]);
+      float acc = 0.0f;
+      for (int k = 0; k < K; ++k) {
+        float yv = bf16_to_f32(f32_to_bf16(xv * scale[topk_rows[i * K + k]]));
+        float prod = w_rows[i * K + k] * yv;
+        acc = acc + prod;
+      }
+      out[i * H + h] = f32_to_bf16(acc);
+    }
+  }
+}
+
+/* ------------------------------------------------------ 7. grad reduce */
+/*
+ * [GR] "Τι συμβαίνει στους gradients κατά την εκπαίδευση": gradients are kept
+ * in fp32; replica slots write to a separate reduce buffer, and reduce_grad
+ * adds the slots belonging to a rank's own experts into the local parameter
+ * gradient and then clears the used slots.  [JA]: replica gradients are folded
+ * back into the primary expert.  Order used: for every element, the home value
+ * first, then each replica of that expert in match order, one fp32 add each:
+ *   g_home[e][j] = ((g_home[e][j] + g_rep[m1][j]) + g_rep[m2][j]) + ...
+ * rep_dtype 0: g_rep is fp32; 1: bf16 (widened exactly to fp32 before the add).
+ * clear != 0 zeroes each used replica row afterwards.
+ */
+void oracle_grad_reduce(float* g_home, void* g_rep, int rep_dtype, int64_t n, int n_rep, const int32_t* rep_expert,
+                        int clear) {
+  for (int m = 0; m < n_rep; ++m) {
+    float* dst = g_home + (int64_t)rep_expert[m] * n;
+    if (rep_dtype == 0) {
+      float* g = (float*)g_rep + (int64_t)m * n;
+      for (int64_t j = 0; j < n; ++j) dst[j] = dst[j] + g[j];
+      if (clear) memset(g, 0, (size_t)n * 4);
+    } else {
+      uint16_t* g = (uint16_t*)g_rep + (int64_t)m * n;
+      for (int64_t j = 0; j < n; ++j) dst[j] = dst[j] + bf16_to_f32(g[j]);
+      if (clear) memset(g, 0, (size_t)n * 2);
+    }
+  }
+}

@@ -1,0 +1,476 @@
+"""Pins for the CPU oracle: checks against facts fixed by the source pages and
+by mathematics, never against the oracle itself.
+
+Each pin takes a loaded oracle library `L` (so the mutation tests can run the
+same pins on deliberately broken copies) and raises AssertionError on failure.
+
+Kinds of pin used:
+  * the hand-worked 4-rank example (tests/golden/hand_example_4rank.json), every
+    value derived by hand from the definitions;
+  * brute force: all P! row permutations of tiny cases, filtered by the
+    layout's defining predicates -- exactly one must survive;
+  * reductions to library routines in special cases (numpy stable argsort,
+    fancy indexing, float32 adds);
+  * closed forms (max_vio of uniform / single-expert routing) and fp64 error
+    bounds for the fp32 sums;
+  * invariants the pages state (S*K rows per rank, routing unchanged, copies of
+    an expert add up to T_e).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle as O
+import workload as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_example_4rank.json")
+
+
+def golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- helpers
+
+def unit_plan(loads, R, S, K, E):
+    """Independent statement of the replica rule at the level of single pairs:
+    list the excess pairs one by one (overloaded ranks ascending, within a rank
+    its home experts by descending id, each expert giving up to what is still
+    in excess), list the missing pairs one by one (underloaded ranks ascending),
+    pair them up position by position, and merge runs of equal (expert, rank)."""
+    ER, SK = E // R, S * K
+    excess_units, deficit_units = [], []
+    for r in range(R):
+        Lr = sum(int(loads[e]) for e in range(r * ER, (r + 1) * ER))
+        if Lr > SK:
+            rem = Lr - SK
+            for e in reversed(range(r * ER, (r + 1) * ER)):
+                take = min(int(loads[e]), rem)
+                excess_units += [e] * take
+                rem -= take
+        elif Lr < SK:
+            deficit_units += [r] * (SK - Lr)
+    assert len(excess_units) == len(deficit_units)
+    reps = []
+    for e, r in zip(excess_units, deficit_units):
+        if reps and reps[-1][0] == e and reps[-1][1] == r:
+            reps[-1][2] += 1
+        else:
+            reps.append([e, r, 1])
+    return reps
+
+
+def slots_from_plan(pl, R, S, K, E):
+    """Buffer slots in order: (slot id, logical expert, first row, rows)."""
+    ER, SK = E // R, S * K
+    out = []
+    for r in range(R):
+        row = r * SK
+        for e in range(r * ER, (r + 1) * ER):
+            out.append((e, e, row, int(pl["home_count"][e])))
+            row += int(pl["home_count"][e])
+        for m in range(pl["n_rep"]):
+            if pl["rep_rank"][m] == r:
+                out.append((E + m, int(pl["rep_expert"][m]), row, int(pl["rep_count"][m])))
+                row += int(pl["rep_count"][m])
+        assert row == (r + 1) * SK, "rank does not hold exactly S*K rows"
+    return out
+
+
+def layout_predicates_hold(pos, topk_flat, pl, R, S, K, E):
+    """The defining predicates of the layout, given the plan."""
+    slots = slots_from_plan(pl, R, S, K, E)
+    P = len(topk_flat)
+    row_slot = np.empty(P, dtype=np.int64)
+    row_expert = np.empty(P, dtype=np.int64)
+    for sid, e, first, n in slots:
+        row_slot[first:first + n] = sid
+        row_expert[first:first + n] = e
+    # routing unchanged: the row's copy is a copy of the pair's expert
+    if not np.array_equal(row_expert[pos], topk_flat):
+        return False
+    # within a slot, rows follow ascending p
+    src = np.empty(P, dtype=np.int64)
+    src[pos] = np.arange(P)
+    for sid, e, first, n in slots:
+        if n > 1 and not np.all(np.diff(src[first:first + n]) > 0):
+            return False
+    # an expert's copies take consecutive ranges of its pairs: home first, then
+    # replicas in match order
+    for e in range(E):
+        copies = [s for s in slots if s[1] == e and s[0] == e] + sorted(
+            [s for s in slots if s[1] == e and s[0] >= E], key=lambda s: s[0])
+        last = -1
+        for sid, _, first, n in copies:
+            if n == 0:
+                continue
+            ps = src[first:first + n]
+            if ps.min() <= last:
+                return False
+            last = ps.max()
+    return True
+
+
+def check_layout_invariants(topk, pl, lo, R, S, K, E):
+    topk_flat = np.asarray(topk, dtype=np.int64).reshape(-1)
+    P = topk_flat.size
+    SK = S * K
+    pos, src = lo["pos"].astype(np.int64), lo["src"].astype(np.int64)
+    # pos is a permutation of [0, P) and src its inverse
+    assert np.array_equal(np.sort(pos), np.arange(P))
+    assert np.array_equal(src[pos], np.arange(P))
+    # S*K rows per rank: every row index in [r*SK, (r+1)*SK) is used once (permutation)
+    # and the slot lengths of each rank add up to S*K
+    cu = lo["cu_seqlens"].astype(np.int64)
+    order = lo["slot_order"]
+    n_rep = pl["n_rep"]
+    assert len(order) == E + n_rep and cu[0] == 0 and cu[-1] == P and np.all(np.diff(cu) >= 0)
+    # slot -> logical expert
+    slot_expert = np.concatenate([np.arange(E), np.asarray(pl["rep_expert"], dtype=np.int64)])
+    assert np.array_equal(slot_expert[lo["pair_slot"]], topk_flat), "routing changed"
+    # each pair's row lies inside its slot's range
+    where = np.empty(E + n_rep, dtype=np.int64)
+    where[order] = np.arange(E + n_rep)
+    i = where[lo["pair_slot"]]
+    assert np.all(cu[i] <= pos) and np.all(pos < cu[i + 1])
+    # rank sizes: slot ranges of rank r stay in [r*SK, (r+1)*SK)
+    ER = E // R
+    for r in range(R):
+        assert np.sum((pos >= r * SK) & (pos < (r + 1) * SK)) == SK
+    # copies of each expert add up to T_e
+    loads = np.bincount(topk_flat, minlength=E)
+    per = np.asarray(pl["home_count"], dtype=np.int64).copy()
+    np.add.at(per, np.asarray(pl["rep_expert"], dtype=np.int64), np.asarray(pl["rep_count"], dtype=np.int64))
+    assert np.array_equal(per, loads)
+    # replicas go from overloaded home ranks to underloaded ranks
+    rank_load = loads.reshape(R, ER).sum(1)
+    for m in range(n_rep):
+        e, r = int(pl["rep_expert"][m]), int(pl["rep_rank"][m])
+        assert rank_load[e // ER] > SK and rank_load[r] < SK and r != e // ER
+        assert pl["rep_count"][m] > 0
+    return True
+
+
+# ------------------------------------------------------------------- pins
+
+def pin_hand_example(L):
+    g = golden()
+    R, S, K, E, bm = g["R"], g["S"], g["K"], g["E"], g["block_m"]
+    topk = np.array(g["topk_ids"], dtype=np.int32)
+    loads, mv, bad = O.route_stats(topk, E, L=L)
+    assert bad == 0
+    assert loads.tolist() == g["loads"]
+    assert mv == g["max_vio"]
+    pl = O.plan(loads, R, S, K, E, L=L)
+    assert [[int(a), int(b), int(c)] for a, b, c in zip(pl["rep_expert"], pl["rep_rank"], pl["rep_count"])] == \
+        g["replicas"]
+    assert pl["home_count"].tolist() == g["home_count"]
+    lo = O.layout(topk, pl, R, S, E, L=L)
+    assert lo["pos"].tolist() == g["pos"]
+    assert lo["slot_order"].tolist() == g["slot_order"]
+    assert lo["cu_seqlens"].tolist() == g["cu_seqlens"]
+    ids, eids, n = O.align_sort(topk, E, bm, L=L)
+    assert n == g["align_num_tokens_post_pad"]
+    assert len(ids) == g["align_capacity"]
+    pre = g["align_sorted_token_ids_prefix"]
+    assert ids[:len(pre)].tolist() == pre
+    assert np.all(ids[len(pre):] == g["align_sentinel"])
+    assert eids.tolist() == g["align_expert_ids"]
+
+
+def pin_max_vio_closed_forms(L):
+    # uniform routing: every expert gets P/E pairs -> 0 (perfect balance)
+    for (T, E, K) in [(64, 16, 2), (96, 8, 4), (256, 64, 8)]:
+        topk, _ = W.routing_from(T, E, K, seed=1, uniform=True)
+        loads, mv, _ = O.route_stats(topk, E, L=L)
+        assert np.all(loads == T * K // E) and mv == 0.0
+    # all tokens on one expert with K = 1: max T_e = P, mean P/E -> E - 1
+    for E in (2, 7, 64):
+        topk = np.full((40, 1), E - 1, dtype=np.int32)
+        loads, mv, _ = O.route_stats(topk, E, L=L)
+        assert loads[E - 1] == 40 and loads[:E - 1].sum() == 0 and mv == float(E - 1)
+    # ids out of range are reported, not counted
+    topk = np.array([[0, 1], [2, 9]], dtype=np.int32)
+    loads, mv, bad = O.route_stats(topk, 4, L=L)
+    assert bad == 1 and loads.tolist() == [1, 1, 1, 0]
+    # a generic case against exact rational arithmetic: max_e T_e / (P/E) - 1
+    topk, _ = W.routing_from(300, 12, 3, seed=5, bias_e=np.linspace(1, -1, 12))
+    loads, mv, _ = O.route_stats(topk, 12, L=L)
+    ref = np.bincount(topk.ravel(), minlength=12)
+    from fractions import Fraction
+    exact = Fraction(int(ref.max()), 1) / Fraction(900, 12) - 1
+    assert loads.tolist() == ref.tolist()
+    assert abs(mv - float(exact)) <= 2 * math.ulp(float(exact) + 1.0)
+
+
+def _rand_loads(rng, R, ER, SK):
+    E = R * ER
+    total = R * SK
+    mode = rng.integers(0, 4)
+    if mode == 0:  # multinomial with a random skew
+        p = rng.dirichlet(np.full(E, rng.uniform(0.1, 3.0)))
+        return rng.multinomial(total, p).astype(np.int32)
+    if mode == 1:  # one hot expert
+        loads = np.zeros(E, dtype=np.int32)
+        loads[rng.integers(0, E)] = total
+        return loads
+    if mode == 2:  # balanced
+        loads = np.zeros(E, dtype=np.int32)
+        for r in range(R):
+            part = rng.multinomial(SK, np.full(ER, 1.0 / ER))
+            loads[r * ER:(r + 1) * ER] = part
+        return loads
+    loads = rng.multinomial(total, np.full(E, 1.0 / E)).astype(np.int32)  # near uniform
+    return loads
+
+
+def pin_plan_unit_restatement(L):
+    rng = np.random.default_rng(1234)
+    for it in range(400):
+        R = int(rng.choice([1, 2, 3, 4, 5, 8]))
+        ER = int(rng.integers(1, 6))
+        SK = int(rng.integers(1, 40))
+        E = R * ER
+        K = int(rng.integers(1, 4))
+        if SK % K:
+            SK = K * max(1, SK // K)
+        S = SK // K
+        loads = _rand_loads(rng, R, ER, SK)
+        pl = O.plan(loads, R, S, K, E, L=L)
+        ref = unit_plan(loads, R, S, K, E)
+        got = [[int(a), int(b), int(c)] for a, b, c in zip(pl["rep_expert"], pl["rep_rank"], pl["rep_count"])]
+        assert got == ref, (loads.tolist(), R, S, K, got, ref)
+        # every rank ends with exactly S*K pairs
+        rows = np.zeros(R, dtype=np.int64)
+        for e in range(E):
+            rows[e // ER] += pl["home_count"][e]
+        for e, r, c in got:
+            rows[r] += c
+        assert np.all(rows == SK)
+        assert np.all(pl["home_count"] >= 0)
+        n_chunks = len({e for e, _, _ in got})
+        n_def = len({r for _, r, _ in got})
+        assert len(got) <= max(0, n_chunks + n_def - 1)
+        assert len(got) <= E + R - 1
+    # uniform loads: no replica at all
+    pl = O.plan(np.full(16, 8, dtype=np.int32), 4, 16, 2, 16, L=L)
+    assert pl["n_rep"] == 0 and np.all(pl["home_count"] == 8)
+
+
+def pin_layout_brute_force(L):
+    """All P! permutations of the rows of tiny cases; exactly one satisfies the
+    layout's defining predicates, and it is the oracle's."""
+    rng = np.random.default_rng(7)
+    cases = []
+    for R, E, S, K in [(2, 2, 2, 2), (2, 4, 2, 2), (2, 4, 4, 1), (2, 2, 4, 1), (1, 3, 2, 2), (2, 4, 1, 2)]:
+        for _ in range(3):
+            T = R * S
+            topk = np.stack([rng.choice(E, size=K, replace=False) for _ in range(T)]).astype(np.int32)
+            cases.append((R, E, S, K, topk))
+    # a degenerate one: all pairs on expert 0
+    cases.append((2, 2, 4, 1, np.zeros((8, 1), dtype=np.int32)))
+    for R, E, S, K, topk in cases:
+        P = R * S * K
+        loads, _, _ = O.route_stats(topk, E, L=L)
+        pl = O.plan(loads, R, S, K, E, L=L)
+        lo = O.layout(topk, pl, R, S, E, L=L)
+        flat = topk.reshape(-1).astype(np.int64)
+        survivors = [np.array(perm) for perm in itertools.permutations(range(P))
+                     if layout_predicates_hold(np.array(perm), flat, pl, R, S, K, E)]
+        assert len(survivors) == 1, (topk.tolist(), len(survivors))
+        assert np.array_equal(survivors[0], lo["pos"])
+
+
+def pin_layout_library_reductions(L):
+    """With no replicas (one rank, or balanced ranks), rows are the pairs sorted
+    by expert, stable in p: the inverse of numpy's stable argsort."""
+    for seed, (R, S, K, E) in enumerate([(1, 50, 3, 7), (1, 300, 8, 64), (4, 10, 2, 8)]):
+        if R == 1:
+            topk, _ = W.routing_from(R * S, E, K, seed=seed, bias_e=np.linspace(2, -2, E))
+        else:
+            topk, _ = W.routing_from(R * S, E, K, seed=seed, uniform=True)
+        loads, _, _ = O.route_stats(topk, E, L=L)
+        pl = O.plan(loads, R, S, K, E, L=L)
+        assert pl["n_rep"] == 0
+        lo = O.layout(topk, pl, R, S, E, L=L)
+        src = np.argsort(topk.reshape(-1), kind="stable")
+        assert np.array_equal(lo["src"], src)
+        assert np.array_equal(lo["pos"][src], np.arange(R * S * K))
+
+
+def pin_layout_invariants(L):
+    rng = np.random.default_rng(99)
+    for it in range(40):
+        R = int(rng.choice([1, 2, 3, 4, 8]))
+        ER = int(rng.integers(1, 7))
+        E = R * ER
+        K = int(rng.integers(1, min(8, E) + 1))
+        S = int(rng.integers(1, 50))
+        variant = rng.integers(0, 3)
+        if variant == 0:
+            topk, _ = W.routing_from(R * S, E, K, seed=it, bias_e=rng.normal(0, 2, E))
+        elif variant == 1:
+            topk, _ = W.routing_from(R * S, E, K, seed=it, uniform=True)
+        else:
+            topk, _ = W.routing_from(R * S, E, K, seed=it, force_expert0=True)
+        loads, _, _ = O.route_stats(topk, E, L=L)
+        pl = O.plan(loads, R, S, K, E, L=L)
+        lo = O.layout(topk, pl, R, S, E, L=L)
+        check_layout_invariants(topk, pl, lo, R, S, K, E)
+
+
+def pin_align_sort(L):
+    # block_m = 1: no padding; the ids are numpy's stable argsort by expert
+    for seed, (T, K, E) in enumerate([(37, 3, 9), (200, 8, 64), (16, 2, 8)]):
+        topk, _ = W.routing_from(T, E, K, seed=seed, bias_e=np.linspace(1.5, -1.5, E))
+        ids, eids, n = O.align_sort(topk, E, 1, L=L)
+        P = T * K
+        assert n == P
+        assert np.array_equal(ids[:P], np.argsort(topk.reshape(-1), kind="stable"))
+        assert np.array_equal(eids[:P], np.sort(topk.reshape(-1)))
+    # invariants at several block sizes, including experts with no pairs
+    rng = np.random.default_rng(3)
+    for it in range(30):
+        E = int(rng.integers(1, 40))
+        K = int(rng.integers(1, min(E, 8) + 1))
+        T = int(rng.integers(0, 200))
+        bm = int(rng.choice([1, 2, 3, 4, 16, 64, 128]))
+        topk, _ = W.routing_from(T, E, K, seed=it, bias_e=rng.normal(0, 2, E)) if T else \
+            (np.zeros((0, K), np.int32), None)
+        P = T * K
+        ids, eids, n = O.align_sort(topk, E, bm, L=L)
+        cap, capb = O.align_sort_capacity(P, E, bm)
+        assert len(ids) == cap and len(eids) == capb
+        assert n % bm == 0
+        counts = np.bincount(topk.reshape(-1), minlength=E)
+        assert n == sum(-(-int(c) // bm) * bm for c in counts)
+        assert np.all(ids[n:] == P) and np.all(eids[n // bm:] == -1)
+        valid = ids[:n][ids[:n] != P]
+        assert np.array_equal(np.sort(valid), np.arange(P))
+        flat = topk.reshape(-1)
+        for b in range(n // bm):
+            blk = ids[b * bm:(b + 1) * bm]
+            blk = blk[blk != P]
+            assert len(blk) > 0  # no block is padding only
+            assert np.all(flat[blk] == eids[b])
+            assert np.all(np.diff(blk) > 0)
+        assert np.all(np.diff(eids[:n // bm]) >= 0)
+
+
+def pin_dispatch(L):
+    rng = np.random.default_rng(11)
+    for (R, S, K, E, H) in [(2, 3, 2, 4, 8), (4, 16, 4, 16, 64), (1, 5, 1, 3, 16)]:
+        topk, _ = W.routing_from(R * S, E, K, seed=int(rng.integers(1 << 30)), bias_e=rng.normal(0, 1, E))
+        loads, _, _ = O.route_stats(topk, E, L=L)
+        pl = O.plan(loads, R, S, K, E, L=L)
+        lo = O.layout(topk, pl, R, S, E, L=L)
+        x = W.hidden(R * S, H, seed=3)
+        buf = O.dispatch(x, lo["pos"], K, R * S * K, L=L)
+        ref = np.zeros_like(buf)
+        ref[lo["pos"]] = np.repeat(x, K, axis=0)  # numpy scatter
+        assert np.array_equal(buf, ref)
+
+
+def pin_combine(L):
+    rng = np.random.default_rng(5)
+    # hand-computed rounding cases, K = 1, y = 1.0: the result is bf16_rn(w).
+    # bf16 keeps 8 significant bits, so in [1, 2) its spacing is 2^-7:
+    #   1 + 2^-8      is halfway between 1 and 1 + 2^-7       -> ties to even: 1.0
+    #   1 + 3*2^-8    is halfway between 1 + 2^-7 and 1 + 2^-6 -> ties to even: 1 + 2^-6
+    #   1 + 2^-8 + 2^-20 is above halfway                       -> 1 + 2^-7
+    #   -(1 + 2^-8)   ties to even, sign kept                    -> -1.0
+    ws = np.array([[1 + 2.0 ** -8], [1 + 3 * 2.0 ** -8], [1 + 2.0 ** -8 + 2.0 ** -20], [-(1 + 2.0 ** -8)]],
+                  dtype=np.float32)
+    one = np.full((4, 1), 0x3F80, dtype=np.uint16)  # bf16 1.0
+    out = O.combine(one, ws, np.arange(4, dtype=np.int32), 1, L=L)
+    assert O.bf16_to_f32(out[:, 0]).tolist() == [1.0, 1 + 2.0 ** -6, 1 + 2.0 ** -7, -1.0]
+    # K = 1, w = 1: out is the y row itself, bit for bit
+    T, H, E = 20, 32, 6
+    topk = rng.integers(0, E, size=(T, 1)).astype(np.int32)
+    y = W.hidden(T, H, seed=9)
+    pos = rng.permutation(T).astype(np.int32)
+    out = O.combine(y, np.ones((T, 1), np.float32), pos, 1, L=L)
+    assert np.array_equal(out, y[pos])
+    # general K: within fp32-sum error bound of the fp64 sum, then one bf16 rounding
+    for (R, S, K, E, H) in [(2, 8, 4, 8, 16), (4, 12, 3, 12, 40), (2, 4, 2, 2, 8)]:
+        T = R * S
+        topk, w = W.routing_from(T, E, K, seed=int(rng.integers(1 << 30)), bias_e=rng.normal(0, 1, E))
+        loads, _, _ = O.route_stats(topk, E, L=L)
+        pl = O.plan(loads, R, S, K, E, L=L)
+        lo = O.layout(topk, pl, R, S, E, L=L)
+        y = W.hidden(T * K, H, seed=17)
+        out = O.combine(y, w, lo["pos"], K, L=L)
+        yf = O.bf16_to_f32(y).astype(np.float64)
+        rows = yf[lo["pos"].reshape(T, K)]                       # [T, K, H]
+        exact = np.einsum("tk,tkh->th", w.astype(np.float64), rows)
+        absum = np.einsum("tk,tkh->th", np.abs(w.astype(np.float64)), np.abs(rows))
+        got = O.bf16_to_f32(out).astype(np.float64)
+        # fp32 error of K products and K-1 adds, plus half a bf16 ulp of the result
+        bound = 2 * K * 2.0 ** -24 * absum + np.abs(exact) * 2.0 ** -8 + 1e-30
+        assert np.all(np.abs(got - exact) <= bound)
+        # the stand-in expert's closed form agrees with the definition through the layout
+        scale = W.expert_scale(E)
+        x = W.hidden(T, H, seed=21)
+        buf = O.dispatch(x, lo["pos"], K, T * K, L=L)
+        y2 = O.expert_standin(buf, lo["src"], topk, scale, L=L)
+        out_def = O.combine(y2, w, lo["pos"], K, L=L)
+        out_cf = O.combine_closed(x, w, topk, scale, L=L)
+        assert np.array_equal(out_def, out_cf)
+        # and the closed form is the bf16 rounding of an fp32 sum within the bound
+        xf = O.bf16_to_f32(x).astype(np.float64)
+        yv = O.bf16_to_f32(
+            _bf16_rne((O.bf16_to_f32(x)[:, None, :] * scale[topk][:, :, None]).astype(np.float32))
+        ).astype(np.float64)
+        exact = np.einsum("tk,tkh->th", w.astype(np.float64), yv)
+        absum = np.einsum("tk,tkh->th", np.abs(w.astype(np.float64)), np.abs(yv))
+        got = O.bf16_to_f32(out_cf).astype(np.float64)
+        assert np.all(np.abs(got - exact) <= 2 * K * 2.0 ** -24 * absum + np.abs(exact) * 2.0 ** -8 + 1e-30)
+        del xf
+
+
+def _bf16_rne(f32):
+    u = np.asarray(f32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def pin_grad_reduce(L):
+    rng = np.random.default_rng(8)
+    E, n = 6, 257
+    g_home = W.grad_rows(1, W.STREAM_GHOME, n, E)
+    # no replica: unchanged
+    gh, _ = O.grad_reduce(g_home, np.zeros((1, n), np.float32), [], L=L)
+    assert np.array_equal(gh, g_home)
+    # one replica: the single fp32 add (numpy float32 addition)
+    g_rep = W.grad_rows(2, W.STREAM_GREP, n, 1)
+    gh, _ = O.grad_reduce(g_home, g_rep, [4], L=L)
+    ref = g_home.copy()
+    ref[4] = (g_home[4] + g_rep[0]).astype(np.float32)
+    assert np.array_equal(gh, ref)
+    # several replicas per expert, in match order, fp32 and bf16 replica rows
+    rep_expert = [2, 2, 5, 0, 2]
+    for dt in ("f32", "bf16"):
+        g_rep = W.grad_rows(3, W.STREAM_GREP, n, len(rep_expert), dtype=dt)
+        gr_f = g_rep if dt == "f32" else O.bf16_to_f32(g_rep)
+        gh, gr2 = O.grad_reduce(g_home, g_rep, rep_expert, clear=True, L=L)
+        ref = g_home.copy()
+        for m, e in enumerate(rep_expert):  # home first, then replicas in match order
+            ref[e] = (ref[e] + gr_f[m]).astype(np.float32)
+        assert np.array_equal(gh, ref)
+        assert not np.any(gr2)  # cleared
+        # fp64 bound: at most 3 fp32 adds per element
+        exact = g_home.astype(np.float64).copy()
+        absum = np.abs(exact).copy()
+        for m, e in enumerate(rep_expert):
+            exact[e] += gr_f[m]
+            absum[e] += np.abs(gr_f[m])
+        assert np.all(np.abs(gh - exact) <= 3 * 2.0 ** -24 * absum + 1e-30)
+        _ = rng
+
+
+ALL_PINS = [pin_hand_example, pin_max_vio_closed_forms, pin_plan_unit_restatement, pin_layout_brute_force,
+            pin_layout_library_reductions, pin_layout_invariants, pin_align_sort, pin_dispatch, pin_combine,
+            pin_grad_reduce]
