@@ -1,0 +1,246 @@
+/*
+ * ep.h -- C ABI of the B200 expert-parallel dispatch library (libep.so).
+ *
+ * The hot path of an expert-parallel MoE layer whose ranks are balanced by
+ * online redundant experts, with the R expert-parallel ranks simulated as R
+ * partitions of one static buffer on one GPU:
+ *
+ *   ep_route_stats -> ep_plan -> ep_layout -> ep_dispatch -> (expert) -> ep_combine
+ *   ep_align_sort (block-aligned expert sort for a grouped GEMM)
+ *   ep_replica_grad_reduce (backward: replica gradients into the home expert)
+ *
+ * Sources, cited by page title and section:
+ *  [GR] "MoonEP: πώς η εξισορρόπηση των AI experts αλλάζει την υποδομή των MoE
+ *       μοντέλων" (twodots.gr)
+ *  [FR] "Moonshot AI открыла код MoonEP — библиотеки для обучения MoE-модели
+ *       Kimi K3" (news.hamidun.com)
+ *  [ZH] the MoE Align & Sort report (新智元报道, los70adestajo.com page)
+ *  [JA] "Xiaohongshuと北京大学がUltraEPを発表、静的MoE負荷分散に挑戦" (remio.ai)
+ *
+ * Notation: R ranks, S tokens per rank, K experts per token (top-K), E experts,
+ * E_R = E/R experts homed contiguously per rank (expert e lives on rank
+ * floor(e/E_R)), H hidden size, T = R*S tokens, P = T*K routed (token, k)
+ * pairs, flattened pair index p = t*K + k.  The dispatch buffer has P rows; rank
+ * r owns rows [r*S*K, (r+1)*S*K).
+ *
+ * Conventions shared by every call:
+ *  - Array arguments are DEVICE pointers, owned by the caller, unless a comment
+ *    says "host".  Bases must be 16-byte aligned; row-major, contiguous.
+ *  - bf16 data are passed as uint16_t bit patterns.
+ *  - Every call that takes a stream only enqueues work on it: no host
+ *    synchronisation, no device or host allocation.  ep_status_read is the one
+ *    call that waits.
+ *  - Return value: EP_OK, or a negative EP_ERR_* code when an argument is
+ *    invalid (nothing is enqueued) or a launch failed.
+ *  - Problems the device detects (an expert id outside [0, E), a row index
+ *    outside the buffer, loads that do not add up, a bounded wait that ran out)
+ *    are OR-ed as EP_DEV_* bits into the caller's int32 *dev_status; the outputs
+ *    are then defined but unspecified, and no write goes out of bounds.
+ *  - Limits: 1 <= K <= min(E, 32), E <= EP_MAX_EXPERTS, R <= EP_MAX_RANKS,
+ *    E % R == 0, H % 8 == 0, P < 2^31.
+ *  - The dispatch buffer and the combine input are views that the next dispatch
+ *    or combine overwrites ([GR] "Ένα ρεαλιστικό πλαίσιο αξιολόγησης πριν από
+ *    την υιοθέτηση": zero-copy views must not be kept past the next dispatch or
+ *    combine, nor saved by autograd).
+ */
+#ifndef TDH_EP_H
+#define TDH_EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EP_OK 0
+#define EP_ERR_ARG (-1)      /* invalid argument; nothing enqueued */
+#define EP_ERR_CAPACITY (-2) /* a caller buffer is too small; nothing enqueued */
+#define EP_ERR_CUDA (-3)     /* a CUDA launch or copy failed */
+
+#define EP_DEV_BAD_EXPERT_ID 0x1     /* a topk id outside [0, E) */
+#define EP_DEV_LOOKBACK_TIMEOUT 0x2  /* a bounded inter-block wait gave up */
+#define EP_DEV_BAD_LOADS 0x4         /* loads do not sum to R*S*K, or are negative */
+#define EP_DEV_BAD_ROW 0x8           /* a row index outside the buffer */
+#define EP_DEV_COPY_TIMEOUT 0x10     /* a bounded wait on an asynchronous copy gave up */
+
+#define EP_MAX_EXPERTS 1024
+#define EP_MAX_RANKS 1024
+
+#define EP_DTYPE_F32 0
+#define EP_DTYPE_BF16 1
+
+/*
+ * Layout of the plan buffer (int32 words) written by ep_plan.  Every field is an
+ * offset, in int32 elements, from the start of the buffer; `words` is its size.
+ * cap = E + R - 1 bounds the number of replicas (each replica ends at a chunk
+ * boundary or a deficit boundary: at most E chunks plus R deficits, minus one).
+ * Slot ids: e for the home copy of expert e, E + m for replica m.
+ */
+typedef struct {
+  int64_t words;      /* total size in int32 elements */
+  int32_t cap;        /* E + R - 1 */
+  int32_t n_rep;      /* [1] number of replicas */
+  int32_t n_chunks;   /* [1] number of replicated experts (chunks) */
+  int32_t rank_load;  /* [R] L_r = sum of T_e over rank r's home experts */
+  int32_t rank_nrep;  /* [R] replicas received by rank r */
+  int32_t rank_rep_first; /* [R] match index of rank r's first received replica
+                             (= replicas received by ranks < r) */
+  int32_t home_count; /* [E] pairs kept by the home copy of e */
+  int32_t home_base;  /* [E] first buffer row of the home copy of e */
+  int32_t copy_first; /* [E] match index of e's first replica (0 if none) */
+  int32_t copy_cnt;   /* [E] number of replicas of e */
+  int32_t rep_expert; /* [cap] logical expert of replica m (match order) */
+  int32_t rep_rank;   /* [cap] receiving rank of replica m */
+  int32_t rep_count;  /* [cap] pairs taken by replica m */
+  int32_t rep_begin;  /* [cap] offset of replica m's range in e's pair list */
+  int32_t rep_base;   /* [cap] first buffer row of replica m */
+  int32_t rep_experts;/* [E] replicated experts in match order (n_chunks valid) */
+  int32_t slot_order; /* [E + cap] slot ids in buffer order; -1 past E + n_rep */
+  int32_t cu_seqlens; /* [E + cap + 1] first row of each slot in buffer order;
+                         entries from E + n_rep on hold R*S*K */
+} EpPlanLayout;
+
+/* Library version string (host). */
+EP_API const char* ep_version(void);
+
+/* Number of CUDA kernels this library has launched in this process (host
+ * counter, incremented at each launch). */
+EP_API uint64_t ep_launch_count(void);
+
+/*
+ * Bytes of scratch (`ws`) that ep_route_stats, ep_layout and ep_align_sort need
+ * for T tokens, K, E.  Host only.  The same ws must be passed to ep_route_stats
+ * and then ep_layout for the same topk_ids: ep_layout reads the per-tile
+ * per-expert prefix counts that ep_route_stats left there.
+ */
+EP_API int ep_workspace_size(int64_t T, int K, int E, size_t* bytes /* host out */);
+
+/* Fill *layout (host) with the plan buffer layout for E, R.  Host only. */
+EP_API int ep_plan_layout(int E, int R, EpPlanLayout* layout /* host out */);
+
+/*
+ * a1. Per-expert loads and imbalance.  [FR] "Pourquoi le parallélisme d'experts
+ * est-il nécessaire": max_vio = max_e(T_e / T̄) - 1, 0 for perfect balance;
+ * T̄ is the mean load P/E.
+ *   topk_ids [T, K] int32: expert of pair p = t*K + k.
+ *   loads    [E] int32 out: T_e = #{p : topk_ids[p] == e}.
+ *   max_vio  [1] double out: (max_e T_e) * E / P - 1 in fp64 (0 when P == 0).
+ *   ws       scratch of ep_workspace_size bytes; keeps per-tile prefix counts.
+ * One histogram pass with a single-pass decoupled look-back scan over tiles;
+ * integer adds only, so the result does not depend on scheduling.
+ */
+EP_API int ep_route_stats(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads, double* max_vio, void* ws,
+                   size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * a2. Replica plan.  [GR] "Η βασική υπόσχεση του MoonEP: σταθερό φορτίο S × K":
+ * every rank ends with exactly S*K pairs, by copying hot experts to other ranks
+ * for this step.  Rule (the pages leave it open; this library's deterministic
+ * reading): rank load L_r; an overloaded rank's excess L_r - S*K is cut into
+ * chunks taken from its home experts in descending id (chunk = min(T_e, excess
+ * left)); underloaded ranks' deficits S*K - L_r are taken in ascending rank;
+ * the two sequences are matched by a merge over their prefix sums, and every
+ * piece of the merge is one replica (expert, receiving rank, count), in "match
+ * order".
+ *   loads [E] int32 (from ep_route_stats); must sum to R*S*K.
+ *   plan  int32 buffer of EpPlanLayout.words elements, written in full.
+ * One block of 1024 threads.
+ */
+EP_API int ep_plan(const int32_t* loads, int R, int64_t S, int K, int E, int32_t* plan, size_t plan_words,
+            int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * a3. Layout.  [GR] "Online planning, zero copy και στατικά σχήματα": each pair
+ * goes straight to its final row, grouped by expert, in a static S*K buffer per
+ * rank.  Stable counting sort by expert, ties in flattened (rank, token, k)
+ * order; the home copy takes an expert's first home_count pairs, its replicas
+ * the following ranges in match order; rank r's rows hold its home experts in
+ * id order, then its received replicas in match order.
+ *   pos       [P] int32 out: row of pair p.
+ *   src       [P] int32 out: pair of row i (inverse of pos).
+ *   pair_slot [P] int32 out, may be NULL: slot id of pair p (e or E + m).
+ *   plan      from ep_plan for the loads of these topk_ids.
+ *   ws        the scratch ep_route_stats filled for these topk_ids.
+ */
+EP_API int ep_layout(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, const int32_t* plan,
+              size_t plan_words, const void* ws, size_t ws_bytes, int32_t* pos, int32_t* src, int32_t* pair_slot,
+              int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * a4. MoE Align & Sort.  [ZH]: sort the routed ids by expert and pad each
+ * expert's group to a multiple of block_m so every block of the grouped GEMM
+ * belongs to one expert.  Readings: the ids are flattened pair indices p
+ * (token = p / K), stable in p; padding holds the sentinel P.
+ *   sorted_token_ids [sorted_cap] int32 out, sorted_cap >= P + E*(block_m-1):
+ *       group of e at off_e = sum_{e'<e} ceil(c_e'/block_m)*block_m, then P
+ *       as padding up to the next multiple of block_m, and P past the end.
+ *   expert_ids [expert_ids_cap] int32 out, >= ceil(sorted_cap / block_m):
+ *       expert of each block, -1 past num_tokens_post_pad / block_m.
+ *   num_tokens_post_pad [1] int32 out: sum_e ceil(c_e/block_m)*block_m.
+ *   ws  scratch of ep_workspace_size bytes (its histogram is rebuilt here).
+ */
+EP_API int ep_align_sort(const int32_t* topk_ids, int64_t T, int K, int E, int block_m, int32_t* sorted_token_ids,
+                  int64_t sorted_cap, int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad,
+                  void* ws, size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * a5. Dispatch.  [GR] "Online planning, zero copy και στατικά σχήματα": rows are
+ * written in place into the expert-grouped buffer, no intermediate copy.
+ *   x   [T, H] bf16; buf [buf_rows, H] bf16 out; buf[pos[p]] = x[p / K] bitwise.
+ *   Rows whose pos is outside [0, buf_rows) are skipped and flagged.
+ * Each token row is read once (TMA bulk copy into shared memory) and written to
+ * its K rows by bulk stores.
+ */
+EP_API int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
+                int64_t buf_rows, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Stand-in for the expert computation (the grouped GEMM is outside this
+ * library's path), for tests and examples: y[i] = bf16_rn(float(buf[i]) *
+ * scale[e]) with e = topk_ids[src[i]], fp32 multiply.  y may alias buf.
+ */
+EP_API int ep_expert_scale(const uint16_t* buf, int64_t rows, int64_t H, const int32_t* src, const int32_t* topk_ids,
+                    int64_t P, const float* scale, int E, uint16_t* y, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * a6. Combine.  out[t] = bf16_rn( sum_{k=0..K-1} w[t,k] * float(y[pos[t*K+k]]) ),
+ * accumulated in fp32 in k order from 0, each product and sum rounded
+ * separately (no fused multiply-add), one rounding to bf16 at the end.
+ *   y [y_rows, H] bf16; w [T, K] fp32; pos [P] int32; out [T, H] bf16 out.
+ *   Pairs whose pos is outside [0, y_rows) contribute nothing and are flagged.
+ */
+EP_API int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* pos, int64_t T, int K, int64_t H,
+               uint16_t* out, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * a7. Replica gradient reduction.  [GR] "Τι συμβαίνει στους gradients κατά την
+ * εκπαίδευση": replica gradients live in a separate reduce buffer in fp32 and
+ * are added into the home expert's gradient, after which the used slots are
+ * cleared.  Per element: g_home[e] = ((g_home[e] + g_rep[m1]) + g_rep[m2]) ...
+ * over e's replicas in match order, fp32, one add at a time.
+ *   g_home [E, n] fp32 in/out.  g_rep [cap, n], row m = replica m, fp32
+ *   (EP_DTYPE_F32) or bf16 (EP_DTYPE_BF16, widened exactly).
+ *   clear_replicas != 0 zeroes the rows of the replicas used.
+ */
+EP_API int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
+                           const int32_t* plan, size_t plan_words, int clear_replicas, int32_t* dev_status,
+                           cudaStream_t stream);
+
+/* Copy *dev_status to *host_status (host) after the work queued on `stream`;
+ * waits for the stream.  The only synchronising call. */
+EP_API int ep_status_read(const int32_t* dev_status, int32_t* host_status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TDH_EP_H */

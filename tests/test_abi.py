@@ -1,0 +1,98 @@
+"""The C ABI library loads and exports every entry point include/ep.h declares,
+and its host-side logic (sizes, plan layout, argument checks) works without a
+GPU.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ep.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    return re.findall(r"EP_API\s+[\w\s\*]+?\b(ep_\w+)\s*\(", text)
+
+
+def test_header_declares_the_path():
+    names = set(declared())
+    for n in ("ep_route_stats", "ep_plan", "ep_layout", "ep_align_sort", "ep_dispatch", "ep_combine",
+              "ep_replica_grad_reduce", "ep_workspace_size", "ep_plan_layout", "ep_status_read"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import token_dispatch_histogram_b200 as tdh
+    L = ctypes.CDLL(tdh.LIB_PATH)
+    for name in declared():
+        assert hasattr(L, name), name
+
+
+def test_binding_has_same_names():
+    import token_dispatch_histogram_b200 as tdh
+    for name in declared():
+        if name in ("ep_version",):
+            continue
+        assert hasattr(tdh, name), name
+
+
+def test_host_only_calls():
+    import token_dispatch_histogram_b200 as tdh
+    assert "sm_100a" in tdh.version()
+    lay = tdh.ep_plan_layout(64, 8)
+    assert lay["cap"] == 64 + 8 - 1
+    offs = sorted(v for k, v in lay.items() if k not in ("words", "cap"))
+    assert len(set(offs)) == len(offs) and offs[-1] < lay["words"]
+    assert all(v % 8 == 0 for k, v in lay.items() if k not in ("words", "cap"))
+    # workspace grows with the tile count and E
+    a = tdh.ep_workspace_size(32768, 6, 64)
+    b = tdh.ep_workspace_size(524288, 8, 384)
+    assert 0 < a < b
+    assert tdh.ep_workspace_size(0, 2, 16) > 0
+
+
+def test_argument_errors_return_before_any_launch():
+    import token_dispatch_histogram_b200 as tdh
+    L = tdh.lib()
+    n = ctypes.c_size_t()
+    assert L.ep_workspace_size(10, 0, 8, ctypes.byref(n)) == tdh.EP_ERR_ARG      # K < 1
+    assert L.ep_workspace_size(10, 9, 8, ctypes.byref(n)) == tdh.EP_ERR_ARG      # K > E
+    assert L.ep_workspace_size(10, 2, 2000, ctypes.byref(n)) == tdh.EP_ERR_ARG   # E > max
+    assert L.ep_workspace_size(1 << 30, 4, 8, ctypes.byref(n)) == tdh.EP_ERR_ARG  # P >= 2^31
+    lay = tdh.EpPlanLayout()
+    assert L.ep_plan_layout(10, 4, ctypes.byref(lay)) == tdh.EP_ERR_ARG          # E % R
+    fake = ctypes.c_void_p(0x1000)
+    # ep_plan: E % R != 0
+    assert L.ep_plan(fake, 3, 4, 2, 8, fake, 1 << 20, None, None) == tdh.EP_ERR_ARG
+    # ep_plan: plan buffer too small
+    assert L.ep_plan(fake, 4, 4, 2, 8, fake, 3, None, None) == tdh.EP_ERR_CAPACITY
+    # ep_route_stats: workspace too small
+    assert L.ep_route_stats(fake, 16, 2, 8, fake, fake, fake, 8, None, None) == tdh.EP_ERR_CAPACITY
+    # ep_layout: R*S != T
+    assert L.ep_layout(fake, 16, 2, 8, 4, 5, fake, 1 << 20, fake, 1 << 20, fake, fake, None, None,
+                       None) == tdh.EP_ERR_ARG
+    # ep_align_sort: sorted capacity too small
+    assert L.ep_align_sort(fake, 16, 2, 8, 4, fake, 10, fake, 100, fake, fake, 1 << 20, None,
+                           None) == tdh.EP_ERR_CAPACITY
+    # ep_dispatch / ep_combine: H not a multiple of 8, misaligned pointers
+    assert L.ep_dispatch(fake, 16, 2, 12, fake, fake, 32, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_dispatch(ctypes.c_void_p(0x1008), 16, 2, 16, fake, fake, 32, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_combine(fake, 32, fake, fake, 16, 2, 12, fake, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_combine(fake, 32, fake, fake, 16, 33, 16, fake, None, None) == tdh.EP_ERR_ARG  # K > 32
+    # grad reduce: bad dtype, plan too small
+    assert L.ep_replica_grad_reduce(fake, fake, 7, 8, 8, 4, fake, 1 << 20, 0, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_replica_grad_reduce(fake, fake, 0, 8, 8, 4, fake, 3, 0, None, None) == tdh.EP_ERR_CAPACITY
+    # zero-size work is a no-op that succeeds without touching the device
+    assert L.ep_dispatch(None, 0, 2, 16, None, None, 0, None, None) == tdh.EP_OK
+    assert L.ep_combine(None, 0, None, None, 0, 2, 16, None, None, None) == tdh.EP_OK
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    t = torch.zeros((4, 2), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        tdh.ep_route_stats(t, 8, torch.zeros(8, dtype=torch.int32), torch.zeros(1, dtype=torch.float64),
+                           torch.zeros(64, dtype=torch.uint8))

@@ -1,0 +1,160 @@
+"""CUDA path vs CPU oracle, element by element, through the C ABI (-m gpu).
+
+Bars: loads, max_vio, plan, layout, align-sort and dispatch bit-exact;
+combine within 1 bf16 ulp per element (the kernel's arithmetic is the
+oracle's, one fp32 multiply and one fp32 add per term in k order, so it is
+also checked to be bit-exact); grad-reduce within 1e-6 relative (the same
+adds in the same order, also checked bit-exact).
+
+Sizes span several histogram tiles (2048-8192 pairs each) with ragged tails,
+plus the degenerate cases: one rank, uniform routing (no replica), every
+token's top-1 on one expert, an expert with no pair, T = 0.
+"""
+import numpy as np
+import pytest
+
+import oracle_pins as PINS
+import workload as W
+from gpu_path import (bf16_ulp_diff, case_inputs, expected_plan_tables, plan_field, run_cuda, run_oracle)
+
+pytestmark = pytest.mark.gpu
+
+
+def _assert_route_parity(cu, orc, R, S, K, E):
+    assert cu["status"] == 0
+    np.testing.assert_array_equal(cu["loads"], orc["loads"])
+    assert cu["max_vio"] == orc["max_vio"]  # fp64, same expression on both sides
+    pl = orc["plan"]
+    n = pl["n_rep"]
+    assert plan_field(cu, "n_rep", 1)[0] == n
+    np.testing.assert_array_equal(plan_field(cu, "rep_expert", n), pl["rep_expert"])
+    np.testing.assert_array_equal(plan_field(cu, "rep_rank", n), pl["rep_rank"])
+    np.testing.assert_array_equal(plan_field(cu, "rep_count", n), pl["rep_count"])
+    np.testing.assert_array_equal(plan_field(cu, "home_count", E), pl["home_count"])
+    lo = orc["layout"]
+    np.testing.assert_array_equal(plan_field(cu, "slot_order", E + n), lo["slot_order"])
+    np.testing.assert_array_equal(plan_field(cu, "cu_seqlens", E + n + 1), lo["cu_seqlens"])
+    exp = expected_plan_tables(pl, lo, R, S, K, E)
+    for name in ("home_base", "copy_cnt", "rank_nrep", "rank_rep_first"):
+        np.testing.assert_array_equal(plan_field(cu, name, len(exp[name])), exp[name], err_msg=name)
+    for name in ("rep_base", "rep_begin"):
+        np.testing.assert_array_equal(plan_field(cu, name, n), exp[name], err_msg=name)
+    has = exp["copy_cnt"] > 0
+    np.testing.assert_array_equal(plan_field(cu, "copy_first", E)[has], exp["copy_first"][has])
+    np.testing.assert_array_equal(cu["pos"], lo["pos"])
+    np.testing.assert_array_equal(cu["src"], lo["src"])
+    np.testing.assert_array_equal(cu["pair_slot"], lo["pair_slot"])
+    np.testing.assert_array_equal(cu["sorted_ids"], orc["sorted_ids"])
+    np.testing.assert_array_equal(cu["expert_ids"], orc["expert_ids"])
+    assert cu["ntpp"] == orc["ntpp"]
+
+
+def test_hand_example_on_gpu():
+    g = PINS.golden()
+    topk = np.array(g["topk_ids"], dtype=np.int32)
+    R, S, K, E = g["R"], g["S"], g["K"], g["E"]
+    cu = run_cuda(topk, None, None, R, S, E, g["block_m"])
+    assert cu["status"] == 0
+    assert cu["loads"].tolist() == g["loads"]
+    assert cu["max_vio"] == g["max_vio"]
+    assert cu["pos"].tolist() == g["pos"]
+    assert plan_field(cu, "cu_seqlens", 12).tolist() == g["cu_seqlens"]
+    assert plan_field(cu, "slot_order", 11).tolist() == g["slot_order"]
+    assert cu["ntpp"] == g["align_num_tokens_post_pad"]
+    assert cu["expert_ids"].tolist() == g["align_expert_ids"]
+
+
+ROUTE_CASES = [
+    # (R, S, K, E, kind, block_m)
+    (4, 64, 2, 16, "zipf", 4),            # the tiny workload's shape
+    (8, 4096, 6, 64, "skew", 64),         # the moderate EP8 workload's shape (96 tiles)
+    (1, 1000, 3, 7, "skew", 16),          # one rank: no replica possible
+    (4, 1024, 8, 32, "uniform", 128),     # uniform: max_vio 0, no replica
+    (16, 613, 8, 256, "single", 128),     # every top-1 on expert 0; ragged tail
+    (3, 777, 5, 9, "skew", 3),            # odd sizes, E/R = 3
+    (2, 1, 1, 2, "skew", 1),
+    (64, 301, 8, 384, "skew", 128),       # fine-grained, ragged
+    (8, 2047, 4, 1024, "skew", 8),        # E at the library limit
+    (1024, 4, 2, 1024, "skew", 4),        # R at the library limit, E/R = 1
+    (4, 0, 2, 16, "skew", 4),             # T = 0
+]
+
+
+@pytest.mark.parametrize("case", ROUTE_CASES, ids=lambda c: "R{}_S{}_K{}_E{}_{}".format(*c[:5]))
+def test_route_plan_layout_align(case):
+    R, S, K, E, kind, bm = case
+    if kind == "zipf":
+        topk, w = W.routing_from(R * S, E, K, seed=0, bias_e=W.bias(1, 0))
+    else:
+        topk, w, _ = case_inputs(R, S, K, E, 0, seed=R * 131 + S, kind=kind, bias_scale=1.5)
+    cu = run_cuda(topk, None, None, R, S, E, bm)
+    orc = run_oracle(topk, None, None, R, S, E, bm)
+    _assert_route_parity(cu, orc, R, S, K, E)
+
+
+def test_route_fuzz():
+    rng = np.random.default_rng(2024)
+    for it in range(60):
+        R = int(rng.choice([1, 2, 3, 4, 8, 16]))
+        ER = int(rng.integers(1, 9))
+        E = R * ER
+        K = int(rng.integers(1, min(8, E) + 1))
+        S = int(rng.integers(0, 3000 // max(1, R)))
+        kind = ["skew", "uniform", "single"][it % 3]
+        bm = int(rng.choice([1, 2, 16, 64, 128]))
+        topk, w, _ = case_inputs(R, S, K, E, 0, seed=it, kind=kind, bias_scale=float(rng.uniform(0.2, 3)))
+        cu = run_cuda(topk, None, None, R, S, E, bm)
+        orc = run_oracle(topk, None, None, R, S, E, bm)
+        _assert_route_parity(cu, orc, R, S, K, E)
+
+
+ROW_CASES = [
+    # (R, S, K, E, H, kind)
+    (4, 64, 2, 16, 128, "zipf"),       # tiny workload
+    (8, 256, 6, 64, 2048, "skew"),     # moderate workload's row width, fewer tokens
+    (4, 300, 8, 32, 7168, "skew"),     # DeepSeek-V3 row width, ragged
+    (2, 50, 1, 4, 64, "skew"),         # K = 1
+    (3, 33, 5, 9, 24, "single"),       # generic-K combine path, narrow rows
+    (16, 64, 8, 256, 4096, "uniform"),
+]
+
+
+@pytest.mark.parametrize("case", ROW_CASES, ids=lambda c: "R{}_S{}_K{}_E{}_H{}_{}".format(*c))
+def test_dispatch_expert_combine(case):
+    R, S, K, E, H, kind = case
+    if kind == "zipf":
+        topk, w = W.routing_from(R * S, E, K, seed=0, bias_e=W.bias(1, 0))
+        x = W.hidden(R * S, H, seed=5)
+    else:
+        topk, w, x = case_inputs(R, S, K, E, H, seed=H + S, kind=kind)
+    scale = W.expert_scale(E)
+    cu = run_cuda(topk, w, x, R, S, E, 4, scale=scale)
+    orc = run_oracle(topk, w, x, R, S, E, 4, scale=scale)
+    assert cu["status"] == 0
+    np.testing.assert_array_equal(cu["pos"], orc["layout"]["pos"])
+    np.testing.assert_array_equal(cu["buf"], orc["buf"])          # dispatch: bitwise
+    np.testing.assert_array_equal(cu["y"], orc["y"])              # stand-in expert: bitwise
+    ulp = bf16_ulp_diff(cu["out"], orc["out"])
+    assert ulp.max() <= 1                                         # combine bar: 1 bf16 ulp
+    assert np.count_nonzero(ulp) == 0                             # and in fact identical
+    # combine against the layout-free closed form too
+    cf = __import__("oracle").combine_closed(x, w, topk, scale)
+    assert bf16_ulp_diff(cu["out"], cf).max() <= 1
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("clear", [False, True])
+def test_grad_reduce(dtype, clear):
+    R, S, K, E = 8, 512, 6, 64
+    topk, w, _ = case_inputs(R, S, K, E, 0, seed=77, bias_scale=1.5)
+    for n in (1000, 4096, 3 * 128 * 64 + 8):  # n % 8 != 0 takes the scalar path
+        cap = E + R - 1
+        g_home = W.grad_rows(3, W.STREAM_GHOME, n, E)
+        g_rep = W.grad_rows(4, W.STREAM_GREP, n, cap, dtype)
+        cu = run_cuda(topk, None, None, R, S, E, 4, g_home=g_home, g_rep=g_rep, clear=clear)
+        orc = run_oracle(topk, None, None, R, S, E, 4, g_home=g_home, g_rep=g_rep, clear=clear)
+        assert orc["plan"]["n_rep"] > 0
+        rel = np.abs(cu["g_home"] - orc["g_home"]) / np.maximum(np.abs(orc["g_home"]), 1e-30)
+        assert rel.max() <= 1e-6
+        np.testing.assert_array_equal(cu["g_home"], orc["g_home"])  # same adds, same order
+        np.testing.assert_array_equal(cu["g_rep"], orc["g_rep"])    # cleared rows (if asked), others untouched

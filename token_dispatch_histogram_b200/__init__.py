@@ -1,0 +1,216 @@
+"""B200 expert-parallel dispatch path: Python binding of libep.so (include/ep.h).
+
+Argument marshalling only: each function below checks tensor dtypes and
+devices, passes data pointers, sizes and the CUDA stream to the C entry point
+of the same name, and turns a negative return code into an exception.  Every
+step of the path runs in the library's sm_100a kernels; there is no fallback.
+If libep.so is missing the import fails.
+
+Device memory and streams come from PyTorch; nothing here computes.
+"""
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libep.so")
+
+EP_OK, EP_ERR_ARG, EP_ERR_CAPACITY, EP_ERR_CUDA = 0, -1, -2, -3
+EP_DEV_BAD_EXPERT_ID = 0x1
+EP_DEV_LOOKBACK_TIMEOUT = 0x2
+EP_DEV_BAD_LOADS = 0x4
+EP_DEV_BAD_ROW = 0x8
+EP_DEV_COPY_TIMEOUT = 0x10
+EP_MAX_EXPERTS = 1024
+EP_MAX_RANKS = 1024
+EP_DTYPE_F32, EP_DTYPE_BF16 = 0, 1
+
+
+class EpError(RuntimeError):
+    def __init__(self, name, code):
+        what = {EP_ERR_ARG: "invalid argument", EP_ERR_CAPACITY: "capacity too small",
+                EP_ERR_CUDA: "CUDA launch failed"}.get(code, "error")
+        super().__init__(f"{name}: {what} ({code})")
+        self.code = code
+
+
+class EpPlanLayout(ctypes.Structure):
+    _fields_ = [("words", ctypes.c_int64), ("cap", ctypes.c_int32)] + [
+        (n, ctypes.c_int32) for n in ("n_rep", "n_chunks", "rank_load", "rank_nrep", "rank_rep_first", "home_count",
+                                      "home_base", "copy_first", "copy_cnt", "rep_expert", "rep_rank", "rep_count",
+                                      "rep_begin", "rep_base", "rep_experts", "slot_order", "cu_seqlens")]
+
+
+_lib = None
+_V, _I, _I64, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+
+_SIGS = {
+    "ep_version": (ctypes.c_char_p, []),
+    "ep_launch_count": (ctypes.c_uint64, []),
+    "ep_workspace_size": (_I, [_I64, _I, _I, _V]),
+    "ep_plan_layout": (_I, [_I, _I, _V]),
+    "ep_route_stats": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
+    "ep_plan": (_I, [_V, _I, _I64, _I, _I, _V, _SZ, _V, _V]),
+    "ep_layout": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _SZ, _V, _SZ, _V, _V, _V, _V, _V]),
+    "ep_align_sort": (_I, [_V, _I64, _I, _I, _I, _V, _I64, _V, _I64, _V, _V, _SZ, _V, _V]),
+    "ep_dispatch": (_I, [_V, _I64, _I, _I64, _V, _V, _I64, _V, _V]),
+    "ep_expert_scale": (_I, [_V, _I64, _I64, _V, _V, _I64, _V, _I, _V, _V, _V]),
+    "ep_combine": (_I, [_V, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
+    "ep_replica_grad_reduce": (_I, [_V, _V, _I, _I64, _I, _I, _V, _SZ, _I, _V, _V]),
+    "ep_status_read": (_I, [_V, _V, _V]),
+}
+
+
+def lib():
+    """The loaded libep.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} not built: run token_dispatch_histogram_b200/build.py "
+                              "(or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+lib()  # fail at import time when the library is missing
+
+
+def _check(name, code):
+    if code != EP_OK:
+        raise EpError(name, code)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(t, *dts):
+    if t.dtype not in dts:
+        raise TypeError(f"dtype {t.dtype}, expected one of {dts}")
+
+
+def version():
+    return lib().ep_version().decode()
+
+
+def ep_launch_count():
+    return int(lib().ep_launch_count())
+
+
+def ep_workspace_size(T, K, E):
+    n = ctypes.c_size_t(0)
+    _check("ep_workspace_size", lib().ep_workspace_size(T, K, E, ctypes.byref(n)))
+    return int(n.value)
+
+
+def ep_plan_layout(E, R):
+    L = EpPlanLayout()
+    _check("ep_plan_layout", lib().ep_plan_layout(E, R, ctypes.byref(L)))
+    return {name: getattr(L, name) for name, _ in EpPlanLayout._fields_}
+
+
+def ep_route_stats(topk_ids, E, loads, max_vio, ws, dev_status=None, stream=None):
+    _dtype(topk_ids, torch.int32)
+    _dtype(loads, torch.int32)
+    _dtype(max_vio, torch.float64)
+    T, K = topk_ids.shape
+    _check("ep_route_stats", lib().ep_route_stats(_p(topk_ids), T, K, E, _p(loads), _p(max_vio), _p(ws),
+                                                  ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
+
+
+def ep_plan(loads, R, S, K, E, plan, dev_status=None, stream=None):
+    _dtype(loads, torch.int32)
+    _dtype(plan, torch.int32)
+    _check("ep_plan", lib().ep_plan(_p(loads), R, S, K, E, _p(plan), plan.numel(), _p(dev_status), _s(stream)))
+
+
+def ep_layout(topk_ids, E, R, S, plan, ws, pos, src, pair_slot=None, dev_status=None, stream=None):
+    for t in (topk_ids, plan, pos, src) + ((pair_slot,) if pair_slot is not None else ()):
+        _dtype(t, torch.int32)
+    T, K = topk_ids.shape
+    _check("ep_layout", lib().ep_layout(_p(topk_ids), T, K, E, R, S, _p(plan), plan.numel(), _p(ws),
+                                        ws.numel() * ws.element_size(), _p(pos), _p(src), _p(pair_slot),
+                                        _p(dev_status), _s(stream)))
+
+
+def ep_align_sort(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_pad, ws, dev_status=None,
+                  stream=None):
+    for t in (topk_ids, sorted_token_ids, expert_ids, num_tokens_post_pad):
+        _dtype(t, torch.int32)
+    T, K = topk_ids.shape
+    _check("ep_align_sort", lib().ep_align_sort(_p(topk_ids), T, K, E, block_m, _p(sorted_token_ids),
+                                                sorted_token_ids.numel(), _p(expert_ids), expert_ids.numel(),
+                                                _p(num_tokens_post_pad), _p(ws), ws.numel() * ws.element_size(),
+                                                _p(dev_status), _s(stream)))
+
+
+def align_sort_capacity(P, E, block_m):
+    cap = P + E * (block_m - 1)
+    return cap, (cap + block_m - 1) // block_m
+
+
+def ep_dispatch(x, K, pos, buf, dev_status=None, stream=None):
+    _dtype(x, torch.bfloat16, torch.int16, torch.uint16)
+    _dtype(buf, torch.bfloat16, torch.int16, torch.uint16)
+    _dtype(pos, torch.int32)
+    T, H = x.shape
+    _check("ep_dispatch", lib().ep_dispatch(_p(x), T, K, H, _p(pos), _p(buf), buf.shape[0], _p(dev_status),
+                                            _s(stream)))
+
+
+def ep_expert_scale(buf, src, topk_ids, scale, y, dev_status=None, stream=None):
+    _dtype(scale, torch.float32)
+    rows, H = buf.shape
+    _check("ep_expert_scale", lib().ep_expert_scale(_p(buf), rows, H, _p(src), _p(topk_ids), topk_ids.numel(),
+                                                    _p(scale), scale.numel(), _p(y), _p(dev_status), _s(stream)))
+
+
+def ep_combine(y, w, pos, out, dev_status=None, stream=None):
+    _dtype(w, torch.float32)
+    _dtype(pos, torch.int32)
+    T, K = w.shape
+    H = y.shape[1]
+    _check("ep_combine", lib().ep_combine(_p(y), y.shape[0], _p(w), _p(pos), T, K, H, _p(out), _p(dev_status),
+                                          _s(stream)))
+
+
+def ep_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False, dev_status=None, stream=None):
+    _dtype(g_home, torch.float32)
+    _dtype(plan, torch.int32)
+    if g_rep.dtype == torch.float32:
+        dt = EP_DTYPE_F32
+    elif g_rep.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        dt = EP_DTYPE_BF16
+    else:
+        raise TypeError(g_rep.dtype)
+    n = g_home.shape[1]
+    _check("ep_replica_grad_reduce", lib().ep_replica_grad_reduce(_p(g_home), _p(g_rep), dt, n, E, R, _p(plan),
+                                                                  plan.numel(), int(bool(clear_replicas)),
+                                                                  _p(dev_status), _s(stream)))
+
+
+def ep_status_read(dev_status, stream=None):
+    h = ctypes.c_int32(0)
+    _check("ep_status_read", lib().ep_status_read(_p(dev_status), ctypes.byref(h), _s(stream)))
+    return int(h.value)
+
+
+from .layer import EpLayer  # noqa: E402  (needs the binding above)

@@ -1,0 +1,213 @@
+// Shared device/host helpers of libep.so (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "ep.h"
+
+namespace ep {
+
+// ---------------------------------------------------------------- host side
+
+extern std::atomic<uint64_t> g_launches;
+
+inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+inline int launch_status() { return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms();  // cached per device
+
+// Pairs per tile of the histogram / rank scatter passes.  The largest of
+// 2048, 4096, 8192 that still gives two tiles per SM (so small problems spread
+// over the GPU and large ones amortise the per-tile scan), never below 2048.
+inline int tile_pairs_for(int64_t P) {
+  const int64_t want = 2 * 148;
+  if (P >= want * 8192) return 8192;
+  if (P >= want * 4096) return 4096;
+  return 2048;
+}
+
+inline int64_t num_tiles(int64_t P, int tile) { return (P + tile - 1) / tile; }
+
+// Workspace layout (bytes): [0,256) header (ticket counter), then the
+// decoupled look-back words u64 [ntiles][E], then tile_excl i32 [ntiles][E],
+// then loads i32 [E] (align-sort's own histogram).
+struct WsLayout {
+  size_t status_off, excl_off, loads_off, bytes, clear_bytes;
+};
+inline WsLayout ws_layout(int64_t P, int E) {
+  const int tile = tile_pairs_for(P);
+  const int64_t nt = num_tiles(P, tile);
+  WsLayout l;
+  l.status_off = 256;
+  l.excl_off = l.status_off + (size_t)nt * E * 8;
+  l.excl_off = (l.excl_off + 255) & ~(size_t)255;
+  l.loads_off = l.excl_off + (size_t)nt * E * 4;
+  l.loads_off = (l.loads_off + 255) & ~(size_t)255;
+  l.bytes = l.loads_off + (size_t)E * 4 + 256;
+  l.clear_bytes = l.status_off + (size_t)nt * E * 8;
+  return l;
+}
+
+// Plan buffer layout: fills EpPlanLayout (offsets in int32 words).
+void plan_layout(int E, int R, EpPlanLayout* L);
+
+// Common argument checks for (T, K, E).
+inline bool valid_tke(int64_t T, int K, int E) {
+  if (T < 0 || K < 1 || K > 32 || E < 1 || E > EP_MAX_EXPERTS || K > E) return false;
+  if (T * (int64_t)K >= ((int64_t)1 << 31)) return false;
+  return true;
+}
+
+// ------------------------------------------------------------- device side
+
+__device__ __forceinline__ void flag(int32_t* dev_status, int32_t bits) {
+  if (dev_status) atomicOr(dev_status, bits);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// fp32 -> bf16 bits, round to nearest even; NaN kept quiet.
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (u >> 16) | 0x40u;
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return u >> 16;
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Wall-clock bound for every wait inside a kernel (a look-back on another
+// CTA, an mbarrier of an asynchronous copy): after it the kernel reports a
+// timeout bit and goes on, so no wait can hang the device.
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// --- mbarrier and bulk-copy (TMA) wrappers --------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// global -> shared bulk copy completing on an mbarrier (bytes % 16 == 0,
+// both addresses 16-byte aligned)
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// shared -> global bulk copy in the calling thread's bulk async-group
+__device__ __forceinline__ void bulk_store(void* gmem_dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_addr(smem_src)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 16-byte global loads that skip L1 allocation (streamed once)
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// Block-wide exclusive scan of one int32 per thread (blockDim.x <= 1024,
+// a multiple of 32).  `warp_sums` is shared scratch of 32 ints.  Returns the
+// exclusive prefix; *total gets the block sum.  Contains __syncthreads.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  int32_t x = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int32_t y = __shfl_up_sync(0xffffffffu, x, d);
+    if (lane >= d) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t s = lane < nwarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, s, d);
+      if (lane >= d) s += y;
+    }
+    if (lane < nwarps) warp_sums[lane] = s;  // inclusive
+  }
+  __syncthreads();
+  int32_t base = warp > 0 ? warp_sums[warp - 1] : 0;
+  int32_t tot = warp_sums[nwarps - 1];
+  __syncthreads();
+  if (total) *total = tot;
+  return base + x - v;
+}
+
+}  // namespace ep

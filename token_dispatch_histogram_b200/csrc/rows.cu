@@ -1,0 +1,266 @@
+// a5. Dispatch and a6. Combine: the HBM-bound row movers.
+//
+// Dispatch ([GR] "Online planning, zero copy και στατικά σχήματα", twodots.gr
+// MoonEP article): each token's hidden row is written straight into the K rows
+// the layout gave its pairs, in the static expert-grouped buffer.
+// buf[pos[t*K + k]] = x[t] for k < K.  Minimal traffic: each x row is read once
+// (T*H*2 bytes) and each buffer row written once (P*H*2 bytes).
+//
+// B200 design: a persistent grid of one-warp CTAs, each with a ring of shared
+// memory stages.  Lane 0 brings a whole row in with one TMA bulk copy
+// (cp.async.bulk global->shared, completion on an mbarrier); once it lands,
+// lanes 0..K-1 each issue one bulk store (shared->global) of that row to one
+// destination.  Loads for the next stages are in flight while the stores
+// drain, so a handful of instructions per row keeps ~200 KB per SM moving.
+//
+// Combine: out[t] = bf16_rn(sum_k w[t,k] * float(y[pos[t*K+k]])), fp32 in k
+// order, separate multiply and add roundings (no FMA).  One thread owns 8
+// consecutive bf16 of one output row (one 16-byte vector); it issues all K
+// 16-byte row loads before using any, so K loads are in flight per thread.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace ep {
+
+constexpr int DISPATCH_MAX_STAGES = 8;
+
+// Wait (bounded by WAIT_LIMIT_NS) for phase `parity` of an mbarrier.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
+  return true;
+}
+
+__global__ void __launch_bounds__(32)
+    k_dispatch(const uint8_t* __restrict__ x, int64_t T, int K, uint32_t row_bytes, const int32_t* __restrict__ pos,
+               int64_t buf_rows, uint8_t* __restrict__ buf, int stages, int32_t* dev_status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t stride_b = (row_bytes + 127u) & ~127u;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stride_b);
+  int32_t* ring = reinterpret_cast<int32_t*>(bars + DISPATCH_MAX_STAGES);  // [stages][K] destination rows
+  const int lane = threadIdx.x;
+  if (lane == 0)
+    for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
+  fence_mbar_init();
+  __syncwarp();
+
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  const int64_t njobs = first < T ? (T - first + step - 1) / step : 0;
+  auto issue = [&](int64_t j) {
+    const int s = (int)(j % stages);
+    const int64_t t = first + j * step;
+    if (lane < K) ring[s * K + lane] = __ldg(pos + t * K + lane);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[s], row_bytes);
+      bulk_load(smem + (size_t)s * stride_b, x + t * (int64_t)row_bytes, row_bytes, &bars[s]);
+    }
+  };
+  const int64_t pro = std::min<int64_t>(stages, njobs);
+  for (int64_t j = 0; j < pro; ++j) issue(j);
+  int64_t issued = pro;
+
+  int32_t bad = 0;
+  bool ok = true;
+  int64_t j = 0;
+  for (; j < njobs; ++j) {
+    const int s = (int)(j % stages);
+    const uint32_t parity = (uint32_t)((j / stages) & 1);
+    const bool landed = mbar_wait_bounded(&bars[s], parity);
+    if (!__all_sync(0xffffffffu, landed)) {
+      ok = false;
+      break;
+    }
+    if (lane < K) {
+      const int32_t row = ring[s * K + lane];
+      if (row >= 0 && row < buf_rows)
+        bulk_store(buf + (int64_t)row * row_bytes, smem + (size_t)s * stride_b, row_bytes);
+      else
+        bad = EP_DEV_BAD_ROW;
+    }
+    bulk_commit();
+    // refill the previous job's stage once its stores have read shared memory
+    if (j >= 1 && issued < njobs) {
+      bulk_wait_read<1>();
+      __syncwarp();
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (!ok) {
+    // a copy did not land in time: report, then give every load still in
+    // flight a bounded chance to land before the CTA (and its smem) goes away
+    if (lane == 0) flag(dev_status, EP_DEV_COPY_TIMEOUT);
+    for (int64_t q = j; q < issued; ++q) {
+      const int s = (int)(q % stages);
+      const uint32_t parity = (uint32_t)((q / stages) & 1);
+      mbar_wait_bounded(&bars[s], parity);
+    }
+  }
+  bulk_wait_all();
+  if (bad) flag(dev_status, bad);
+}
+
+// y[i] = bf16_rn(float(buf[i]) * scale[topk[src[i]]])  (stand-in expert)
+__global__ void __launch_bounds__(256)
+    k_expert_scale(const uint16_t* __restrict__ buf, int64_t rows, int64_t H, const int32_t* __restrict__ src,
+                   const int32_t* __restrict__ topk, int64_t P, const float* __restrict__ scale, int E,
+                   uint16_t* __restrict__ y, int32_t* dev_status) {
+  const int64_t nvec = H / 8;
+  const int tpr = (int)std::min<int64_t>(256, (nvec + 31) / 32 * 32);  // threads per row
+  const int rows_per_cta = 256 / tpr;
+  const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
+  int32_t bad = 0;
+  for (int64_t r = (int64_t)blockIdx.x * rows_per_cta + sub; r < rows; r += (int64_t)gridDim.x * rows_per_cta) {
+    if (sub >= rows_per_cta) break;
+    const int32_t p = __ldg(src + r);
+    int e = (p >= 0 && p < P) ? __ldg(topk + p) : -1;
+    if (e < 0 || e >= E) {
+      bad = EP_DEV_BAD_ROW;
+      continue;
+    }
+    const float s = __ldg(scale + e);
+    for (int64_t v = v0; v < nvec; v += tpr) {
+      const uint4 in = ld_stream_v4(buf + r * H + v * 8);
+      const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = f32_to_bf16_bits(__fmul_rn(bf16_bits_to_f32(w[q] & 0xFFFFu), s));
+        const uint32_t hi = f32_to_bf16_bits(__fmul_rn(bf16_bits_to_f32(w[q] >> 16), s));
+        o[q] = lo | (hi << 16);
+      }
+      st_v4(y + r * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+  if (bad) flag(dev_status, bad);
+}
+
+template <int KT>
+__global__ void __launch_bounds__(256)
+    k_combine(const uint16_t* __restrict__ y, int64_t y_rows, const float* __restrict__ w,
+              const int32_t* __restrict__ pos, int64_t T, int Kd, int64_t H, uint16_t* __restrict__ out,
+              int32_t* dev_status) {
+  constexpr int KMAX = KT > 0 ? KT : 32;
+  const int K = KT > 0 ? KT : Kd;
+  const int64_t nvec = H / 8;
+  const int tpr = (int)std::min<int64_t>(256, (nvec + 31) / 32 * 32);  // threads per token
+  const int toks_per_cta = 256 / tpr;
+  const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
+  int32_t bad = 0;
+  if (sub >= toks_per_cta) return;
+  for (int64_t t = (int64_t)blockIdx.x * toks_per_cta + sub; t < T; t += (int64_t)gridDim.x * toks_per_cta) {
+    int32_t rows[KMAX];
+    float wk[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < K) {
+        rows[k] = __ldg(pos + t * K + k);
+        wk[k] = __ldg(w + t * K + k);
+        if (rows[k] < 0 || rows[k] >= y_rows) {
+          rows[k] = -1;
+          bad = EP_DEV_BAD_ROW;
+        }
+      }
+    }
+    for (int64_t v = v0; v < nvec; v += tpr) {
+      uint4 in[KMAX];
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k)
+        if (k < K) in[k] = rows[k] >= 0 ? ld_stream_v4(y + (int64_t)rows[k] * H + v * 8) : make_uint4(0, 0, 0, 0);
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        if (k < K && rows[k] >= 0) {
+          const uint32_t wd[4] = {in[k].x, in[k].y, in[k].z, in[k].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(wk[k], bf16_bits_to_f32(wd[q] & 0xFFFFu)));
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(wk[k], bf16_bits_to_f32(wd[q] >> 16)));
+          }
+        }
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) o[q] = f32_to_bf16_bits(acc[2 * q]) | (f32_to_bf16_bits(acc[2 * q + 1]) << 16);
+      st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+  if (bad) flag(dev_status, bad);
+}
+
+int occupancy_grid(const void* fn, int threads, size_t smem, int64_t work_items, int cap_per_sm) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  per_sm = std::min(per_sm, cap_per_sm);
+  int64_t g = (int64_t)num_sms() * per_sm;
+  g = std::min<int64_t>(g, std::max<int64_t>(1, work_items));
+  return (int)g;
+}
+
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
+                           int64_t buf_rows, int32_t* dev_status, cudaStream_t stream) {
+  if (T < 0 || K < 1 || K > 32 || H < 8 || H % 8 || buf_rows < 0) return EP_ERR_ARG;
+  if (H * 2 > (1 << 20)) return EP_ERR_ARG;  // one row per bulk copy, at most 1 MiB
+  if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (T == 0) return EP_OK;
+  if (!x || !pos || !buf || !aligned16(x) || !aligned16(buf)) return EP_ERR_ARG;
+  const uint32_t row_bytes = (uint32_t)(H * 2);
+  const uint32_t stride_b = (row_bytes + 127u) & ~127u;
+  // stages: as many rows as fit in ~48 KB, 2..8
+  int stages = (int)std::max<uint32_t>(2, std::min<uint32_t>(DISPATCH_MAX_STAGES, (48u * 1024u) / stride_b));
+  size_t smem = (size_t)stages * stride_b + DISPATCH_MAX_STAGES * 8 + (size_t)stages * K * 4;
+  if (smem > 200 * 1024) return EP_ERR_ARG;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_dispatch, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return EP_ERR_CUDA;
+  const int grid = occupancy_grid((const void*)k_dispatch, 32, smem, T, 32);
+  k_dispatch<<<grid, 32, smem, stream>>>(reinterpret_cast<const uint8_t*>(x), T, K, row_bytes, pos, buf_rows,
+                                         reinterpret_cast<uint8_t*>(buf), stages, dev_status);
+  count_launch();
+  return launch_status();
+}
+
+extern "C" int ep_expert_scale(const uint16_t* buf, int64_t rows, int64_t H, const int32_t* src,
+                               const int32_t* topk_ids, int64_t P, const float* scale, int E, uint16_t* y,
+                               int32_t* dev_status, cudaStream_t stream) {
+  if (rows < 0 || H < 8 || H % 8 || E < 1 || P < 0) return EP_ERR_ARG;
+  if (rows == 0) return EP_OK;
+  if (!buf || !src || !topk_ids || !scale || !y || !aligned16(buf) || !aligned16(y)) return EP_ERR_ARG;
+  const int grid = occupancy_grid((const void*)k_expert_scale, 256, 0, rows, 8);
+  k_expert_scale<<<grid, 256, 0, stream>>>(buf, rows, H, src, topk_ids, P, scale, E, y, dev_status);
+  count_launch();
+  return launch_status();
+}
+
+extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* pos, int64_t T, int K,
+                          int64_t H, uint16_t* out, int32_t* dev_status, cudaStream_t stream) {
+  if (T < 0 || K < 1 || K > 32 || H < 8 || H % 8 || y_rows < 0) return EP_ERR_ARG;
+  if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (T == 0) return EP_OK;
+  if (!y || !w || !pos || !out || !aligned16(y) || !aligned16(out)) return EP_ERR_ARG;
+  const void* fn;
+  switch (K) {
+    case 1: fn = (const void*)k_combine<1>; break;
+    case 2: fn = (const void*)k_combine<2>; break;
+    case 4: fn = (const void*)k_combine<4>; break;
+    case 6: fn = (const void*)k_combine<6>; break;
+    case 8: fn = (const void*)k_combine<8>; break;
+    default: fn = (const void*)k_combine<0>; break;
+  }
+  const int grid = occupancy_grid(fn, 256, 0, T, 8);
+  void* args[] = {(void*)&y, (void*)&y_rows, (void*)&w, (void*)&pos, (void*)&T, (void*)&K, (void*)&H, (void*)&out,
+                  (void*)&dev_status};
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+  count_launch();
+  return launch_status();
+}

@@ -1,0 +1,154 @@
+// a1. Per-expert loads T_e and max_vio, plus the per-tile per-expert prefix
+// counts that the stable layout and the align-sort scatter read back.
+//
+// [FR] "Pourquoi le parallélisme d'experts est-il nécessaire" (news.hamidun.com
+// MoonEP article): max_vio = max_e(T_e / T̄) - 1, zero for perfect balance, T̄
+// the mean load P/E.
+//
+// One kernel, one pass over topk_ids:
+//  - each CTA takes a tile of consecutive flattened pairs (tile index from an
+//    atomic ticket, so a CTA only ever waits on tiles that started earlier),
+//  - builds the tile's histogram in shared memory, one shared-memory add per
+//    distinct expert per warp (__match_any_sync aggregation),
+//  - publishes it and resolves its exclusive prefix over earlier tiles with a
+//    decoupled look-back (Merrill & Garland, "Single-pass Parallel Prefix Scan
+//    with Decoupled Look-back", 2016), one 64-bit {flag, value} word per
+//    (tile, expert), every wait bounded,
+//  - the last tile's inclusive prefix is T_e; it also reduces max_e T_e.
+// Only integer adds feed the outputs, so they do not depend on scheduling.
+#include "common.cuh"
+
+namespace ep {
+
+constexpr int HIST_THREADS = 512;
+constexpr uint64_t FLAG_AGGREGATE = 1ull << 32;
+constexpr uint64_t FLAG_PREFIX = 2ull << 32;
+
+__global__ void __launch_bounds__(HIST_THREADS)
+    k_hist_lookback(const int32_t* __restrict__ topk, int64_t P, int E, int tile, int ntiles, uint32_t* ticket,
+                    uint64_t* status, int32_t* __restrict__ tile_excl, int32_t* __restrict__ loads,
+                    double* __restrict__ max_vio, int32_t* dev_status) {
+  extern __shared__ int32_t s_hist[];  // [E]
+  __shared__ int s_tile, s_bad;
+  __shared__ int32_t s_max[HIST_THREADS / 32];
+  if (threadIdx.x == 0) {
+    s_tile = (int)atomicAdd(ticket, 1u);
+    s_bad = 0;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+  const int t = s_tile;
+  const int lane = threadIdx.x & 31;
+  const int64_t p0 = (int64_t)t * tile;
+  const int64_t p1 = min(P, p0 + tile);
+
+  for (int64_t base = p0; base < p1; base += blockDim.x) {
+    const int64_t p = base + threadIdx.x;
+    int e = -1;
+    if (p < p1) {
+      e = __ldg(topk + p);
+      if (e < 0 || e >= E) {
+        e = -1;
+        s_bad = 1;
+      }
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[e], __popc(peers));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_EXPERT_ID);
+
+  int32_t my_max = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t agg = s_hist[e];
+    int32_t excl = 0;
+    uint64_t* mine = status + (int64_t)t * E + e;
+    if (t == 0) {
+      st_relaxed_u64(mine, FLAG_PREFIX | (uint32_t)agg);
+    } else {
+      st_relaxed_u64(mine, FLAG_AGGREGATE | (uint32_t)agg);
+      int j = t - 1;
+      int spins = 0;
+      uint64_t t0 = 0;
+      while (j >= 0) {
+        const uint64_t w = ld_relaxed_u64(status + (int64_t)j * E + e);
+        const uint64_t f = w & (3ull << 32);
+        if (f == 0) {  // predecessor not published yet: bounded wait
+          if (++spins > 32) {
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) {
+              t0 = now;
+            } else if (now - t0 > WAIT_LIMIT_NS) {
+              flag(dev_status, EP_DEV_LOOKBACK_TIMEOUT);
+              break;
+            }
+            __nanosleep(100);
+          }
+          continue;
+        }
+        excl += (int32_t)(uint32_t)w;
+        if (f == FLAG_PREFIX) break;
+        --j;
+      }
+      st_relaxed_u64(mine, FLAG_PREFIX | (uint32_t)(excl + agg));
+    }
+    tile_excl[(int64_t)t * E + e] = excl;
+    if (t == ntiles - 1) {
+      const int32_t total = excl + agg;
+      if (loads) loads[e] = total;
+      my_max = max(my_max, total);
+    }
+  }
+  if (t == ntiles - 1 && max_vio) {
+#pragma unroll
+    for (int d = 16; d; d >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, d));
+    if (lane == 0) s_max[threadIdx.x >> 5] = my_max;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int32_t m = 0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, s_max[w]);
+      // (max_e T_e) * E / P - 1, fp64, each step rounded once (product exact)
+      *max_vio = __dsub_rn(__ddiv_rn(__dmul_rn((double)m, (double)E), (double)P), 1.0);
+    }
+  }
+}
+
+// Histogram of topk_ids into ws (+ optional loads/max_vio).  Shared by
+// ep_route_stats and ep_align_sort.
+int run_hist(const int32_t* topk, int64_t P, int E, void* ws, int32_t* loads, double* max_vio, int32_t* dev_status,
+             cudaStream_t st) {
+  const WsLayout l = ws_layout(P, E);
+  const int tile = tile_pairs_for(P);
+  const int64_t nt = num_tiles(P, tile);
+  if (nt == 0) {
+    if (loads && cudaMemsetAsync(loads, 0, (size_t)E * 4, st) != cudaSuccess) return EP_ERR_CUDA;
+    if (max_vio && cudaMemsetAsync(max_vio, 0, sizeof(double), st) != cudaSuccess) return EP_ERR_CUDA;
+    return EP_OK;
+  }
+  char* w = static_cast<char*>(ws);
+  if (cudaMemsetAsync(w, 0, l.clear_bytes, st) != cudaSuccess) return EP_ERR_CUDA;
+  k_hist_lookback<<<(unsigned)nt, HIST_THREADS, (size_t)E * 4, st>>>(
+      topk, P, E, tile, (int)nt, reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint64_t*>(w + l.status_off),
+      reinterpret_cast<int32_t*>(w + l.excl_off), loads, max_vio, dev_status);
+  count_launch();
+  return launch_status();
+}
+
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" int ep_workspace_size(int64_t T, int K, int E, size_t* bytes) {
+  if (!bytes || !valid_tke(T, K, E)) return EP_ERR_ARG;
+  *bytes = ws_layout(T * K, E).bytes;
+  return EP_OK;
+}
+
+extern "C" int ep_route_stats(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads, double* max_vio,
+                              void* ws, size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
+  if (!valid_tke(T, K, E) || !loads || !max_vio || !ws) return EP_ERR_ARG;
+  const int64_t P = T * K;
+  if (P > 0 && !topk_ids) return EP_ERR_ARG;
+  if (ws_bytes < ws_layout(P, E).bytes) return EP_ERR_CAPACITY;
+  return run_hist(topk_ids, P, E, ws, loads, max_vio, dev_status, stream);
+}

@@ -1,0 +1,102 @@
+"""EpLayer: one expert-parallel MoE layer's dispatch path on static buffers.
+
+Allocates every buffer once at its static capacity (the S*K-per-rank contract
+makes all shapes known in advance: [GR] "Online planning, zero copy και
+στατικά σχήματα", twodots.gr MoonEP article) and runs the path as a fixed
+sequence of libep.so calls on one stream, with no host synchronisation:
+
+  ep_route_stats -> ep_plan -> ep_layout -> ep_align_sort -> ep_dispatch
+  -> [expert: outside the path] -> ep_combine -> ep_replica_grad_reduce
+
+`step()` is one pass of that sequence over the resident inputs; `run_host()`
+is the same pass fed from pinned host buffers (copies in, result out).
+Plumbing only: every computation happens in the library's kernels.
+"""
+import torch
+
+from . import (align_sort_capacity, ep_align_sort, ep_combine, ep_dispatch, ep_expert_scale, ep_layout,
+               ep_plan, ep_plan_layout, ep_replica_grad_reduce, ep_route_stats, ep_status_read, ep_workspace_size)
+
+
+class EpLayer:
+    def __init__(self, R, S, K, E, H, block_m, device="cuda", grad_n=0, grad_dtype=torch.float32,
+                 with_pair_slot=False):
+        self.R, self.S, self.K, self.E, self.H, self.block_m = R, S, K, E, H, block_m
+        self.T = R * S
+        self.P = self.T * K
+        self.device = torch.device(device)
+        dev = self.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.topk_ids = torch.zeros((self.T, K), **i32)
+        self.w = torch.zeros((self.T, K), dtype=torch.float32, device=dev)
+        self.x = torch.zeros((self.T, H), dtype=torch.bfloat16, device=dev)
+        self.loads = torch.zeros(E, **i32)
+        self.max_vio = torch.zeros(1, dtype=torch.float64, device=dev)
+        self.ws = torch.zeros(ep_workspace_size(self.T, K, E), dtype=torch.uint8, device=dev)
+        self.plan_layout = ep_plan_layout(E, R)
+        self.plan = torch.zeros(self.plan_layout["words"], **i32)
+        self.pos = torch.zeros(self.P, **i32)
+        self.src = torch.zeros(self.P, **i32)
+        self.pair_slot = torch.zeros(self.P, **i32) if with_pair_slot else None
+        self.buf = torch.zeros((self.P, H), dtype=torch.bfloat16, device=dev)  # dispatch output / combine input
+        self.out = torch.zeros((self.T, H), dtype=torch.bfloat16, device=dev)
+        cap, capb = align_sort_capacity(self.P, E, block_m)
+        self.sorted_token_ids = torch.zeros(cap, **i32)
+        self.expert_ids = torch.zeros(capb, **i32)
+        self.num_tokens_post_pad = torch.zeros(1, **i32)
+        self.dev_status = torch.zeros(1, **i32)
+        self.grad_n = grad_n
+        if grad_n:
+            self.g_home = torch.zeros((E, grad_n), dtype=torch.float32, device=dev)
+            self.g_rep = torch.zeros((self.plan_layout["cap"], grad_n), dtype=grad_dtype, device=dev)
+        else:
+            self.g_home = self.g_rep = None
+
+    # --- the path ---------------------------------------------------------
+    def route(self, stream=None):
+        """a1-a4: loads/max_vio, plan, layout, align-sort."""
+        ep_route_stats(self.topk_ids, self.E, self.loads, self.max_vio, self.ws, self.dev_status, stream)
+        ep_plan(self.loads, self.R, self.S, self.K, self.E, self.plan, self.dev_status, stream)
+        ep_layout(self.topk_ids, self.E, self.R, self.S, self.plan, self.ws, self.pos, self.src, self.pair_slot,
+                  self.dev_status, stream)
+        ep_align_sort(self.topk_ids, self.E, self.block_m, self.sorted_token_ids, self.expert_ids,
+                      self.num_tokens_post_pad, self.ws, self.dev_status, stream)
+
+    def dispatch(self, stream=None):
+        ep_dispatch(self.x, self.K, self.pos, self.buf, self.dev_status, stream)
+
+    def expert_standin(self, scale, stream=None):
+        """y = bf16(buf * s_e) in place (stands in for the grouped GEMM)."""
+        ep_expert_scale(self.buf, self.src, self.topk_ids, scale, self.buf, self.dev_status, stream)
+
+    def combine(self, stream=None):
+        ep_combine(self.buf, self.w, self.pos, self.out, self.dev_status, stream)
+
+    def grad_reduce(self, clear=False, stream=None):
+        if self.grad_n:
+            ep_replica_grad_reduce(self.g_home, self.g_rep, self.E, self.R, self.plan, clear, self.dev_status, stream)
+
+    def step(self, stream=None, grads=True):
+        """One pass of the whole path over the resident inputs."""
+        self.route(stream)
+        self.dispatch(stream)
+        self.combine(stream)
+        if grads:
+            self.grad_reduce(False, stream)
+
+    def run_host(self, topk_h, w_h, x_h, out_h, stream=None, grads=True):
+        """The step fed from (pinned) host buffers: host->device copies of the
+        routing and hidden rows, the path, and the combined rows back to host."""
+        self.topk_ids.copy_(topk_h, non_blocking=True)
+        self.w.copy_(w_h, non_blocking=True)
+        self.x.copy_(x_h, non_blocking=True)
+        self.step(stream, grads)
+        out_h.copy_(self.out, non_blocking=True)
+
+    def status(self, stream=None):
+        return ep_status_read(self.dev_status, stream)
+
+    # --- plan views -------------------------------------------------------
+    def plan_view(self, name, count):
+        off = self.plan_layout[name]
+        return self.plan[off:off + count]
