@@ -1,0 +1,434 @@
+"""Benchmark of the expert-parallel dispatch path on B200.
+
+One step = one pass of the whole path over one layer's synthetic batch:
+  ep_route_stats -> ep_plan -> ep_layout -> ep_align_sort -> ep_dispatch
+  -> ep_combine -> ep_replica_grad_reduce
+(the expert GEMM between dispatch and combine is outside the path; combine
+reads the dispatched rows).  Metric: routed (token, k) pairs per second.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (default): the moderate EP8 layer, R=8 simulated ranks x S=4096
+tokens, E=64 experts, top-K=6, H=2048 bf16, block_m=64, replica gradients of
+3*2048*1024 fp32 per expert; router logits N(0,1)+b_e with b_e ~ N(0,0.5^2).
+
+`value`: device-resident inputs, CUDA events around each step on the launching
+stream, L2 flushed (a 512 MB write) between steps outside the events, max over
+ranks.  `e2e`: the same steps through the public API (EpLayer.run_host) from
+pinned host buffers: routing, gate weights and hidden rows copied in, the
+combined rows copied out, inside the timed region.  Under torchrun each rank
+runs its own independent layer (weak scaling, no data-path collective).
+
+--impl reference times the CPU oracle (the plain single-threaded definition of
+the same path) on the host, on the same workload and metric.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed (token,k) pairs/s for plan+dispatch+combine; achieved HBM GB/s vs peak"
+UNIT = "pairs/s"
+OPS = ["route_stats", "plan", "layout", "align_sort", "dispatch", "combine", "grad_reduce"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2, help="workload number (1-5); 2 is the headline")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_desc(c):
+    g = f", replica grads {c['grad_n']} {c['grad_dtype']} per expert" if c["grad_n"] else ""
+    return (f"{c['name']}: R={c['R']} simulated EP ranks x S={c['S']} tokens, E={c['E']} experts, top-K={c['K']}, "
+            f"H={c['H']} bf16, block_m={c['block_m']}, router bias {c['bias']}{g}")
+
+
+def config_obj(c, l2):
+    return {"workload": workload_desc(c), "R": c["R"], "S": c["S"], "E": c["E"], "K": c["K"], "H": c["H"],
+            "tokens_per_step": c["T"], "pairs_per_step": c["P"], "block_m": c["block_m"], "l2": l2,
+            "step": "+".join(OPS)}
+
+
+def algorithmic_bytes(c, n_rep, n_chunks):
+    """Bytes each op must move (read + write) for one step."""
+    T, P, E, H, K = c["T"], c["P"], c["E"], c["H"], c["K"]
+    bm = c["block_m"]
+    n = c["grad_n"] or 0
+    gb = 4 if c["grad_dtype"] == "f32" else 2
+    return {
+        "route_stats": 4 * P + 4 * E,
+        "plan": 4 * E,
+        "layout": 4 * P + 8 * P,                      # read ids, write pos + src
+        "align_sort": 4 * P + 4 * P + 4 * (P + E * (bm - 1)),  # read ids twice, write padded ids
+        "dispatch": 2 * T * H + 2 * P * H + 4 * P,    # x once, every buffer row once, pos
+        "combine": 2 * P * H + 8 * P + 2 * T * H,     # every buffer row, w + pos, out once
+        "grad_reduce": n_chunks * 8 * n + n_rep * gb * n,
+    }
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our arm
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_record(kernel):
+    """ncu DRAM bytes per launch for `kernel`, if the committed capture was taken
+    on the current source of that kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha"]:
+        return None
+    return rec
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import token_dispatch_histogram_b200 as tdh
+    import workload as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    c = W.shape(args.config)
+    seed = args.seed + 1000 * rank  # every rank: its own independent layer
+    R, S, E, K, H, T, P = c["R"], c["S"], c["E"], c["K"], c["H"], c["T"], c["P"]
+    gdt = torch.float32 if c["grad_dtype"] in ("f32", None) else torch.bfloat16
+    layer = tdh.EpLayer(R, S, K, E, H, c["block_m"], device=dev, grad_n=c["grad_n"] or 0, grad_dtype=gdt)
+
+    # inputs: host-generated routing and hidden rows (pinned), device-generated grads
+    topk_np, w_np = W.routing(args.config, seed)
+    x_np = W.hidden(T, H, seed)
+    topk_h = torch.from_numpy(topk_np).pin_memory()
+    w_h = torch.from_numpy(w_np).pin_memory()
+    x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    layer.topk_ids.copy_(topk_h)
+    layer.w.copy_(w_h)
+    layer.x.copy_(x_h)
+    if layer.grad_n:
+        W.fill_device(layer.g_home, seed, W.STREAM_GHOME)
+        W.fill_device(layer.g_rep, seed, W.STREAM_GREP)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 512 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        layer.step(stream)
+    torch.cuda.synchronize()
+    status = layer.status(stream)
+    if status:
+        raise RuntimeError(f"device status {status:#x} after warm-up")
+    n_rep = int(layer.plan_view("n_rep", 1).item())
+    n_chunks = int(layer.plan_view("n_chunks", 1).item())
+    max_vio = float(layer.max_vio.item())
+
+    # ---- device-resident timed region
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = tdh.ep_launch_count()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)  # outside the step's events
+        e = ev[i]
+        e[0].record(stream)
+        tdh.ep_route_stats(layer.topk_ids, E, layer.loads, layer.max_vio, layer.ws, layer.dev_status, stream)
+        e[1].record(stream)
+        tdh.ep_plan(layer.loads, R, S, K, E, layer.plan, layer.dev_status, stream)
+        e[2].record(stream)
+        tdh.ep_layout(layer.topk_ids, E, R, S, layer.plan, layer.ws, layer.pos, layer.src, None, layer.dev_status,
+                      stream)
+        e[3].record(stream)
+        tdh.ep_align_sort(layer.topk_ids, E, layer.block_m, layer.sorted_token_ids, layer.expert_ids,
+                          layer.num_tokens_post_pad, layer.ws, layer.dev_status, stream)
+        e[4].record(stream)
+        tdh.ep_dispatch(layer.x, K, layer.pos, layer.buf, layer.dev_status, stream)
+        e[5].record(stream)
+        tdh.ep_combine(layer.buf, layer.w, layer.pos, layer.out, layer.dev_status, stream)
+        e[6].record(stream)
+        layer.grad_reduce(False, stream)
+        e[7].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = tdh.ep_launch_count() - launches0
+    clk = clocks.stop()
+    per_op = {op: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j, op in enumerate(OPS)}
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    status = layer.status(stream)
+    if status:
+        raise RuntimeError(f"device status {status:#x} in the timed region")
+
+    # ---- end to end through the public API, pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        for _ in range(min(3, args.warmup)):
+            layer.run_host(topk_h, w_h, x_h, out_h, stream)
+        torch.cuda.synchronize()
+        barrier()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            layer.run_host(topk_h, w_h, x_h, out_h, stream)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item())
+        bi = topk_h.numel() * 4 + w_h.numel() * 4 + x_h.numel() * 2
+        bo = out_h.numel() * 2
+        e2e = {"value": world * P * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
+
+    # ---- roofline of the dominant kernel and the per-op breakdown
+    ab = algorithmic_bytes(c, n_rep, n_chunks)
+    peak, peak_kind = peaks()
+    mean_ms = {op: sum(v) / len(v) for op, v in per_op.items()}
+    dom = max(("dispatch", "combine", "grad_reduce"), key=lambda op: mean_ms[op])
+    kernel_of = {"dispatch": "k_dispatch", "combine": "k_combine", "grad_reduce": "k_grad_reduce"}
+    achieved = ab[dom] / (mean_ms[dom] / 1e3) / 1e9
+    tr = traffic_record(kernel_of[dom])
+    roofline = {"bound": "hbm", "kernel": kernel_of[dom], "achieved": round(achieved, 1), "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "algorithmic_bytes_per_launch": ab[dom],
+                "traffic": (tr["dram_bytes_per_launch"] if tr else None),
+                "traffic_source": (tr["capture"] if tr else None)}
+    breakdown = {op: {"ms": round(mean_ms[op], 5), "GB_s": round(ab[op] / (mean_ms[op] / 1e3) / 1e9, 1)}
+                 for op in OPS}
+    step_bytes = sum(ab.values())
+    value = world * P * args.steps / (total_ms / 1e3)
+    d_c_ms = mean_ms["dispatch"] + mean_ms["combine"]
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox; see DESIGN.md input recipe)",
+        "config": config_obj(c, "flushed between steps (512 MB write, outside the step events)"),
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "breakdown": breakdown,
+        "step_hbm": {"bytes": step_bytes, "GB_s": round(step_bytes / (total_ms / args.steps / 1e3) / 1e9, 1),
+                     "frac": round(step_bytes / (total_ms / args.steps / 1e3) / 1e9 / peak, 4)},
+        "dispatch_combine": {"ms": round(d_c_ms, 5),
+                             "GB_s": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9, 1),
+                             "frac": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9 / peak, 4)},
+        "routing": {"max_vio": max_vio, "n_rep": n_rep, "replicated_experts": n_chunks},
+    }
+    return res, (topk_np, w_np, x_np, c, seed)
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_step(c, topk, w, x, gh, gr, rep_expert_local):
+    """One pass of the path through the CPU oracle (single thread)."""
+    import oracle as O
+    loads, mv, _ = O.route_stats(topk, c["E"])
+    pl = O.plan(loads, c["R"], c["S"], c["K"], c["E"])
+    lo = O.layout(topk, pl, c["R"], c["S"], c["E"])
+    O.align_sort(topk, c["E"], c["block_m"])
+    buf = O.dispatch(x, lo["pos"], c["K"], c["P"])
+    O.combine(buf, w, lo["pos"], c["K"])
+    if gh is not None:
+        O.grad_reduce(gh, gr, rep_expert_local)
+    return pl
+
+
+def oracle_inputs(c, seed, topk):
+    """Gradient rows the oracle's grad-reduce touches: the replicated experts'
+    home rows and the replica rows, with the replica->expert map remapped to
+    the compact home block (same adds, fewer untouched rows generated)."""
+    import oracle as O
+    import workload as W
+    if not c["grad_n"]:
+        return None, None, None
+    loads, _, _ = O.route_stats(topk, c["E"])
+    pl = O.plan(loads, c["R"], c["S"], c["K"], c["E"])
+    experts = sorted(set(pl["rep_expert"].tolist()))
+    idx = {e: i for i, e in enumerate(experts)}
+    n = c["grad_n"]
+    gh = W.grad_rows(seed, W.STREAM_GHOME, n, max(1, len(experts)))
+    gr = W.grad_rows(seed, W.STREAM_GREP, n, max(1, pl["n_rep"]), c["grad_dtype"])
+    local = np.array([idx[e] for e in pl["rep_expert"]], dtype=np.int32)
+    return gh, gr, local
+
+
+def time_oracle(c, seed, steps, topk=None, w=None, x=None, budget_s=None):
+    import workload as W
+    if topk is None:
+        raise ValueError("routing required")
+    if x is None:
+        x = W.hidden(c["T"], c["H"], seed)
+    gh, gr, local = oracle_inputs(c, seed, topk)
+    times = []
+    t_begin = time.perf_counter()
+    for i in range(steps):
+        t0 = time.perf_counter()
+        oracle_step(c, topk, w, x, gh, gr, local)
+        times.append(time.perf_counter() - t0)
+        if budget_s is not None and time.perf_counter() - t_begin > budget_s:
+            break
+    return times
+
+
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args):
+    import workload as W
+    c = W.shape(args.config)
+    topk, w = W.routing(args.config, args.seed)
+    x = W.hidden(c["T"], c["H"], args.seed)
+    time_oracle(c, args.seed, args.warmup, topk, w, x)
+    times = time_oracle(c, args.seed, args.steps, topk, w, x)
+    total = sum(times)
+    value = c["P"] * len(times) / total
+    sample = (f"the full step on the full workload, {len(times)} timed steps after {args.warmup} warm-up, "
+              f"single thread, {cpu_model()}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": len(times),
+        "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox)",
+        "config": config_obj(c, "n/a (CPU)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res, (topk, w, x, c, seed) = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times = time_oracle(c, seed, 3, topk, w, x, budget_s=20.0)
+        v = c["P"] * len(times) / sum(times)
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                               "sample": f"{len(times)} full steps of the same workload and seed, single thread, "
+                                         f"{cpu_model()} ({os.cpu_count()} cores on the host)"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()
