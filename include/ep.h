@@ -235,6 +235,30 @@ EP_API int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtyp
                            const int32_t* plan, size_t plan_words, int clear_replicas, int32_t* dev_status,
                            cudaStream_t stream);
 
+/*
+ * ep_route_stats without a scratch argument, for callers that cannot allocate
+ * device memory for it: hosts that pass a kernel only its inputs and outputs at
+ * enqueue time and forbid allocation there, or runtimes whose device memory is
+ * all planned in advance.  The source pages have no counterpart of this call;
+ * it computes the same loads and max_vio as ep_route_stats, bit for bit.
+ *   Scratch: a fixed array of EP_NOALLOC_SCRATCH_BYTES inside the library,
+ *   present on every GPU that loads it until the process exits.  The problem
+ *   must fit: about 12 * ceil(T*K / tile) * E + 4*E + 512 bytes, tile = 2048,
+ *   4096 or 8192 pairs (as ep_workspace_size reports for the same T, K, E);
+ *   larger problems get EP_ERR_CAPACITY and nothing is enqueued.
+ *   The first call on a device (with that device current) looks the array's
+ *   device address up with cudaGetSymbolAddress; make that first call before
+ *   any stream capture.  No call allocates (no cudaMalloc, cudaFree or
+ *   allocating library routine).
+ *   All calls share the one array and it keeps the previous call's contents:
+ *   calls whose work overlaps on the GPU (other streams, other threads) race
+ *   on it and must be serialised by the caller.  ep_layout cannot use this
+ *   call's per-tile counts; use ep_route_stats with a workspace for that.
+ */
+#define EP_NOALLOC_SCRATCH_BYTES (4u << 20)
+EP_API int ep_route_stats_noalloc(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads, double* max_vio,
+                                  int32_t* dev_status, cudaStream_t stream);
+
 /* Copy *dev_status to *host_status (host) after the work queued on `stream`;
  * waits for the stream.  The only synchronising call. */
 EP_API int ep_status_read(const int32_t* dev_status, int32_t* host_status, cudaStream_t stream);

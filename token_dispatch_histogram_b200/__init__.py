@@ -51,6 +51,7 @@ _SIGS = {
     "ep_workspace_size": (_I, [_I64, _I, _I, _V]),
     "ep_plan_layout": (_I, [_I, _I, _V]),
     "ep_route_stats": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
+    "ep_route_stats_noalloc": (_I, [_V, _I64, _I, _I, _V, _V, _V, _V]),
     "ep_plan": (_I, [_V, _I, _I64, _I, _I, _V, _SZ, _V, _V]),
     "ep_layout": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _SZ, _V, _SZ, _V, _V, _V, _V, _V]),
     "ep_align_sort": (_I, [_V, _I64, _I, _I, _I, _V, _I64, _V, _I64, _V, _V, _SZ, _V, _V]),
@@ -134,6 +135,17 @@ def ep_route_stats(topk_ids, E, loads, max_vio, ws, dev_status=None, stream=None
     T, K = topk_ids.shape
     _check("ep_route_stats", lib().ep_route_stats(_p(topk_ids), T, K, E, _p(loads), _p(max_vio), _p(ws),
                                                   ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
+
+
+def ep_route_stats_noalloc(topk_ids, E, loads, max_vio, dev_status=None, stream=None):
+    """ep_route_stats with the library's fixed internal scratch instead of a
+    caller workspace (for callers that cannot allocate one)."""
+    _dtype(topk_ids, torch.int32)
+    _dtype(loads, torch.int32)
+    _dtype(max_vio, torch.float64)
+    T, K = topk_ids.shape
+    _check("ep_route_stats_noalloc", lib().ep_route_stats_noalloc(_p(topk_ids), T, K, E, _p(loads), _p(max_vio),
+                                                                  _p(dev_status), _s(stream)))
 
 
 def ep_plan(loads, R, S, K, E, plan, dev_status=None, stream=None):

@@ -16,6 +16,8 @@
 //    (tile, expert), every wait bounded,
 //  - the last tile's inclusive prefix is T_e; it also reduces max_e T_e.
 // Only integer adds feed the outputs, so they do not depend on scheduling.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace ep {
@@ -151,4 +153,53 @@ extern "C" int ep_route_stats(const int32_t* topk_ids, int64_t T, int K, int E, 
   if (P > 0 && !topk_ids) return EP_ERR_ARG;
   if (ws_bytes < ws_layout(P, E).bytes) return EP_ERR_CAPACITY;
   return run_hist(topk_ids, P, E, ws, loads, max_vio, dev_status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of ep_route_stats.
+//
+// Some callers cannot hand this library a scratch buffer: hosts that give a
+// kernel only its input and output tensors at enqueue time and forbid device
+// allocation there (plugin-style interfaces), or runtimes whose device memory is
+// planned once up front.  For them ep_route_stats_noalloc keeps its scratch in
+// the fixed array below, which exists on every GPU that loads this library
+// until the process exits.  Its device address is looked up once per device
+// (cudaGetSymbolAddress) on the first call made with that device current.  All
+// calls share the array and it keeps the last call's contents; the part that
+// must start at zero (the look-back words and the tile counter) is cleared on
+// the call's stream, so calls must not overlap on the GPU: two calls running at
+// the same time race on the array.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EP_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {nullptr};
+
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return EP_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return EP_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return EP_OK;
+}
+}  // namespace
+
+
+extern "C" int ep_route_stats_noalloc(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads,
+                                      double* max_vio, int32_t* dev_status, cudaStream_t stream) {
+  using namespace ep;
+  if (!valid_tke(T, K, E) || !loads || !max_vio) return EP_ERR_ARG;
+  const int64_t P = T * K;
+  if (P > 0 && !topk_ids) return EP_ERR_ARG;
+  if (ws_layout(P, E).bytes > (size_t)EP_NOALLOC_SCRATCH_BYTES) return EP_ERR_CAPACITY;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != EP_OK) return rc;
+  return run_hist(topk_ids, P, E, scratch, loads, max_vio, dev_status, stream);
 }
