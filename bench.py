@@ -138,6 +138,28 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------ multi-rank host logic
+
+def rank_seed(base, rank):
+    """Every rank runs its own independent layer (weak scaling): its own seed."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(value_ms, world, device):
+    """Max of a per-rank device time over all ranks (the job's time)."""
+    import torch
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, pairs_per_step, steps, job_ms):
+    """Whole-job pairs/s: all ranks' pairs over the slowest rank's time."""
+    return world * pairs_per_step * steps / (job_ms / 1e3)
+
+
 # --------------------------------------------------------------- our arm
 
 def peaks():
@@ -172,7 +194,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     c = W.shape(args.config)
-    seed = args.seed + 1000 * rank  # every rank: its own independent layer
+    seed = rank_seed(args.seed, rank)
     R, S, E, K, H, T, P = c["R"], c["S"], c["E"], c["K"], c["H"], c["T"], c["P"]
     gdt = torch.float32 if c["grad_dtype"] in ("f32", None) else torch.bfloat16
     layer = tdh.EpLayer(R, S, K, E, H, c["block_m"], device=dev, grad_n=c["grad_n"] or 0, grad_dtype=gdt)
@@ -242,11 +264,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     per_op = {op: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j, op in enumerate(OPS)}
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     status = layer.status(stream)
     if status:
         raise RuntimeError(f"device status {status:#x} in the timed region")
@@ -267,14 +285,10 @@ def run_ours(args, rank, world, local_rank):
             ends[i].record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item())
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
         bi = topk_h.numel() * 4 + w_h.numel() * 4 + x_h.numel() * 2
         bo = out_h.numel() * 2
-        e2e = {"value": world * P * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": bi,
+        e2e = {"value": job_throughput(world, P, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
 
     # ---- roofline of the dominant kernel and the per-op breakdown
@@ -293,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
     breakdown = {op: {"ms": round(mean_ms[op], 5), "GB_s": round(ab[op] / (mean_ms[op] / 1e3) / 1e9, 1)}
                  for op in OPS}
     step_bytes = sum(ab.values())
-    value = world * P * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, P, args.steps, total_ms)
     d_c_ms = mean_ms["dispatch"] + mean_ms["combine"]
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -259,6 +259,18 @@ EP_API int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtyp
 EP_API int ep_route_stats_noalloc(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads, double* max_vio,
                                   int32_t* dev_status, cudaStream_t stream);
 
+/*
+ * Self-test of failure detection (no counterpart on the pages): runs
+ * ep_route_stats' kernel with its first tile never scheduled, so every other
+ * tile's look-back waits on a flag that nothing sets.  The waits run out after
+ * about one second, EP_DEV_LOOKBACK_TIMEOUT is OR-ed into *dev_status, and the
+ * CUDA context stays usable.  Needs T*K above one tile (> 2048 pairs).  Waits
+ * for the stream before returning.  loads and max_vio come out wrong by design.
+ */
+EP_API int ep_selftest_lookback_timeout(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads,
+                                        double* max_vio, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                        cudaStream_t stream);
+
 /* Copy *dev_status to *host_status (host) after the work queued on `stream`;
  * waits for the stream.  The only synchronising call. */
 EP_API int ep_status_read(const int32_t* dev_status, int32_t* host_status, cudaStream_t stream);

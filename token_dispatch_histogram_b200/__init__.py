@@ -60,6 +60,7 @@ _SIGS = {
     "ep_combine": (_I, [_V, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
     "ep_replica_grad_reduce": (_I, [_V, _V, _I, _I64, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_status_read": (_I, [_V, _V, _V]),
+    "ep_selftest_lookback_timeout": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
 }
 
 
@@ -217,6 +218,14 @@ def ep_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False, dev_
     _check("ep_replica_grad_reduce", lib().ep_replica_grad_reduce(_p(g_home), _p(g_rep), dt, n, E, R, _p(plan),
                                                                   plan.numel(), int(bool(clear_replicas)),
                                                                   _p(dev_status), _s(stream)))
+
+
+def ep_selftest_lookback_timeout(topk_ids, E, loads, max_vio, ws, dev_status, stream=None):
+    """Failure-detection self-test: a look-back wait that runs out (see ep.h)."""
+    T, K = topk_ids.shape
+    _check("ep_selftest_lookback_timeout",
+           lib().ep_selftest_lookback_timeout(_p(topk_ids), T, K, E, _p(loads), _p(max_vio), _p(ws),
+                                              ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
 
 
 def ep_status_read(dev_status, stream=None):

@@ -93,7 +93,7 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
 // Wall-clock bound for every wait inside a kernel (a look-back on another
 // CTA, an mbarrier of an asynchronous copy): after it the kernel reports a
 // timeout bit and goes on, so no wait can hang the device.
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -136,9 +136,40 @@ int run_hist(const int32_t* topk, int64_t P, int E, void* ws, int32_t* loads, do
   return launch_status();
 }
 
+// Self-test of the bounded look-back: the tile counter starts at 1 and one CTA
+// fewer is launched, so tile 0 is never processed and its flag is never set.
+// Every later tile's wait on it runs out after WAIT_LIMIT_NS and reports
+// EP_DEV_LOOKBACK_TIMEOUT; all accesses stay inside the workspace.
+int run_hist_skip_first_tile(const int32_t* topk, int64_t P, int E, void* ws, int32_t* loads, double* max_vio,
+                             int32_t* dev_status, cudaStream_t st) {
+  const WsLayout l = ws_layout(P, E);
+  const int tile = tile_pairs_for(P);
+  const int64_t nt = num_tiles(P, tile);
+  if (nt < 2) return EP_ERR_ARG;
+  char* w = static_cast<char*>(ws);
+  if (cudaMemsetAsync(w, 0, l.clear_bytes, st) != cudaSuccess) return EP_ERR_CUDA;
+  const uint32_t one = 1;
+  if (cudaMemcpyAsync(w, &one, sizeof(one), cudaMemcpyHostToDevice, st) != cudaSuccess) return EP_ERR_CUDA;
+  k_hist_lookback<<<(unsigned)(nt - 1), HIST_THREADS, (size_t)E * 4, st>>>(
+      topk, P, E, tile, (int)nt, reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint64_t*>(w + l.status_off),
+      reinterpret_cast<int32_t*>(w + l.excl_off), loads, max_vio, dev_status);
+  count_launch();
+  if (cudaStreamSynchronize(st) != cudaSuccess) return EP_ERR_CUDA;  // `one` lives on this stack frame
+  return launch_status();
+}
+
 }  // namespace ep
 
 using namespace ep;
+
+extern "C" int ep_selftest_lookback_timeout(const int32_t* topk_ids, int64_t T, int K, int E, int32_t* loads,
+                                            double* max_vio, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                            cudaStream_t stream) {
+  if (!valid_tke(T, K, E) || !topk_ids || !loads || !max_vio || !ws || !dev_status) return EP_ERR_ARG;
+  const int64_t P = T * K;
+  if (ws_bytes < ws_layout(P, E).bytes) return EP_ERR_CAPACITY;
+  return run_hist_skip_first_tile(topk_ids, P, E, ws, loads, max_vio, dev_status, stream);
+}
 
 extern "C" int ep_workspace_size(int64_t T, int K, int E, size_t* bytes) {
   if (!bytes || !valid_tke(T, K, E)) return EP_ERR_ARG;
