@@ -39,7 +39,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "routed (token,k) pairs/s for plan+dispatch+combine; achieved HBM GB/s vs peak"
 UNIT = "pairs/s"
-OPS = ["route_stats", "plan", "layout", "align_sort", "dispatch", "combine", "grad_reduce"]
+OPS = ["route", "dispatch", "combine", "grad_reduce"]
+ROUTE_PARTS = ["route_stats", "plan", "layout", "align_sort"]
 
 
 def parse():
@@ -52,6 +53,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--route", choices=["fused", "separate"], default="fused",
+                    help="route phase as one cooperative launch (ep_route_fused) or the four separate calls")
     return ap.parse_args()
 
 
@@ -64,7 +67,7 @@ def workload_desc(c):
 def config_obj(c, l2):
     return {"workload": workload_desc(c), "R": c["R"], "S": c["S"], "E": c["E"], "K": c["K"], "H": c["H"],
             "tokens_per_step": c["T"], "pairs_per_step": c["P"], "block_m": c["block_m"], "l2": l2,
-            "step": "+".join(OPS)}
+            "step": "route(" + "+".join(ROUTE_PARTS) + ")+dispatch+combine+grad_reduce"}
 
 
 def algorithmic_bytes(c, n_rep, n_chunks):
@@ -73,11 +76,14 @@ def algorithmic_bytes(c, n_rep, n_chunks):
     bm = c["block_m"]
     n = c["grad_n"] or 0
     gb = 4 if c["grad_dtype"] == "f32" else 2
-    return {
+    parts = {
         "route_stats": 4 * P + 4 * E,
         "plan": 4 * E,
         "layout": 4 * P + 8 * P,                      # read ids, write pos + src
         "align_sort": 4 * P + 4 * P + 4 * (P + E * (bm - 1)),  # read ids twice, write padded ids
+    }
+    return {
+        "route": sum(parts.values()),
         "dispatch": 2 * T * H + 2 * P * H + 4 * P,    # x once, every buffer row once, pos
         "combine": 2 * P * H + 8 * P + 2 * T * H,     # every buffer row, w + pos, out once
         "grad_reduce": n_chunks * 8 * n + n_rep * gb * n,
@@ -221,8 +227,9 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    fused = args.route == "fused"
     for _ in range(args.warmup):
-        layer.step(stream)
+        layer.step(stream, fused=fused)
     torch.cuda.synchronize()
     status = layer.status(stream)
     if status:
@@ -242,22 +249,14 @@ def run_ours(args, rank, world, local_rank):
         flush.fill_(i & 0xFF)  # outside the step's events
         e = ev[i]
         e[0].record(stream)
-        tdh.ep_route_stats(layer.topk_ids, E, layer.loads, layer.max_vio, layer.ws, layer.dev_status, stream)
+        layer.route(stream, fused=fused)
         e[1].record(stream)
-        tdh.ep_plan(layer.loads, R, S, K, E, layer.plan, layer.dev_status, stream)
-        e[2].record(stream)
-        tdh.ep_layout(layer.topk_ids, E, R, S, layer.plan, layer.ws, layer.pos, layer.src, None, layer.dev_status,
-                      stream)
-        e[3].record(stream)
-        tdh.ep_align_sort(layer.topk_ids, E, layer.block_m, layer.sorted_token_ids, layer.expert_ids,
-                          layer.num_tokens_post_pad, layer.ws, layer.dev_status, stream)
-        e[4].record(stream)
         tdh.ep_dispatch(layer.x, K, layer.pos, layer.buf, layer.dev_status, stream)
-        e[5].record(stream)
+        e[2].record(stream)
         tdh.ep_combine(layer.buf, layer.w, layer.pos, layer.out, layer.dev_status, stream)
-        e[6].record(stream)
+        e[3].record(stream)
         layer.grad_reduce(False, stream)
-        e[7].record(stream)
+        e[4].record(stream)
     torch.cuda.synchronize()
     barrier()
     launches = tdh.ep_launch_count() - launches0
@@ -273,7 +272,7 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         for _ in range(min(3, args.warmup)):
-            layer.run_host(topk_h, w_h, x_h, out_h, stream)
+            layer.run_host(topk_h, w_h, x_h, out_h, stream, fused=fused)
         torch.cuda.synchronize()
         barrier()
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -281,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             starts[i].record(stream)
-            layer.run_host(topk_h, w_h, x_h, out_h, stream)
+            layer.run_host(topk_h, w_h, x_h, out_h, stream, fused=fused)
             ends[i].record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -325,6 +324,7 @@ def run_ours(args, rank, world, local_rank):
                              "GB_s": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9, 1),
                              "frac": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9 / peak, 4)},
         "routing": {"max_vio": max_vio, "n_rep": n_rep, "replicated_experts": n_chunks},
+        "route_path": args.route,
     }
     return res, (topk_np, w_np, x_np, c, seed)
 

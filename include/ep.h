@@ -193,6 +193,22 @@ EP_API int ep_align_sort(const int32_t* topk_ids, int64_t T, int K, int E, int b
                   void* ws, size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * a1-a4 in one launch: the outputs of ep_route_stats, ep_plan, ep_layout and
+ * (when sorted_token_ids is not NULL) ep_align_sort, bit for bit, from one
+ * cooperative kernel whose CTAs meet at grid barriers (all waits bounded).
+ * The route phase moves only a few bytes per pair, so it is latency-bound; one
+ * resident grid replaces four launches and the serial look-back.  When the
+ * grid cannot be co-resident it runs the four separate calls instead.
+ * Arguments as in those calls; ws is ep_workspace_size bytes (its contents
+ * afterwards are not the per-tile prefixes ep_layout reads).
+ */
+EP_API int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
+                          double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
+                          int32_t* pair_slot, int block_m, int32_t* sorted_token_ids, int64_t sorted_cap,
+                          int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad, void* ws,
+                          size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
  * a5. Dispatch.  [GR] "Online planning, zero copy και στατικά σχήματα": rows are
  * written in place into the expert-grouped buffer, no intermediate copy.
  *   x   [T, H] bf16; buf [buf_rows, H] bf16 out; buf[pos[p]] = x[p / K] bitwise.

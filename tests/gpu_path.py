@@ -12,7 +12,8 @@ def _torch():
     return torch
 
 
-def run_cuda(topk, w, x, R, S, E, block_m, scale=None, g_home=None, g_rep=None, clear=False, with_y=True):
+def run_cuda(topk, w, x, R, S, E, block_m, scale=None, g_home=None, g_rep=None, clear=False, with_y=True,
+             fused=False):
     """All outputs of one pass: stats, plan, layout, align-sort, dispatch,
     stand-in expert, combine, grad-reduce.  x: uint16 [T,H] (or None)."""
     torch = _torch()
@@ -28,17 +29,20 @@ def run_cuda(topk, w, x, R, S, E, block_m, scale=None, g_home=None, g_rep=None, 
     ws = torch.full((tdh.ep_workspace_size(T, K, E),), 0xAB, dtype=torch.uint8, device=dev)
     lay = tdh.ep_plan_layout(E, R)
     plan = torch.full((lay["words"],), -7, dtype=torch.int32, device=dev)
-    tdh.ep_route_stats(t_topk, E, loads, mv, ws, status)
-    tdh.ep_plan(loads, R, S, K, E, plan, status)
     pos = torch.full((P,), -7, dtype=torch.int32, device=dev)
     src = torch.full((P,), -7, dtype=torch.int32, device=dev)
     slot = torch.full((P,), -7, dtype=torch.int32, device=dev)
-    tdh.ep_layout(t_topk, E, R, S, plan, ws, pos, src, slot, status)
     cap, capb = tdh.align_sort_capacity(P, E, block_m)
     sids = torch.full((cap,), -7, dtype=torch.int32, device=dev)
     eids = torch.full((capb,), -7, dtype=torch.int32, device=dev)
     ntpp = torch.full((1,), -7, dtype=torch.int32, device=dev)
-    tdh.ep_align_sort(t_topk, E, block_m, sids, eids, ntpp, ws, status)
+    if fused:
+        tdh.ep_route_fused(t_topk, E, R, S, loads, mv, plan, pos, src, ws, slot, block_m, sids, eids, ntpp, status)
+    else:
+        tdh.ep_route_stats(t_topk, E, loads, mv, ws, status)
+        tdh.ep_plan(loads, R, S, K, E, plan, status)
+        tdh.ep_layout(t_topk, E, R, S, plan, ws, pos, src, slot, status)
+        tdh.ep_align_sort(t_topk, E, block_m, sids, eids, ntpp, ws, status)
     out.update(loads=loads.cpu().numpy(), max_vio=float(mv.cpu().numpy()[0]), plan=plan.cpu().numpy(), layout=lay,
                pos=pos.cpu().numpy(), src=src.cpu().numpy(), pair_slot=slot.cpu().numpy(),
                sorted_ids=sids.cpu().numpy(), expert_ids=eids.cpu().numpy(), ntpp=int(ntpp.cpu().numpy()[0]))

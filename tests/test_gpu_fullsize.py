@@ -82,7 +82,7 @@ def _check_rows(layer, c, topk, w, lo, seed, layer_id, rng):
     assert np.count_nonzero(ulp) == 0
 
 
-def _run_layer(cfg, seed, layer_id=0, variant="default", rows=True, grads=False):
+def _run_layer(cfg, seed, layer_id=0, variant="default", rows=True, grads=False, fused=True):
     import torch
     c = W.shape(cfg)
     dev = torch.device("cuda")
@@ -92,7 +92,7 @@ def _run_layer(cfg, seed, layer_id=0, variant="default", rows=True, grads=False)
     layer.w.copy_(torch.from_numpy(w))
     if rows:
         W.fill_device(layer.x, seed, W.STREAM_X + layer_id)
-    layer.route()
+    layer.route(fused=fused)
     if rows:
         layer.dispatch()
     assert layer.status() == 0
@@ -103,16 +103,18 @@ def _run_layer(cfg, seed, layer_id=0, variant="default", rows=True, grads=False)
     return layer, c, pl, lo, mv
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
 @pytest.mark.parametrize("cfg", [2, 3, 5])
-def test_full_size_layer(cfg):
-    layer, c, pl, lo, mv = _run_layer(cfg, seed=0)
+def test_full_size_layer(cfg, fused):
+    layer, c, pl, lo, mv = _run_layer(cfg, seed=0, rows=fused, fused=fused)
     assert pl["n_rep"] > 0
     del layer
 
 
 def test_full_size_fine_grained_eight_layers():
     for layer_id in range(8):
-        layer, c, pl, lo, mv = _run_layer(4, seed=0, layer_id=layer_id, rows=layer_id in (0, 7))
+        layer, c, pl, lo, mv = _run_layer(4, seed=0, layer_id=layer_id, rows=layer_id in (0, 7),
+                                          fused=layer_id % 2 == 0)
         del layer
 
 

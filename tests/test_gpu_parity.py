@@ -49,11 +49,12 @@ def _assert_route_parity(cu, orc, R, S, K, E):
     assert cu["ntpp"] == orc["ntpp"]
 
 
-def test_hand_example_on_gpu():
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_hand_example_on_gpu(fused):
     g = PINS.golden()
     topk = np.array(g["topk_ids"], dtype=np.int32)
     R, S, K, E = g["R"], g["S"], g["K"], g["E"]
-    cu = run_cuda(topk, None, None, R, S, E, g["block_m"])
+    cu = run_cuda(topk, None, None, R, S, E, g["block_m"], fused=fused)
     assert cu["status"] == 0
     assert cu["loads"].tolist() == g["loads"]
     assert cu["max_vio"] == g["max_vio"]
@@ -80,19 +81,21 @@ ROUTE_CASES = [
 ]
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("case", ROUTE_CASES, ids=lambda c: "R{}_S{}_K{}_E{}_{}".format(*c[:5]))
-def test_route_plan_layout_align(case):
+def test_route_plan_layout_align(case, fused):
     R, S, K, E, kind, bm = case
     if kind == "zipf":
         topk, w = W.routing_from(R * S, E, K, seed=0, bias_e=W.bias(1, 0))
     else:
         topk, w, _ = case_inputs(R, S, K, E, 0, seed=R * 131 + S, kind=kind, bias_scale=1.5)
-    cu = run_cuda(topk, None, None, R, S, E, bm)
+    cu = run_cuda(topk, None, None, R, S, E, bm, fused=fused)
     orc = run_oracle(topk, None, None, R, S, E, bm)
     _assert_route_parity(cu, orc, R, S, K, E)
 
 
-def test_route_fuzz():
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_route_fuzz(fused):
     rng = np.random.default_rng(2024)
     for it in range(60):
         R = int(rng.choice([1, 2, 3, 4, 8, 16]))
@@ -103,7 +106,7 @@ def test_route_fuzz():
         kind = ["skew", "uniform", "single"][it % 3]
         bm = int(rng.choice([1, 2, 16, 64, 128]))
         topk, w, _ = case_inputs(R, S, K, E, 0, seed=it, kind=kind, bias_scale=float(rng.uniform(0.2, 3)))
-        cu = run_cuda(topk, None, None, R, S, E, bm)
+        cu = run_cuda(topk, None, None, R, S, E, bm, fused=fused)
         orc = run_oracle(topk, None, None, R, S, E, bm)
         _assert_route_parity(cu, orc, R, S, K, E)
 

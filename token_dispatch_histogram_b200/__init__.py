@@ -55,6 +55,8 @@ _SIGS = {
     "ep_plan": (_I, [_V, _I, _I64, _I, _I, _V, _SZ, _V, _V]),
     "ep_layout": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _SZ, _V, _SZ, _V, _V, _V, _V, _V]),
     "ep_align_sort": (_I, [_V, _I64, _I, _I, _I, _V, _I64, _V, _I64, _V, _V, _SZ, _V, _V]),
+    "ep_route_fused": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _V, _V, _SZ, _V, _V, _V, _I, _V, _I64, _V, _I64, _V,
+                            _V, _SZ, _V, _V]),
     "ep_dispatch": (_I, [_V, _I64, _I, _I64, _V, _V, _I64, _V, _V]),
     "ep_expert_scale": (_I, [_V, _I64, _I64, _V, _V, _I64, _V, _I, _V, _V, _V]),
     "ep_combine": (_I, [_V, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
@@ -173,6 +175,22 @@ def ep_align_sort(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens
                                                 sorted_token_ids.numel(), _p(expert_ids), expert_ids.numel(),
                                                 _p(num_tokens_post_pad), _p(ws), ws.numel() * ws.element_size(),
                                                 _p(dev_status), _s(stream)))
+
+
+def ep_route_fused(topk_ids, E, R, S, loads, max_vio, plan, pos, src, ws, pair_slot=None, block_m=0,
+                   sorted_token_ids=None, expert_ids=None, num_tokens_post_pad=None, dev_status=None, stream=None):
+    """ep_route_stats + ep_plan + ep_layout (+ ep_align_sort when
+    sorted_token_ids is given) in one cooperative launch."""
+    for t in (topk_ids, loads, plan, pos, src):
+        _dtype(t, torch.int32)
+    _dtype(max_vio, torch.float64)
+    T, K = topk_ids.shape
+    align = sorted_token_ids is not None
+    _check("ep_route_fused", lib().ep_route_fused(
+        _p(topk_ids), T, K, E, R, S, _p(loads), _p(max_vio), _p(plan), plan.numel(), _p(pos), _p(src),
+        _p(pair_slot), block_m, _p(sorted_token_ids), sorted_token_ids.numel() if align else 0,
+        _p(expert_ids), expert_ids.numel() if align else 0, _p(num_tokens_post_pad), _p(ws),
+        ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
 
 
 def align_sort_capacity(P, E, block_m):

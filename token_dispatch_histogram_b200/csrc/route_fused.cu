@@ -1,0 +1,440 @@
+// The whole route phase -- a1 stats, a2 plan, a3 layout, a4 align-sort -- in
+// ONE cooperative launch.  Same outputs as ep_route_stats + ep_plan + ep_layout
+// + ep_align_sort, bit for bit.
+//
+// Why: every step of the route phase moves only a few MB (4-12 bytes per pair),
+// so on B200 it is bound by latency chains, not HBM: launch gaps, the serial
+// look-back, one CTA planning while the GPU idles.  Here all CTAs stay resident
+// (cooperative launch) and meet at grid barriers instead:
+//   1. each CTA counts its tile per warp (__match_any_sync aggregation) and
+//      writes the tile's per-expert counts, column-major [E][tiles];
+//   -- grid barrier --
+//   2. the per-expert columns are scanned in parallel (one CTA per expert
+//      column): exclusive tile prefixes, and the column totals are T_e;
+//   -- grid barrier --
+//   3. CTA 0 runs the planner (plan_block.cuh) and max_vio and raises a flag;
+//      meanwhile every CTA walks its tile once for the align-sort ranks (which
+//      need only T_e), writing sorted ids, padding and block experts;
+//   4. after the flag, every CTA walks its tile again for the layout ranks and
+//      writes pos / src / pair_slot from the plan.
+// A pair's stable rank within its expert = (its tile's prefix) + (earlier warps
+// of the tile) + (earlier chunks of its warp) + popc(peers & lanemask_lt):
+// integer adds only, so nothing depends on scheduling.  Every wait is bounded.
+#include <algorithm>
+
+#include "plan_block.cuh"
+
+namespace ep {
+
+int fused_route_separate(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
+                         double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
+                         int32_t* pair_slot, int block_m, int32_t* sorted_ids, int64_t sorted_cap,
+                         int32_t* expert_ids, int64_t expert_ids_cap, int32_t* ntpp, void* ws, size_t ws_bytes,
+                         int32_t* dev_status, cudaStream_t stream);
+
+constexpr int FUSED_THREADS = 512;
+constexpr int FUSED_WARPS = FUSED_THREADS / 32;
+
+struct FusedArgs {
+  const int32_t* topk;
+  int64_t P;
+  int E, R;
+  int32_t SK;
+  int tile, ntiles;
+  uint32_t* sync;  // [0] barrier arrivals, [1] plan-ready flag
+  int32_t* counts; // [E][ntiles] tile counts, then exclusive tile prefixes
+  int32_t* loads;
+  double* max_vio;
+  int32_t* plan;
+  EpPlanLayout L;
+  int32_t* pos;
+  int32_t* src;
+  int32_t* pair_slot;
+  int block_m;
+  int32_t* sorted_ids;
+  int64_t sorted_cap;
+  int32_t* expert_ids;
+  int64_t expert_ids_cap;
+  int32_t* ntpp;
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Thread 0 waits (bounded) until *ctr >= target; the block follows.
+__device__ void wait_at_least(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
+  if (threadIdx.x == 0 && ld_acquire_u32(ctr) < target) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_u32(ctr) < target) {
+      __nanosleep(32);
+      if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+        flag(dev_status, EP_DEV_LOOKBACK_TIMEOUT);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Barrier over all CTAs of the cooperative grid (they are co-resident).
+__device__ void grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+  }
+  wait_at_least(ctr, target, dev_status);
+}
+
+// Walk this warp's part of the tile in flattened order; `run` is the warp's
+// running per-expert count (initialised to the rank of its first pair).
+template <class Emit>
+__device__ __forceinline__ void walk_warp(const int32_t* __restrict__ topk, int64_t P, int E, int64_t wp0, int sub,
+                                          int32_t* run, Emit emit, int* s_bad) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = lanemask_lt();
+  int64_t p = wp0 + lane;
+  int nxt = (sub > 0 && p < P) ? __ldg(topk + p) : -1;
+  for (int c = 0; c < sub; c += 32, p += 32) {
+    int e = nxt;
+    if (c + 32 < sub && p + 32 < P) nxt = __ldg(topk + p + 32);
+    if (p >= P) e = -1;
+    else if (e < 0 || e >= E) e = -2;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    int32_t base = 0;
+    if (e >= 0) base = run[e];
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) run[e] = base + __popc(peers);
+    __syncwarp();
+    if (e >= 0)
+      emit(p, e, base + __popc(peers & lt));
+    else if (e == -2)
+      *s_bad = 1;
+  }
+}
+
+__global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
+  extern __shared__ int32_t sm[];
+  const int E = a.E, tile = a.tile, G = gridDim.x, t = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int sub = tile / FUSED_WARPS;
+  const int cap = a.L.cap;
+  const int region_a = max(FUSED_WARPS * E, plan_work_words(E, a.R));
+  int32_t* s_wb = sm;                          // [16][E] per-warp exclusive counts within the tile
+  int32_t* s_run = s_wb + FUSED_WARPS * E;     // region A: running counters, or the planner's work space
+  int32_t* s_loads = s_run + region_a;         // [E]
+  int32_t* s_excl = s_loads + E;               // [E] this tile's prefix per expert
+  int32_t* s_off = s_excl + E;                 // [E + 1] align-sort group offsets
+  int32_t* s_hc = s_off + E + 1;               // [E] home_count
+  int32_t* s_hb = s_hc + E;                    // [E] home_base
+  int32_t* s_cf = s_hb + E;                    // [E] copy_first
+  int32_t* s_cc = s_cf + E;                    // [E] copy_cnt
+  int32_t* s_rb = s_cc + E;                    // [cap] rep_begin
+  int32_t* s_rc = s_rb + cap;                  // [cap] rep_count
+  int32_t* s_rbase = s_rc + cap;               // [cap] rep_base
+  __shared__ int32_t warp_sums[32];
+  __shared__ int s_bad, s_badrow;
+  __shared__ int32_t s_max[FUSED_WARPS];
+  const int64_t p0 = (int64_t)t * tile;
+  const int64_t wp0 = p0 + (int64_t)warp * sub;
+
+  // ---- 1. per-warp counts of this tile
+  if (tid == 0) {
+    s_bad = 0;
+    s_badrow = 0;
+  }
+  for (int i = tid; i < FUSED_WARPS * E; i += FUSED_THREADS) s_wb[i] = 0;
+  __syncthreads();
+  {
+    int32_t* my = s_wb + warp * E;
+    int64_t p = wp0 + lane;
+    int nxt = p < a.P ? __ldg(a.topk + p) : -1;
+    for (int c = 0; c < sub; c += 32, p += 32) {
+      int e = nxt;
+      if (c + 32 < sub && p + 32 < a.P) nxt = __ldg(a.topk + p + 32);
+      if (p >= a.P || e < 0 || e >= E) e = -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += FUSED_THREADS) {
+    int32_t run = 0;
+    for (int w = 0; w < FUSED_WARPS; ++w) {
+      const int32_t c = s_wb[w * E + e];
+      s_wb[w * E + e] = run;
+      run += c;
+    }
+    a.counts[(int64_t)e * G + t] = run;
+  }
+  grid_barrier(a.sync, (uint32_t)G, a.dev_status);
+
+  // ---- 2. exclusive scan of every expert column over the tiles; totals = T_e
+  for (int e = t; e < E; e += G) {
+    const int32_t total = block_scan_inplace(a.counts + (int64_t)e * G, G, warp_sums);
+    if (tid == 0) a.loads[e] = total;
+  }
+  grid_barrier(a.sync, 2u * G, a.dev_status);
+
+  // ---- 3. planner on CTA 0; align-sort ranks everywhere
+  for (int e = tid; e < E; e += FUSED_THREADS) {
+    s_loads[e] = __ldcg(a.loads + e);
+    s_excl[e] = __ldcg(a.counts + (int64_t)e * G + t);
+  }
+  __syncthreads();
+  if (t == 0) {
+    int32_t m = 0;
+    for (int e = tid; e < E; e += FUSED_THREADS) m = max(m, s_loads[e]);
+#pragma unroll
+    for (int d = 16; d; d >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, d));
+    if (lane == 0) s_max[warp] = m;
+    __syncthreads();
+    if (tid == 0) {
+      int32_t mx = 0;
+      for (int w = 0; w < FUSED_WARPS; ++w) mx = max(mx, s_max[w]);
+      *a.max_vio = a.P > 0 ? __dsub_rn(__ddiv_rn(__dmul_rn((double)mx, (double)E), (double)a.P), 1.0) : 0.0;
+    }
+    plan_block(s_loads, a.R, a.SK, E, a.plan, a.L, s_run, a.dev_status);
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release_u32(a.sync + 1, 1u);
+    }
+  }
+  if (a.sorted_ids) {
+    const int bm = a.block_m;
+    for (int e = tid; e < E; e += FUSED_THREADS) s_off[e] = (s_loads[e] + bm - 1) / bm * bm;
+    __syncthreads();
+    const int32_t total = block_scan_inplace(s_off, E, warp_sums);
+    if (tid == 0) s_off[E] = total;
+    for (int i = tid; i < FUSED_WARPS * E; i += FUSED_THREADS) s_run[i] = s_wb[i] + s_excl[i % E];
+    __syncthreads();
+    int32_t* sorted_ids = a.sorted_ids;
+    walk_warp(a.topk, a.P, E, wp0, sub, s_run + warp * E,
+              [&](int64_t p, int e, int32_t g) { sorted_ids[s_off[e] + g] = (int32_t)p; }, &s_bad);
+    const int32_t sentinel = (int32_t)a.P;
+    for (int e = t; e < E; e += G)
+      for (int32_t i = s_off[e] + s_loads[e] + tid; i < s_off[e + 1]; i += FUSED_THREADS) sorted_ids[i] = sentinel;
+    const int64_t gt = (int64_t)t * FUSED_THREADS + tid, gs = (int64_t)G * FUSED_THREADS;
+    for (int64_t i = total + gt; i < a.sorted_cap; i += gs) sorted_ids[i] = sentinel;
+    const int64_t nblocks = total / bm;
+    for (int64_t b = gt; b < a.expert_ids_cap; b += gs) {
+      int32_t owner = -1;
+      if (b < nblocks) {
+        const int32_t v = (int32_t)(b * bm);
+        int lo = 0, hi = E - 1;  // last expert whose group starts at or before v
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (s_off[mid] <= v)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        owner = lo;
+      }
+      a.expert_ids[b] = owner;
+    }
+    if (t == 0 && tid == 0) *a.ntpp = total;
+    __syncthreads();
+  }
+
+  // ---- 4. layout ranks once the plan is out
+  wait_at_least(a.sync + 1, 1u, a.dev_status);
+  const EpPlanLayout& L = a.L;
+  const int n_rep = min(max(__ldcg(a.plan + L.n_rep), 0), cap);
+  for (int e = tid; e < E; e += FUSED_THREADS) {
+    s_hc[e] = __ldcg(a.plan + L.home_count + e);
+    s_hb[e] = __ldcg(a.plan + L.home_base + e);
+    s_cf[e] = __ldcg(a.plan + L.copy_first + e);
+    s_cc[e] = __ldcg(a.plan + L.copy_cnt + e);
+  }
+  for (int m = tid; m < n_rep; m += FUSED_THREADS) {
+    s_rb[m] = __ldcg(a.plan + L.rep_begin + m);
+    s_rc[m] = __ldcg(a.plan + L.rep_count + m);
+    s_rbase[m] = __ldcg(a.plan + L.rep_base + m);
+  }
+  for (int i = tid; i < FUSED_WARPS * E; i += FUSED_THREADS) s_run[i] = s_wb[i] + s_excl[i % E];
+  __syncthreads();
+  int32_t* pos = a.pos;
+  int32_t* src = a.src;
+  int32_t* pair_slot = a.pair_slot;
+  const int64_t P = a.P;
+  walk_warp(a.topk, P, E, wp0, sub, s_run + warp * E,
+            [&](int64_t p, int e, int32_t g) {
+              int32_t row = -1, slot = -1;
+              if (g < s_hc[e]) {
+                row = s_hb[e] + g;
+                slot = e;
+              } else if (s_cc[e] > 0) {
+                int lo = s_cf[e], hi = s_cf[e] + s_cc[e] - 1;  // last replica with rep_begin <= g
+                if (lo >= 0 && hi < n_rep) {
+                  while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_rb[mid] <= g)
+                      lo = mid;
+                    else
+                      hi = mid - 1;
+                  }
+                  const int32_t off = g - s_rb[lo];
+                  if (off >= 0 && off < s_rc[lo]) {
+                    row = s_rbase[lo] + off;
+                    slot = E + lo;
+                  }
+                }
+              }
+              if (row < 0 || row >= P) {
+                s_badrow = 1;
+                pos[p] = -1;
+                if (pair_slot) pair_slot[p] = -1;
+                return;
+              }
+              pos[p] = row;
+              src[row] = (int32_t)p;
+              if (pair_slot) pair_slot[p] = slot;
+            },
+            &s_bad);
+  // pairs with an invalid id: pos = -1 (their rank walk skipped them)
+  __syncthreads();
+  if (s_bad) {
+    for (int64_t p = wp0 + lane, c = 0; c < sub; c += 32, p += 32) {
+      if (p >= P) break;
+      const int e = __ldg(a.topk + p);
+      if (e < 0 || e >= E) {
+        pos[p] = -1;
+        if (pair_slot) pair_slot[p] = -1;
+      }
+    }
+  }
+  if (tid == 0) {
+    if (s_bad) flag(a.dev_status, EP_DEV_BAD_EXPERT_ID);
+    if (s_badrow) flag(a.dev_status, EP_DEV_BAD_ROW);
+  }
+}
+
+size_t fused_smem_bytes(int E, int R) {
+  const int cap = E + R - 1;
+  const size_t words = (size_t)FUSED_WARPS * E + std::max(FUSED_WARPS * E, plan_work_words(E, R)) + 3 * (size_t)E +
+                       1 + 4 * (size_t)E + 3 * (size_t)cap;
+  return words * sizeof(int32_t);
+}
+
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
+                              double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
+                              int32_t* pair_slot, int block_m, int32_t* sorted_token_ids, int64_t sorted_cap,
+                              int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad, void* ws,
+                              size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
+  if (!valid_tke(T, K, E) || R < 1 || R > EP_MAX_RANKS || E % R || S < 0 || (int64_t)R * S != T) return EP_ERR_ARG;
+  if (!loads || !max_vio || !plan || !ws) return EP_ERR_ARG;
+  const int64_t P = T * K;
+  if (P > 0 && (!topk_ids || !pos || !src)) return EP_ERR_ARG;
+  const bool align = sorted_token_ids != nullptr;
+  if (align) {
+    if (!expert_ids || !num_tokens_post_pad || block_m < 1 || block_m > (1 << 16)) return EP_ERR_ARG;
+    const int64_t need = P + (int64_t)E * (block_m - 1);
+    if (need >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+    if (sorted_cap < need || expert_ids_cap < (sorted_cap + block_m - 1) / block_m) return EP_ERR_CAPACITY;
+  }
+  EpPlanLayout L;
+  plan_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  const WsLayout wl = ws_layout(P, E);
+  if (ws_bytes < wl.bytes) return EP_ERR_CAPACITY;
+
+  // grid: at most two resident CTAs per SM, tiles a multiple of 512 pairs
+  const size_t smem = fused_smem_bytes(E, R);
+  int occ = 0;
+  if (P > 0 && smem <= 227 * 1024) {
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_route_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return EP_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_route_fused, FUSED_THREADS, smem) != cudaSuccess)
+      occ = 0;
+  }
+  const int64_t resident = (int64_t)num_sms() * std::min(occ, 2);
+  int64_t tile = 0, ntiles = 0;
+  if (resident > 0) {
+    tile = (P + resident - 1) / resident;
+    tile = std::max<int64_t>(512, (tile + 511) / 512 * 512);
+    ntiles = (P + tile - 1) / tile;
+  }
+  // the [E][tiles] counts must fit where the separate path keeps its look-back words
+  const bool fits = resident > 0 && ntiles <= resident && tile <= (1 << 20) &&
+                    256 + (size_t)E * ntiles * 4 <= wl.excl_off;
+  if (!fits)
+    return fused_route_separate(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot,
+                                block_m, sorted_token_ids, sorted_cap, expert_ids, expert_ids_cap,
+                                num_tokens_post_pad, ws, ws_bytes, dev_status, stream);
+  char* w = static_cast<char*>(ws);
+  if (cudaMemsetAsync(w, 0, 256, stream) != cudaSuccess) return EP_ERR_CUDA;
+  FusedArgs args;
+  args.topk = topk_ids;
+  args.P = P;
+  args.E = E;
+  args.R = R;
+  args.SK = (int32_t)(S * K);
+  args.tile = (int)tile;
+  args.ntiles = (int)ntiles;
+  args.sync = reinterpret_cast<uint32_t*>(w);
+  args.counts = reinterpret_cast<int32_t*>(w + 256);
+  args.loads = loads;
+  args.max_vio = max_vio;
+  args.plan = plan;
+  args.L = L;
+  args.pos = pos;
+  args.src = src;
+  args.pair_slot = pair_slot;
+  args.block_m = block_m;
+  args.sorted_ids = align ? sorted_token_ids : nullptr;
+  args.sorted_cap = sorted_cap;
+  args.expert_ids = expert_ids;
+  args.expert_ids_cap = expert_ids_cap;
+  args.ntpp = num_tokens_post_pad;
+  args.dev_status = dev_status;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ntiles);
+  cfg.blockDim = dim3(FUSED_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_route_fused, args) != cudaSuccess) return EP_ERR_CUDA;
+  count_launch();
+  return launch_status();
+}
+
+namespace ep {
+
+// Same outputs through the separate entry points (when the cooperative grid
+// cannot be resident, or P == 0).
+int fused_route_separate(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
+                         double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
+                         int32_t* pair_slot, int block_m, int32_t* sorted_ids, int64_t sorted_cap,
+                         int32_t* expert_ids, int64_t expert_ids_cap, int32_t* ntpp, void* ws, size_t ws_bytes,
+                         int32_t* dev_status, cudaStream_t stream) {
+  int rc = ep_route_stats(topk_ids, T, K, E, loads, max_vio, ws, ws_bytes, dev_status, stream);
+  if (rc == EP_OK) rc = ep_plan(loads, R, S, K, E, plan, plan_words, dev_status, stream);
+  if (rc == EP_OK)
+    rc = ep_layout(topk_ids, T, K, E, R, S, plan, plan_words, ws, ws_bytes, pos, src, pair_slot, dev_status, stream);
+  if (rc == EP_OK && sorted_ids)
+    rc = ep_align_sort(topk_ids, T, K, E, block_m, sorted_ids, sorted_cap, expert_ids, expert_ids_cap, ntpp, ws,
+                       ws_bytes, dev_status, stream);
+  return rc;
+}
+
+}  // namespace ep

@@ -5,8 +5,8 @@ makes all shapes known in advance: [GR] "Online planning, zero copy και
 στατικά σχήματα", twodots.gr MoonEP article) and runs the path as a fixed
 sequence of libep.so calls on one stream, with no host synchronisation:
 
-  ep_route_stats -> ep_plan -> ep_layout -> ep_align_sort -> ep_dispatch
-  -> [expert: outside the path] -> ep_combine -> ep_replica_grad_reduce
+  ep_route_fused (= ep_route_stats -> ep_plan -> ep_layout -> ep_align_sort)
+  -> ep_dispatch -> [expert: outside the path] -> ep_combine -> ep_replica_grad_reduce
 
 `step()` is one pass of that sequence over the resident inputs; `run_host()`
 is the same pass fed from pinned host buffers (copies in, result out).
@@ -15,7 +15,8 @@ Plumbing only: every computation happens in the library's kernels.
 import torch
 
 from . import (align_sort_capacity, ep_align_sort, ep_combine, ep_dispatch, ep_expert_scale, ep_layout,
-               ep_plan, ep_plan_layout, ep_replica_grad_reduce, ep_route_stats, ep_status_read, ep_workspace_size)
+               ep_plan, ep_plan_layout, ep_replica_grad_reduce, ep_route_fused, ep_route_stats, ep_status_read,
+               ep_workspace_size)
 
 
 class EpLayer:
@@ -53,8 +54,14 @@ class EpLayer:
             self.g_home = self.g_rep = None
 
     # --- the path ---------------------------------------------------------
-    def route(self, stream=None):
-        """a1-a4: loads/max_vio, plan, layout, align-sort."""
+    def route(self, stream=None, fused=True):
+        """a1-a4: loads/max_vio, plan, layout, align-sort (one cooperative
+        launch when fused, else the four separate entry points)."""
+        if fused:
+            ep_route_fused(self.topk_ids, self.E, self.R, self.S, self.loads, self.max_vio, self.plan, self.pos,
+                           self.src, self.ws, self.pair_slot, self.block_m, self.sorted_token_ids, self.expert_ids,
+                           self.num_tokens_post_pad, self.dev_status, stream)
+            return
         ep_route_stats(self.topk_ids, self.E, self.loads, self.max_vio, self.ws, self.dev_status, stream)
         ep_plan(self.loads, self.R, self.S, self.K, self.E, self.plan, self.dev_status, stream)
         ep_layout(self.topk_ids, self.E, self.R, self.S, self.plan, self.ws, self.pos, self.src, self.pair_slot,
@@ -76,21 +83,21 @@ class EpLayer:
         if self.grad_n:
             ep_replica_grad_reduce(self.g_home, self.g_rep, self.E, self.R, self.plan, clear, self.dev_status, stream)
 
-    def step(self, stream=None, grads=True):
+    def step(self, stream=None, grads=True, fused=True):
         """One pass of the whole path over the resident inputs."""
-        self.route(stream)
+        self.route(stream, fused)
         self.dispatch(stream)
         self.combine(stream)
         if grads:
             self.grad_reduce(False, stream)
 
-    def run_host(self, topk_h, w_h, x_h, out_h, stream=None, grads=True):
+    def run_host(self, topk_h, w_h, x_h, out_h, stream=None, grads=True, fused=True):
         """The step fed from (pinned) host buffers: host->device copies of the
         routing and hidden rows, the path, and the combined rows back to host."""
         self.topk_ids.copy_(topk_h, non_blocking=True)
         self.w.copy_(w_h, non_blocking=True)
         self.x.copy_(x_h, non_blocking=True)
-        self.step(stream, grads)
+        self.step(stream, grads, fused)
         out_h.copy_(self.out, non_blocking=True)
 
     def status(self, stream=None):
