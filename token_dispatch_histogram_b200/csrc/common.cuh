@@ -107,6 +107,28 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Lanes of the warp holding the same key as this lane (the result of
+// __match_any_sync), built from one ballot per key bit: for every bit, keep the
+// lanes that agree with this lane on it.  Keys must lie in [0, 2^nbits).  A
+// fixed, short run of pipelined ballots, whatever the number of distinct keys
+// in the warp.  All 32 lanes must call it with the same nbits.
+__device__ __forceinline__ uint32_t warp_match(uint32_t key, int nbits) {
+  uint32_t m = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const uint32_t bit = (key >> b) & 1u;
+    const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
+// Bits needed for keys 0..n-1.
+__host__ __device__ __forceinline__ int key_bits(int n) {
+  int b = 1;
+  while ((1 << b) < n) ++b;
+  return b;
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

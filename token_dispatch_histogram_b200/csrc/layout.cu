@@ -8,8 +8,8 @@
 // per-warp counts, and walks its pairs in order: a pair's stable rank is
 //   tile_excl[tile][e] + (pairs of e in earlier warps of the tile)
 //                      + (pairs of e earlier in this warp's sub-tile).
-// The last term comes from __match_any_sync over 32 consecutive pairs plus a
-// per-warp running counter.  No atomics feed any output.
+// The last term comes from a warp match over 32 consecutive pairs (one ballot
+// per key bit, common.cuh) plus a per-warp running counter.  No atomics feed any output.
 //
 // Layout  ([GR] "Online planning, zero copy και στατικά σχήματα", twodots.gr
 // MoonEP article): an expert's home copy takes its first home_count pairs, its
@@ -49,10 +49,11 @@ __device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ to
   __syncthreads();
 
   const int sub = tile / SCAT_WARPS;  // pairs per warp, a multiple of 32
+  const int nbits = key_bits(E + 2);  // keys e + 2: -2 (invalid id), -1 (past the end), experts
   int32_t* my = s_whist + warp * E;
   for (int c = 0; c < sub; c += 32) {
     const int e = s_ids[warp * sub + c + lane];
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const uint32_t peers = warp_match((uint32_t)(e + 2), nbits);
     if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
     __syncwarp();
   }
@@ -71,7 +72,7 @@ __device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ to
   for (int c = 0; c < sub; c += 32) {
     const int i = warp * sub + c + lane;
     const int e = s_ids[i];
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const uint32_t peers = warp_match((uint32_t)(e + 2), nbits);
     int32_t base = 0;
     if (e >= 0) base = my[e];
     __syncwarp();

@@ -11,10 +11,10 @@
 // sequences are merged and every piece between consecutive breakpoints is one
 // replica (expert, receiving rank, count), numbered in merge ("match") order.
 //
-// Parallel form: per-rank walks (<= E/R steps each) strided over threads, four
-// rank-length prefix sums in one block scan, then a merge-path: each breakpoint
-// finds its merged position by binary search in the other list, so all replicas
-// are emitted independently.
+// Parallel form: closed-form chunks from a prefix sum of the loads, rank
+// prefix sums in one block scan, then a merge-path: each breakpoint finds its
+// merged position by binary search in the other list, so all replicas are
+// emitted independently.
 #pragma once
 
 #include "common.cuh"
@@ -103,112 +103,126 @@ __device__ __forceinline__ int32_t block_scan_inplace(int32_t* a, int n, int32_t
 }
 
 // Words of shared scratch plan_block needs.
-__host__ __device__ __forceinline__ int plan_work_words(int E, int R) { return 9 * R + 5 * E + 16; }
+__host__ __device__ __forceinline__ int plan_work_words(int E, int R) { return 7 * E + 7 * R + 24; }
 
 // Writes the whole plan buffer from loads in shared memory.  Every thread of
 // the block must call it.  Returns n_rep (or 0 when the loads are invalid, in
 // which case EP_DEV_BAD_LOADS is reported and an empty plan is written).
+//
+// No thread walks a rank serially: with pre[] the prefix sum of T_e in expert
+// order, rank r's load is L_r = pre[(r+1)E_R] - pre[r E_R] and the pairs its
+// home experts with a higher id hold are above(e) = pre[(r+1)E_R] - pre[e+1].
+// Since the excess X_r is cut from the highest id down, expert e gives
+//   take_e = clamp(X_r - above(e), 0, T_e),
+// its chunk starts at X_prefix[r] + min(X_r, above(e)) in the excess sequence,
+// and its home copy begins min(X_r, above(e) + T_e) - X_r + (pre[e] - pre[r E_R])
+// rows after rank r's first row.  Chunk numbers come from one scan of the chunk
+// flags in chunk order (ranks ascending, ids descending within a rank).
 static __device__ int plan_block(const int32_t* s_loads, int R, int32_t SK, int E, int32_t* __restrict__ plan,
-                          const EpPlanLayout& L, int32_t* work, int32_t* dev_status) {
+                                 const EpPlanLayout& L, int32_t* work, int32_t* dev_status) {
   __shared__ int4 warp_sums4[32];
   __shared__ int32_t warp_sums[32];
   __shared__ int s_bad;
   const int ER = E / R;
   const int tid = threadIdx.x, nt = blockDim.x;
-  int32_t* r_L = work;                  // [R]
-  int32_t* r_X = r_L + R;               // [R + 1] excess, then its exclusive prefix
-  int32_t* r_D = r_X + R + 1;           // [R + 1] deficit, then prefix
-  int32_t* r_nch = r_D + R + 1;         // [R + 1] chunk count, then prefix
-  int32_t* r_def = r_nch + R + 1;       // [R + 1] is-underloaded, then prefix
-  int32_t* ch_e = r_def + R + 1;        // [E]
-  int32_t* ch_start = ch_e + E;         // [E + 1]
-  int32_t* ch_first = ch_start + E + 1; // [E + 1]
-  int32_t* chunk_of = ch_first + E + 1; // [E]
-  int32_t* home = chunk_of + E;         // [E]
-  int32_t* df_rank = home + E;          // [R]
-  int32_t* df_start = df_rank + R;      // [R + 1]
-  int32_t* df_first = df_start + R + 1; // [R + 1]
-  int32_t* df_coinc = df_first + R + 1; // [R + 1]
+  int32_t* pre = work;                   // [E + 1] exclusive prefix of T_e, expert order
+  int32_t* qf = pre + E + 1;             // [E + 1] chunk flags in chunk order, then their prefix
+  int32_t* ch_e = qf + E + 1;            // [E] expert of chunk c
+  int32_t* ch_start = ch_e + E;          // [E + 1] chunk start in the excess sequence
+  int32_t* ch_first = ch_start + E + 1;  // [E + 1] first match index of chunk c
+  int32_t* home = ch_first + E + 1;      // [E] home_count
+  int32_t* chunk_of = home + E;          // [E] chunk of expert e or -1
+  int32_t* r_X = chunk_of + E;           // [R + 1] exclusive prefix of the excess X_r
+  int32_t* r_D = r_X + R + 1;            // [R + 1] exclusive prefix of the deficit D_r
+  int32_t* r_di = r_D + R + 1;           // [R + 1] exclusive count of underloaded ranks
+  int32_t* df_rank = r_di + R + 1;       // [R] rank of deficit d
+  int32_t* df_start = df_rank + R;       // [R + 1] deficit start
+  int32_t* df_first = df_start + R + 1;  // [R + 1] first match index of deficit d
+  int32_t* df_coinc = df_first + R + 1;  // [R + 1] exclusive count of deficit starts that are chunk starts
 
+  // 1. prefix of the loads
   if (tid == 0) s_bad = 0;
   __syncthreads();
   for (int e = tid; e < E; e += nt) {
-    chunk_of[e] = -1;
-    if (s_loads[e] < 0) s_bad = 1;
+    const int32_t v = s_loads[e];
+    pre[e] = v;
+    if (v < 0) s_bad = 1;
   }
-  // per-rank quantities, then their prefix sums in one pass (segments per thread)
+  __syncthreads();
+  const int32_t total = block_scan_inplace(pre, E, warp_sums);
+  if (tid == 0) {
+    pre[E] = total;
+    if (total != R * SK) s_bad = 1;
+  }
+  __syncthreads();
+  const bool bad = s_bad != 0;
+
+  // 2. per-rank excess, deficit, underloaded flag, and their prefixes (one scan)
   const int per = (R + nt - 1) / nt;
   const int rb = min(R, tid * per), re = min(R, rb + per);
   int4 seg = make_int4(0, 0, 0, 0);
   for (int r = rb; r < re; ++r) {
-    int32_t Lr = 0;
-    for (int e = r * ER; e < (r + 1) * ER; ++e) Lr += s_loads[e];
+    const int32_t Lr = bad ? SK : pre[(r + 1) * ER] - pre[r * ER];
     const int32_t X = Lr > SK ? Lr - SK : 0, D = Lr < SK ? SK - Lr : 0;
-    int32_t rem = X, nch = 0;
-    for (int e = (r + 1) * ER - 1; e >= r * ER && rem > 0; --e) {
-      const int32_t take = min(s_loads[e], rem);
-      if (take > 0) {
-        ++nch;
-        rem -= take;
-      }
-    }
-    r_L[r] = Lr;
     r_X[r] = X;
     r_D[r] = D;
-    r_nch[r] = nch;
-    r_def[r] = D > 0;
+    r_di[r] = D > 0;
     seg.x += X;
     seg.y += D;
-    seg.z += nch;
-    seg.w += D > 0;
+    seg.z += D > 0;
   }
   int4 tot;
   int4 run = block_exclusive_scan4(seg, warp_sums4, &tot);
   for (int r = rb; r < re; ++r) {
-    const int4 v = make_int4(r_X[r], r_D[r], r_nch[r], r_def[r]);
+    const int3 v = make_int3(r_X[r], r_D[r], r_di[r]);
     r_X[r] = run.x;
     r_D[r] = run.y;
-    r_nch[r] = run.z;
-    r_def[r] = run.w;
+    r_di[r] = run.z;
     run.x += v.x;
     run.y += v.y;
     run.z += v.z;
-    run.w += v.w;
   }
   if (tid == 0) {
     r_X[R] = tot.x;
     r_D[R] = tot.y;
-    r_nch[R] = tot.z;
-    r_def[R] = tot.w;
-    if (tot.x != tot.y) s_bad = 1;  // sum_r (L_r - S*K) != 0: loads do not add up to R*S*K
+    r_di[R] = tot.z;
   }
   __syncthreads();
-  const bool bad = s_bad != 0;
-  const int nC = bad ? 0 : r_nch[R], nD = bad ? 0 : r_def[R];
+  const int nD = r_di[R];
   const int32_t Xtot = r_X[R];
 
-  // chunks (descending id per overloaded rank), home counts, deficits
-  for (int r = tid; r < R; r += nt) {
-    for (int e = r * ER; e < (r + 1) * ER; ++e) home[e] = bad ? 0 : s_loads[e];
-    if (bad) continue;
-    const int32_t Lr = r_L[r];
-    int32_t rem = Lr > SK ? Lr - SK : 0, start = r_X[r];
-    int c = r_nch[r];
-    for (int e = (r + 1) * ER - 1; e >= r * ER && rem > 0; --e) {
-      const int32_t take = min(s_loads[e], rem);
-      if (take > 0) {
-        ch_e[c] = e;
-        ch_start[c] = start;
-        chunk_of[e] = c;
-        home[e] = s_loads[e] - take;
-        start += take;
-        rem -= take;
-        ++c;
-      }
+  // 3. what each expert gives up, and the chunk flags in chunk order
+  for (int e = tid; e < E; e += nt) {
+    const int r = e / ER, i = e - r * ER;
+    const int32_t T_e = bad ? 0 : s_loads[e];
+    const int32_t Lr = bad ? SK : pre[(r + 1) * ER] - pre[r * ER];
+    const int32_t X = Lr > SK ? Lr - SK : 0;
+    const int32_t above = pre[(r + 1) * ER] - pre[e + 1];
+    const int32_t take = bad ? 0 : min(max(X - above, 0), T_e);
+    home[e] = T_e - take;
+    chunk_of[e] = -1;
+    qf[r * ER + (ER - 1 - i)] = take > 0;
+  }
+  __syncthreads();
+  const int nC = block_scan_inplace(qf, E, warp_sums);
+  for (int e = tid; e < E; e += nt) {
+    const int r = e / ER, i = e - r * ER;
+    const int32_t T_e = bad ? 0 : s_loads[e];
+    const int32_t Lr = bad ? SK : pre[(r + 1) * ER] - pre[r * ER];
+    const int32_t X = Lr > SK ? Lr - SK : 0;
+    const int32_t above = pre[(r + 1) * ER] - pre[e + 1];
+    if (!bad && min(max(X - above, 0), T_e) > 0) {
+      const int c = qf[r * ER + (ER - 1 - i)];
+      ch_e[c] = e;
+      ch_start[c] = r_X[r] + min(X, above);
+      chunk_of[e] = c;
     }
+  }
+  for (int r = tid; r < R; r += nt) {
+    const int32_t Lr = bad ? SK : pre[(r + 1) * ER] - pre[r * ER];
     if (Lr < SK) {
-      df_rank[r_def[r]] = r;
-      df_start[r_def[r]] = r_D[r];
+      df_rank[r_di[r]] = r;
+      df_start[r_di[r]] = r_D[r];
     }
   }
   if (tid == 0) {
@@ -217,7 +231,8 @@ static __device__ int plan_block(const int32_t* s_loads, int R, int32_t SK, int 
     if (bad) flag(dev_status, EP_DEV_BAD_LOADS);
   }
   __syncthreads();
-  // deficit starts that coincide with a chunk start share one breakpoint
+
+  // 4. deficit starts that coincide with a chunk start share one breakpoint
   for (int d = tid; d < nD; d += nt) {
     const int32_t v = df_start[d];
     const int i = lower_bound_i32(ch_start, nC, v);
@@ -229,6 +244,7 @@ static __device__ int plan_block(const int32_t* s_loads, int R, int32_t SK, int 
   __syncthreads();
   const int n_rep = nC + nD - ncoinc;
 
+  // 5. merge-path: one replica per breakpoint, with its slot in buffer order
   int32_t* rep_expert = plan + L.rep_expert;
   int32_t* rep_rank = plan + L.rep_rank;
   int32_t* rep_count = plan + L.rep_count;
@@ -238,11 +254,15 @@ static __device__ int plan_block(const int32_t* s_loads, int R, int32_t SK, int 
     const int32_t end = min(ch_start[c + 1], df_start[d + 1]);
     const int e = ch_e[c];
     const int rr = df_rank[d];
+    const int32_t Lrr = pre[(rr + 1) * ER] - pre[rr * ER];
+    const int32_t base = rr * SK + Lrr + (v - df_start[d]);  // the receiver is underloaded: its home rows = L_r
     rep_expert[m] = e;
     rep_rank[m] = rr;
     rep_count[m] = end - v;
     rep_begin[m] = home[e] + (v - ch_start[c]);
-    rep_base[m] = rr * SK + r_L[rr] + (v - df_start[d]);  // the receiver is underloaded: its home rows = L_r
+    rep_base[m] = base;
+    plan[L.slot_order + (rr + 1) * ER + m] = E + m;  // after the receiver's home slots and earlier replicas
+    plan[L.cu_seqlens + (rr + 1) * ER + m] = base;
   };
   for (int c = tid; c < nC; c += nt) {
     const int32_t v = ch_start[c];
@@ -267,35 +287,32 @@ static __device__ int plan_block(const int32_t* s_loads, int R, int32_t SK, int 
   }
   __syncthreads();
 
+  // 6. per-expert and per-rank tables, home slots, tails
   for (int e = tid; e < E; e += nt) {
+    const int r = e / ER;
     const int c = chunk_of[e];
     plan[L.home_count + e] = home[e];
     plan[L.copy_first + e] = c >= 0 ? ch_first[c] : 0;
     plan[L.copy_cnt + e] = c >= 0 ? ch_first[c + 1] - ch_first[c] : 0;
     plan[L.rep_experts + e] = e < nC ? ch_e[e] : -1;
+    int32_t hb = r * SK;
+    if (!bad) {
+      const int32_t Lr = pre[(r + 1) * ER] - pre[r * ER];
+      const int32_t X = Lr > SK ? Lr - SK : 0;
+      const int32_t from_e = pre[(r + 1) * ER] - pre[e];  // pairs of ids >= e on rank r
+      hb += (pre[e] - pre[r * ER]) - (X - min(X, from_e));
+    }
+    const int slot = e + df_first[r_di[r]];  // home slots of rank r follow the replicas of ranks < r
+    plan[L.home_base + e] = hb;
+    plan[L.slot_order + slot] = e;
+    plan[L.cu_seqlens + slot] = hb;
   }
   for (int r = tid; r < R; r += nt) {
-    const int32_t Lr = bad ? 0 : r_L[r];
-    const int di = bad ? 0 : r_def[r];
-    const int32_t first = bad ? 0 : df_first[di];
-    const int32_t nrecv = (bad || Lr >= SK) ? 0 : df_first[di + 1] - df_first[di];
+    const int32_t Lr = bad ? 0 : pre[(r + 1) * ER] - pre[r * ER];
+    const int di = r_di[r];
     plan[L.rank_load + r] = Lr;
-    plan[L.rank_rep_first + r] = first;
-    plan[L.rank_nrep + r] = nrecv;
-    int32_t row = r * SK;
-    const int sbase = r * ER + first;
-    for (int i = 0; i < ER; ++i) {
-      const int e = r * ER + i;
-      plan[L.home_base + e] = row;
-      plan[L.slot_order + sbase + i] = e;
-      plan[L.cu_seqlens + sbase + i] = row;
-      row += home[e];
-    }
-    for (int j = 0; j < nrecv; ++j) {
-      const int m = first + j;
-      plan[L.slot_order + sbase + ER + j] = E + m;
-      plan[L.cu_seqlens + sbase + ER + j] = rep_base[m];
-    }
+    plan[L.rank_rep_first + r] = df_first[di];
+    plan[L.rank_nrep + r] = (!bad && Lr < SK) ? df_first[di + 1] - df_first[di] : 0;
   }
   for (int i = E + n_rep + tid; i <= E + L.cap; i += nt) {
     plan[L.cu_seqlens + i] = R * SK;

@@ -12,9 +12,10 @@
 //   2. the per-expert columns are scanned in parallel (one CTA per expert
 //      column): exclusive tile prefixes, and the column totals are T_e;
 //   -- grid barrier --
-//   3. CTA 0 runs the planner (plan_block.cuh) and max_vio and raises a flag;
-//      meanwhile every CTA walks its tile once for the align-sort ranks (which
-//      need only T_e), writing sorted ids, padding and block experts;
+//   3. one extra CTA with no tile runs the planner (plan_block.cuh) and
+//      max_vio and raises a flag; meanwhile every tile CTA walks its tile once
+//      for the align-sort ranks (which need only T_e), writing sorted ids,
+//      padding and block experts;
 //   4. after the flag, every CTA walks its tile again for the layout ranks and
 //      writes pos / src / pair_slot from the plan.
 // A pair's stable rank within its expert = (its tile's prefix) + (earlier warps
@@ -94,36 +95,53 @@ __device__ void grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_status
   wait_at_least(ctr, target, dev_status);
 }
 
+constexpr int WALK_UNROLL = 8;  // tile loads each lane keeps in flight during a walk
+
 // Walk this warp's part of the tile in flattened order; `run` is the warp's
-// running per-expert count (initialised to the rank of its first pair).
+// running per-expert count (initialised to the rank of its first pair).  Ids
+// are loaded WALK_UNROLL chunks at a time so the loads overlap.
 template <class Emit>
 __device__ __forceinline__ void walk_warp(const int32_t* __restrict__ topk, int64_t P, int E, int64_t wp0, int sub,
                                           int32_t* run, Emit emit, int* s_bad) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
-  int64_t p = wp0 + lane;
-  int nxt = (sub > 0 && p < P) ? __ldg(topk + p) : -1;
-  for (int c = 0; c < sub; c += 32, p += 32) {
-    int e = nxt;
-    if (c + 32 < sub && p + 32 < P) nxt = __ldg(topk + p + 32);
-    if (p >= P) e = -1;
-    else if (e < 0 || e >= E) e = -2;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    int32_t base = 0;
-    if (e >= 0) base = run[e];
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) run[e] = base + __popc(peers);
-    __syncwarp();
-    if (e >= 0)
-      emit(p, e, base + __popc(peers & lt));
-    else if (e == -2)
-      *s_bad = 1;
+  const int nbits = key_bits(E + 2);
+  for (int c0 = 0; c0 < sub; c0 += 32 * WALK_UNROLL) {
+    int ids[WALK_UNROLL];
+#pragma unroll
+    for (int u = 0; u < WALK_UNROLL; ++u) {
+      const int64_t p = wp0 + c0 + u * 32 + lane;
+      ids[u] = (c0 + u * 32 < sub && p < P) ? __ldg(topk + p) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < WALK_UNROLL; ++u) {
+      if (c0 + u * 32 >= sub) break;  // warp-uniform
+      const int64_t p = wp0 + c0 + u * 32 + lane;
+      int e = ids[u];
+      if (p >= P)
+        e = -1;
+      else if (e < 0 || e >= E)
+        e = -2;
+      const uint32_t peers = warp_match((uint32_t)(e + 2), nbits);
+      int32_t base = 0;
+      if (e >= 0) base = run[e];
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) run[e] = base + __popc(peers);
+      __syncwarp();
+      if (e >= 0)
+        emit(p, e, base + __popc(peers & lt));
+      else if (e == -2)
+        *s_bad = 1;
+    }
   }
 }
 
 __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   extern __shared__ int32_t sm[];
-  const int E = a.E, tile = a.tile, G = gridDim.x, t = blockIdx.x, tid = threadIdx.x;
+  // CTAs 0..NT-1 own one tile each; the last CTA (NT) owns none and runs the
+  // planner, so the plan overlaps the align-sort walks of the others.
+  const int E = a.E, tile = a.tile, G = gridDim.x, NT = a.ntiles, t = blockIdx.x, tid = threadIdx.x;
+  const bool has_tile = t < NT, planner = t == NT;
   const int warp = tid >> 5, lane = tid & 31;
   const int sub = tile / FUSED_WARPS;
   const int cap = a.L.cap;
@@ -153,34 +171,43 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   }
   for (int i = tid; i < FUSED_WARPS * E; i += FUSED_THREADS) s_wb[i] = 0;
   __syncthreads();
-  {
+  if (has_tile) {
     int32_t* my = s_wb + warp * E;
-    int64_t p = wp0 + lane;
-    int nxt = p < a.P ? __ldg(a.topk + p) : -1;
-    for (int c = 0; c < sub; c += 32, p += 32) {
-      int e = nxt;
-      if (c + 32 < sub && p + 32 < a.P) nxt = __ldg(a.topk + p + 32);
-      if (p >= a.P || e < 0 || e >= E) e = -1;
-      const uint32_t peers = __match_any_sync(0xffffffffu, e);
-      if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-      __syncwarp();
+    const int nbits1 = key_bits(E + 1);
+    for (int c0 = 0; c0 < sub; c0 += 32 * WALK_UNROLL) {
+      int ids[WALK_UNROLL];
+#pragma unroll
+      for (int u = 0; u < WALK_UNROLL; ++u) {
+        const int64_t p = wp0 + c0 + u * 32 + lane;
+        ids[u] = (c0 + u * 32 < sub && p < a.P) ? __ldg(a.topk + p) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < WALK_UNROLL; ++u) {
+        if (c0 + u * 32 >= sub) break;  // warp-uniform
+        const int e = (ids[u] >= 0 && ids[u] < E) ? ids[u] : -1;
+        const uint32_t peers = warp_match((uint32_t)(e + 1), nbits1);
+        if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+        __syncwarp();
+      }
     }
   }
   __syncthreads();
-  for (int e = tid; e < E; e += FUSED_THREADS) {
-    int32_t run = 0;
-    for (int w = 0; w < FUSED_WARPS; ++w) {
-      const int32_t c = s_wb[w * E + e];
-      s_wb[w * E + e] = run;
-      run += c;
+  if (has_tile) {
+    for (int e = tid; e < E; e += FUSED_THREADS) {
+      int32_t run = 0;
+      for (int w = 0; w < FUSED_WARPS; ++w) {
+        const int32_t c = s_wb[w * E + e];
+        s_wb[w * E + e] = run;
+        run += c;
+      }
+      a.counts[(int64_t)e * NT + t] = run;
     }
-    a.counts[(int64_t)e * G + t] = run;
   }
   grid_barrier(a.sync, (uint32_t)G, a.dev_status);
 
   // ---- 2. exclusive scan of every expert column over the tiles; totals = T_e
   for (int e = t; e < E; e += G) {
-    const int32_t total = block_scan_inplace(a.counts + (int64_t)e * G, G, warp_sums);
+    const int32_t total = block_scan_inplace(a.counts + (int64_t)e * NT, NT, warp_sums);
     if (tid == 0) a.loads[e] = total;
   }
   grid_barrier(a.sync, 2u * G, a.dev_status);
@@ -188,10 +215,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   // ---- 3. planner on CTA 0; align-sort ranks everywhere
   for (int e = tid; e < E; e += FUSED_THREADS) {
     s_loads[e] = __ldcg(a.loads + e);
-    s_excl[e] = __ldcg(a.counts + (int64_t)e * G + t);
+    s_excl[e] = has_tile ? __ldcg(a.counts + (int64_t)e * NT + t) : 0;
   }
   __syncthreads();
-  if (t == 0) {
+  if (planner) {
     int32_t m = 0;
     for (int e = tid; e < E; e += FUSED_THREADS) m = max(m, s_loads[e]);
 #pragma unroll
@@ -210,7 +237,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
       st_release_u32(a.sync + 1, 1u);
     }
   }
-  if (a.sorted_ids) {
+  if (a.sorted_ids && has_tile) {
     const int bm = a.block_m;
     for (int e = tid; e < E; e += FUSED_THREADS) s_off[e] = (s_loads[e] + bm - 1) / bm * bm;
     __syncthreads();
@@ -222,9 +249,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
     walk_warp(a.topk, a.P, E, wp0, sub, s_run + warp * E,
               [&](int64_t p, int e, int32_t g) { sorted_ids[s_off[e] + g] = (int32_t)p; }, &s_bad);
     const int32_t sentinel = (int32_t)a.P;
-    for (int e = t; e < E; e += G)
+    for (int e = t; e < E; e += NT)
       for (int32_t i = s_off[e] + s_loads[e] + tid; i < s_off[e + 1]; i += FUSED_THREADS) sorted_ids[i] = sentinel;
-    const int64_t gt = (int64_t)t * FUSED_THREADS + tid, gs = (int64_t)G * FUSED_THREADS;
+    const int64_t gt = (int64_t)t * FUSED_THREADS + tid, gs = (int64_t)NT * FUSED_THREADS;
     for (int64_t i = total + gt; i < a.sorted_cap; i += gs) sorted_ids[i] = sentinel;
     const int64_t nblocks = total / bm;
     for (int64_t b = gt; b < a.expert_ids_cap; b += gs) {
@@ -243,11 +270,12 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
       }
       a.expert_ids[b] = owner;
     }
-    if (t == 0 && tid == 0) *a.ntpp = total;
+    if (t == 0 && tid == 0) *a.ntpp = total;  // tile 0 always exists when P > 0
     __syncthreads();
   }
 
   // ---- 4. layout ranks once the plan is out
+  if (!has_tile) return;
   wait_at_least(a.sync + 1, 1u, a.dev_status);
   const EpPlanLayout& L = a.L;
   const int n_rep = min(max(__ldcg(a.plan + L.n_rep), 0), cap);
@@ -365,13 +393,13 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   }
   const int64_t resident = (int64_t)num_sms() * std::min(occ, 2);
   int64_t tile = 0, ntiles = 0;
-  if (resident > 0) {
-    tile = (P + resident - 1) / resident;
+  if (resident > 1) {  // one CTA per tile plus the planner CTA
+    tile = (P + resident - 2) / (resident - 1);
     tile = std::max<int64_t>(512, (tile + 511) / 512 * 512);
     ntiles = (P + tile - 1) / tile;
   }
   // the [E][tiles] counts must fit where the separate path keeps its look-back words
-  const bool fits = resident > 0 && ntiles <= resident && tile <= (1 << 20) &&
+  const bool fits = resident > 1 && ntiles + 1 <= resident && tile <= (1 << 20) &&
                     256 + (size_t)E * ntiles * 4 <= wl.excl_off;
   if (!fits)
     return fused_route_separate(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot,
@@ -404,7 +432,7 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   args.ntpp = num_tokens_post_pad;
   args.dev_status = dev_status;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ntiles);
+  cfg.gridDim = dim3((unsigned)ntiles + 1);
   cfg.blockDim = dim3(FUSED_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;

@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(32)
       bulk_load(smem + (size_t)s * stride_b, x + t * (int64_t)row_bytes, row_bytes, &bars[s]);
     }
   };
-  const int64_t pro = std::min<int64_t>(stages, njobs);
+  const int64_t pro = njobs < stages ? njobs : (int64_t)stages;
   for (int64_t j = 0; j < pro; ++j) issue(j);
   int64_t issued = pro;
 
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(256)
                    const int32_t* __restrict__ topk, int64_t P, const float* __restrict__ scale, int E,
                    uint16_t* __restrict__ y, int32_t* dev_status) {
   const int64_t nvec = H / 8;
-  const int tpr = (int)std::min<int64_t>(256, (nvec + 31) / 32 * 32);  // threads per row
+  const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);  // threads per row
   const int rows_per_cta = 256 / tpr;
   const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
   int32_t bad = 0;
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(256)
   constexpr int KMAX = KT > 0 ? KT : 32;
   const int K = KT > 0 ? KT : Kd;
   const int64_t nvec = H / 8;
-  const int tpr = (int)std::min<int64_t>(256, (nvec + 31) / 32 * 32);  // threads per token
+  const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);  // threads per token
   const int toks_per_cta = 256 / tpr;
   const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
   int32_t bad = 0;

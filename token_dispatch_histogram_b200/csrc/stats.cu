@@ -9,7 +9,7 @@
 //  - each CTA takes a tile of consecutive flattened pairs (tile index from an
 //    atomic ticket, so a CTA only ever waits on tiles that started earlier),
 //  - builds the tile's histogram in shared memory, one shared-memory add per
-//    distinct expert per warp (__match_any_sync aggregation),
+//    distinct expert per warp (warp_match aggregation: one ballot per key bit),
 //  - publishes it and resolves its exclusive prefix over earlier tiles with a
 //    decoupled look-back (Merrill & Garland, "Single-pass Parallel Prefix Scan
 //    with Decoupled Look-back", 2016), one 64-bit {flag, value} word per
@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(HIST_THREADS)
   const int64_t p0 = (int64_t)t * tile;
   const int64_t p1 = min(P, p0 + tile);
 
+  const int nbits = key_bits(E + 1);
   for (int64_t base = p0; base < p1; base += blockDim.x) {
     const int64_t p = base + threadIdx.x;
     int e = -1;
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(HIST_THREADS)
         s_bad = 1;
       }
     }
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const uint32_t peers = warp_match((uint32_t)(e + 1), nbits);
     if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[e], __popc(peers));
   }
   __syncthreads();
