@@ -119,6 +119,8 @@ ROW_CASES = [
     (2, 50, 1, 4, 64, "skew"),         # K = 1
     (3, 33, 5, 9, 24, "single"),       # generic-K combine path, narrow rows
     (16, 64, 8, 256, 4096, "uniform"),
+    (2, 40, 12, 16, 64, "skew"),       # K > 8: the generic combine kernel
+    (8, 512, 8, 64, 7168, "single"),   # K = 8, wide rows, a dominant expert
 ]
 
 

@@ -11,12 +11,14 @@
 // (cp.async.bulk global->shared, completion on an mbarrier); once it lands,
 // lanes 0..K-1 each issue one bulk store (shared->global) of that row to one
 // destination.  Loads for the next stages are in flight while the stores
-// drain, so a handful of instructions per row keeps ~200 KB per SM moving.
+// drain; the launch sizes stages x CTAs so about 32 KB of loads are in flight
+// per SM, which measured fastest.
 //
 // Combine: out[t] = bf16_rn(sum_k w[t,k] * float(y[pos[t*K+k]])), fp32 in k
 // order, separate multiply and add roundings (no FMA).  One thread owns 8
 // consecutive bf16 of one output row (one 16-byte vector); it issues all K
-// 16-byte row loads before using any, so K loads are in flight per thread.
+// 16-byte row loads before using any, so K loads are in flight per thread,
+// with the token's row indices and weights already staged in shared memory.
 #include <algorithm>
 
 #include "common.cuh"
@@ -138,57 +140,113 @@ __global__ void __launch_bounds__(256)
   if (bad) flag(dev_status, bad);
 }
 
-template <int KT>
-__global__ void __launch_bounds__(256)
+// Combine with the indices and gate weights of a CTA's tokens staged in shared
+// memory one iteration ahead (double buffer), so each thread's K 16-byte row
+// loads issue back to back without waiting on index loads, and registers stay
+// within 64 (four 256-thread CTAs per SM).
+template <int K>
+__global__ void __launch_bounds__(256, 4)
     k_combine(const uint16_t* __restrict__ y, int64_t y_rows, const float* __restrict__ w,
-              const int32_t* __restrict__ pos, int64_t T, int Kd, int64_t H, uint16_t* __restrict__ out,
+              const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ out,
               int32_t* dev_status) {
-  constexpr int KMAX = KT > 0 ? KT : 32;
-  const int K = KT > 0 ? KT : Kd;
+  constexpr int MAXT = 8;  // tokens per CTA iteration (rows narrower than 256 vectors)
+  __shared__ int32_t s_rows[2][MAXT][K];
+  __shared__ float s_w[2][MAXT][K];
+  __shared__ int s_bad;
   const int64_t nvec = H / 8;
   const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);  // threads per token
-  const int toks_per_cta = 256 / tpr;
+  const int tpc = 256 / tpr <= MAXT ? 256 / tpr : MAXT;                // tokens per CTA iteration
   const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
-  int32_t bad = 0;
-  if (sub >= toks_per_cta) return;
-  for (int64_t t = (int64_t)blockIdx.x * toks_per_cta + sub; t < T; t += (int64_t)gridDim.x * toks_per_cta) {
-    int32_t rows[KMAX];
-    float wk[KMAX];
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-      if (k < K) {
-        rows[k] = __ldg(pos + t * K + k);
-        wk[k] = __ldg(w + t * K + k);
-        if (rows[k] < 0 || rows[k] >= y_rows) {
-          rows[k] = -1;
-          bad = EP_DEV_BAD_ROW;
+  const int64_t step = (int64_t)gridDim.x * tpc;
+  if (threadIdx.x == 0) s_bad = 0;
+  auto stage = [&](int b, int64_t tb) {
+    if (threadIdx.x < tpc * K) {
+      const int s = threadIdx.x / K, k = threadIdx.x - s * K;
+      const int64_t t = tb + s;
+      int32_t r = -1;
+      float wk = 0.0f;
+      if (t < T) {
+        r = __ldg(pos + t * K + k);
+        wk = __ldg(w + t * K + k);
+        if (r < 0 || r >= y_rows) {
+          r = -1;
+          s_bad = 1;
         }
       }
+      s_rows[b][s][k] = r;
+      s_w[b][s][k] = wk;
     }
-    for (int64_t v = v0; v < nvec; v += tpr) {
-      uint4 in[KMAX];
+  };
+  int64_t tb = (int64_t)blockIdx.x * tpc;
+  stage(0, tb);
+  __syncthreads();
+  for (int b = 0; tb < T; tb += step, b ^= 1) {
+    stage(b ^ 1, tb + step);
+    const int64_t t = tb + sub;
+    if (sub < tpc && t < T) {
+      for (int64_t v = v0; v < nvec; v += tpr) {
+        uint4 in[K];
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k)
-        if (k < K) in[k] = rows[k] >= 0 ? ld_stream_v4(y + (int64_t)rows[k] * H + v * 8) : make_uint4(0, 0, 0, 0);
-      float acc[8];
+        for (int k = 0; k < K; ++k) {
+          const int32_t r = s_rows[b][sub][k];
+          in[k] = r >= 0 ? ld_stream_v4(y + (int64_t)r * H + v * 8) : make_uint4(0, 0, 0, 0);
+        }
+        float acc[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+        for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k) {
-        if (k < K && rows[k] >= 0) {
+        for (int k = 0; k < K; ++k) {
+          if (s_rows[b][sub][k] < 0) continue;  // an invalid row contributes nothing
+          const float wk = s_w[b][sub][k];
           const uint32_t wd[4] = {in[k].x, in[k].y, in[k].z, in[k].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(wk[k], bf16_bits_to_f32(wd[q] & 0xFFFFu)));
-            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(wk[k], bf16_bits_to_f32(wd[q] >> 16)));
+            acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(wk, bf16_bits_to_f32(wd[q] & 0xFFFFu)));
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(wk, bf16_bits_to_f32(wd[q] >> 16)));
           }
         }
-      }
-      uint32_t o[4];
+        uint32_t o[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) o[q] = f32_to_bf16_bits(acc[2 * q]) | (f32_to_bf16_bits(acc[2 * q + 1]) << 16);
-      st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+        for (int q = 0; q < 4; ++q) o[q] = f32_to_bf16_bits(acc[2 * q]) | (f32_to_bf16_bits(acc[2 * q + 1]) << 16);
+        st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+      }
     }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_ROW);
+}
+
+// Any K up to 32, one row at a time (no K-wide register arrays).
+__global__ void __launch_bounds__(256)
+    k_combine_any(const uint16_t* __restrict__ y, int64_t y_rows, const float* __restrict__ w,
+                  const int32_t* __restrict__ pos, int64_t T, int K, int64_t H, uint16_t* __restrict__ out,
+                  int32_t* dev_status) {
+  const int64_t nvec = H / 8;
+  int32_t bad = 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T * nvec; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / nvec, v = i - t * nvec;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      const int32_t r = __ldg(pos + t * K + k);
+      if (r < 0 || r >= y_rows) {
+        bad = EP_DEV_BAD_ROW;
+        continue;
+      }
+      const float wk = __ldg(w + t * K + k);
+      const uint4 in = ld_stream_v4(y + (int64_t)r * H + v * 8);
+      const uint32_t wd[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(wk, bf16_bits_to_f32(wd[q] & 0xFFFFu)));
+        acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(wk, bf16_bits_to_f32(wd[q] >> 16)));
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o[q] = f32_to_bf16_bits(acc[2 * q]) | (f32_to_bf16_bits(acc[2 * q + 1]) << 16);
+    st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
   }
   if (bad) flag(dev_status, bad);
 }
@@ -216,14 +274,20 @@ extern "C" int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const
   if (!x || !pos || !buf || !aligned16(x) || !aligned16(buf)) return EP_ERR_ARG;
   const uint32_t row_bytes = (uint32_t)(H * 2);
   const uint32_t stride_b = (row_bytes + 127u) & ~127u;
-  // stages: as many rows as fit in ~48 KB, 2..8
-  int stages = (int)std::max<uint32_t>(2, std::min<uint32_t>(DISPATCH_MAX_STAGES, (48u * 1024u) / stride_b));
+  // Measured on B200: the scatter runs fastest with about 32 KB of row loads
+  // in flight per SM (e.g. 2 stages x 4 CTAs of 4 KB rows: 6.0 TB/s, against
+  // 5.5 TB/s with 48 KB per CTA and 6 CTAs); more concurrency only adds
+  // read/write contention at the memory.  Small rows use 4 stages so the
+  // per-SM target is reached within 32 CTAs.
+  const uint32_t target = 32u * 1024u;
+  const int stages = stride_b * 2u * 16u <= target ? 4 : 2;
+  const int per_sm = (int)std::min<uint32_t>(32, std::max<uint32_t>(1, (target + stages * stride_b - 1) / (stages * stride_b)));
   size_t smem = (size_t)stages * stride_b + DISPATCH_MAX_STAGES * 8 + (size_t)stages * K * 4;
   if (smem > 200 * 1024) return EP_ERR_ARG;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(k_dispatch, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EP_ERR_CUDA;
-  const int grid = occupancy_grid((const void*)k_dispatch, 32, smem, T, 32);
+  const int grid = occupancy_grid((const void*)k_dispatch, 32, smem, T, per_sm);
   k_dispatch<<<grid, 32, smem, stream>>>(reinterpret_cast<const uint8_t*>(x), T, K, row_bytes, pos, buf_rows,
                                          reinterpret_cast<uint8_t*>(buf), stages, dev_status);
   count_launch();
@@ -248,19 +312,27 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
   if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
   if (T == 0) return EP_OK;
   if (!y || !w || !pos || !out || !aligned16(y) || !aligned16(out)) return EP_ERR_ARG;
-  const void* fn;
+  const void* fn = nullptr;
   switch (K) {
     case 1: fn = (const void*)k_combine<1>; break;
     case 2: fn = (const void*)k_combine<2>; break;
+    case 3: fn = (const void*)k_combine<3>; break;
     case 4: fn = (const void*)k_combine<4>; break;
+    case 5: fn = (const void*)k_combine<5>; break;
     case 6: fn = (const void*)k_combine<6>; break;
+    case 7: fn = (const void*)k_combine<7>; break;
     case 8: fn = (const void*)k_combine<8>; break;
-    default: fn = (const void*)k_combine<0>; break;
+    default: break;
   }
-  const int grid = occupancy_grid(fn, 256, 0, T, 8);
-  void* args[] = {(void*)&y, (void*)&y_rows, (void*)&w, (void*)&pos, (void*)&T, (void*)&K, (void*)&H, (void*)&out,
-                  (void*)&dev_status};
-  if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (fn) {
+    const int grid = occupancy_grid(fn, 256, 0, T, 4);
+    void* args[] = {(void*)&y, (void*)&y_rows, (void*)&w, (void*)&pos, (void*)&T, (void*)&H, (void*)&out,
+                    (void*)&dev_status};
+    if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+  } else {
+    const int grid = occupancy_grid((const void*)k_combine_any, 256, 0, T * (H / 8) / 256 + 1, 8);
+    k_combine_any<<<grid, 256, 0, stream>>>(y, y_rows, w, pos, T, K, H, out, dev_status);
+  }
   count_launch();
   return launch_status();
 }
