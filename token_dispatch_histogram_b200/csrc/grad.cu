@@ -7,10 +7,11 @@
 // micro-batch.  Per element, home first and then the replicas in match order,
 // one fp32 add each:  g_home[e] = ((g_home[e] + g_rep[m1]) + g_rep[m2]) + ...
 //
-// Work = (replicated expert, 8-element vector) items; the replicated experts and
-// each one's replica range come from the plan on the device (no host sync).
-// A persistent grid walks the items in units of 2048 elements; each thread keeps
-// two 32-byte groups of loads in flight per replica step.
+// Work = (replicated expert, 4096-element unit) items; the replicated experts
+// and each one's replica range come from the plan on the device (no host sync),
+// read once per unit into shared memory.  Each thread owns two 8-element
+// vectors of a unit and loads up to four replica vectors before adding them in
+// match order, so several 32-byte loads are in flight per thread.
 #include <algorithm>
 
 #include "common.cuh"
@@ -18,7 +19,20 @@
 namespace ep {
 
 constexpr int GRAD_THREADS = 256;
-constexpr int64_t GRAD_UNIT = GRAD_THREADS * 8;  // elements per work unit
+constexpr int GRAD_VECS = 2;                                   // 8-element vectors per thread per unit
+constexpr int64_t GRAD_UNIT = (int64_t)GRAD_THREADS * 8 * GRAD_VECS;  // elements per work unit
+constexpr int GRAD_BATCH = 4;                                  // replica rows loaded before adding
+
+__device__ __forceinline__ void add_f32x8(float (&a)[8], uint4 lo, uint4 hi) {
+  a[0] = __fadd_rn(a[0], __uint_as_float(lo.x));
+  a[1] = __fadd_rn(a[1], __uint_as_float(lo.y));
+  a[2] = __fadd_rn(a[2], __uint_as_float(lo.z));
+  a[3] = __fadd_rn(a[3], __uint_as_float(lo.w));
+  a[4] = __fadd_rn(a[4], __uint_as_float(hi.x));
+  a[5] = __fadd_rn(a[5], __uint_as_float(hi.y));
+  a[6] = __fadd_rn(a[6], __uint_as_float(hi.z));
+  a[7] = __fadd_rn(a[7], __uint_as_float(hi.w));
+}
 
 __device__ __forceinline__ void add_bf16x8(float (&a)[8], uint4 v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -29,9 +43,59 @@ __device__ __forceinline__ void add_bf16x8(float (&a)[8], uint4 v) {
   }
 }
 
-__global__ void __launch_bounds__(GRAD_THREADS)
-    k_grad_reduce(float* __restrict__ g_home, void* __restrict__ g_rep, int rep_dtype, int64_t n,
-                  const int32_t* __restrict__ plan, EpPlanLayout L, int E, int clear, int32_t* dev_status) {
+// One 8-element vector of one replicated expert: home + replicas m0..m0+mc-1
+// in match order.  Up to GRAD_BATCH replica vectors are loaded before any add,
+// so their loads overlap; the adds still go in match order.
+template <bool BF16, bool CLEAR>
+__device__ __forceinline__ void reduce_vec8(float* __restrict__ home, void* __restrict__ g_rep, int64_t n, int64_t j,
+                                            int m0, int mc) {
+  float a[8];
+  const float4 h0 = *reinterpret_cast<const float4*>(home + j);
+  const float4 h1 = *reinterpret_cast<const float4*>(home + j + 4);
+  a[0] = h0.x; a[1] = h0.y; a[2] = h0.z; a[3] = h0.w;
+  a[4] = h1.x; a[5] = h1.y; a[6] = h1.z; a[7] = h1.w;
+  for (int mb = m0; mb < m0 + mc; mb += GRAD_BATCH) {
+    uint4 r[GRAD_BATCH][BF16 ? 1 : 2];
+#pragma unroll
+    for (int q = 0; q < GRAD_BATCH; ++q) {
+      if (mb + q < m0 + mc) {
+        if (BF16) {
+          r[q][0] = ld_stream_v4(static_cast<const uint16_t*>(g_rep) + (int64_t)(mb + q) * n + j);
+        } else {
+          const float* rp = static_cast<const float*>(g_rep) + (int64_t)(mb + q) * n + j;
+          r[q][0] = ld_stream_v4(rp);
+          r[q][BF16 ? 0 : 1] = ld_stream_v4(rp + 4);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < GRAD_BATCH; ++q) {
+      if (mb + q < m0 + mc) {
+        if (BF16)
+          add_bf16x8(a, r[q][0]);
+        else
+          add_f32x8(a, r[q][0], r[q][BF16 ? 0 : 1]);
+        if (CLEAR) {
+          if (BF16) {
+            st_v4(static_cast<uint16_t*>(g_rep) + (int64_t)(mb + q) * n + j, make_uint4(0, 0, 0, 0));
+          } else {
+            float* rp = static_cast<float*>(g_rep) + (int64_t)(mb + q) * n + j;
+            st_v4(rp, make_uint4(0, 0, 0, 0));
+            st_v4(rp + 4, make_uint4(0, 0, 0, 0));
+          }
+        }
+      }
+    }
+  }
+  *reinterpret_cast<float4*>(home + j) = make_float4(a[0], a[1], a[2], a[3]);
+  *reinterpret_cast<float4*>(home + j + 4) = make_float4(a[4], a[5], a[6], a[7]);
+}
+
+template <bool BF16, bool CLEAR>
+__global__ void __launch_bounds__(GRAD_THREADS, 4)
+    k_grad_reduce(float* __restrict__ g_home, void* __restrict__ g_rep, int64_t n, const int32_t* __restrict__ plan,
+                  EpPlanLayout L, int E, int32_t* dev_status) {
+  __shared__ int s_e, s_m0, s_mc;
   const int nC = min(max(plan[L.n_chunks], 0), E);
   const int64_t units_per_expert = (n + GRAD_UNIT - 1) / GRAD_UNIT;
   const int64_t total = (int64_t)nC * units_per_expert;
@@ -39,61 +103,47 @@ __global__ void __launch_bounds__(GRAD_THREADS)
   for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
     const int c = (int)(u / units_per_expert);
     const int64_t j0 = (u - (int64_t)c * units_per_expert) * GRAD_UNIT;
-    const int e = plan[L.rep_experts + c];
-    if (e < 0 || e >= E) {
-      if (threadIdx.x == 0) flag(dev_status, EP_DEV_BAD_ROW);
-      continue;
+    __syncthreads();  // the previous unit is done with s_e, s_m0, s_mc
+    if (threadIdx.x == 0) {
+      const int e = plan[L.rep_experts + c];
+      int m0 = 0, mc = 0;
+      if (e >= 0 && e < E) {
+        m0 = plan[L.copy_first + e];
+        mc = plan[L.copy_cnt + e];
+      }
+      if (e < 0 || e >= E || m0 < 0 || mc < 0 || m0 + mc > L.cap) {
+        flag(dev_status, EP_DEV_BAD_ROW);
+        s_e = -1;
+      } else {
+        s_e = e;
+        s_m0 = m0;
+        s_mc = mc;
+      }
     }
-    const int m0 = plan[L.copy_first + e], mc = plan[L.copy_cnt + e];
-    if (m0 < 0 || mc < 0 || m0 + mc > L.cap) {
-      if (threadIdx.x == 0) flag(dev_status, EP_DEV_BAD_ROW);
-      continue;
-    }
+    __syncthreads();
+    const int e = s_e;
+    if (e < 0) continue;
+    const int m0 = s_m0, mc = s_mc;
     float* home = g_home + (int64_t)e * n;
     if (vec) {
-      const int64_t j = j0 + (int64_t)threadIdx.x * 8;
-      if (j >= n) continue;
-      float a[8];
-      const float4 h0 = *reinterpret_cast<const float4*>(home + j);
-      const float4 h1 = *reinterpret_cast<const float4*>(home + j + 4);
-      a[0] = h0.x; a[1] = h0.y; a[2] = h0.z; a[3] = h0.w;
-      a[4] = h1.x; a[5] = h1.y; a[6] = h1.z; a[7] = h1.w;
-      for (int m = m0; m < m0 + mc; ++m) {
-        if (rep_dtype == EP_DTYPE_F32) {
-          const float* r = static_cast<const float*>(g_rep) + (int64_t)m * n + j;
-          const uint4 r0 = ld_stream_v4(r), r1 = ld_stream_v4(r + 4);
-          a[0] = __fadd_rn(a[0], __uint_as_float(r0.x));
-          a[1] = __fadd_rn(a[1], __uint_as_float(r0.y));
-          a[2] = __fadd_rn(a[2], __uint_as_float(r0.z));
-          a[3] = __fadd_rn(a[3], __uint_as_float(r0.w));
-          a[4] = __fadd_rn(a[4], __uint_as_float(r1.x));
-          a[5] = __fadd_rn(a[5], __uint_as_float(r1.y));
-          a[6] = __fadd_rn(a[6], __uint_as_float(r1.z));
-          a[7] = __fadd_rn(a[7], __uint_as_float(r1.w));
-          if (clear) {
-            st_v4((void*)r, make_uint4(0, 0, 0, 0));
-            st_v4((void*)(r + 4), make_uint4(0, 0, 0, 0));
-          }
-        } else {
-          const uint16_t* r = static_cast<const uint16_t*>(g_rep) + (int64_t)m * n + j;
-          add_bf16x8(a, ld_stream_v4(r));
-          if (clear) st_v4((void*)r, make_uint4(0, 0, 0, 0));
-        }
+#pragma unroll
+      for (int vv = 0; vv < GRAD_VECS; ++vv) {
+        const int64_t j = j0 + ((int64_t)vv * GRAD_THREADS + threadIdx.x) * 8;
+        if (j >= n) break;
+        reduce_vec8<BF16, CLEAR>(home, g_rep, n, j, m0, mc);
       }
-      *reinterpret_cast<float4*>(home + j) = make_float4(a[0], a[1], a[2], a[3]);
-      *reinterpret_cast<float4*>(home + j + 4) = make_float4(a[4], a[5], a[6], a[7]);
     } else {
       for (int64_t j = j0 + threadIdx.x; j < min(n, j0 + GRAD_UNIT); j += blockDim.x) {
         float a = home[j];
         for (int m = m0; m < m0 + mc; ++m) {
-          if (rep_dtype == EP_DTYPE_F32) {
+          if (!BF16) {
             float* r = static_cast<float*>(g_rep) + (int64_t)m * n + j;
             a = __fadd_rn(a, *r);
-            if (clear) *r = 0.0f;
+            if (CLEAR) *r = 0.0f;
           } else {
             uint16_t* r = static_cast<uint16_t*>(g_rep) + (int64_t)m * n + j;
             a = __fadd_rn(a, bf16_bits_to_f32(*r));
-            if (clear) *r = 0;
+            if (CLEAR) *r = 0;
           }
         }
         home[j] = a;
@@ -120,9 +170,14 @@ extern "C" int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_
   if (n == 0) return EP_OK;
   if (!g_home || !g_rep || !aligned16(g_home) || !aligned16(g_rep)) return EP_ERR_ARG;
   const int64_t units = (int64_t)E * ((n + GRAD_UNIT - 1) / GRAD_UNIT);  // upper bound (n_chunks <= E)
-  const int grid = occupancy_grid((const void*)k_grad_reduce, GRAD_THREADS, 0, units, 8);
-  k_grad_reduce<<<grid, GRAD_THREADS, 0, stream>>>(g_home, const_cast<void*>(g_rep), rep_dtype, n, plan, L, E,
-                                                   clear_replicas, dev_status);
+  // 4 CTAs per SM measured best
+  const void* fn = rep_dtype == EP_DTYPE_F32
+                       ? (clear_replicas ? (const void*)k_grad_reduce<false, true> : (const void*)k_grad_reduce<false, false>)
+                       : (clear_replicas ? (const void*)k_grad_reduce<true, true> : (const void*)k_grad_reduce<true, false>);
+  const int grid = occupancy_grid(fn, GRAD_THREADS, 0, units, 4);
+  void* gr = const_cast<void*>(g_rep);
+  void* args[] = {(void*)&g_home, (void*)&gr, (void*)&n, (void*)&plan, (void*)&L, (void*)&E, (void*)&dev_status};
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(GRAD_THREADS), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }
