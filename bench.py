@@ -12,9 +12,11 @@ Workload (default): the moderate EP8 layer, R=8 simulated ranks x S=4096
 tokens, E=64 experts, top-K=6, H=2048 bf16, block_m=64, replica gradients of
 3*2048*1024 fp32 per expert; router logits N(0,1)+b_e with b_e ~ N(0,0.5^2).
 
-`value`: device-resident inputs, CUDA events around each step on the launching
-stream, L2 flushed (a 512 MB write) between steps outside the events, max over
-ranks.  `e2e`: the same steps through the public API (EpLayer.run_host) from
+`value`: device-resident inputs; the step is captured once as a CUDA graph and
+replayed K times, with CUDA events around each replay on the launching stream,
+L2 flushed (a 512 MB write) between replays outside the events, max over ranks.
+The per-op breakdown and the roofline come from an eager pass of the same K
+steps with CUDA events between the ops.  `e2e`: the same steps through the public API (EpLayer.run_host) from
 pinned host buffers: routing, gate weights and hidden rows copied in, the
 combined rows copied out, inside the timed region.  Under torchrun each rank
 runs its own independent layer (weak scaling, no data-path collective).
@@ -53,6 +55,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the eager per-op pass only (default: the headline value comes from replaying the "
+                         "step as one captured CUDA graph; the per-op breakdown from the eager pass)")
     ap.add_argument("--route", choices=["fused", "separate"], default="fused",
                     help="route phase as one cooperative launch (ep_route_fused) or the four separate calls")
     return ap.parse_args()
@@ -60,12 +65,13 @@ def parse():
 
 def workload_desc(c):
     g = f", replica grads {c['grad_n']} {c['grad_dtype']} per expert" if c["grad_n"] else ""
+    lay = f", {c['layers']} layers per step" if c["layers"] > 1 else ""
     return (f"{c['name']}: R={c['R']} simulated EP ranks x S={c['S']} tokens, E={c['E']} experts, top-K={c['K']}, "
-            f"H={c['H']} bf16, block_m={c['block_m']}, router bias {c['bias']}{g}")
+            f"H={c['H']} bf16, block_m={c['block_m']}, router bias {c['bias']}{g}{lay}")
 
 
 def config_obj(c, l2):
-    return {"workload": workload_desc(c), "R": c["R"], "S": c["S"], "E": c["E"], "K": c["K"], "H": c["H"],
+    return {"workload": workload_desc(c), "layers": c["layers"], "R": c["R"], "S": c["S"], "E": c["E"], "K": c["K"], "H": c["H"],
             "tokens_per_step": c["T"], "pairs_per_step": c["P"], "block_m": c["block_m"], "l2": l2,
             "step": "route(" + "+".join(ROUTE_PARTS) + ")+dispatch+combine+grad_reduce"}
 
@@ -193,7 +199,6 @@ def traffic_record(kernel):
 
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
     import token_dispatch_histogram_b200 as tdh
     import workload as W
 
@@ -202,19 +207,27 @@ def run_ours(args, rank, world, local_rank):
     c = W.shape(args.config)
     seed = rank_seed(args.seed, rank)
     R, S, E, K, H, T, P = c["R"], c["S"], c["E"], c["K"], c["H"], c["T"], c["P"]
+    nl = c["layers"]
     gdt = torch.float32 if c["grad_dtype"] in ("f32", None) else torch.bfloat16
-    layer = tdh.EpLayer(R, S, K, E, H, c["block_m"], device=dev, grad_n=c["grad_n"] or 0, grad_dtype=gdt)
+    layers = []
+    for i in range(nl):  # consecutive layers share the large buffers
+        layers.append(tdh.EpLayer(R, S, K, E, H, c["block_m"], device=dev, grad_n=c["grad_n"] or 0, grad_dtype=gdt,
+                                  share=layers[0] if layers else None))
+    layer = layers[0]
 
-    # inputs: host-generated routing and hidden rows (pinned), device-generated grads
-    topk_np, w_np = W.routing(args.config, seed)
-    x_np = W.hidden(T, H, seed)
-    topk_h = torch.from_numpy(topk_np).pin_memory()
-    w_h = torch.from_numpy(w_np).pin_memory()
-    x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    layer.topk_ids.copy_(topk_h)
-    layer.w.copy_(w_h)
-    layer.x.copy_(x_h)
+    # inputs: host-generated routing (per layer) and hidden rows (pinned when the
+    # end-to-end pass runs), device-generated gradients
+    routes = [W.routing(args.config, seed, i) for i in range(nl)]
+    for ly, (tk, ww) in zip(layers, routes):
+        ly.topk_ids.copy_(torch.from_numpy(tk))
+        ly.w.copy_(torch.from_numpy(ww))
+    host_x = T * H * 2 <= (4 << 30)
+    if host_x:
+        x_np = W.hidden(T, H, seed)
+        layer.x.copy_(torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16))
+    else:
+        x_np = None
+        W.fill_device(layer.x, seed, W.STREAM_X)
     if layer.grad_n:
         W.fill_device(layer.g_home, seed, W.STREAM_GHOME)
         W.fill_device(layer.g_rep, seed, W.STREAM_GREP)
@@ -225,21 +238,52 @@ def run_ours(args, rank, world, local_rank):
 
     def barrier():
         if world > 1:
+            import torch.distributed as dist
             dist.barrier()
 
     fused = args.route == "fused"
-    for _ in range(args.warmup):
-        layer.step(stream, fused=fused)
-    torch.cuda.synchronize()
-    status = layer.status(stream)
-    if status:
-        raise RuntimeError(f"device status {status:#x} after warm-up")
-    n_rep = int(layer.plan_view("n_rep", 1).item())
-    n_chunks = int(layer.plan_view("n_chunks", 1).item())
-    max_vio = float(layer.max_vio.item())
 
-    # ---- device-resident timed region
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(args.steps)]
+    def step(rec=None, st=stream):
+        # st=None: the binding uses torch's current stream (the capture stream
+        # while a CUDA graph is being recorded)
+        for ly in layers:
+            if rec:
+                rec("route")
+            ly.route(st, fused=fused)
+            if rec:
+                rec("dispatch")
+            tdh.ep_dispatch(ly.x, K, ly.pos, ly.buf, ly.dev_status, st)
+            if rec:
+                rec("combine")
+            tdh.ep_combine(ly.buf, ly.w, ly.pos, ly.out, ly.dev_status, st)
+            if ly.grad_n:
+                if rec:
+                    rec("grad_reduce")
+                ly.grad_reduce(False, st)
+        if rec:
+            rec(None)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for ly in layers:
+        st = ly.status(stream)
+        if st:
+            raise RuntimeError(f"device status {st:#x} after warm-up")
+    n_rep = [int(ly.plan_view("n_rep", 1).item()) for ly in layers]
+    n_chunks = [int(ly.plan_view("n_chunks", 1).item()) for ly in layers]
+    max_vio = [float(ly.max_vio.item()) for ly in layers]
+
+    # ---- device-resident timed region: per-op CUDA events on the launching stream
+    marks = []  # per step: list of (op, event)
+
+    def recorder(lst):
+        def rec(op):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            lst.append((op, e))
+        return rec
+
     clocks = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
@@ -247,30 +291,69 @@ def run_ours(args, rank, world, local_rank):
     launches0 = tdh.ep_launch_count()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)  # outside the step's events
-        e = ev[i]
-        e[0].record(stream)
-        layer.route(stream, fused=fused)
-        e[1].record(stream)
-        tdh.ep_dispatch(layer.x, K, layer.pos, layer.buf, layer.dev_status, stream)
-        e[2].record(stream)
-        tdh.ep_combine(layer.buf, layer.w, layer.pos, layer.out, layer.dev_status, stream)
-        e[3].record(stream)
-        layer.grad_reduce(False, stream)
-        e[4].record(stream)
+        lst = []
+        step(recorder(lst))
+        marks.append(lst)
     torch.cuda.synchronize()
     barrier()
     launches = tdh.ep_launch_count() - launches0
     clk = clocks.stop()
-    per_op = {op: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j, op in enumerate(OPS)}
-    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
+    per_op = {op: 0.0 for op in OPS}
+    step_ms = []
+    for lst in marks:
+        for (op, e0), (_, e1) in zip(lst[:-1], lst[1:]):
+            per_op[op] += e0.elapsed_time(e1)
+        step_ms.append(lst[0][1].elapsed_time(lst[-1][1]))
     total_ms = max_over_ranks(sum(step_ms), world, dev)
-    status = layer.status(stream)
-    if status:
-        raise RuntimeError(f"device status {status:#x} in the timed region")
+    for ly in layers:
+        st = ly.status(stream)
+        if st:
+            raise RuntimeError(f"device status {st:#x} in the timed region")
+
+    # ---- the same step replayed as one captured CUDA graph: the headline timing
+    graph = None
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize()
+            c0 = tdh.ep_launch_count()
+            with torch.cuda.graph(g):
+                step(st=None)
+            per_replay = tdh.ep_launch_count() - c0
+            g.replay()
+            torch.cuda.synchronize()
+            gs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+            ge = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+            clocks_g = ClockSampler(local_rank)
+            barrier()
+            torch.cuda.synchronize()
+            clocks_g.start()
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                gs[i].record(stream)
+                g.replay()
+                ge[i].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            clk_g = clocks_g.stop()
+            g_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(gs, ge)), world, dev)
+            graph = {"ms": g_ms, "launches": int(per_replay * args.steps), "clocks": clk_g}
+            del g
+            for ly in layers:
+                st = ly.status(stream)
+                if st:
+                    raise RuntimeError(f"device status {st:#x} in the graph replays")
+        except RuntimeError as exc:  # capture unsupported here: keep the eager timing
+            graph = None
+            print(f"graph capture unavailable: {exc}", file=sys.stderr)
 
     # ---- end to end through the public API, pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and host_x and nl == 1:
+        topk_h = torch.from_numpy(routes[0][0]).pin_memory()
+        w_h = torch.from_numpy(routes[0][1]).pin_memory()
+        x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+        out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
         for _ in range(min(3, args.warmup)):
             layer.run_host(topk_h, w_h, x_h, out_h, stream, fused=fused)
         torch.cuda.synchronize()
@@ -290,43 +373,54 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": job_throughput(world, P, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
 
-    # ---- roofline of the dominant kernel and the per-op breakdown
-    ab = algorithmic_bytes(c, n_rep, n_chunks)
+    # ---- roofline of the dominant kernel and the per-op breakdown (bytes summed over layers)
+    abs_ = [algorithmic_bytes(c, nr, nc) for nr, nc in zip(n_rep, n_chunks)]
+    ab = {op: sum(a[op] for a in abs_) for op in OPS}
     peak, peak_kind = peaks()
-    mean_ms = {op: sum(v) / len(v) for op, v in per_op.items()}
+    calls = args.steps
+    mean_ms = {op: per_op[op] / calls for op in OPS}  # per step (all layers)
     dom = max(("dispatch", "combine", "grad_reduce"), key=lambda op: mean_ms[op])
     kernel_of = {"dispatch": "k_dispatch", "combine": "k_combine", "grad_reduce": "k_grad_reduce"}
-    achieved = ab[dom] / (mean_ms[dom] / 1e3) / 1e9
-    tr = traffic_record(kernel_of[dom])
+    achieved = ab[dom] / (mean_ms[dom] / 1e3) / 1e9 if mean_ms[dom] else 0.0
+    tr = traffic_record(kernel_of[dom]) if args.config == 2 else None
     roofline = {"bound": "hbm", "kernel": kernel_of[dom], "achieved": round(achieved, 1), "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "algorithmic_bytes_per_launch": ab[dom],
+                "algorithmic_bytes_per_launch": ab[dom] // nl,
                 "traffic": (tr["dram_bytes_per_launch"] if tr else None),
                 "traffic_source": (tr["capture"] if tr else None)}
-    breakdown = {op: {"ms": round(mean_ms[op], 5), "GB_s": round(ab[op] / (mean_ms[op] / 1e3) / 1e9, 1)}
+    breakdown = {op: {"ms": round(mean_ms[op], 5),
+                      "GB_s": round(ab[op] / (mean_ms[op] / 1e3) / 1e9, 1) if mean_ms[op] else None}
                  for op in OPS}
     step_bytes = sum(ab.values())
-    value = job_throughput(world, P, args.steps, total_ms)
+    eager = {"value": job_throughput(world, nl * P, args.steps, total_ms), "ms_per_step": total_ms / args.steps,
+             "gpu_launches": int(launches)}
+    timed_ms = graph["ms"] if graph else total_ms
+    value = job_throughput(world, nl * P, args.steps, timed_ms)
     d_c_ms = mean_ms["dispatch"] + mean_ms["combine"]
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": timed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox; see DESIGN.md input recipe)",
         "config": config_obj(c, "flushed between steps (512 MB write, outside the step events)"),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": int(launches),
-        "clocks": clk,
+        "gpu_launches": graph["launches"] if graph else int(launches),
+        "clocks": graph["clocks"] if graph else clk,
+        "timing": ("one captured CUDA graph per step, replayed; CUDA events around each replay"
+                   if graph else "eager launches; CUDA events around each step"),
+        "eager": eager,
         "breakdown": breakdown,
-        "step_hbm": {"bytes": step_bytes, "GB_s": round(step_bytes / (total_ms / args.steps / 1e3) / 1e9, 1),
-                     "frac": round(step_bytes / (total_ms / args.steps / 1e3) / 1e9 / peak, 4)},
+        "step_hbm": {"bytes": step_bytes, "GB_s": round(step_bytes / (timed_ms / args.steps / 1e3) / 1e9, 1),
+                     "frac": round(step_bytes / (timed_ms / args.steps / 1e3) / 1e9 / peak, 4)},
         "dispatch_combine": {"ms": round(d_c_ms, 5),
                              "GB_s": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9, 1),
                              "frac": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9 / peak, 4)},
-        "routing": {"max_vio": max_vio, "n_rep": n_rep, "replicated_experts": n_chunks},
+        "routing": {"max_vio": max_vio if nl > 1 else max_vio[0], "n_rep": n_rep if nl > 1 else n_rep[0],
+                    "replicated_experts": n_chunks if nl > 1 else n_chunks[0]},
+        "layers_per_step": nl,
         "route_path": args.route,
     }
-    return res, (topk_np, w_np, x_np, c, seed)
+    return res, (routes[0][0], routes[0][1], x_np, c, seed)
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -430,7 +524,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     res, (topk, w, x, c, seed) = run_ours(args, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and x is not None and c["P"] * c["H"] <= (1 << 30):
         times = time_oracle(c, seed, 3, topk, w, x, budget_s=20.0)
         v = c["P"] * len(times) / sum(times)
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",

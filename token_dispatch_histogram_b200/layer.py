@@ -21,7 +21,11 @@ from . import (align_sort_capacity, ep_align_sort, ep_combine, ep_dispatch, ep_e
 
 class EpLayer:
     def __init__(self, R, S, K, E, H, block_m, device="cuda", grad_n=0, grad_dtype=torch.float32,
-                 with_pair_slot=False):
+                 with_pair_slot=False, share=None):
+        """share: another EpLayer of the same shape whose row buffers (x, the
+        dispatch buffer, out), workspace and gradients this layer reuses --
+        consecutive layers of a model run one after another, so one set of the
+        large buffers serves them all."""
         self.R, self.S, self.K, self.E, self.H, self.block_m = R, S, K, E, H, block_m
         self.T = R * S
         self.P = self.T * K
@@ -30,24 +34,30 @@ class EpLayer:
         i32 = dict(dtype=torch.int32, device=dev)
         self.topk_ids = torch.zeros((self.T, K), **i32)
         self.w = torch.zeros((self.T, K), dtype=torch.float32, device=dev)
-        self.x = torch.zeros((self.T, H), dtype=torch.bfloat16, device=dev)
+        self.x = share.x if share is not None else torch.zeros((self.T, H), dtype=torch.bfloat16, device=dev)
         self.loads = torch.zeros(E, **i32)
         self.max_vio = torch.zeros(1, dtype=torch.float64, device=dev)
-        self.ws = torch.zeros(ep_workspace_size(self.T, K, E), dtype=torch.uint8, device=dev)
+        self.ws = share.ws if share is not None else torch.zeros(ep_workspace_size(self.T, K, E), dtype=torch.uint8,
+                                                                 device=dev)
         self.plan_layout = ep_plan_layout(E, R)
         self.plan = torch.zeros(self.plan_layout["words"], **i32)
         self.pos = torch.zeros(self.P, **i32)
         self.src = torch.zeros(self.P, **i32)
         self.pair_slot = torch.zeros(self.P, **i32) if with_pair_slot else None
-        self.buf = torch.zeros((self.P, H), dtype=torch.bfloat16, device=dev)  # dispatch output / combine input
-        self.out = torch.zeros((self.T, H), dtype=torch.bfloat16, device=dev)
+        if share is not None:
+            self.buf, self.out = share.buf, share.out
+        else:
+            self.buf = torch.zeros((self.P, H), dtype=torch.bfloat16, device=dev)  # dispatch output / combine input
+            self.out = torch.zeros((self.T, H), dtype=torch.bfloat16, device=dev)
         cap, capb = align_sort_capacity(self.P, E, block_m)
         self.sorted_token_ids = torch.zeros(cap, **i32)
         self.expert_ids = torch.zeros(capb, **i32)
         self.num_tokens_post_pad = torch.zeros(1, **i32)
         self.dev_status = torch.zeros(1, **i32)
         self.grad_n = grad_n
-        if grad_n:
+        if grad_n and share is not None and share.grad_n == grad_n:
+            self.g_home, self.g_rep = share.g_home, share.g_rep
+        elif grad_n:
             self.g_home = torch.zeros((E, grad_n), dtype=torch.float32, device=dev)
             self.g_rep = torch.zeros((self.plan_layout["cap"], grad_n), dtype=grad_dtype, device=dev)
         else:
