@@ -48,6 +48,10 @@ def _bind(L):
     L.oracle_combine.argtypes = [P, P, P, _c.c_int64, _c.c_int, _c.c_int64, P]
     L.oracle_combine_closed.restype = None
     L.oracle_combine_closed.argtypes = [P, P, P, _c.c_int64, _c.c_int, _c.c_int64, P, P]
+    L.oracle_dispatch_backward.restype = None
+    L.oracle_dispatch_backward.argtypes = [P, P, _c.c_int64, _c.c_int, _c.c_int64, P]
+    L.oracle_combine_backward.restype = None
+    L.oracle_combine_backward.argtypes = [P, P, P, P, _c.c_int64, _c.c_int, _c.c_int64, P, P]
     L.oracle_grad_reduce.restype = None
     L.oracle_grad_reduce.argtypes = [P, P, _c.c_int, _c.c_int64, _c.c_int, P, _c.c_int]
     return L
@@ -184,6 +188,30 @@ def grad_reduce(g_home, g_rep, rep_expert, clear=False, L=None):
     re = _i32(rep_expert) if len(rep_expert) else np.zeros(1, np.int32)
     L.oracle_grad_reduce(_p(gh), _p(gr), dt, n, len(rep_expert), _p(re), int(clear))
     return gh, gr
+
+
+def dispatch_backward(dbuf, pos, T, K, L=None):
+    """dx [T, H]: the unpermute gradient of dispatch."""
+    L = L or lib()
+    dbuf = np.ascontiguousarray(dbuf, dtype=np.uint16)
+    H = dbuf.shape[1]
+    dx = np.empty((T, H), dtype=np.uint16)
+    L.oracle_dispatch_backward(_p(dbuf), _p(_i32(pos)), T, K, H, _p(dx))
+    return dx
+
+
+def combine_backward(dout, w, y, pos, dy_init=None, L=None):
+    """(dy [rows, H] uint16, dw [T, K] float64): the gradient of combine."""
+    L = L or lib()
+    dout = np.ascontiguousarray(dout, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    y = np.ascontiguousarray(y, dtype=np.uint16)
+    T, H = dout.shape
+    K = w.shape[1]
+    dy = np.zeros_like(y) if dy_init is None else np.array(dy_init, dtype=np.uint16, copy=True)
+    dw = np.empty((T, K), dtype=np.float64)
+    L.oracle_combine_backward(_p(dout), _p(w), _p(y), _p(_i32(pos)), T, K, H, _p(dy), _p(dw))
+    return dy, dw
 
 
 def bf16_to_f32(u16):

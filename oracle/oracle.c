@@ -412,3 +412,57 @@ void oracle_grad_reduce(float* g_home, void* g_rep, int rep_dtype, int64_t n, in
     }
   }
 }
+
+/* ------------------------------------------------------ 8. backward */
+/*
+ * The MoE Align & Sort report [ZH] recalls that the permute which records the
+ * source -> destination mapping has unpermute as its gradient.  Dispatch is
+ * that permute (every token row copied to K rows) and combine its weighted
+ * inverse, so their gradients are:
+ *
+ * backward of dispatch (unpermute): dx[t] = bf16_rn( sum_{k=0..K-1}
+ *   float(dbuf[pos[t*K+k]]) ), accumulated in fp32 in k order from 0, one add
+ *   per term, one rounding to bf16.  Pairs with pos < 0 contribute nothing.
+ */
+void oracle_dispatch_backward(const uint16_t* dbuf, const int32_t* pos, int64_t T, int K, int64_t H, uint16_t* dx) {
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t h = 0; h < H; ++h) {
+      float acc = 0.0f;
+      for (int k = 0; k < K; ++k) {
+        int32_t row = pos[t * K + k];
+        if (row < 0) continue;
+        acc = acc + bf16_to_f32(dbuf[(int64_t)row * H + h]);
+      }
+      dx[t * H + h] = f32_to_bf16(acc);
+    }
+  }
+}
+
+/*
+ * backward of combine, given dout [T, H] (bf16):
+ *   dy[pos[t*K+k]] = bf16_rn( w[t,k] * float(dout[t]) )   one fp32 multiply per element;
+ *   dw[t,k] = sum_h float(dout[t,h]) * float(y[pos[t*K+k], h])
+ * dw is accumulated in fp64 (each product of two bf16 values is exact in fp64;
+ * the sum carries only fp64 rounding), the reference against which an fp32
+ * reduction in any order is bounded.  Rows of dy not addressed by any pair are
+ * left untouched.
+ */
+void oracle_combine_backward(const uint16_t* dout, const float* w, const uint16_t* y, const int32_t* pos, int64_t T,
+                             int K, int64_t H, uint16_t* dy, double* dw) {
+  for (int64_t t = 0; t < T; ++t) {
+    for (int k = 0; k < K; ++k) {
+      int32_t row = pos[t * K + k];
+      if (row < 0) {
+        dw[t * K + k] = 0.0;
+        continue;
+      }
+      double s = 0.0;
+      for (int64_t h = 0; h < H; ++h) {
+        float g = bf16_to_f32(dout[t * H + h]);
+        dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K + k] * g);
+        s += (double)g * (double)bf16_to_f32(y[(int64_t)row * H + h]);
+      }
+      dw[t * K + k] = s;
+    }
+  }
+}

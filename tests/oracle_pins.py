@@ -471,6 +471,63 @@ def pin_grad_reduce(L):
         _ = rng
 
 
+def pin_dispatch_backward(L):
+    rng = np.random.default_rng(21)
+    # K = 1: the gradient of a pure permutation is the inverse permutation
+    T, H = 30, 24
+    dbuf = W.hidden(T, H, seed=31)
+    pos = rng.permutation(T).astype(np.int32)
+    np.testing.assert_array_equal(O.dispatch_backward(dbuf, pos, T, 1, L=L), dbuf[pos])
+    # backward of dispatch applied to dispatch(x): every token gets K copies of x,
+    # and j*x is exact in fp32 for a bf16 x, so dx = bf16_rn(K * x) in closed form
+    for K in (2, 3, 4, 6, 8):
+        T, H = 20, 16
+        x = W.hidden(T, H, seed=K)
+        pos = rng.permutation(T * K).astype(np.int32)
+        buf = O.dispatch(x, pos, K, T * K, L=L)
+        dx = O.dispatch_backward(buf, pos, T, K, L=L)
+        ref = _bf16_rne(O.bf16_to_f32(x) * np.float32(K))
+        np.testing.assert_array_equal(dx, ref)
+    # general rows: fp32 sum of K terms within its error bound of the fp64 sum
+    T, K, H = 25, 5, 40
+    dbuf = W.hidden(T * K, H, seed=41)
+    pos = rng.permutation(T * K).astype(np.int32)
+    pos[7] = -1  # a pair without a row contributes nothing
+    dx = O.bf16_to_f32(O.dispatch_backward(dbuf, pos, T, K, L=L)).astype(np.float64)
+    rows = O.bf16_to_f32(dbuf).astype(np.float64)[np.maximum(pos, 0)].reshape(T, K, H)
+    rows[7 // K, 7 % K] = 0.0
+    exact = rows.sum(1)
+    assert np.all(np.abs(dx - exact) <= K * 2.0 ** -24 * np.abs(rows).sum(1) + np.abs(exact) * 2.0 ** -8 + 1e-30)
+
+
+def pin_combine_backward(L):
+    rng = np.random.default_rng(22)
+    T, K, H = 16, 3, 32
+    P = T * K
+    dout = W.hidden(T, H, seed=51)
+    y = W.hidden(P, H, seed=52)
+    pos = rng.permutation(P).astype(np.int32)
+    # w = 1: dy rows are dout rows, exactly
+    dy, dw = O.combine_backward(dout, np.ones((T, K), np.float32), y, pos, L=L)
+    np.testing.assert_array_equal(dy[pos].reshape(T, K, H), np.repeat(dout[:, None, :], K, axis=1))
+    # general weights: dy = bf16_rn(float32 product), dw = the fp64 dot product
+    w = rng.uniform(-2, 2, (T, K)).astype(np.float32)
+    init = np.full((P + 5, H), 0x1234, dtype=np.uint16)
+    y5 = np.concatenate([y, W.hidden(5, H, seed=53)])
+    dy, dw = O.combine_backward(dout, w, y5, pos, dy_init=init, L=L)
+    ref = _bf16_rne(O.bf16_to_f32(dout)[:, None, :] * w[:, :, None])       # [T, K, H]
+    np.testing.assert_array_equal(dy[pos].reshape(T, K, H), ref)
+    assert np.all(dy[P:] == 0x1234)  # rows no pair addresses are left alone
+    dref = np.einsum("th,tkh->tk", O.bf16_to_f32(dout).astype(np.float64),
+                     O.bf16_to_f32(y5).astype(np.float64)[pos].reshape(T, K, H))
+    np.testing.assert_allclose(dw, dref, rtol=1e-12, atol=1e-12)
+    # y rows equal to their token's dout row: dw is the squared norm
+    y_same = np.repeat(dout, K, axis=0)[np.argsort(pos)]
+    _, dw2 = O.combine_backward(dout, w, y_same, pos, L=L)
+    sq = (O.bf16_to_f32(dout).astype(np.float64) ** 2).sum(1)
+    np.testing.assert_allclose(dw2, np.repeat(sq[:, None], K, axis=1), rtol=1e-12)
+
+
 ALL_PINS = [pin_hand_example, pin_max_vio_closed_forms, pin_plan_unit_restatement, pin_layout_brute_force,
             pin_layout_library_reductions, pin_layout_invariants, pin_align_sort, pin_dispatch, pin_combine,
-            pin_grad_reduce]
+            pin_grad_reduce, pin_dispatch_backward, pin_combine_backward]

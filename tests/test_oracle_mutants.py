@@ -43,12 +43,19 @@ MUTANTS = [
      "float prod = w[k * T + t] * bf16_to_f32(y[(int64_t)row * H + h]);"),
     ("combine_wrong_sign", "        float prod = w[t * K + k] * bf16_to_f32(y[(int64_t)row * H + h]);\n        acc = acc + prod;",
      "        float prod = w[t * K + k] * bf16_to_f32(y[(int64_t)row * H + h]);\n        acc = acc - prod;"),
-    ("combine_first_term_dropped", "      for (int k = 0; k < K; ++k) {\n        int32_t row = pos[t * K + k];",
-     "      for (int k = 1; k < K; ++k) {\n        int32_t row = pos[t * K + k];"),
+    ("combine_first_term_dropped",
+     "      for (int k = 0; k < K; ++k) {\n        int32_t row = pos[t * K + k];\n        if (row < 0) continue;\n        float prod",
+     "      for (int k = 1; k < K; ++k) {\n        int32_t row = pos[t * K + k];\n        if (row < 0) continue;\n        float prod"),
     ("bf16_round_half_up", "  uint32_t lsb = (u >> 16) & 1u;\n  u += 0x7FFFu + lsb;", "  uint32_t lsb = 1u;\n  u += 0x7FFFu + lsb;"),
     ("grad_home_dropped", "for (int64_t j = 0; j < n; ++j) dst[j] = dst[j] + g[j];", "for (int64_t j = 0; j < n; ++j) dst[j] = g[j];"),
     ("grad_bf16_wrong_widen", "dst[j] = dst[j] + bf16_to_f32(g[j]);", "dst[j] = dst[j] + (float)g[j];"),
     ("grad_no_clear", "if (clear) memset(g, 0, (size_t)n * 4);", "if (0) memset(g, 0, (size_t)n * 4);"),
+    ("dispatch_bwd_first_term_dropped", "        acc = acc + bf16_to_f32(dbuf[(int64_t)row * H + h]);",
+     "        if (k > 0) acc = acc + bf16_to_f32(dbuf[(int64_t)row * H + h]);"),
+    ("combine_bwd_weight_index", "dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K + k] * g);",
+     "dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K] * g);"),
+    ("combine_bwd_dw_wrong_row", "s += (double)g * (double)bf16_to_f32(y[(int64_t)row * H + h]);",
+     "s += (double)g * (double)bf16_to_f32(y[(int64_t)(t * K + k) * H + h]);"),
 ]
 
 RUNNER = r"""
