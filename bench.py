@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing the backward of dispatch and combine")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the eager per-op pass only (default: the headline value comes from replaying the "
                          "step as one captured CUDA graph; the per-op breakdown from the eager pass)")
@@ -347,6 +348,41 @@ def run_ours(args, rank, world, local_rank):
             graph = None
             print(f"graph capture unavailable: {exc}", file=sys.stderr)
 
+    # ---- backward of combine and of dispatch (timed apart from the step)
+    backward = None
+    if not args.no_backward and 2 * P * H <= (20 << 30):
+        dy = torch.empty_like(layer.buf)
+        dx = torch.empty_like(layer.x)
+        dw = torch.empty((T, K), dtype=torch.float32, device=dev)
+        ops_b = {
+            "combine_backward": (lambda: tdh.ep_combine_backward(layer.out, layer.w, layer.buf, layer.pos, dy, dw,
+                                                                 layer.dev_status, stream),
+                                 2 * T * H + 2 * 2 * P * H + 12 * P + 4 * P),
+            "dispatch_backward": (lambda: tdh.ep_dispatch_backward(layer.buf, layer.pos, T, K, dx, layer.dev_status,
+                                                                   stream),
+                                  2 * P * H + 4 * P + 2 * T * H),
+        }
+        backward = {}
+        for name, (fn, nbytes) in ops_b.items():
+            for _ in range(3):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                fn()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / args.steps
+            gbs = nbytes / (ms / 1e3) / 1e9
+            backward[name] = {"ms": round(ms, 5), "GB_s": round(gbs, 1), "frac": round(gbs / peaks()[0], 4),
+                              "algorithmic_bytes": nbytes}
+        st = layer.status(stream)
+        if st:
+            raise RuntimeError(f"device status {st:#x} in the backward timing")
+        del dy, dx, dw
+
     # ---- end to end through the public API, pinned host buffers
     e2e = None
     if not args.no_e2e and host_x and nl == 1:
@@ -417,6 +453,7 @@ def run_ours(args, rank, world, local_rank):
                              "frac": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9 / peak, 4)},
         "routing": {"max_vio": max_vio if nl > 1 else max_vio[0], "n_rep": n_rep if nl > 1 else n_rep[0],
                     "replicated_experts": n_chunks if nl > 1 else n_chunks[0]},
+        "backward": backward,
         "layers_per_step": nl,
         "route_path": args.route,
     }

@@ -238,6 +238,29 @@ EP_API int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, const i
                uint16_t* out, int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * Backward of dispatch: the MoE Align & Sort report [ZH] recalls that the
+ * permute recording the source -> destination mapping has unpermute as its
+ * gradient.  dx[t] = bf16_rn( sum_{k} float(dbuf[pos[t*K+k]]) ), fp32 in k
+ * order, one rounding (combine with unit weights).
+ *   dbuf [buf_rows, H] bf16 (gradient w.r.t. the dispatched rows); dx [T, H] out.
+ */
+EP_API int ep_dispatch_backward(const uint16_t* dbuf, int64_t buf_rows, const int32_t* pos, int64_t T, int K,
+                                int64_t H, uint16_t* dx, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Backward of combine, given dout [T, H] bf16 (gradient w.r.t. out):
+ *   dy[pos[t*K+k]] = bf16_rn(w[t,k] * float(dout[t]))   (gradient w.r.t. the expert rows)
+ *   dw[t,k] = sum_h float(dout[t,h]) * float(y[pos[t*K+k], h])   fp32, summation
+ *             order unspecified (within H * 2^-24 * sum|dout*y| of the exact value)
+ *   y [y_rows, H] bf16 (combine's input); dy [y_rows, H] out (rows no pair
+ *   addresses are left untouched); dw [T, K] fp32 out; 1 <= K <= 8.
+ * Each dout row is read once, each y row once, each dy row written once.
+ */
+EP_API int ep_combine_backward(const uint16_t* dout, const float* w, const uint16_t* y, int64_t y_rows,
+                               const int32_t* pos, int64_t T, int K, int64_t H, uint16_t* dy, float* dw,
+                               int32_t* dev_status, cudaStream_t stream);
+
+/*
  * a7. Replica gradient reduction.  [GR] "Τι συμβαίνει στους gradients κατά την
  * εκπαίδευση": replica gradients live in a separate reduce buffer in fp32 and
  * are added into the home expert's gradient, after which the used slots are

@@ -59,6 +59,8 @@ _SIGS = {
                             _V, _SZ, _V, _V]),
     "ep_dispatch": (_I, [_V, _I64, _I, _I64, _V, _V, _I64, _V, _V]),
     "ep_expert_scale": (_I, [_V, _I64, _I64, _V, _V, _I64, _V, _I, _V, _V, _V]),
+    "ep_dispatch_backward": (_I, [_V, _I64, _V, _I64, _I, _I64, _V, _V, _V]),
+    "ep_combine_backward": (_I, [_V, _V, _V, _I64, _V, _I64, _I, _I64, _V, _V, _V, _V]),
     "ep_combine": (_I, [_V, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
     "ep_replica_grad_reduce": (_I, [_V, _V, _I, _I64, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_status_read": (_I, [_V, _V, _V]),
@@ -221,6 +223,25 @@ def ep_combine(y, w, pos, out, dev_status=None, stream=None):
     H = y.shape[1]
     _check("ep_combine", lib().ep_combine(_p(y), y.shape[0], _p(w), _p(pos), T, K, H, _p(out), _p(dev_status),
                                           _s(stream)))
+
+
+def ep_dispatch_backward(dbuf, pos, T, K, dx, dev_status=None, stream=None):
+    """dx[t] = sum_k dbuf[pos[t*K+k]] (the unpermute gradient of dispatch)."""
+    _dtype(pos, torch.int32)
+    H = dbuf.shape[1]
+    _check("ep_dispatch_backward", lib().ep_dispatch_backward(_p(dbuf), dbuf.shape[0], _p(pos), T, K, H, _p(dx),
+                                                              _p(dev_status), _s(stream)))
+
+
+def ep_combine_backward(dout, w, y, pos, dy, dw, dev_status=None, stream=None):
+    """dy[pos[t,k]] = w[t,k] * dout[t]; dw[t,k] = <dout[t], y[pos[t,k]]>."""
+    _dtype(w, torch.float32)
+    _dtype(dw, torch.float32)
+    _dtype(pos, torch.int32)
+    T, K = w.shape
+    H = dout.shape[1]
+    _check("ep_combine_backward", lib().ep_combine_backward(_p(dout), _p(w), _p(y), y.shape[0], _p(pos), T, K, H,
+                                                            _p(dy), _p(dw), _p(dev_status), _s(stream)))
 
 
 def ep_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False, dev_status=None, stream=None):

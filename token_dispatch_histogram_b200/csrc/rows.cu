@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(256, 4)
       float wk = 0.0f;
       if (t < T) {
         r = __ldg(pos + t * K + k);
-        wk = __ldg(w + t * K + k);
+        wk = w ? __ldg(w + t * K + k) : 1.0f;  // no weights: the unpermute (x 1.0f is exact)
         if (r < 0 || r >= y_rows) {
           r = -1;
           s_bad = 1;
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(256)
         bad = EP_DEV_BAD_ROW;
         continue;
       }
-      const float wk = __ldg(w + t * K + k);
+      const float wk = w ? __ldg(w + t * K + k) : 1.0f;
       const uint4 in = ld_stream_v4(y + (int64_t)r * H + v * 8);
       const uint32_t wd[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
@@ -249,6 +249,115 @@ __global__ void __launch_bounds__(256)
     st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
   }
   if (bad) flag(dev_status, bad);
+}
+
+// Backward of combine.  For every pair (t, k) with row r = pos[t*K+k]:
+//   dy[r]    = bf16_rn(w[t,k] * float(dout[t]))          (one fp32 multiply per element)
+//   dw[t,k]  = sum_h float(dout[t,h]) * float(y[r,h])     (fp32; any summation order)
+// A thread owns one 16-byte vector of the token's row: it loads the dout vector
+// and the K y vectors, writes the K scaled dy vectors and keeps K partial dot
+// products; those are reduced over the token's threads (warp shuffles, then
+// shared memory) once the row is done.
+template <int K>
+__global__ void __launch_bounds__(256, 4)
+    k_combine_bwd(const uint16_t* __restrict__ dout, const float* __restrict__ w, const uint16_t* __restrict__ y,
+                  int64_t y_rows, const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ dy,
+                  float* __restrict__ dw, int32_t* dev_status) {
+  constexpr int MAXT = 8;
+  __shared__ int32_t s_rows[2][MAXT][K];
+  __shared__ float s_w[2][MAXT][K];
+  __shared__ float s_part[8][K];  // per warp partial dot products
+  __shared__ int s_bad;
+  const int64_t nvec = H / 8;
+  const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);
+  const int tpc = 256 / tpr <= MAXT ? 256 / tpr : MAXT;
+  const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t step = (int64_t)gridDim.x * tpc;
+  if (threadIdx.x == 0) s_bad = 0;
+  auto stage = [&](int b, int64_t tb) {
+    if (threadIdx.x < tpc * K) {
+      const int s = threadIdx.x / K, k = threadIdx.x - s * K;
+      const int64_t t = tb + s;
+      int32_t r = -1;
+      float wk = 0.0f;
+      if (t < T) {
+        r = __ldg(pos + t * K + k);
+        wk = __ldg(w + t * K + k);
+        if (r < 0 || r >= y_rows) {
+          r = -1;
+          s_bad = 1;
+        }
+      }
+      s_rows[b][s][k] = r;
+      s_w[b][s][k] = wk;
+    }
+  };
+  int64_t tb = (int64_t)blockIdx.x * tpc;
+  stage(0, tb);
+  __syncthreads();
+  for (int b = 0; tb < T; tb += step, b ^= 1) {
+    stage(b ^ 1, tb + step);
+    const int64_t t = tb + sub;
+    const bool live = sub < tpc && t < T;
+    float part[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) part[k] = 0.0f;
+    if (live) {
+      for (int64_t v = v0; v < nvec; v += tpr) {
+        const uint4 g = ld_stream_v4(dout + t * H + v * 8);
+        uint4 in[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const int32_t r = s_rows[b][sub][k];
+          in[k] = r >= 0 ? ld_stream_v4(y + (int64_t)r * H + v * 8) : make_uint4(0, 0, 0, 0);
+        }
+        const uint32_t gd[4] = {g.x, g.y, g.z, g.w};
+        float gf[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gf[2 * q] = bf16_bits_to_f32(gd[q] & 0xFFFFu);
+          gf[2 * q + 1] = bf16_bits_to_f32(gd[q] >> 16);
+        }
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const int32_t r = s_rows[b][sub][k];
+          if (r < 0) continue;
+          const float wk = s_w[b][sub][k];
+          const uint32_t yd[4] = {in[k].x, in[k].y, in[k].z, in[k].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            o[q] = f32_to_bf16_bits(__fmul_rn(wk, gf[2 * q])) | (f32_to_bf16_bits(__fmul_rn(wk, gf[2 * q + 1])) << 16);
+            part[k] = fmaf(gf[2 * q], bf16_bits_to_f32(yd[q] & 0xFFFFu), part[k]);
+            part[k] = fmaf(gf[2 * q + 1], bf16_bits_to_f32(yd[q] >> 16), part[k]);
+          }
+          st_v4(dy + (int64_t)r * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+      }
+    }
+    // reduce the K partial dot products over the token's threads
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      float v = part[k];
+#pragma unroll
+      for (int d = 16; d; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+      if (lane == 0) s_part[warp][k] = v;
+    }
+    __syncthreads();
+    const int wpt = tpr / 32;  // warps per token
+    if (threadIdx.x < tpc * K) {
+      const int s = threadIdx.x / K, k = threadIdx.x - s * K;
+      const int64_t tt = tb + s;
+      if (tt < T) {
+        float acc = 0.0f;
+        for (int i = 0; i < wpt; ++i) acc += s_part[s * wpt + i][k];
+        dw[tt * K + k] = s_rows[b][s][k] >= 0 ? acc : 0.0f;
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_ROW);
 }
 
 int occupancy_grid(const void* fn, int threads, size_t smem, int64_t work_items, int cap_per_sm) {
@@ -311,7 +420,7 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
   if (T < 0 || K < 1 || K > 32 || H < 8 || H % 8 || y_rows < 0) return EP_ERR_ARG;
   if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
   if (T == 0) return EP_OK;
-  if (!y || !w || !pos || !out || !aligned16(y) || !aligned16(out)) return EP_ERR_ARG;
+  if (!y || !pos || !out || !aligned16(y) || !aligned16(out)) return EP_ERR_ARG;  // w == NULL: unit weights
   const void* fn = nullptr;
   switch (K) {
     case 1: fn = (const void*)k_combine<1>; break;
@@ -333,6 +442,38 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
     const int grid = occupancy_grid((const void*)k_combine_any, 256, 0, T * (H / 8) / 256 + 1, 8);
     k_combine_any<<<grid, 256, 0, stream>>>(y, y_rows, w, pos, T, K, H, out, dev_status);
   }
+  count_launch();
+  return launch_status();
+}
+
+extern "C" int ep_dispatch_backward(const uint16_t* dbuf, int64_t buf_rows, const int32_t* pos, int64_t T, int K,
+                                    int64_t H, uint16_t* dx, int32_t* dev_status, cudaStream_t stream) {
+  // dx[t] = sum_k dbuf[pos[t*K+k]]: the combine kernel with unit weights
+  return ep_combine(dbuf, buf_rows, nullptr, pos, T, K, H, dx, dev_status, stream);
+}
+
+extern "C" int ep_combine_backward(const uint16_t* dout, const float* w, const uint16_t* y, int64_t y_rows,
+                                   const int32_t* pos, int64_t T, int K, int64_t H, uint16_t* dy, float* dw,
+                                   int32_t* dev_status, cudaStream_t stream) {
+  if (T < 0 || K < 1 || K > 8 || H < 8 || H % 8 || y_rows < 0) return EP_ERR_ARG;
+  if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (T == 0) return EP_OK;
+  if (!dout || !w || !y || !pos || !dy || !dw || !aligned16(dout) || !aligned16(y) || !aligned16(dy)) return EP_ERR_ARG;
+  const void* fn = nullptr;
+  switch (K) {
+    case 1: fn = (const void*)k_combine_bwd<1>; break;
+    case 2: fn = (const void*)k_combine_bwd<2>; break;
+    case 3: fn = (const void*)k_combine_bwd<3>; break;
+    case 4: fn = (const void*)k_combine_bwd<4>; break;
+    case 5: fn = (const void*)k_combine_bwd<5>; break;
+    case 6: fn = (const void*)k_combine_bwd<6>; break;
+    case 7: fn = (const void*)k_combine_bwd<7>; break;
+    default: fn = (const void*)k_combine_bwd<8>; break;
+  }
+  const int grid = occupancy_grid(fn, 256, 0, T, 4);
+  void* args[] = {(void*)&dout, (void*)&w, (void*)&y, (void*)&y_rows, (void*)&pos, (void*)&T, (void*)&H, (void*)&dy,
+                  (void*)&dw, (void*)&dev_status};
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }
