@@ -18,7 +18,8 @@ L2 flushed (a 512 MB write) between replays outside the events, max over ranks.
 The per-op breakdown and the roofline come from an eager pass of the same K
 steps with CUDA events between the ops.  `e2e`: the same steps through the public API (EpLayer.run_host) from
 pinned host buffers: routing, gate weights and hidden rows copied in, the
-combined rows copied out, inside the timed region.  Under torchrun each rank
+combined rows copied out, inside the timed region (run_host pipelines the
+copies in token slices over two copy streams).  Under torchrun each rank
 runs its own independent layer (weak scaling, no data-path collective).
 
 --impl reference times the CPU oracle (the plain single-threaded definition of

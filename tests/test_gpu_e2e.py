@@ -1,0 +1,37 @@
+"""The public end-to-end call (EpLayer.run_host) gives the same result as the
+device-resident step, whether or not it pipelines the host copies in slices,
+and matches the oracle (-m gpu)."""
+import numpy as np
+import pytest
+
+import oracle as O
+import workload as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 8])
+def test_run_host_matches_oracle(chunks):
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    c = W.shape(2)
+    R, S, E, K, H, T = c["R"], c["S"], c["E"], c["K"], c["H"], c["T"]
+    S2 = 512  # a smaller token count with the workload's shape
+    T2 = R * S2
+    topk, w = W.routing_from(T2, E, K, seed=3, bias_e=W.bias(2, 0))
+    x = W.hidden(T2, H, seed=4)
+    layer = tdh.EpLayer(R, S2, K, E, H, c["block_m"], device="cuda")
+    topk_h = torch.from_numpy(topk).pin_memory()
+    w_h = torch.from_numpy(w).pin_memory()
+    x_h = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_h = torch.zeros((T2, H), dtype=torch.bfloat16).pin_memory()
+    layer.run_host(topk_h, w_h, x_h, out_h, grads=False, chunks=chunks)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    loads, mv, _ = O.route_stats(topk, E)
+    pl = O.plan(loads, R, S2, K, E)
+    lo = O.layout(topk, pl, R, S2, E)
+    buf = O.dispatch(x, lo["pos"], K, T2 * K)
+    ref = O.combine(buf, w, lo["pos"], K)
+    np.testing.assert_array_equal(out_h.view(torch.int16).numpy().view(np.uint16), ref)
+    _ = (S, T)

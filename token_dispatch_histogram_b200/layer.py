@@ -9,7 +9,8 @@ sequence of libep.so calls on one stream, with no host synchronisation:
   -> ep_dispatch -> [expert: outside the path] -> ep_combine -> ep_replica_grad_reduce
 
 `step()` is one pass of that sequence over the resident inputs; `run_host()`
-is the same pass fed from pinned host buffers (copies in, result out).
+is the same pass fed from pinned host buffers (copies in, result out),
+pipelined in token slices so the host transfers overlap.
 Plumbing only: every computation happens in the library's kernels.
 """
 import torch
@@ -101,14 +102,55 @@ class EpLayer:
         if grads:
             self.grad_reduce(False, stream)
 
-    def run_host(self, topk_h, w_h, x_h, out_h, stream=None, grads=True, fused=True):
-        """The step fed from (pinned) host buffers: host->device copies of the
-        routing and hidden rows, the path, and the combined rows back to host."""
-        self.topk_ids.copy_(topk_h, non_blocking=True)
-        self.w.copy_(w_h, non_blocking=True)
-        self.x.copy_(x_h, non_blocking=True)
-        self.step(stream, grads, fused)
-        out_h.copy_(self.out, non_blocking=True)
+    def run_host(self, topk_h, w_h, x_h, out_h, stream=None, grads=True, fused=True, chunks=8):
+        """The step fed from pinned host buffers: host->device copies of the
+        routing and hidden rows, the path, and the combined rows back to host.
+
+        With chunks > 1 the token rows move in `chunks` slices on two copy
+        streams: slice i is copied in, dispatched and combined while slice i+1
+        is still arriving and slice i-1 is already going out (the host link is
+        full duplex), so the transfers overlap each other and the kernels.
+        Dispatch and combine of a token slice touch only that slice's pairs, so
+        the slices are independent.  The caller's stream waits for the last copy
+        out before anything queued after this call."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if chunks <= 1 or self.T < chunks:
+            with torch.cuda.stream(main):
+                self.topk_ids.copy_(topk_h, non_blocking=True)
+                self.w.copy_(w_h, non_blocking=True)
+                self.x.copy_(x_h, non_blocking=True)
+                self.step(main, grads, fused)
+                out_h.copy_(self.out, non_blocking=True)
+            return
+        if not hasattr(self, "_h2d"):
+            self._h2d = torch.cuda.Stream(self.device)
+            self._d2h = torch.cuda.Stream(self.device)
+        h2d, d2h = self._h2d, self._d2h
+        h2d.wait_stream(main)  # buffers are free once the caller's earlier work is done
+        d2h.wait_stream(main)
+        with torch.cuda.stream(main):
+            self.topk_ids.copy_(topk_h, non_blocking=True)
+            self.w.copy_(w_h, non_blocking=True)
+            self.route(main, fused)
+        bounds = [self.T * i // chunks for i in range(chunks + 1)]
+        K = self.K
+        for t0, t1 in zip(bounds[:-1], bounds[1:]):
+            with torch.cuda.stream(h2d):
+                self.x[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(h2d)
+            main.wait_event(arrived)
+            ep_dispatch(self.x[t0:t1], K, self.pos[t0 * K:t1 * K], self.buf, self.dev_status, main)
+            ep_combine(self.buf, self.w[t0:t1], self.pos[t0 * K:t1 * K], self.out[t0:t1], self.dev_status, main)
+            combined = torch.cuda.Event()
+            combined.record(main)
+            d2h.wait_event(combined)
+            with torch.cuda.stream(d2h):
+                out_h[t0:t1].copy_(self.out[t0:t1], non_blocking=True)
+        if grads:
+            self.grad_reduce(False, main)
+        main.wait_stream(d2h)
+        main.wait_stream(h2d)
 
     def status(self, stream=None):
         return ep_status_read(self.dev_status, stream)
