@@ -52,6 +52,8 @@ def _bind(L):
     L.oracle_dispatch_backward.argtypes = [P, P, _c.c_int64, _c.c_int, _c.c_int64, P]
     L.oracle_combine_backward.restype = None
     L.oracle_combine_backward.argtypes = [P, P, P, P, _c.c_int64, _c.c_int, _c.c_int64, P, P]
+    L.oracle_prefetch_slots.restype = None
+    L.oracle_prefetch_slots.argtypes = [_c.c_int, P, _c.c_int, _c.c_int, _c.c_int, P, P]
     L.oracle_grad_reduce.restype = None
     L.oracle_grad_reduce.argtypes = [P, P, _c.c_int, _c.c_int64, _c.c_int, P, _c.c_int]
     return L
@@ -212,6 +214,17 @@ def combine_backward(dout, w, y, pos, dy_init=None, L=None):
     dw = np.empty((T, K), dtype=np.float64)
     L.oracle_combine_backward(_p(dout), _p(w), _p(y), _p(_i32(pos)), T, K, H, _p(dy), _p(dw))
     return dy, dw
+
+
+def prefetch_slots(pl, E, R, B, L=None):
+    """(slot [n_rep] int32: E + j or -1, n_remote [R] int32)."""
+    L = L or lib()
+    n = pl["n_rep"]
+    rr = _i32(pl["rep_rank"]) if n else np.zeros(1, np.int32)
+    slot = np.empty(max(n, 1), dtype=np.int32)
+    nrem = np.empty(R, dtype=np.int32)
+    L.oracle_prefetch_slots(n, _p(rr), E, R, B, _p(slot), _p(nrem))
+    return slot[:n].copy(), nrem
 
 
 def bf16_to_f32(u16):

@@ -466,3 +466,30 @@ void oracle_combine_backward(const uint16_t* dout, const float* w, const uint16_
     }
   }
 }
+
+/* ------------------------------------------------ 9. prefetch slots */
+/*
+ * [GR] "Το memory contract που πρέπει να καταλάβει η τεχνική ομάδα": each rank's
+ * grouped-GEMM weight tensor is [E+B, H, H'], rows 0..E-1 for the ranks' own
+ * experts and rows E..E+B-1 as local prefetch slots; when a rank needs more
+ * remote experts than it has slots, the rest are read from their home rank
+ * (correct, slower).  Reading used: replicas take a rank's slots in match order,
+ * so the j-th replica a rank receives gets slot E + j while j < B, and -1
+ * (read from the home rank) after that.  The token layout does not change.
+ * slot[m] for m < n_rep; n_remote[r] = replicas rank r reads from home.
+ */
+void oracle_prefetch_slots(int n_rep, const int32_t* rep_rank, int E, int R, int B, int32_t* slot, int32_t* n_remote) {
+  int32_t* seen = (int32_t*)calloc((size_t)R, sizeof(int32_t));
+  for (int r = 0; r < R; ++r) n_remote[r] = 0;
+  for (int m = 0; m < n_rep; ++m) {
+    int r = rep_rank[m];
+    int j = seen[r]++;
+    if (j < B) {
+      slot[m] = E + j;
+    } else {
+      slot[m] = -1;
+      n_remote[r] += 1;
+    }
+  }
+  free(seen);
+}

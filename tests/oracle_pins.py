@@ -528,6 +528,34 @@ def pin_combine_backward(L):
     np.testing.assert_allclose(dw2, np.repeat(sq[:, None], K, axis=1), rtol=1e-12)
 
 
+def pin_prefetch_slots(L):
+    g = golden()
+    R, S, K, E = g["R"], g["S"], g["K"], g["E"]
+    topk = np.array(g["topk_ids"], dtype=np.int32)
+    loads, _, _ = O.route_stats(topk, E, L=L)
+    pl = O.plan(loads, R, S, K, E, L=L)
+    # hand example: m0 -> rank 1, m1 and m2 -> rank 3
+    assert O.prefetch_slots(pl, E, R, 2, L=L)[0].tolist() == [8, 8, 9]
+    slot, nrem = O.prefetch_slots(pl, E, R, 1, L=L)
+    assert slot.tolist() == [8, 8, -1] and nrem.tolist() == [0, 0, 0, 1]
+    slot, nrem = O.prefetch_slots(pl, E, R, 0, L=L)
+    assert slot.tolist() == [-1, -1, -1] and nrem.tolist() == [0, 1, 0, 2]
+    # random plans: slots on a rank are E, E+1, ... in match order up to B; the
+    # remote count is what does not fit
+    rng = np.random.default_rng(17)
+    for it in range(100):
+        R = int(rng.choice([2, 4, 8])); ER = int(rng.integers(1, 5)); E = R * ER
+        SK = int(rng.integers(4, 40)); loads = _rand_loads(rng, R, ER, SK)
+        pl = O.plan(loads, R, SK, 1, E, L=L)
+        B = int(rng.integers(0, 4))
+        slot, nrem = O.prefetch_slots(pl, E, R, B, L=L)
+        for r in range(R):
+            mine = [m for m in range(pl["n_rep"]) if pl["rep_rank"][m] == r]
+            want = [E + j if j < B else -1 for j in range(len(mine))]
+            assert [int(slot[m]) for m in mine] == want
+            assert nrem[r] == max(0, len(mine) - B)
+
+
 ALL_PINS = [pin_hand_example, pin_max_vio_closed_forms, pin_plan_unit_restatement, pin_layout_brute_force,
             pin_layout_library_reductions, pin_layout_invariants, pin_align_sort, pin_dispatch, pin_combine,
-            pin_grad_reduce, pin_dispatch_backward, pin_combine_backward]
+            pin_grad_reduce, pin_dispatch_backward, pin_combine_backward, pin_prefetch_slots]
