@@ -53,7 +53,7 @@ def _bind(L):
     L.oracle_combine_backward.restype = None
     L.oracle_combine_backward.argtypes = [P, P, P, P, _c.c_int64, _c.c_int, _c.c_int64, P, P]
     L.oracle_prefetch_slots.restype = None
-    L.oracle_prefetch_slots.argtypes = [_c.c_int, P, _c.c_int, _c.c_int, _c.c_int, P, P]
+    L.oracle_prefetch_slots.argtypes = [_c.c_int, P, P, P, _c.c_int, _c.c_int, _c.c_int64, _c.c_int, P, P, P]
     L.oracle_grad_reduce.restype = None
     L.oracle_grad_reduce.argtypes = [P, P, _c.c_int, _c.c_int64, _c.c_int, P, _c.c_int]
     return L
@@ -216,15 +216,17 @@ def combine_backward(dout, w, y, pos, dy_init=None, L=None):
     return dy, dw
 
 
-def prefetch_slots(pl, E, R, B, L=None):
-    """(slot [n_rep] int32: E + j or -1, n_remote [R] int32)."""
+def prefetch_slots(pl, E, R, B, SK=0, L=None):
+    """(slot [n_rep] int32: E + j or -1, n_remote [R] int32, load_capped [R]
+    int64: rank loads when slotless replicas' pairs stay home; needs SK = S*K)."""
     L = L or lib()
     n = pl["n_rep"]
-    rr = _i32(pl["rep_rank"]) if n else np.zeros(1, np.int32)
+    re, rr, rc = (_i32(pl[k]) if n else np.zeros(1, np.int32) for k in ("rep_expert", "rep_rank", "rep_count"))
     slot = np.empty(max(n, 1), dtype=np.int32)
     nrem = np.empty(R, dtype=np.int32)
-    L.oracle_prefetch_slots(n, _p(rr), E, R, B, _p(slot), _p(nrem))
-    return slot[:n].copy(), nrem
+    capped = np.empty(R, dtype=np.int64)
+    L.oracle_prefetch_slots(n, _p(re), _p(rr), _p(rc), E, R, SK, B, _p(slot), _p(nrem), _p(capped))
+    return slot[:n].copy(), nrem, capped
 
 
 def bf16_to_f32(u16):

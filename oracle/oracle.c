@@ -477,10 +477,22 @@ void oracle_combine_backward(const uint16_t* dout, const float* w, const uint16_
  * so the j-th replica a rank receives gets slot E + j while j < B, and -1
  * (read from the home rank) after that.  The token layout does not change.
  * slot[m] for m < n_rep; n_remote[r] = replicas rank r reads from home.
+ *
+ * load_capped (may be NULL): the other reading of the overflow, where a
+ * replica without a slot is not made at all and its pairs stay with the
+ * expert's home rank e / (E/R).  Rank r then holds S*K, less the pairs of its
+ * own slotless replicas, plus the pairs of slotless replicas of its experts.
+ * B = 0 gives back the unplanned rank loads; B >= every rank's replica count
+ * gives S*K everywhere.
  */
-void oracle_prefetch_slots(int n_rep, const int32_t* rep_rank, int E, int R, int B, int32_t* slot, int32_t* n_remote) {
+void oracle_prefetch_slots(int n_rep, const int32_t* rep_expert, const int32_t* rep_rank, const int32_t* rep_count,
+                           int E, int R, int64_t SK, int B, int32_t* slot, int32_t* n_remote, int64_t* load_capped) {
   int32_t* seen = (int32_t*)calloc((size_t)R, sizeof(int32_t));
-  for (int r = 0; r < R; ++r) n_remote[r] = 0;
+  int ER = E / R;
+  for (int r = 0; r < R; ++r) {
+    n_remote[r] = 0;
+    if (load_capped) load_capped[r] = SK;
+  }
   for (int m = 0; m < n_rep; ++m) {
     int r = rep_rank[m];
     int j = seen[r]++;
@@ -489,6 +501,10 @@ void oracle_prefetch_slots(int n_rep, const int32_t* rep_rank, int E, int R, int
     } else {
       slot[m] = -1;
       n_remote[r] += 1;
+      if (load_capped) {
+        load_capped[r] -= rep_count[m];
+        load_capped[rep_expert[m] / ER] += rep_count[m];
+      }
     }
   }
   free(seen);

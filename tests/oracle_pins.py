@@ -531,29 +531,40 @@ def pin_combine_backward(L):
 def pin_prefetch_slots(L):
     g = golden()
     R, S, K, E = g["R"], g["S"], g["K"], g["E"]
+    SK = S * K
     topk = np.array(g["topk_ids"], dtype=np.int32)
     loads, _, _ = O.route_stats(topk, E, L=L)
     pl = O.plan(loads, R, S, K, E, L=L)
-    # hand example: m0 -> rank 1, m1 and m2 -> rank 3
-    assert O.prefetch_slots(pl, E, R, 2, L=L)[0].tolist() == [8, 8, 9]
-    slot, nrem = O.prefetch_slots(pl, E, R, 1, L=L)
+    # hand example: m0 (expert 1, 4 pairs) -> rank 1; m1 (expert 0, 2 pairs) and
+    # m2 (expert 5, 4 pairs) -> rank 3
+    slot, nrem, capped = O.prefetch_slots(pl, E, R, 2, SK, L=L)
+    assert slot.tolist() == [8, 8, 9] and nrem.tolist() == [0, 0, 0, 0] and capped.tolist() == [8, 8, 8, 8]
+    slot, nrem, capped = O.prefetch_slots(pl, E, R, 1, SK, L=L)
     assert slot.tolist() == [8, 8, -1] and nrem.tolist() == [0, 0, 0, 1]
-    slot, nrem = O.prefetch_slots(pl, E, R, 0, L=L)
+    assert capped.tolist() == [8, 8, 12, 4]  # expert 5's 4 pairs back on rank 2
+    slot, nrem, capped = O.prefetch_slots(pl, E, R, 0, SK, L=L)
     assert slot.tolist() == [-1, -1, -1] and nrem.tolist() == [0, 1, 0, 2]
+    assert capped.tolist() == g["rank_loads"]  # no replica: the unplanned loads
     # random plans: slots on a rank are E, E+1, ... in match order up to B; the
-    # remote count is what does not fit
+    # remote count is what does not fit; B = 0 gives each rank the sum of its
+    # experts' loads, a B above every rank's replica count gives S*K, and the
+    # capped loads always sum to R*S*K
     rng = np.random.default_rng(17)
     for it in range(100):
         R = int(rng.choice([2, 4, 8])); ER = int(rng.integers(1, 5)); E = R * ER
         SK = int(rng.integers(4, 40)); loads = _rand_loads(rng, R, ER, SK)
         pl = O.plan(loads, R, SK, 1, E, L=L)
         B = int(rng.integers(0, 4))
-        slot, nrem = O.prefetch_slots(pl, E, R, B, L=L)
+        slot, nrem, capped = O.prefetch_slots(pl, E, R, B, SK, L=L)
         for r in range(R):
             mine = [m for m in range(pl["n_rep"]) if pl["rep_rank"][m] == r]
             want = [E + j if j < B else -1 for j in range(len(mine))]
             assert [int(slot[m]) for m in mine] == want
             assert nrem[r] == max(0, len(mine) - B)
+        assert int(capped.sum()) == R * SK
+        unplanned = loads.reshape(R, ER).sum(axis=1)
+        assert O.prefetch_slots(pl, E, R, 0, SK, L=L)[2].tolist() == unplanned.tolist()
+        assert O.prefetch_slots(pl, E, R, E + R, SK, L=L)[2].tolist() == [SK] * R
 
 
 ALL_PINS = [pin_hand_example, pin_max_vio_closed_forms, pin_plan_unit_restatement, pin_layout_brute_force,

@@ -54,6 +54,7 @@ MUTANTS = [
      "        if (k > 0) acc = acc + bf16_to_f32(dbuf[(int64_t)row * H + h]);"),
     ("combine_bwd_weight_index", "dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K + k] * g);",
      "dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K] * g);"),
+    ("capped_home_by_mod", "load_capped[rep_expert[m] / ER]", "load_capped[rep_expert[m] % R]"),
     ("prefetch_slot_off_by_one", "    if (j < B) {\n      slot[m] = E + j;", "    if (j <= B) {\n      slot[m] = E + j;"),
     ("combine_bwd_dw_wrong_row", "s += (double)g * (double)bf16_to_f32(y[(int64_t)row * H + h]);",
      "s += (double)g * (double)bf16_to_f32(y[(int64_t)(t * K + k) * H + h]);"),
