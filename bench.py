@@ -384,6 +384,47 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device status {st:#x} in the backward timing")
         del dy, dx, dw
 
+    # ---- prefetch slots under a per-rank budget B (one small launch, timed
+    # apart as device time: 20 launches in one captured graph, replayed):
+    # replicas whose weights are read from the home rank, and the rank loads if
+    # slotless replicas' pairs stayed home instead (B = 0: the unplanned loads)
+    prefetch = {}
+    SK = S * K
+    cap = layer.plan_layout["cap"]
+    pf_slot = torch.empty(cap, dtype=torch.int32, device=dev)
+    pf_rem = torch.empty(R, dtype=torch.int32, device=dev)
+    pf_load = torch.empty(R, dtype=torch.int64, device=dev)
+    for B in sorted({0, 3, 4, E // R}):
+        rem, worst = [], []
+        for ly in layers:
+            tdh.ep_prefetch_slots(ly.plan, E, R, SK, B, pf_slot, pf_rem, pf_load, stream)
+            torch.cuda.synchronize()
+            rem.append(int(pf_rem.sum().item()))
+            worst.append(round(int(pf_load.max().item()) / SK, 4))
+        us = None
+        if not args.no_graph:
+            try:
+                gp = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gp):
+                    for _ in range(20):
+                        tdh.ep_prefetch_slots(layer.plan, E, R, SK, B, pf_slot, pf_rem, pf_load)
+                gp.replay()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(args.steps):
+                    gp.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                us = round(e0.elapsed_time(e1) * 1e3 / (20 * args.steps), 2)
+                del gp
+            except RuntimeError as exc:
+                print(f"graph capture unavailable: {exc}", file=sys.stderr)
+        prefetch[f"B={B}"] = {"us_per_launch": us,
+                              "replicas_read_from_home": rem if nl > 1 else rem[0],
+                              "max_rank_load_if_pairs_stay_home_over_SK": worst if nl > 1 else worst[0]}
+    del pf_slot, pf_rem, pf_load
+
     # ---- end to end through the public API, pinned host buffers
     e2e = None
     if not args.no_e2e and host_x and nl == 1:
@@ -455,6 +496,7 @@ def run_ours(args, rank, world, local_rank):
         "routing": {"max_vio": max_vio if nl > 1 else max_vio[0], "n_rep": n_rep if nl > 1 else n_rep[0],
                     "replicated_experts": n_chunks if nl > 1 else n_chunks[0]},
         "backward": backward,
+        "prefetch_slots": prefetch,
         "layers_per_step": nl,
         "route_path": args.route,
     }

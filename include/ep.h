@@ -159,6 +159,28 @@ EP_API int ep_plan(const int32_t* loads, int R, int64_t S, int K, int E, int32_t
             int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * Prefetch slots under a per-rank budget B.  [GR] "Το memory contract που
+ * πρέπει να καταλάβει η τεχνική ομάδα": each rank's grouped-GEMM weights are
+ * [E+B, H, H'], rows E..E+B-1 being local prefetch slots, and replicas beyond
+ * the slots read their weights from the home rank (B = E/R for training, 3-4
+ * for inference).  The j-th replica a rank receives, in match order, gets
+ * weight row E + j while j < B, else -1; the token layout is unchanged.
+ *   plan         from ep_plan (device).
+ *   SK           S*K, the pairs per rank.
+ *   slot         [cap] int32 out (device; -1 past n_rep too).
+ *   n_remote     [R] int32 out (device): replicas rank r reads from home.
+ *   load_capped  [R] int64 out (device) or NULL: the other reading of the
+ *                overflow, where a replica without a slot is not made and its
+ *                pairs stay with the expert's home rank; rank r's load is then
+ *                S*K - (pairs of its slotless replicas) + (pairs of slotless
+ *                replicas of its own experts).
+ * One launch, nothing allocated.  EP_ERR_ARG for a bad shape, B < 0 or a
+ * NULL required pointer; EP_ERR_CAPACITY when plan_words is short.
+ */
+EP_API int ep_prefetch_slots(const int32_t* plan, size_t plan_words, int E, int R, int64_t SK, int B,
+                             int32_t* slot, int32_t* n_remote, int64_t* load_capped, cudaStream_t stream);
+
+/*
  * a3. Layout.  [GR] "Online planning, zero copy και στατικά σχήματα": each pair
  * goes straight to its final row, grouped by expert, in a static S*K buffer per
  * rank.  Stable counting sort by expert, ties in flattened (rank, token, k)

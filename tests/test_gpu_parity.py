@@ -163,3 +163,36 @@ def test_grad_reduce(dtype, clear):
         assert rel.max() <= 1e-6
         np.testing.assert_array_equal(cu["g_home"], orc["g_home"])  # same adds, same order
         np.testing.assert_array_equal(cu["g_rep"], orc["g_rep"])    # cleared rows (if asked), others untouched
+
+
+@pytest.mark.parametrize("B", [0, 1, 3, 8])
+def test_prefetch_slots(B):
+    """Slot per replica, remote count and capped loads, bit-exact, on the hand
+    example and the routings of three workloads."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    import oracle as O
+    g = PINS.golden()
+    cases = [(g["R"], g["S"], g["K"], g["E"], 4, np.array(g["topk_ids"], dtype=np.int32))]
+    for cfg in (1, 2, 5):
+        c = W.shape(cfg)
+        cases.append((c["R"], c["S"], c["K"], c["E"], c["block_m"], W.routing(cfg, 0)[0]))
+    for R, S, K, E, block_m, topk in cases:
+        layer = tdh.EpLayer(R, S, K, E, 8, block_m, device="cuda")
+        layer.topk_ids.copy_(torch.from_numpy(topk))
+        layer.route()
+        cap = layer.plan_layout["cap"]
+        slot = torch.full((cap,), -7, dtype=torch.int32, device="cuda")
+        nrem = torch.full((R,), -7, dtype=torch.int32, device="cuda")
+        capped = torch.full((R,), -7, dtype=torch.int64, device="cuda")
+        tdh.ep_prefetch_slots(layer.plan, E, R, S * K, B, slot, nrem, capped)
+        loads, _, _ = O.route_stats(topk, E)
+        pl = O.plan(loads, R, S, K, E)
+        ref, ref_rem, ref_capped = O.prefetch_slots(pl, E, R, B, S * K)
+        got = slot.cpu().numpy()
+        np.testing.assert_array_equal(got[:pl["n_rep"]], ref)
+        assert np.all(got[pl["n_rep"]:] == -1)
+        np.testing.assert_array_equal(nrem.cpu().numpy(), ref_rem)
+        np.testing.assert_array_equal(capped.cpu().numpy(), ref_capped)
+        tdh.ep_prefetch_slots(layer.plan, E, R, S * K, B, slot, nrem)  # load_capped is optional
+        np.testing.assert_array_equal(slot.cpu().numpy()[:pl["n_rep"]], ref)

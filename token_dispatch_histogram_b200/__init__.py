@@ -53,6 +53,7 @@ _SIGS = {
     "ep_route_stats": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
     "ep_route_stats_noalloc": (_I, [_V, _I64, _I, _I, _V, _V, _V, _V]),
     "ep_plan": (_I, [_V, _I, _I64, _I, _I, _V, _SZ, _V, _V]),
+    "ep_prefetch_slots": (_I, [_V, _SZ, _I, _I, _I64, _I, _V, _V, _V, _V]),
     "ep_layout": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _SZ, _V, _SZ, _V, _V, _V, _V, _V]),
     "ep_align_sort": (_I, [_V, _I64, _I, _I, _I, _V, _I64, _V, _I64, _V, _V, _SZ, _V, _V]),
     "ep_route_fused": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _V, _V, _SZ, _V, _V, _V, _I, _V, _I64, _V, _I64, _V,
@@ -157,6 +158,18 @@ def ep_plan(loads, R, S, K, E, plan, dev_status=None, stream=None):
     _dtype(loads, torch.int32)
     _dtype(plan, torch.int32)
     _check("ep_plan", lib().ep_plan(_p(loads), R, S, K, E, _p(plan), plan.numel(), _p(dev_status), _s(stream)))
+
+
+def ep_prefetch_slots(plan, E, R, SK, B, slot, n_remote, load_capped=None, stream=None):
+    """Weight row (E + j or -1) of every replica under a per-rank slot budget B,
+    replicas each rank reads from home, and optionally the rank loads when
+    slotless replicas' pairs stay home."""
+    for t in (plan, slot, n_remote):
+        _dtype(t, torch.int32)
+    if load_capped is not None:
+        _dtype(load_capped, torch.int64)
+    _check("ep_prefetch_slots", lib().ep_prefetch_slots(_p(plan), plan.numel(), E, R, SK, B, _p(slot), _p(n_remote),
+                                                        _p(load_capped), _s(stream)))
 
 
 def ep_layout(topk_ids, E, R, S, plan, ws, pos, src, pair_slot=None, dev_status=None, stream=None):

@@ -39,6 +39,47 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   plan_block(s_loads, R, SK, E, plan, L, work, dev_status);
 }
 
+// Prefetch slots under a per-rank budget B: replica m is the j-th replica its
+// rank receives, j = m - rank_rep_first[rank] (replicas of a rank are
+// consecutive in match order); it gets weight row E + j while j < B, else -1
+// (its weights are read from the home rank).  With load_capped, also the rank
+// loads when a slotless replica's pairs stay with the expert's home rank:
+// integer atomics in shared memory, so the sums do not depend on their order.
+// One CTA: cap = E + R - 1 < 2048.
+__global__ void __launch_bounds__(1024)
+    k_prefetch_slots(const int32_t* __restrict__ plan, EpPlanLayout L, int E, int R, int64_t SK, int B,
+                     int32_t* __restrict__ slot, int32_t* __restrict__ n_remote, int64_t* __restrict__ load_capped) {
+  __shared__ unsigned long long s_load[EP_MAX_RANKS];
+  const int ER = E / R;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    s_load[r] = (unsigned long long)SK;
+    n_remote[r] = max(0, plan[L.rank_nrep + r] - B);
+  }
+  __syncthreads();
+  const int n_rep = min(max(plan[L.n_rep], 0), L.cap);
+  for (int m = threadIdx.x; m < L.cap; m += blockDim.x) {
+    int32_t s = -1;
+    if (m < n_rep) {
+      const int r = plan[L.rep_rank + m];
+      const int e = plan[L.rep_expert + m];
+      if (r >= 0 && r < R && e >= 0 && e < E) {
+        const int j = m - plan[L.rank_rep_first + r];
+        if (j >= 0 && j < B) {
+          s = E + j;
+        } else if (load_capped) {
+          const unsigned long long c = (unsigned long long)(int64_t)plan[L.rep_count + m];
+          atomicAdd(&s_load[r], 0ull - c);
+          atomicAdd(&s_load[e / ER], c);
+        }
+      }
+    }
+    slot[m] = s;
+  }
+  if (!load_capped) return;
+  __syncthreads();
+  for (int r = threadIdx.x; r < R; r += blockDim.x) load_capped[r] = (int64_t)s_load[r];
+}
+
 void plan_layout(int E, int R, EpPlanLayout* L) {
   const int cap = E + R - 1;
   int32_t o = 0;
@@ -93,6 +134,19 @@ extern "C" int ep_plan(const int32_t* loads, int R, int64_t S, int K, int E, int
       cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EP_ERR_CUDA;
   k_plan<<<1, PLAN_THREADS, smem, stream>>>(loads, R, (int32_t)(S * K), E, plan, L, dev_status);
+  count_launch();
+  return launch_status();
+}
+
+extern "C" int ep_prefetch_slots(const int32_t* plan, size_t plan_words, int E, int R, int64_t SK, int B,
+                                 int32_t* slot, int32_t* n_remote, int64_t* load_capped, cudaStream_t stream) {
+  if (!plan || !slot || !n_remote || R < 1 || R > EP_MAX_RANKS || E < 1 || E > EP_MAX_EXPERTS || E % R || B < 0 ||
+      SK < 0)
+    return EP_ERR_ARG;
+  EpPlanLayout L;
+  plan_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  k_prefetch_slots<<<1, 1024, 0, stream>>>(plan, L, E, R, SK, B, slot, n_remote, load_capped);
   count_launch();
   return launch_status();
 }
