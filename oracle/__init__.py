@@ -54,6 +54,14 @@ def _bind(L):
     L.oracle_combine_backward.argtypes = [P, P, P, P, _c.c_int64, _c.c_int, _c.c_int64, P, P]
     L.oracle_prefetch_slots.restype = None
     L.oracle_prefetch_slots.argtypes = [_c.c_int, P, P, P, _c.c_int, _c.c_int, _c.c_int64, _c.c_int, P, P, P]
+    L.oracle_load_matrix.restype = None
+    L.oracle_load_matrix.argtypes = [P, _c.c_int, _c.c_int64, _c.c_int, P]
+    L.oracle_quota_plan_at.restype = _c.c_int
+    L.oracle_quota_plan_at.argtypes = [P, _c.c_int, _c.c_int, _c.c_int64, _c.c_int, P, P, P, P]
+    L.oracle_quota_threshold.restype = _c.c_int64
+    L.oracle_quota_threshold.argtypes = [P, _c.c_int, _c.c_int, _c.c_int64, _c.c_int]
+    L.oracle_quota_layout.restype = _c.c_int
+    L.oracle_quota_layout.argtypes = [P, _c.c_int, _c.c_int64, _c.c_int, _c.c_int, P, P, P, P, P, P, P, P, P, P]
     L.oracle_grad_reduce.restype = None
     L.oracle_grad_reduce.argtypes = [P, P, _c.c_int, _c.c_int64, _c.c_int, P, _c.c_int]
     return L
@@ -227,6 +235,62 @@ def prefetch_slots(pl, E, R, B, SK=0, L=None):
     capped = np.empty(R, dtype=np.int64)
     L.oracle_prefetch_slots(n, _p(re), _p(rr), _p(rc), E, R, SK, B, _p(slot), _p(nrem), _p(capped))
     return slot[:n].copy(), nrem, capped
+
+
+def load_matrix(topk, R, S, K, E, L=None):
+    """int32 [R, E]: pairs of each source rank per expert."""
+    L = L or lib()
+    topk = _i32(topk)
+    Lm = np.empty((R, E), dtype=np.int32)
+    L.oracle_load_matrix(_p(topk), R, S * K, E, _p(Lm))
+    return Lm
+
+
+def quota_plan_at(loads, E, R, tau, B, L=None):
+    """The quota plan at threshold tau (dict), or None when tau is infeasible."""
+    L = L or lib()
+    loads = _i32(loads)
+    cap = E + R - 1
+    re = np.full(cap, -1, dtype=np.int32)
+    rr = np.full(cap, -1, dtype=np.int32)
+    rc = np.zeros(cap, dtype=np.int32)
+    hq = np.zeros(E, dtype=np.int32)
+    n = L.oracle_quota_plan_at(_p(loads), E, R, int(tau), int(B), _p(re), _p(rr), _p(rc), _p(hq))
+    if n < 0:
+        return None
+    return dict(tau=int(tau), n_rep=n, rep_expert=re[:n].copy(), rep_rank=rr[:n].copy(), rep_count=rc[:n].copy(),
+                home_quota=hq)
+
+
+def quota_threshold(loads, E, R, P, B, L=None):
+    L = L or lib()
+    return int(L.oracle_quota_threshold(_p(_i32(loads)), E, R, int(P), int(B)))
+
+
+def quota_plan(loads, R, S, K, E, B, L=None):
+    """Threshold search then the plan at tau*."""
+    tau = quota_threshold(loads, E, R, R * S * K, B, L=L)
+    return quota_plan_at(loads, E, R, tau, B, L=L)
+
+
+def quota_layout(topk, qp, R, S, K, E, L=None):
+    """dict(pos [P], src [P], slot_order, cu_seqlens, rank_load [R], n_local)."""
+    L = L or lib()
+    topk = _i32(topk)
+    P = R * S * K
+    n = qp["n_rep"]
+    pos = np.full(P, -1, dtype=np.int32)
+    src = np.full(P, -1, dtype=np.int32)
+    order = np.empty(E + n, dtype=np.int32)
+    cu = np.empty(E + n + 1, dtype=np.int32)
+    rl = np.empty(R, dtype=np.int32)
+    nl = np.zeros(1, dtype=np.int64)
+    re, rr, rc = (_i32(qp[k]) if n else np.zeros(1, np.int32) for k in ("rep_expert", "rep_rank", "rep_count"))
+    code = L.oracle_quota_layout(_p(topk), R, S * K, E, n, _p(re), _p(rr), _p(rc), _p(_i32(qp["home_quota"])),
+                                 _p(pos), _p(src), _p(order), _p(cu), _p(rl), _p(nl))
+    if code != 0:
+        raise ValueError(f"quota layout failed ({code})")
+    return dict(pos=pos, src=src, slot_order=order, cu_seqlens=cu, rank_load=rl, n_local=int(nl[0]))
 
 
 def bf16_to_f32(u16):

@@ -509,3 +509,272 @@ void oracle_prefetch_slots(int n_rep, const int32_t* rep_expert, const int32_t* 
   }
   free(seen);
 }
+
+/* ----------------------------------------------- 10. quota planner */
+/*
+ * [JA] "その仕組みは高速なエキスパート複製に依存する" (remio.ai UltraEP article):
+ * planning starts from the exact load matrix produced by routing (how many
+ * tokens of each source rank chose each logical expert); a target load
+ * threshold is searched for that keeps every rank below it within the replica
+ * slots available; a quota-driven planner then decides in one step which heavy
+ * experts get copies, on which ranks, and how many tokens each instance takes;
+ * a copy exists only when it is given work; tokens use the capacity of a local
+ * instance before the rest of the demand is sent elsewhere; the aggregated
+ * quotas become per-token destinations by a lookup on cumulative quotas.
+ *
+ * The page prints no formula.  Readings used here:
+ *   - source rank of pair p = p / (S*K); home rank of expert e = e / E_R;
+ *     H_r = sum of T_e over rank r's home experts;
+ *   - at threshold tau, rank r sheds X_r = max(0, H_r - tau) pairs, taken from
+ *     its home experts HEAVIEST FIRST (ties: lower id), chunk = min(T_e, excess
+ *     left); rank r has room C_r = max(0, tau - H_r);
+ *   - chunks (overloaded ranks ascending) are matched to rooms (ranks
+ *     ascending) as in the MoonEP walk, one replica per match, except that a
+ *     rank stops taking pieces once it holds B of them (its slot budget);
+ *     tau is feasible when every chunk is placed;
+ *   - tau* is the smallest feasible tau from ceil(P/R) up (the largest H_r is
+ *     always feasible: nothing is shed);
+ *   - instances of expert e: its home copy, then its replicas in match order;
+ *     instance i on rank r_i with quota q_i first takes its local pairs -- the
+ *     first min(q_i, L[r_i][e]) pairs of e from source rank r_i, in pair order
+ *     -- and the remaining pairs of e, in pair order, fill the instances' left
+ *     quotas by cumulative lookup in instance order;
+ *   - layout: rank r's rows follow rank r-1's (each rank holds its load, at
+ *     most tau*); within a rank, home experts in id order then received
+ *     replicas in match order; within an instance, local pairs then looked-up
+ *     pairs, each in pair order.
+ */
+
+/* Lm[s*E + e] = pairs of source rank s (pairs [s*SK, (s+1)*SK)) routed to e. */
+void oracle_load_matrix(const int32_t* topk, int R, int64_t SK, int E, int32_t* Lm) {
+  for (int64_t i = 0; i < (int64_t)R * E; ++i) Lm[i] = 0;
+  for (int64_t p = 0; p < (int64_t)R * SK; ++p) {
+    int e = topk[p];
+    if (e >= 0 && e < E) Lm[(p / SK) * E + e] += 1;
+  }
+}
+
+/*
+ * The quota plan at threshold tau with at most B replicas per rank.  Returns
+ * n_rep, or -1 when tau is not feasible.  rep_* hold at least E + R - 1 entries.
+ */
+int oracle_quota_plan_at(const int32_t* loads, int E, int R, int64_t tau, int B, int32_t* rep_expert,
+                         int32_t* rep_rank, int32_t* rep_count, int32_t* home_quota) {
+  int ER = E / R;
+  int64_t* H = (int64_t*)calloc((size_t)R, sizeof(int64_t));
+  for (int e = 0; e < E; ++e) H[e / ER] += loads[e];
+
+  /* chunks: overloaded ranks ascending, each rank's experts heaviest first */
+  int32_t* ch_e = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+  int64_t* ch_n = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+  char* used = (char*)calloc((size_t)E, 1);
+  int nch = 0;
+  for (int r = 0; r < R; ++r) {
+    int64_t rem = H[r] - tau;
+    while (rem > 0) {
+      int best = -1;
+      for (int e = r * ER; e < (r + 1) * ER; ++e)
+        if (!used[e] && (best < 0 || loads[e] > loads[best])) best = e;
+      if (best < 0 || loads[best] <= 0) break;
+      used[best] = 1;
+      int64_t take = loads[best] < rem ? loads[best] : rem;
+      ch_e[nch] = best;
+      ch_n[nch] = take;
+      ++nch;
+      rem -= take;
+    }
+  }
+  /* rooms: ranks below tau, ascending */
+  int32_t* rm_r = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+  int64_t* rm_n = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
+  int nrm = 0;
+  for (int r = 0; r < R; ++r) {
+    if (tau - H[r] > 0) {
+      rm_r[nrm] = r;
+      rm_n[nrm] = tau - H[r];
+      ++nrm;
+    }
+  }
+  /* the walk; a room closes when full or when it holds B pieces */
+  int nrep = 0, i = 0, j = 0, pieces = 0;
+  int64_t left_c = nch ? ch_n[0] : 0, left_r = nrm ? rm_n[0] : 0;
+  if (B <= 0) j = nrm; /* no slot anywhere */
+  while (i < nch && j < nrm) {
+    int64_t take = left_c < left_r ? left_c : left_r;
+    rep_expert[nrep] = ch_e[i];
+    rep_rank[nrep] = rm_r[j];
+    rep_count[nrep] = (int32_t)take;
+    ++nrep;
+    ++pieces;
+    left_c -= take;
+    left_r -= take;
+    if (left_c == 0) {
+      ++i;
+      if (i < nch) left_c = ch_n[i];
+    }
+    if (left_r == 0 || pieces == B) {
+      ++j;
+      pieces = 0;
+      if (j < nrm) left_r = rm_n[j];
+    }
+  }
+  int ok = (i == nch);
+  if (ok) {
+    for (int e = 0; e < E; ++e) home_quota[e] = loads[e];
+    for (int m = 0; m < nrep; ++m) home_quota[rep_expert[m]] -= rep_count[m];
+  }
+  free(H);
+  free(ch_e);
+  free(ch_n);
+  free(used);
+  free(rm_r);
+  free(rm_n);
+  return ok ? nrep : -1;
+}
+
+/* tau*: the smallest feasible threshold from ceil(P/R) up. */
+int64_t oracle_quota_threshold(const int32_t* loads, int E, int R, int64_t P, int B) {
+  int cap = E + R - 1;
+  int32_t* a = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  int32_t* b = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  int32_t* c = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  int32_t* h = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+  int64_t tau = (P + R - 1) / R;
+  while (oracle_quota_plan_at(loads, E, R, tau, B, a, b, c, h) < 0) ++tau;
+  free(a);
+  free(b);
+  free(c);
+  free(h);
+  return tau;
+}
+
+/*
+ * Per-pair destinations of a quota plan.  pos[p] = row of pair p, src[row] = p,
+ * slot_order / cu_seqlens over the E + n_rep slots in buffer order (slot id e
+ * for e's home copy, E + m for replica m), rank_load[r] = rows of rank r,
+ * *n_local = pairs placed on their own source rank.  Returns 0, -1 when an
+ * expert would have two instances on one rank or a quota goes negative, -2 on
+ * an expert id outside [0, E).
+ */
+int oracle_quota_layout(const int32_t* topk, int R, int64_t SK, int E, int n_rep, const int32_t* rep_expert,
+                        const int32_t* rep_rank, const int32_t* rep_count, const int32_t* home_quota, int32_t* pos,
+                        int32_t* src, int32_t* slot_order, int32_t* cu_seqlens, int32_t* rank_load,
+                        int64_t* n_local) {
+  int ER = E / R;
+  int64_t P = (int64_t)R * SK;
+  int n_inst = E + n_rep;
+  for (int64_t p = 0; p < P; ++p)
+    if (topk[p] < 0 || topk[p] >= E) return -2;
+  int32_t* Lm = (int32_t*)malloc(sizeof(int32_t) * (size_t)R * (size_t)E);
+  oracle_load_matrix(topk, R, SK, E, Lm);
+
+  int32_t* ie = (int32_t*)malloc(sizeof(int32_t) * (size_t)n_inst); /* expert */
+  int32_t* ir = (int32_t*)malloc(sizeof(int32_t) * (size_t)n_inst); /* rank */
+  int64_t* iq = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_inst); /* quota */
+  int64_t* il = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_inst); /* local pairs */
+  int64_t* ic = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_inst); /* cumulative left quota before it */
+  int64_t* ib = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_inst); /* first row */
+  int32_t* at = (int32_t*)malloc(sizeof(int32_t) * (size_t)E * (size_t)R); /* instance of e on r */
+  int32_t* lst = (int32_t*)malloc(sizeof(int32_t) * (size_t)n_inst);        /* instances grouped by expert */
+  int32_t* lst_off = (int32_t*)calloc((size_t)E + 1, sizeof(int32_t));
+  int64_t* seen_se = (int64_t*)calloc((size_t)R * (size_t)E, sizeof(int64_t));
+  int64_t* seen_e = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+  int64_t* rl = (int64_t*)calloc((size_t)R, sizeof(int64_t));
+  int rc = 0;
+
+  for (int e = 0; e < E; ++e) {
+    ie[e] = e;
+    ir[e] = e / ER;
+    iq[e] = home_quota[e];
+  }
+  for (int m = 0; m < n_rep; ++m) {
+    ie[E + m] = rep_expert[m];
+    ir[E + m] = rep_rank[m];
+    iq[E + m] = rep_count[m];
+  }
+  for (int64_t k = 0; k < (int64_t)E * R; ++k) at[k] = -1;
+  for (int i = 0; i < n_inst; ++i) {
+    if (iq[i] < 0 || at[ie[i] * R + ir[i]] >= 0) rc = -1;
+    at[ie[i] * R + ir[i]] = i;
+    il[i] = iq[i] < Lm[ir[i] * E + ie[i]] ? iq[i] : Lm[ir[i] * E + ie[i]];
+    lst_off[ie[i] + 1] += 1;
+  }
+  if (rc == 0) {
+    /* instance lists per expert: home first, then replicas in match order */
+    for (int e = 0; e < E; ++e) lst_off[e + 1] += lst_off[e];
+    int32_t* fill = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+    for (int i = 0; i < n_inst; ++i) lst[lst_off[ie[i]] + fill[ie[i]]++] = i;
+    free(fill);
+    for (int e = 0; e < E; ++e) {
+      int64_t run = 0;
+      for (int k = lst_off[e]; k < lst_off[e + 1]; ++k) {
+        ic[lst[k]] = run;
+        run += iq[lst[k]] - il[lst[k]];
+      }
+    }
+    /* rows: ranks in order; home experts by id, then received replicas by m */
+    for (int i = 0; i < n_inst; ++i) rl[ir[i]] += iq[i];
+    int64_t row = 0;
+    int ns = 0;
+    cu_seqlens[0] = 0;
+    for (int r = 0; r < R; ++r) {
+      for (int e = r * ER; e < (r + 1) * ER; ++e) {
+        ib[e] = row;
+        row += iq[e];
+        slot_order[ns] = e;
+        cu_seqlens[++ns] = (int32_t)row;
+      }
+      for (int m = 0; m < n_rep; ++m) {
+        if (rep_rank[m] != r) continue;
+        ib[E + m] = row;
+        row += iq[E + m];
+        slot_order[ns] = E + m;
+        cu_seqlens[++ns] = (int32_t)row;
+      }
+      rank_load[r] = (int32_t)rl[r];
+    }
+    /* pairs in order: local first, then the cumulative-quota lookup */
+    *n_local = 0;
+    for (int64_t p = 0; p < P; ++p) {
+      int e = topk[p];
+      int s = (int)(p / SK);
+      int64_t ls = seen_se[(int64_t)s * E + e]++;
+      int i = at[e * R + s];
+      int64_t r;
+      if (i >= 0 && ls < il[i]) {
+        r = ib[i] + ls;
+        *n_local += 1;
+      } else {
+        int64_t jj = seen_e[e]++;
+        r = -1;
+        for (int k = lst_off[e]; k < lst_off[e + 1]; ++k) {
+          int c = lst[k];
+          if (jj >= ic[c] && jj < ic[c] + (iq[c] - il[c])) {
+            r = ib[c] + il[c] + (jj - ic[c]);
+            break;
+          }
+        }
+        if (r < 0) {
+          rc = -1;
+          break;
+        }
+      }
+      pos[p] = (int32_t)r;
+      src[r] = (int32_t)p;
+    }
+  }
+  free(Lm);
+  free(ie);
+  free(ir);
+  free(iq);
+  free(il);
+  free(ic);
+  free(ib);
+  free(at);
+  free(lst);
+  free(lst_off);
+  free(seen_se);
+  free(seen_e);
+  free(rl);
+  return rc;
+}

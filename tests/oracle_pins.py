@@ -27,6 +27,7 @@ import oracle as O
 import workload as W
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_example_4rank.json")
+QUOTA_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quota_hand_example_4rank.json")
 
 
 def golden():
@@ -567,6 +568,145 @@ def pin_prefetch_slots(L):
         assert O.prefetch_slots(pl, E, R, E + R, SK, L=L)[2].tolist() == [SK] * R
 
 
+# ------------------------------------------------------- quota planner
+
+def pin_quota_hand_example(L):
+    g = golden()
+    with open(QUOTA_GOLDEN) as f:
+        q = json.load(f)
+    R, S, K, E = g["R"], g["S"], g["K"], g["E"]
+    topk = np.array(g["topk_ids"], dtype=np.int32)
+    assert O.load_matrix(topk, R, S, K, E, L=L).tolist() == q["load_matrix"]
+    loads = np.array(g["loads"], dtype=np.int32)
+    for key, B in (("B1", 1), ("B2", 2), ("B0", 0)):
+        want = q[key]
+        qp = O.quota_plan(loads, R, S, K, E, B, L=L)
+        assert qp["tau"] == want["tau"], (key, qp["tau"])
+        reps = [[int(a), int(b), int(c)] for a, b, c in zip(qp["rep_expert"], qp["rep_rank"], qp["rep_count"])]
+        assert reps == want["replicas"], (key, reps)
+        if "home_quota" in want:
+            assert qp["home_quota"].tolist() == want["home_quota"]
+        lo = O.quota_layout(topk, qp, R, S, K, E, L=L)
+        assert lo["rank_load"].tolist() == want["rank_load"]
+        assert lo["n_local"] == want["n_local"]
+        for name in ("pos", "slot_order", "cu_seqlens"):
+            if name in want:
+                assert lo[name].tolist() == want[name], (key, name)
+
+
+def pin_quota_threshold_closed_forms(L):
+    """R = 2: one rank sheds, the other takes every chunk as one piece, so tau is
+    feasible iff the B heaviest experts of the heavier rank cover its excess:
+    tau* = max(ceil(P/2), H_o - (sum of its B largest loads)).  Any R: B = 0
+    leaves only tau = max H_r (nothing shed); unlimited slots make ceil(P/R)
+    feasible (the rooms then hold at least the excess)."""
+    rng = np.random.default_rng(31)
+    for it in range(300):
+        R = 2 if it < 200 else int(rng.choice([3, 4, 8]))
+        ER = int(rng.integers(1, 6))
+        E = R * ER
+        P = int(rng.integers(1, 200))
+        loads = rng.multinomial(P, rng.dirichlet(np.full(E, rng.uniform(0.1, 3.0)))).astype(np.int32)
+        H = loads.reshape(R, ER).sum(axis=1)
+        lo = -(-P // R)
+        B = int(rng.integers(0, ER + 2))
+        if R == 2:
+            o = int(np.argmax(H))
+            top = int(np.sort(loads[o * ER:(o + 1) * ER])[::-1][:B].sum())
+            assert O.quota_threshold(loads, E, R, P, B, L=L) == max(lo, int(H[o]) - top), (loads.tolist(), B)
+        assert O.quota_threshold(loads, E, R, P, 0, L=L) == max(lo, int(H.max()))
+        assert O.quota_threshold(loads, E, R, P, E + R, L=L) == lo
+
+
+def _quota_case(rng, it):
+    R = int(rng.choice([1, 2, 3, 4, 8]))
+    ER = int(rng.integers(1, 5))
+    E = R * ER
+    S = int(rng.integers(1, 24))
+    K = int(rng.integers(1, min(E, 4) + 1))
+    bias = rng.normal(0.0, rng.uniform(0.0, 3.0), E).astype(np.float32)
+    topk, _ = W.routing_from(R * S, E, K, seed=500 + it, bias_e=bias)
+    return R, S, K, E, ER, topk
+
+
+def pin_quota_invariants(L):
+    """What the page states (every rank at or under the threshold, copies only
+    with work, a replica budget per rank, local instances first, routing
+    unchanged), checked on random routings with numpy doing the counting."""
+    rng = np.random.default_rng(32)
+    for it in range(80):
+        R, S, K, E, ER, topk = _quota_case(rng, it)
+        SK, P = S * K, R * S * K
+        loads = np.bincount(topk.ravel(), minlength=E).astype(np.int32)
+        H = loads.reshape(R, ER).sum(axis=1)
+        B = int(rng.integers(0, 4))
+        qp = O.quota_plan(loads, R, S, K, E, B, L=L)
+        tau, n = qp["tau"], qp["n_rep"]
+        re, rr, rc, hq = qp["rep_expert"], qp["rep_rank"], qp["rep_count"], qp["home_quota"]
+        assert -(-P // R) <= tau <= max(-(-P // R), int(H.max()))
+        assert np.all(rc > 0) and np.all(hq >= 0)
+        assert np.all(np.bincount(rr, minlength=R) <= B)
+        assert all(H[rr[m]] < tau and H[re[m] // ER] > tau for m in range(n))
+        assert np.array_equal(hq + np.bincount(re, weights=rc, minlength=E).astype(np.int64), loads)
+        assert O.quota_plan_at(loads, E, R, tau - 1, B, L=L) is None or tau == -(-P // R)
+        lo = O.quota_layout(topk, qp, R, S, K, E, L=L)
+        pos, src = lo["pos"], lo["src"]
+        assert np.array_equal(np.sort(pos), np.arange(P)) and np.array_equal(src[pos], np.arange(P))
+        order, cu = lo["slot_order"], lo["cu_seqlens"]
+        q = np.diff(cu)
+        slot_e = np.where(order < E, order, re[np.maximum(order - E, 0)] if n else order)
+        slot_r = np.where(order < E, order // ER, rr[np.maximum(order - E, 0)] if n else order // ER)
+        row_slot = np.repeat(np.arange(len(order)), q)
+        assert np.array_equal(slot_e[row_slot[pos]], topk.ravel())  # routing unchanged
+        row_rank = slot_r[row_slot]
+        assert np.all(np.diff(row_rank) >= 0)  # ranks in order
+        assert np.array_equal(np.bincount(row_rank, minlength=R), lo["rank_load"])
+        assert np.all(lo["rank_load"] <= tau) and lo["rank_load"].sum() == P
+        for r in range(R):  # home experts by id, then received replicas by match order
+            mine = order[slot_r == r]
+            homes = mine[mine < E]
+            assert homes.tolist() == list(range(r * ER, (r + 1) * ER))
+            assert mine[ER:].tolist() == sorted(mine[ER:].tolist()) and np.all(mine[ER:] >= E)
+        Lm = np.zeros((R, E), dtype=np.int64)
+        np.add.at(Lm, (np.arange(P) // SK, topk.ravel()), 1)
+        want_local = 0
+        for i, sid in enumerate(order):
+            ps = src[cu[i]:cu[i + 1]]
+            e, r = slot_e[i], slot_r[i]
+            nloc = int(min(q[i], Lm[r, e]))
+            want_local += nloc
+            assert np.all(ps[:nloc] // SK == r)  # local pairs first
+            assert np.all(np.diff(ps[:nloc]) > 0) and np.all(np.diff(ps[nloc:]) > 0)
+        assert lo["n_local"] == want_local == int(np.sum(row_rank[pos] == np.arange(P) // SK))
+        for e in range(E):  # the looked-up pairs of e, instance after instance, are e's other pairs in order
+            inst = [i for i in range(len(order)) if slot_e[i] == e]
+            inst.sort(key=lambda i: (order[i] >= E, order[i]))
+            rest = np.concatenate([src[cu[i] + int(min(q[i], Lm[slot_r[i], e])):cu[i + 1]] for i in inst])
+            local = set(np.concatenate([src[cu[i]:cu[i] + int(min(q[i], Lm[slot_r[i], e]))] for i in inst]).tolist())
+            mine = [p for p in np.flatnonzero(topk.ravel() == e).tolist() if p not in local]
+            assert rest.tolist() == mine
+
+
+def pin_quota_no_replica_is_a_sort(L):
+    """B = 0: no copy, so the layout is a stable sort by (expert, pair not from
+    the expert's home rank) -- numpy's lexsort."""
+    rng = np.random.default_rng(33)
+    for it in range(40):
+        R, S, K, E, ER, topk = _quota_case(rng, 100 + it)
+        SK, P = S * K, R * S * K
+        loads = np.bincount(topk.ravel(), minlength=E).astype(np.int32)
+        qp = O.quota_plan(loads, R, S, K, E, 0, L=L)
+        assert qp["n_rep"] == 0
+        lo = O.quota_layout(topk, qp, R, S, K, E, L=L)
+        e = topk.ravel()
+        p = np.arange(P)
+        order = np.lexsort((p, (p // SK) != (e // ER), e))
+        want = np.empty(P, dtype=np.int64)
+        want[order] = p
+        assert np.array_equal(lo["pos"], want)
+
+
 ALL_PINS = [pin_hand_example, pin_max_vio_closed_forms, pin_plan_unit_restatement, pin_layout_brute_force,
             pin_layout_library_reductions, pin_layout_invariants, pin_align_sort, pin_dispatch, pin_combine,
-            pin_grad_reduce, pin_dispatch_backward, pin_combine_backward, pin_prefetch_slots]
+            pin_grad_reduce, pin_dispatch_backward, pin_combine_backward, pin_prefetch_slots, pin_quota_hand_example,
+            pin_quota_threshold_closed_forms, pin_quota_invariants, pin_quota_no_replica_is_a_sort]

@@ -54,6 +54,18 @@ MUTANTS = [
      "        if (k > 0) acc = acc + bf16_to_f32(dbuf[(int64_t)row * H + h]);"),
     ("combine_bwd_weight_index", "dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K + k] * g);",
      "dy[(int64_t)row * H + h] = f32_to_bf16(w[t * K] * g);"),
+    ("quota_ties_to_higher_id", "if (!used[e] && (best < 0 || loads[e] > loads[best])) best = e;",
+     "if (!used[e] && (best < 0 || loads[e] >= loads[best])) best = e;"),
+    ("quota_descending_id_chunks", "if (!used[e] && (best < 0 || loads[e] > loads[best])) best = e;",
+     "if (!used[e] && (best < 0 || e > best)) best = e;"),
+    ("quota_no_slot_budget", "if (left_r == 0 || pieces == B) {", "if (left_r == 0) {"),
+    ("quota_zero_rooms", "if (tau - H[r] > 0) {\n      rm_r[nrm] = r;", "if (tau - H[r] >= 0) {\n      rm_r[nrm] = r;"),
+    ("quota_scan_from_above", "int64_t tau = (P + R - 1) / R;", "int64_t tau = (P + R - 1) / R + 1;"),
+    ("quota_no_locality", "if (i >= 0 && ls < il[i]) {", "if (i >= 0 && ls < 0) {"),
+    ("quota_local_not_capped", "il[i] = iq[i] < Lm[ir[i] * E + ie[i]] ? iq[i] : Lm[ir[i] * E + ie[i]];",
+     "il[i] = Lm[ir[i] * E + ie[i]];"),
+    ("quota_lookup_off_by_one", "if (jj >= ic[c] && jj < ic[c] + (iq[c] - il[c])) {",
+     "if (jj > ic[c] && jj <= ic[c] + (iq[c] - il[c])) {"),
     ("capped_home_by_mod", "load_capped[rep_expert[m] / ER]", "load_capped[rep_expert[m] % R]"),
     ("prefetch_slot_off_by_one", "    if (j < B) {\n      slot[m] = E + j;", "    if (j <= B) {\n      slot[m] = E + j;"),
     ("combine_bwd_dw_wrong_row", "s += (double)g * (double)bf16_to_f32(y[(int64_t)row * H + h]);",
