@@ -109,6 +109,36 @@ typedef struct {
                          entries from E + n_rep on hold R*S*K */
 } EpPlanLayout;
 
+/*
+ * Layout of the quota-plan buffer written by ep_quota_route: offsets in int32
+ * elements into one int32 array, each region 32-byte aligned.  Instance i of
+ * the plan is the home copy of expert i for i < E and replica i - E after.
+ */
+typedef struct {
+  int64_t words;          /* total size in int32 elements */
+  int32_t cap;            /* E + R - 1 */
+  int32_t tau;            /* [1] tau*, the rank-load threshold met (-1: no plan) */
+  int32_t n_rep;          /* [1] number of replicas */
+  int32_t n_local;        /* [1] pairs placed on their own source rank */
+  int32_t rank_load;      /* [R] rows of rank r (<= tau) */
+  int32_t rank_off;       /* [R] first buffer row of rank r */
+  int32_t rank_nrep;      /* [R] replicas received by rank r */
+  int32_t rank_rep_first; /* [R] replicas received by ranks < r */
+  int32_t home_quota;     /* [E] pairs taken by the home copy of e */
+  int32_t rep_first;      /* [E] match index of e's first replica (0 if none) */
+  int32_t rep_cnt;        /* [E] number of replicas of e */
+  int32_t rep_expert;     /* [cap] logical expert of replica m (match order) */
+  int32_t rep_rank;       /* [cap] receiving rank of replica m */
+  int32_t rep_count;      /* [cap] quota of replica m */
+  int32_t inst_local;     /* [E + cap] local pairs of instance i: min(quota, L[rank][e]) */
+  int32_t inst_cum;       /* [E + cap] looked-up pairs of e's earlier instances */
+  int32_t inst_base;      /* [E + cap] first buffer row of instance i */
+  int32_t inst_lpre;      /* [E + cap] pairs of e from source ranks below instance i's rank */
+  int32_t slot_order;     /* [E + cap] instance ids in buffer order; -1 past E + n_rep */
+  int32_t cu_seqlens;     /* [E + cap + 1] first row of each slot in buffer order;
+                             entries from E + n_rep on hold R*S*K */
+} EpQuotaLayout;
+
 /* Library version string (host). */
 EP_API const char* ep_version(void);
 
@@ -157,6 +187,52 @@ EP_API int ep_route_stats(const int32_t* topk_ids, int64_t T, int K, int E, int3
  */
 EP_API int ep_plan(const int32_t* loads, int R, int64_t S, int K, int E, int32_t* plan, size_t plan_words,
             int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Quota-driven replica planning with a per-rank replica budget.  [JA]
+ * "その仕組みは高速なエキスパート複製に依存する" (remio.ai UltraEP article):
+ * from the exact load matrix after routing (pairs of each source rank per
+ * expert), a load threshold is searched for that every rank can stay under
+ * within the replica slots available; the planner decides which heavy experts
+ * get copies, on which ranks, and how many pairs each instance takes; copies
+ * exist only with work; pairs use a local instance first and the rest of the
+ * demand is placed by lookup on cumulative quotas; all on the GPU.
+ * Rule (this library's reading; the page prints none):
+ *   - source rank of pair p = p / (S*K); home rank of e = e / (E/R); H_r = the
+ *     loads of rank r's home experts;
+ *   - at threshold tau, rank r sheds max(0, H_r - tau) pairs from its home
+ *     experts heaviest first (ties: lower id), each chunk = min(T_e, excess
+ *     left); ranks with H_r < tau take pieces in ascending rank order (one
+ *     replica per piece) until full or holding B pieces; tau is feasible when
+ *     every chunk is placed;
+ *   - tau* = the smallest feasible tau from ceil(P/R) up (max H_r always is);
+ *   - instances of e: home, then its replicas in match order.  Instance i on
+ *     rank r_i takes the first min(q_i, L[r_i][e]) pairs of e from source rank
+ *     r_i; the other pairs of e, in pair order, fill the instances' remaining
+ *     quotas in instance order;
+ *   - rows: rank after rank (rank r holds rank_load[r] <= tau* rows); within a
+ *     rank home experts by id then received replicas by match order; within an
+ *     instance its local pairs then its looked-up pairs, each in pair order.
+ * Arguments:
+ *   topk_ids [T, K] int32 device, T = R*S.
+ *   B        replicas a rank may hold (>= 0).
+ *   loads    [E] int32 device out: T_e.
+ *   plan     int32 device out, layout from ep_quota_plan_layout.
+ *   pos, src [T*K] int32 device out: row of each pair, pair of each row.
+ *   ws       device scratch of ep_quota_workspace_size bytes (contents need
+ *            not be initialised).
+ * Four launches (rank-aligned tile histogram, column scan, threshold search
+ * over all candidates at once, stable-rank walk); integer work only, so the
+ * result does not depend on scheduling.  EP_ERR_ARG for bad shapes (E % R,
+ * K > E, ...) or B < 0; EP_ERR_CAPACITY when plan_words or ws_bytes is short.
+ * Expert ids outside [0, E) set EP_DEV_BAD_EXPERT_ID and leave tau = -1 and
+ * pos = -1.
+ */
+EP_API int ep_quota_workspace_size(int64_t T, int K, int E, int R, size_t* bytes /* host out */);
+EP_API int ep_quota_plan_layout(int E, int R, EpQuotaLayout* layout /* host out */);
+EP_API int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int B, int32_t* loads,
+                          int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src, void* ws, size_t ws_bytes,
+                          int32_t* dev_status, cudaStream_t stream);
 
 /*
  * Prefetch slots under a per-rank budget B.  [GR] "Το memory contract που

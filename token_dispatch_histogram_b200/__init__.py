@@ -42,6 +42,14 @@ class EpPlanLayout(ctypes.Structure):
                                       "rep_begin", "rep_base", "rep_experts", "slot_order", "cu_seqlens")]
 
 
+class EpQuotaLayout(ctypes.Structure):
+    _fields_ = [("words", ctypes.c_int64), ("cap", ctypes.c_int32)] + [
+        (n, ctypes.c_int32) for n in ("tau", "n_rep", "n_local", "rank_load", "rank_off", "rank_nrep",
+                                      "rank_rep_first", "home_quota", "rep_first", "rep_cnt", "rep_expert", "rep_rank",
+                                      "rep_count", "inst_local", "inst_cum", "inst_base", "inst_lpre", "slot_order",
+                                      "cu_seqlens")]
+
+
 _lib = None
 _V, _I, _I64, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 
@@ -53,6 +61,9 @@ _SIGS = {
     "ep_route_stats": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
     "ep_route_stats_noalloc": (_I, [_V, _I64, _I, _I, _V, _V, _V, _V]),
     "ep_plan": (_I, [_V, _I, _I64, _I, _I, _V, _SZ, _V, _V]),
+    "ep_quota_workspace_size": (_I, [_I64, _I, _I, _I, _V]),
+    "ep_quota_plan_layout": (_I, [_I, _I, _V]),
+    "ep_quota_route": (_I, [_V, _I64, _I, _I, _I, _I64, _I, _V, _V, _SZ, _V, _V, _V, _SZ, _V, _V]),
     "ep_prefetch_slots": (_I, [_V, _SZ, _I, _I, _I64, _I, _V, _V, _V, _V]),
     "ep_layout": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _SZ, _V, _SZ, _V, _V, _V, _V, _V]),
     "ep_align_sort": (_I, [_V, _I64, _I, _I, _I, _V, _I64, _V, _I64, _V, _V, _SZ, _V, _V]),
@@ -158,6 +169,29 @@ def ep_plan(loads, R, S, K, E, plan, dev_status=None, stream=None):
     _dtype(loads, torch.int32)
     _dtype(plan, torch.int32)
     _check("ep_plan", lib().ep_plan(_p(loads), R, S, K, E, _p(plan), plan.numel(), _p(dev_status), _s(stream)))
+
+
+def ep_quota_workspace_size(T, K, E, R):
+    n = ctypes.c_size_t(0)
+    _check("ep_quota_workspace_size", lib().ep_quota_workspace_size(T, K, E, R, ctypes.byref(n)))
+    return int(n.value)
+
+
+def ep_quota_plan_layout(E, R):
+    L = EpQuotaLayout()
+    _check("ep_quota_plan_layout", lib().ep_quota_plan_layout(E, R, ctypes.byref(L)))
+    return {name: getattr(L, name) for name, _ in EpQuotaLayout._fields_}
+
+
+def ep_quota_route(topk_ids, E, R, S, B, loads, plan, pos, src, ws, dev_status=None, stream=None):
+    """Quota-driven replica plan under a per-rank replica budget B, and the
+    local-first per-pair layout (see ep.h)."""
+    for t in (topk_ids, loads, plan, pos, src):
+        _dtype(t, torch.int32)
+    T, K = topk_ids.shape
+    _check("ep_quota_route", lib().ep_quota_route(_p(topk_ids), T, K, E, R, S, B, _p(loads), _p(plan), plan.numel(),
+                                                  _p(pos), _p(src), _p(ws), ws.numel() * ws.element_size(),
+                                                  _p(dev_status), _s(stream)))
 
 
 def ep_prefetch_slots(plan, E, R, SK, B, slot, n_remote, load_capped=None, stream=None):

@@ -232,4 +232,22 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return base + x - v;
 }
 
+// Block-wide exclusive scan of a[0..n) in shared memory (any n), in place;
+// returns the total.  Each thread scans a contiguous segment.
+__device__ __forceinline__ int32_t block_scan_array(int32_t* a, int n, int32_t* warp_sums) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int b = threadIdx.x * per, e = min(n, b + per);
+  int32_t s = 0;
+  for (int i = b; i < e; ++i) s += a[i];
+  int32_t total;
+  int32_t run = block_exclusive_scan(s, warp_sums, &total);
+  for (int i = b; i < e; ++i) {
+    const int32_t v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  __syncthreads();
+  return total;
+}
+
 }  // namespace ep

@@ -17,75 +17,12 @@
 // first row.  Outputs pos (pair -> row), src (row -> pair), pair_slot.
 // Align & Sort ([ZH] MoE Align & Sort report): groups padded to block_m;
 // sorted_token_ids[off_e + rank] = p; padding and tail hold the sentinel P.
-#include "common.cuh"
+#include "tile_ranks.cuh"
 
 namespace ep {
 
 int run_hist(const int32_t* topk, int64_t P, int E, void* ws, int32_t* loads, double* max_vio, int32_t* dev_status,
              cudaStream_t st);
-
-constexpr int SCAT_THREADS = 512;
-constexpr int SCAT_WARPS = SCAT_THREADS / 32;
-
-// Stable ranks of the pairs of tile `t`; calls emit(p, e, g) for every valid
-// pair (g = rank of p among all pairs of expert e) and bad(p) for pairs whose
-// id is outside [0, E).  s_ids: [tile] ints, s_whist: [SCAT_WARPS][E] ints.
-template <class Emit, class Bad>
-__device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ topk, int64_t P, int E, int tile, int t,
-                                                  const int32_t* __restrict__ tile_excl, int32_t* s_ids,
-                                                  int32_t* s_whist, Emit emit, Bad bad) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t p0 = (int64_t)t * tile;
-  const int n = (int)min((int64_t)tile, P - p0);
-  for (int i = threadIdx.x; i < tile; i += blockDim.x) {
-    int e = -1;
-    if (i < n) {
-      e = __ldg(topk + p0 + i);
-      if (e < 0 || e >= E) e = -2;  // invalid id (reported by bad())
-    }
-    s_ids[i] = e;
-  }
-  for (int i = threadIdx.x; i < SCAT_WARPS * E; i += blockDim.x) s_whist[i] = 0;
-  __syncthreads();
-
-  const int sub = tile / SCAT_WARPS;  // pairs per warp, a multiple of 32
-  const int nbits = key_bits(E + 2);  // keys e + 2: -2 (invalid id), -1 (past the end), experts
-  int32_t* my = s_whist + warp * E;
-  for (int c = 0; c < sub; c += 32) {
-    const int e = s_ids[warp * sub + c + lane];
-    const uint32_t peers = warp_match((uint32_t)(e + 2), nbits);
-    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t run = tile_excl[(int64_t)t * E + e];
-#pragma unroll 4
-    for (int w = 0; w < SCAT_WARPS; ++w) {
-      const int32_t c = s_whist[w * E + e];
-      s_whist[w * E + e] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  const uint32_t lt = lanemask_lt();
-  for (int c = 0; c < sub; c += 32) {
-    const int i = warp * sub + c + lane;
-    const int e = s_ids[i];
-    const uint32_t peers = warp_match((uint32_t)(e + 2), nbits);
-    int32_t base = 0;
-    if (e >= 0) base = my[e];
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) my[e] = base + __popc(peers);
-    __syncwarp();
-    if (i < n) {
-      if (e >= 0)
-        emit(p0 + i, e, base + __popc(peers & lt));
-      else
-        bad(p0 + i);
-    }
-  }
-}
 
 __global__ void __launch_bounds__(SCAT_THREADS)
     k_layout(const int32_t* __restrict__ topk, int64_t P, int E, int tile, const int32_t* __restrict__ tile_excl,
@@ -154,27 +91,11 @@ __global__ void __launch_bounds__(SCAT_THREADS)
     pos[p] = -1;
     if (pair_slot) pair_slot[p] = -1;
   };
-  tile_stable_ranks(topk, P, E, tile, blockIdx.x, tile_excl, s_ids, s_whist, emit, bad);
+  const int64_t p0 = (int64_t)blockIdx.x * tile;
+  tile_stable_ranks(topk, E, tile, p0, (int)min((int64_t)tile, P - p0), tile_excl + (int64_t)blockIdx.x * E, s_ids,
+                    s_whist, emit, bad);
   __syncthreads();
   if (threadIdx.x == 0 && s_flags) flag(dev_status, s_flags);
-}
-
-// Block-wide exclusive scan of a[0..n) in shared memory (any n), in place;
-// returns the total.  Each thread scans a contiguous segment.
-__device__ int32_t block_scan_array(int32_t* a, int n, int32_t* warp_sums) {
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int b = threadIdx.x * per, e = min(n, b + per);
-  int32_t s = 0;
-  for (int i = b; i < e; ++i) s += a[i];
-  int32_t total;
-  int32_t run = block_exclusive_scan(s, warp_sums, &total);
-  for (int i = b; i < e; ++i) {
-    const int32_t v = a[i];
-    a[i] = run;
-    run += v;
-  }
-  __syncthreads();
-  return total;
 }
 
 __global__ void __launch_bounds__(SCAT_THREADS)
@@ -202,7 +123,11 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   auto emit = [&](int64_t p, int e, int32_t g) { sorted_ids[s_off[e] + g] = (int32_t)p; };
   auto bad = [&](int64_t) { atomicOr(&s_flags, EP_DEV_BAD_EXPERT_ID); };
   const int ntiles = (int)((P + tile - 1) / tile);
-  if ((int)blockIdx.x < ntiles) tile_stable_ranks(topk, P, E, tile, blockIdx.x, tile_excl, s_ids, s_whist, emit, bad);
+  if ((int)blockIdx.x < ntiles) {
+    const int64_t p0 = (int64_t)blockIdx.x * tile;
+    tile_stable_ranks(topk, E, tile, p0, (int)min((int64_t)tile, P - p0), tile_excl + (int64_t)blockIdx.x * E, s_ids,
+                      s_whist, emit, bad);
+  }
   __syncthreads();
   // padding of each group, the tail past the padded total, and expert_ids
   const int32_t sentinel = (int32_t)P;
