@@ -57,6 +57,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the backward of dispatch and combine")
+    ap.add_argument("--no-quota", action="store_true", help="skip timing the quota-driven planner")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the eager per-op pass only (default: the headline value comes from replaying the "
                          "step as one captured CUDA graph; the per-op breakdown from the eager pass)")
@@ -384,6 +385,82 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device status {st:#x} in the backward timing")
         del dy, dx, dw
 
+    # ---- the quota-driven planner (a per-rank replica budget B) in place of
+    # the exact-S*K plan: the same step (route, dispatch, combine, replica
+    # gradients) and the route alone, each as one captured graph, replayed
+    quota = {}
+    if not args.no_graph and not args.no_quota:
+        q_lay = tdh.ep_quota_plan_layout(E, R)
+        q_plans = [torch.zeros(q_lay["words"], dtype=torch.int32, device=dev) for _ in layers]
+        q_loads = torch.zeros(E, dtype=torch.int32, device=dev)
+        q_pos = torch.zeros(P, dtype=torch.int32, device=dev)
+        q_src = torch.zeros(P, dtype=torch.int32, device=dev)
+        q_ws = torch.zeros(tdh.ep_quota_workspace_size(T, K, E, R), dtype=torch.uint8, device=dev)
+
+        def q_route(B, li, ly):
+            tdh.ep_quota_route(ly.topk_ids, E, R, S, B, q_loads, q_plans[li], q_pos, q_src, q_ws, ly.dev_status)
+
+        def q_step(B):
+            for li, ly in enumerate(layers):
+                q_route(B, li, ly)
+                tdh.ep_dispatch(ly.x, K, q_pos, ly.buf, ly.dev_status)
+                tdh.ep_combine(ly.buf, ly.w, q_pos, ly.out, ly.dev_status)
+                if ly.grad_n:
+                    tdh.ep_quota_replica_grad_reduce(ly.g_home, ly.g_rep, E, R, q_plans[li], False, ly.dev_status)
+
+        def q_routes(B):
+            for li, ly in enumerate(layers):
+                q_route(B, li, ly)
+
+        def replay_ms(fn, flush_between):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            g.replay()
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for i in range(args.steps):
+                if flush_between:
+                    flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                g.replay()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            del g
+            return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / args.steps
+
+        try:
+            for B in sorted({1, 3, E // R}):
+                for _ in range(2):
+                    q_step(B)
+                torch.cuda.synchronize()
+                step_ms_q = replay_ms(lambda: q_step(B), True)
+                route_ms_q = replay_ms(lambda: q_routes(B), True)
+                taus, nreps, locs = [], [], []
+                for li in range(nl):
+                    pl = q_plans[li]
+                    taus.append(round(int(pl[q_lay["tau"]].item()) * R / P, 4))
+                    nreps.append(int(pl[q_lay["n_rep"]].item()))
+                    locs.append(round(int(pl[q_lay["n_local"]].item()) / P, 4))
+                one = nl == 1
+                quota[f"B={B}"] = {
+                    "ms_per_step": round(step_ms_q, 5),
+                    "value": job_throughput(world, nl * P, 1, step_ms_q), "unit": UNIT,
+                    "route_us": round(route_ms_q * 1e3 / nl, 2),
+                    "max_rank_load_over_SK": taus[0] if one else taus,
+                    "n_rep": nreps[0] if one else nreps,
+                    "local_pair_fraction": locs[0] if one else locs}
+            for ly in layers:
+                st = ly.status(stream)
+                if st:
+                    raise RuntimeError(f"device status {st:#x} in the quota-planner timing")
+        except RuntimeError as exc:
+            if "device status" in str(exc):
+                raise
+            print(f"graph capture unavailable: {exc}", file=sys.stderr)
+        del q_plans, q_pos, q_src, q_ws
+
     # ---- prefetch slots under a per-rank budget B (one small launch, timed
     # apart as device time: 20 launches in one captured graph, replayed):
     # replicas whose weights are read from the home rank, and the rank loads if
@@ -497,6 +574,7 @@ def run_ours(args, rank, world, local_rank):
                     "replicated_experts": n_chunks if nl > 1 else n_chunks[0]},
         "backward": backward,
         "prefetch_slots": prefetch,
+        "quota_planner": quota,
         "layers_per_step": nl,
         "route_path": args.route,
     }

@@ -120,6 +120,7 @@ typedef struct {
   int32_t tau;            /* [1] tau*, the rank-load threshold met (-1: no plan) */
   int32_t n_rep;          /* [1] number of replicas */
   int32_t n_local;        /* [1] pairs placed on their own source rank */
+  int32_t n_chunks;       /* [1] number of replicated experts */
   int32_t rank_load;      /* [R] rows of rank r (<= tau) */
   int32_t rank_off;       /* [R] first buffer row of rank r */
   int32_t rank_nrep;      /* [R] replicas received by rank r */
@@ -127,6 +128,7 @@ typedef struct {
   int32_t home_quota;     /* [E] pairs taken by the home copy of e */
   int32_t rep_first;      /* [E] match index of e's first replica (0 if none) */
   int32_t rep_cnt;        /* [E] number of replicas of e */
+  int32_t rep_experts;    /* [E] replicated experts in match order (n_chunks valid, -1 after) */
   int32_t rep_expert;     /* [cap] logical expert of replica m (match order) */
   int32_t rep_rank;       /* [cap] receiving rank of replica m */
   int32_t rep_count;      /* [cap] quota of replica m */
@@ -134,6 +136,7 @@ typedef struct {
   int32_t inst_cum;       /* [E + cap] looked-up pairs of e's earlier instances */
   int32_t inst_base;      /* [E + cap] first buffer row of instance i */
   int32_t inst_lpre;      /* [E + cap] pairs of e from source ranks below instance i's rank */
+  int32_t rep_local_incl; /* [cap] local pairs of e's replicas up to and including m */
   int32_t slot_order;     /* [E + cap] instance ids in buffer order; -1 past E + n_rep */
   int32_t cu_seqlens;     /* [E + cap + 1] first row of each slot in buffer order;
                              entries from E + n_rep on hold R*S*K */
@@ -233,6 +236,16 @@ EP_API int ep_quota_plan_layout(int E, int R, EpQuotaLayout* layout /* host out 
 EP_API int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int B, int32_t* loads,
                           int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src, void* ws, size_t ws_bytes,
                           int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * ep_replica_grad_reduce for a plan from ep_quota_route: the same reduction
+ * (g_home[e] += each replica's row of e in match order, fp32), the replica
+ * list read from the quota plan.  Arguments as in ep_replica_grad_reduce;
+ * g_rep has at least n_rep rows.
+ */
+EP_API int ep_quota_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
+                                        const int32_t* plan, size_t plan_words, int clear_replicas,
+                                        int32_t* dev_status, cudaStream_t stream);
 
 /*
  * Prefetch slots under a per-rank budget B.  [GR] "Το memory contract που

@@ -66,6 +66,9 @@ def check_quota(topk, R, S, E, B):
     np.testing.assert_array_equal(f("rep_rank", n), qp["rep_rank"])
     np.testing.assert_array_equal(f("rep_count", n), qp["rep_count"])
     np.testing.assert_array_equal(f("home_quota", E), qp["home_quota"])
+    rep_experts = [int(e) for e in dict.fromkeys(qp["rep_expert"].tolist())]  # replicated experts, match order
+    assert int(f("n_chunks", 1)[0]) == len(rep_experts)
+    assert f("rep_experts", E)[:len(rep_experts)].tolist() == rep_experts
     np.testing.assert_array_equal(f("rank_load", R), lo["rank_load"])
     off = np.concatenate([[0], np.cumsum(lo["rank_load"])[:-1]])
     np.testing.assert_array_equal(f("rank_off", R), off)
@@ -195,3 +198,33 @@ def test_quota_rows_through_dispatch_and_combine():
     assert tdh.ep_status_read(status) == 0
     want = O.combine_closed(x, w, topk, scale)
     np.testing.assert_array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+@pytest.mark.parametrize("gdt", ["f32", "bf16"])
+def test_quota_grad_reduce(gdt):
+    """Replica gradients into their home expert, in match order, read from the
+    quota plan: bit-exact against the oracle's fp32 adds in the same order."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    for (R, S, K, E, B, n) in [(8, 300, 6, 64, 1, 1000), (16, 200, 8, 64, 3, 4096 + 520)]:
+        bias = np.random.default_rng(R).normal(0.0, 2.0, E).astype(np.float32)
+        topk, _ = W.routing_from(R * S, E, K, seed=21, bias_e=bias)
+        cu = run_quota(topk, R, S, E, B)
+        assert cu["status"] == 0
+        loads = np.bincount(topk.ravel(), minlength=E).astype(np.int32)
+        qp = O.quota_plan(loads, R, S, K, E, B)
+        cap = E + R - 1
+        gh = W.grad_rows(3, W.STREAM_GHOME, n, E, "f32")
+        gr = W.grad_rows(3, W.STREAM_GREP, n, cap, gdt)
+        dev = torch.device("cuda")
+        t_gh = torch.from_numpy(gh.copy()).to(dev)
+        t_gr = (torch.from_numpy(gr.view(np.int16).copy()).to(dev).view(torch.bfloat16) if gdt == "bf16"
+                else torch.from_numpy(gr.copy()).to(dev))
+        lay = tdh.ep_quota_plan_layout(E, R)
+        plan = torch.from_numpy(cu["plan"]).to(dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        tdh.ep_quota_replica_grad_reduce(t_gh, t_gr, E, R, plan, False, status)
+        assert tdh.ep_status_read(status) == 0
+        want_h, _ = O.grad_reduce(gh, gr, qp["rep_expert"])
+        np.testing.assert_array_equal(t_gh.cpu().numpy(), want_h)
+        assert lay["words"] == plan.numel()

@@ -44,9 +44,11 @@ class EpPlanLayout(ctypes.Structure):
 
 class EpQuotaLayout(ctypes.Structure):
     _fields_ = [("words", ctypes.c_int64), ("cap", ctypes.c_int32)] + [
-        (n, ctypes.c_int32) for n in ("tau", "n_rep", "n_local", "rank_load", "rank_off", "rank_nrep",
-                                      "rank_rep_first", "home_quota", "rep_first", "rep_cnt", "rep_expert", "rep_rank",
-                                      "rep_count", "inst_local", "inst_cum", "inst_base", "inst_lpre", "slot_order",
+        (n, ctypes.c_int32) for n in ("tau", "n_rep", "n_local", "n_chunks", "rank_load", "rank_off", "rank_nrep",
+                                      "rank_rep_first", "home_quota", "rep_first", "rep_cnt", "rep_experts",
+                                      "rep_expert", "rep_rank",
+                                      "rep_count", "inst_local", "inst_cum", "inst_base", "inst_lpre", "rep_local_incl",
+                                      "slot_order",
                                       "cu_seqlens")]
 
 
@@ -63,6 +65,7 @@ _SIGS = {
     "ep_plan": (_I, [_V, _I, _I64, _I, _I, _V, _SZ, _V, _V]),
     "ep_quota_workspace_size": (_I, [_I64, _I, _I, _I, _V]),
     "ep_quota_plan_layout": (_I, [_I, _I, _V]),
+    "ep_quota_replica_grad_reduce": (_I, [_V, _V, _I, _I64, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_quota_route": (_I, [_V, _I64, _I, _I, _I, _I64, _I, _V, _V, _SZ, _V, _V, _V, _SZ, _V, _V]),
     "ep_prefetch_slots": (_I, [_V, _SZ, _I, _I, _I64, _I, _V, _V, _V, _V]),
     "ep_layout": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _SZ, _V, _SZ, _V, _V, _V, _V, _V]),
@@ -291,19 +294,31 @@ def ep_combine_backward(dout, w, y, pos, dy, dw, dev_status=None, stream=None):
                                                             _p(dy), _p(dw), _p(dev_status), _s(stream)))
 
 
-def ep_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False, dev_status=None, stream=None):
+def _grad_dtype(g_home, g_rep, plan):
     _dtype(g_home, torch.float32)
     _dtype(plan, torch.int32)
     if g_rep.dtype == torch.float32:
-        dt = EP_DTYPE_F32
-    elif g_rep.dtype in (torch.bfloat16, torch.int16, torch.uint16):
-        dt = EP_DTYPE_BF16
-    else:
-        raise TypeError(g_rep.dtype)
+        return EP_DTYPE_F32
+    if g_rep.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return EP_DTYPE_BF16
+    raise TypeError(g_rep.dtype)
+
+
+def ep_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False, dev_status=None, stream=None):
+    dt = _grad_dtype(g_home, g_rep, plan)
     n = g_home.shape[1]
     _check("ep_replica_grad_reduce", lib().ep_replica_grad_reduce(_p(g_home), _p(g_rep), dt, n, E, R, _p(plan),
                                                                   plan.numel(), int(bool(clear_replicas)),
                                                                   _p(dev_status), _s(stream)))
+
+
+def ep_quota_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False, dev_status=None, stream=None):
+    """ep_replica_grad_reduce for a plan written by ep_quota_route."""
+    dt = _grad_dtype(g_home, g_rep, plan)
+    n = g_home.shape[1]
+    _check("ep_quota_replica_grad_reduce",
+           lib().ep_quota_replica_grad_reduce(_p(g_home), _p(g_rep), dt, n, E, R, _p(plan), plan.numel(),
+                                              int(bool(clear_replicas)), _p(dev_status), _s(stream)))
 
 
 def ep_selftest_lookback_timeout(topk_ids, E, loads, max_vio, ws, dev_status, stream=None):

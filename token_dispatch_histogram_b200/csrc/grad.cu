@@ -158,15 +158,13 @@ int occupancy_grid(const void* fn, int threads, size_t smem, int64_t work_items,
 
 using namespace ep;
 
-extern "C" int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
-                                      const int32_t* plan, size_t plan_words, int clear_replicas,
-                                      int32_t* dev_status, cudaStream_t stream) {
-  if (n < 0 || E < 1 || E > EP_MAX_EXPERTS || R < 1 || R > EP_MAX_RANKS || E % R) return EP_ERR_ARG;
-  if (rep_dtype != EP_DTYPE_F32 && rep_dtype != EP_DTYPE_BF16) return EP_ERR_ARG;
-  if (!plan) return EP_ERR_ARG;
-  EpPlanLayout L;
-  plan_layout(E, R, &L);
-  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+namespace ep {
+void quota_layout(int E, int R, EpQuotaLayout* L);
+
+// The plan fields the reduction reads: replicated experts in match order, and
+// each expert's first replica and replica count.
+static int run_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, const int32_t* plan,
+                           EpPlanLayout L, int clear_replicas, int32_t* dev_status, cudaStream_t stream) {
   if (n == 0) return EP_OK;
   if (!g_home || !g_rep || !aligned16(g_home) || !aligned16(g_rep)) return EP_ERR_ARG;
   const int64_t units = (int64_t)E * ((n + GRAD_UNIT - 1) / GRAD_UNIT);  // upper bound (n_chunks <= E)
@@ -180,4 +178,36 @@ extern "C" int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_
   if (cudaLaunchKernel(fn, dim3(grid), dim3(GRAD_THREADS), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
+}
+}  // namespace ep
+
+extern "C" int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
+                                      const int32_t* plan, size_t plan_words, int clear_replicas,
+                                      int32_t* dev_status, cudaStream_t stream) {
+  if (n < 0 || E < 1 || E > EP_MAX_EXPERTS || R < 1 || R > EP_MAX_RANKS || E % R) return EP_ERR_ARG;
+  if (rep_dtype != EP_DTYPE_F32 && rep_dtype != EP_DTYPE_BF16) return EP_ERR_ARG;
+  if (!plan) return EP_ERR_ARG;
+  EpPlanLayout L;
+  plan_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, dev_status, stream);
+}
+
+extern "C" int ep_quota_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
+                                            const int32_t* plan, size_t plan_words, int clear_replicas,
+                                            int32_t* dev_status, cudaStream_t stream) {
+  if (n < 0 || E < 1 || E > EP_MAX_EXPERTS || R < 1 || R > EP_MAX_RANKS || E % R) return EP_ERR_ARG;
+  if (rep_dtype != EP_DTYPE_F32 && rep_dtype != EP_DTYPE_BF16) return EP_ERR_ARG;
+  if (!plan) return EP_ERR_ARG;
+  EpQuotaLayout Q;
+  quota_layout(E, R, &Q);
+  if ((int64_t)plan_words < Q.words) return EP_ERR_CAPACITY;
+  EpPlanLayout L{};
+  L.words = Q.words;
+  L.cap = Q.cap;
+  L.n_chunks = Q.n_chunks;
+  L.rep_experts = Q.rep_experts;
+  L.copy_first = Q.rep_first;
+  L.copy_cnt = Q.rep_cnt;
+  return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, dev_status, stream);
 }

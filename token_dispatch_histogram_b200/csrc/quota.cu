@@ -35,11 +35,11 @@ namespace ep {
 
 int num_sms();
 
-constexpr int Q_SCAN_THREADS = 256;
+constexpr int Q_SCAN_THREADS = 512;
 constexpr int Q_SEARCH_THREADS = 256;
 
 // header words of the quota workspace
-enum : int { QH_TICKET_SCAN = 0, QH_TICKET_SEARCH = 1, QH_BEST = 2, QH_TAU_LO = 3, QH_TAU_HI = 4, QH_VALID = 5 };
+enum : int { QH_TICKET_SEARCH = 0, QH_BEST = 1 };
 
 struct QTiles {
   int tile;       // pairs per tile, a multiple of 512
@@ -64,7 +64,7 @@ inline QTiles q_tiles(int64_t SK, int R) {
 }
 
 struct QWs {
-  size_t hdr, cnt, excl, H, ord, bytes;
+  size_t hdr, cnt, excl, bytes;
 };
 inline QWs q_ws(int64_t ntiles, int E, int R) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -72,9 +72,7 @@ inline QWs q_ws(int64_t ntiles, int E, int R) {
   w.hdr = 0;
   w.cnt = 256;
   w.excl = al(w.cnt + sizeof(int32_t) * (size_t)E * (size_t)std::max<int64_t>(ntiles, 1));
-  w.H = al(w.excl + sizeof(int32_t) * (size_t)E * (size_t)(ntiles + 1));
-  w.ord = al(w.H + sizeof(int32_t) * (size_t)R);
-  w.bytes = al(w.ord + sizeof(int32_t) * (size_t)E);
+  w.bytes = al(w.excl + sizeof(int32_t) * (size_t)E * (size_t)(ntiles + 1));
   return w;
 }
 
@@ -90,6 +88,7 @@ void quota_layout(int E, int R, EpQuotaLayout* L) {
   L->tau = take(1);
   L->n_rep = take(1);
   L->n_local = take(1);
+  L->n_chunks = take(1);
   L->rank_load = take(R);
   L->rank_off = take(R);
   L->rank_nrep = take(R);
@@ -97,6 +96,7 @@ void quota_layout(int E, int R, EpQuotaLayout* L) {
   L->home_quota = take(E);
   L->rep_first = take(E);
   L->rep_cnt = take(E);
+  L->rep_experts = take(E);
   L->rep_expert = take(cap);
   L->rep_rank = take(cap);
   L->rep_count = take(cap);
@@ -104,6 +104,7 @@ void quota_layout(int E, int R, EpQuotaLayout* L) {
   L->inst_cum = take(E + cap);
   L->inst_base = take(E + cap);
   L->inst_lpre = take(E + cap);
+  L->rep_local_incl = take(cap);
   L->slot_order = take(E + cap);
   L->cu_seqlens = take(E + cap + 1);
   L->words = o;
@@ -111,6 +112,9 @@ void quota_layout(int E, int R, EpQuotaLayout* L) {
 
 // ------------------------------------------------------------------ 1. count
 
+constexpr int Q_ITEMS = 16;  // keys per thread: tiles of up to 512 * 16 = 8192 pairs
+
+// Counts are order-free, so plain shared-memory adds do (no warp aggregation).
 __global__ void __launch_bounds__(SCAT_THREADS)
     k_q_count(const int32_t* __restrict__ topk, int64_t SK, int E, int tile, int tpr, int64_t ntiles,
               int32_t* __restrict__ cnt, uint32_t* __restrict__ hdr, int32_t* dev_status) {
@@ -118,141 +122,121 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   __shared__ int s_bad;
   const int64_t t = blockIdx.x;
   if (t == 0 && threadIdx.x == 0) {
-    hdr[QH_TICKET_SCAN] = 0;
     hdr[QH_TICKET_SEARCH] = 0;
+    hdr[QH_BEST] = 0xffffffffu;
   }
   if (t >= ntiles) return;
   if (threadIdx.x == 0) s_bad = 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
-  __syncthreads();
   const int64_t r = t / tpr, lt = t % tpr;
   const int64_t p0 = r * SK + lt * tile;
   const int n = (int)min((int64_t)tile, SK - lt * tile);
-  const int lane = threadIdx.x & 31;
-  const int nbits = key_bits(E + 1);
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    int e = -1;
-    if (i < n) {
-      e = __ldg(topk + p0 + i);
-      if (e < 0 || e >= E) {
-        e = -1;
-        s_bad = 1;
-      }
-    }
-    const uint32_t peers = warp_match((uint32_t)(e + 1), nbits);
-    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[e], __popc(peers));
+  int key[Q_ITEMS];
+#pragma unroll
+  for (int k = 0; k < Q_ITEMS; ++k) {  // every load issued before the first add
+    const int i = k * SCAT_THREADS + threadIdx.x;
+    key[k] = i < n ? __ldg(topk + p0 + i) : 0;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(int64_t)e * ntiles + t] = s_hist[e];
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < Q_ITEMS; ++k) {
+    const int i = k * SCAT_THREADS + threadIdx.x;
+    if (i < n) {
+      const int e = key[k];
+      if (e >= 0 && e < E)
+        atomicAdd(&s_hist[e], 1);
+      else
+        bad = true;
+    }
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[t * E + e] = s_hist[e];
   if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_EXPERT_ID);
 }
 
 // ------------------------------------------------------------------- 2. scan
 
+constexpr int Q_SCAN_WARPS = Q_SCAN_THREADS / 32;
+
+// Lanes = 32 consecutive experts, warps = consecutive ranges of tiles: per-warp
+// sums, a scan over the warps, then each warp writes its exclusive prefixes.
+// Row ntiles of excl and loads get T_e.
 __global__ void __launch_bounds__(Q_SCAN_THREADS)
-    k_q_scan(const int32_t* __restrict__ cnt, int64_t ntiles, int E, int R, int64_t P, int32_t* __restrict__ excl,
-             int32_t* __restrict__ loads, int32_t* __restrict__ H_out, int32_t* __restrict__ ord,
-             uint32_t* __restrict__ hdr) {
-  extern __shared__ int32_t sm[];
-  int32_t* s_T = sm;      // [E]
-  int32_t* s_H = sm + E;  // [R]
-  __shared__ int s_last;
-  __shared__ unsigned long long s_total;
-  __shared__ int s_maxH;
+    k_q_scan(const int32_t* __restrict__ cnt, int64_t ntiles, int E, int32_t* __restrict__ excl,
+             int32_t* __restrict__ loads) {
+  __shared__ int32_t s_part[Q_SCAN_WARPS][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int e = blockIdx.x * (Q_SCAN_THREADS / 32) + warp;
+  const int e = blockIdx.x * 32 + lane;
+  const int64_t span = (ntiles + Q_SCAN_WARPS - 1) / Q_SCAN_WARPS;
+  const int64_t t0 = min(ntiles, warp * span), t1 = min(ntiles, t0 + span);
+  int32_t sum = 0;
   if (e < E) {
+#pragma unroll 8
+    for (int64_t t = t0; t < t1; ++t) sum += cnt[t * E + e];
+  }
+  s_part[warp][lane] = sum;
+  __syncthreads();
+  if (warp == 0) {
     int32_t run = 0;
-    for (int64_t b = 0; b < ntiles; b += 32) {
-      const int64_t t = b + lane;
-      const int32_t v = t < ntiles ? cnt[(int64_t)e * ntiles + t] : 0;
-      int32_t x = v;
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t y = __shfl_up_sync(0xffffffffu, x, d);
-        if (lane >= d) x += y;
-      }
-      if (t < ntiles) excl[t * E + e] = run + x - v;
-      run += __shfl_sync(0xffffffffu, x, 31);
+    for (int w = 0; w < Q_SCAN_WARPS; ++w) {
+      const int32_t v = s_part[w][lane];
+      s_part[w][lane] = run;
+      run += v;
     }
-    if (lane == 0) {
+    if (e < E) {
       excl[ntiles * E + e] = run;
       loads[e] = run;
     }
   }
-  // the last CTA to finish prepares the threshold search
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&hdr[QH_TICKET_SCAN], 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (threadIdx.x == 0) {
-    s_total = 0;
-    s_maxH = 0;
-  }
-  for (int r = threadIdx.x; r < R; r += blockDim.x) s_H[r] = 0;
-  __syncthreads();
-  const int ER = E / R;
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
-    const int32_t v = __ldcg(loads + x);
-    s_T[x] = v;
-    atomicAdd(&s_total, (unsigned long long)v);
-    atomicAdd(&s_H[x / ER], v);
-  }
-  __syncthreads();
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    H_out[r] = s_H[r];
-    atomicMax(&s_maxH, s_H[r]);
-  }
-  // each rank's experts heaviest first, ties to the lower id
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
-    const int r = x / ER;
-    const int32_t v = s_T[x];
-    int k = 0;
-    for (int y = r * ER; y < (r + 1) * ER; ++y) {
-      const int32_t w = s_T[y];
-      k += (w > v) || (w == v && y < x);
+  if (e < E) {
+    int32_t run = s_part[warp][lane];
+#pragma unroll 8
+    for (int64_t t = t0; t < t1; ++t) {
+      const int32_t v = cnt[t * E + e];
+      excl[t * E + e] = run;
+      run += v;
     }
-    ord[r * ER + k] = x;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int64_t lo = (P + R - 1) / R;
-    const int64_t hi = (int64_t)s_maxH > lo ? (int64_t)s_maxH : lo;
-    hdr[QH_TAU_LO] = (uint32_t)lo;
-    hdr[QH_TAU_HI] = (uint32_t)hi;
-    hdr[QH_BEST] = (uint32_t)hi;
-    hdr[QH_VALID] = s_total == (unsigned long long)P;
-    hdr[QH_TICKET_SCAN] = 0;
   }
 }
 
 // --------------------------------------------------------- 3. search + build
 
-// Whether every chunk finds room at threshold tau (the chunk/room walk).
-__device__ bool q_feasible(int64_t tau, const int32_t* s_T, const int32_t* s_H, const int32_t* s_ord, int R, int ER,
-                           int B) {
+// Whether every chunk finds room at threshold tau: the chunk/room walk over
+// this CTA's lists of possibly overloaded ranks (H and offset of its sorted
+// loads) and possible rooms (H), both in ascending rank order.  All values fit
+// in 32 bits (they are at most P < 2^31).
+__device__ __forceinline__ bool q_feasible(int32_t tau, const int32_t* s_sT, const int32_t* s_oH,
+                                           const int32_t* s_oOff, int novr, const int32_t* s_mH, int nroom, int ER,
+                                           int B) {
+  if (B <= 0) {
+    for (int a = 0; a < novr; ++a)
+      if (s_oH[a] > tau) return false;
+    return true;
+  }
   int j = 0;
-  while (j < R && s_H[j] >= tau) ++j;
-  int64_t room = j < R ? tau - s_H[j] : 0;
+  while (j < nroom && s_mH[j] >= tau) ++j;
+  int32_t room = j < nroom ? tau - s_mH[j] : 0;
   int pieces = 0;
-  for (int r = 0; r < R; ++r) {
-    int64_t rem = (int64_t)s_H[r] - tau;
+  for (int a = 0; a < novr; ++a) {
+    int32_t rem = s_oH[a] - tau;
+    const int32_t* st = s_sT + s_oOff[a];
     for (int i = 0; i < ER && rem > 0; ++i) {
-      int64_t c = min((int64_t)s_T[s_ord[r * ER + i]], rem);
+      int32_t c = min(st[i], rem);
       if (c <= 0) break;
       rem -= c;
       while (c > 0) {
-        if (j >= R || B <= 0) return false;
-        const int64_t take = min(c, room);
+        if (j >= nroom) return false;
+        const int32_t take = min(c, room);
         c -= take;
         room -= take;
         if (++pieces == B || room == 0) {
           ++j;
-          while (j < R && s_H[j] >= tau) ++j;
-          room = j < R ? tau - s_H[j] : 0;
+          while (j < nroom && s_mH[j] >= tau) ++j;
+          room = j < nroom ? tau - s_mH[j] : 0;
           pieces = 0;
         }
       }
@@ -261,38 +245,110 @@ __device__ bool q_feasible(int64_t tau, const int32_t* s_T, const int32_t* s_H, 
   return true;
 }
 
+inline size_t q_search_smem(int E, int R) {
+  const size_t cap = (size_t)E + R - 1;
+  return sizeof(int32_t) * (9 * (size_t)E + 12 * (size_t)R + 3 * cap + ((size_t)E + cap));
+}
+
 __global__ void __launch_bounds__(Q_SEARCH_THREADS)
-    k_q_search(const int32_t* __restrict__ loads, const int32_t* __restrict__ H_in, const int32_t* __restrict__ ord,
-               const int32_t* __restrict__ excl, int tpr, int E, int R, int B, int64_t P, uint32_t* hdr,
-               int32_t* __restrict__ plan, EpQuotaLayout L) {
+    k_q_search(const int32_t* __restrict__ loads, const int32_t* __restrict__ excl, int tpr, int E, int R, int B,
+               int64_t P, uint32_t* hdr, int32_t* __restrict__ plan, EpQuotaLayout L) {
   extern __shared__ int32_t sm[];
-  int32_t* s_T = sm;            // [E]
-  int32_t* s_ord = s_T + E;     // [E]
-  int32_t* s_rfirst = s_ord + E;  // [E] (build)
-  int32_t* s_rcnt = s_rfirst + E;  // [E] (build)
-  int32_t* s_hq = s_rcnt + E;   // [E] (build)
-  int32_t* s_H = s_hq + E;      // [R]
-  int32_t* s_rnrep = s_H + R;   // [R] (build)
-  int32_t* s_rrf = s_rnrep + R;  // [R] (build)
-  int32_t* s_rl = s_rrf + R;    // [R] (build)
-  __shared__ int s_last, s_nrep;
+  const int cap = L.cap;
+  int32_t* s_T = sm;                // [E]
+  int32_t* s_sT = s_T + E;          // [E] each rank's loads, heaviest first
+  int32_t* s_ord = s_sT + E;        // [E] the matching expert ids
+  int32_t* s_rfirst = s_ord + E;    // [E] (build)
+  int32_t* s_rcnt = s_rfirst + E;   // [E] (build)
+  int32_t* s_hq = s_rcnt + E;       // [E] (build)
+  int32_t* s_H = s_hq + E;          // [R]
+  int32_t* s_oH = s_H + R;          // [R] possibly overloaded ranks: H
+  int32_t* s_oOff = s_oH + R;       // [R]   and r * E/R
+  int32_t* s_mH = s_oOff + R;       // [R] possible rooms: H
+  int32_t* s_mR = s_mH + R;         // [R]   and rank
+  int32_t* s_rnrep = s_mR + R;      // [R] (build)
+  int32_t* s_rrf = s_rnrep + R;     // [R] (build)
+  int32_t* s_rl = s_rrf + R;        // [R] (build)
+  int32_t* s_re = s_rl + R;         // [cap]
+  int32_t* s_rr = s_re + cap;       // [cap]
+  int32_t* s_rc = s_rr + cap;       // [cap]
+  int32_t* s_loc = s_rc + cap;      // [E + cap]
+  int32_t* s_chE = s_loc + E + cap; // [E] chunks at tau*: expert
+  int32_t* s_chB = s_chE + E;       // [E]   first position in the excess sequence
+  int32_t* s_chN = s_chB + E;       // [E]   size
+  int32_t* s_wS = s_chN + E;        // [R] room windows at tau*: start
+  int32_t* s_wE = s_wS + R;         // [R]   end
+  int32_t* s_wR = s_wE + R;         // [R]   rank
+  int32_t* s_wP = s_wR + R;         // [R]   first piece
+  __shared__ int s_last, s_nrep, s_novr, s_nroom, s_maxH, s_nwin;
   __shared__ int32_t warp_sums[32];
-  __shared__ unsigned long long s_local;
+  __shared__ int32_t s_total, s_local;
   const int ER = E / R;
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
-    s_T[x] = loads[x];
-    s_ord[x] = ord[x];
+  // every CTA derives the rank loads, each rank's order and the range itself
+  if (threadIdx.x == 0) {
+    s_total = 0;
+    s_maxH = 0;
   }
-  for (int r = threadIdx.x; r < R; r += blockDim.x) s_H[r] = H_in[r];
+  for (int r = threadIdx.x; r < R; r += blockDim.x) s_H[r] = 0;
   __syncthreads();
-  const int64_t lo = hdr[QH_TAU_LO], hi = hdr[QH_TAU_HI];
-  const bool valid = hdr[QH_VALID] != 0;
+  {
+    int32_t part = 0;  // loads count valid pairs only, so every sum stays below 2^31
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {
+      const int32_t v = loads[x];
+      s_T[x] = v;
+      part += v;
+      atomicAdd(&s_H[x / ER], v);
+    }
+    for (int d = 16; d > 0; d >>= 1) part += __shfl_down_sync(0xffffffffu, part, d);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&s_total, part);
+  }
+  __syncthreads();
+  const int64_t lo = (P + R - 1) / R;
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {  // heaviest first, ties to the lower id
+    const int r = x / ER;
+    if (s_H[r] <= lo) {  // never sheds: the order is not needed
+      s_sT[x] = s_T[x];
+      s_ord[x] = x;
+      continue;
+    }
+    const int32_t v = s_T[x];
+    int k = 0;
+    for (int y = r * ER; y < (r + 1) * ER; ++y) {
+      const int32_t w = s_T[y];
+      k += (w > v) || (w == v && y < x);
+    }
+    s_sT[r * ER + k] = v;
+    s_ord[r * ER + k] = x;
+  }
+  for (int r = threadIdx.x; r < R; r += blockDim.x) atomicMax(&s_maxH, s_H[r]);
+  __syncthreads();
+  const bool valid = (int64_t)s_total == P;
+  const int64_t hi = (int64_t)s_maxH > lo ? (int64_t)s_maxH : lo;
+  const int64_t tmin = lo + (int64_t)blockIdx.x * blockDim.x;  // this CTA's smallest candidate
+  if (threadIdx.x == 0) {
+    if (valid && blockIdx.x == 0) atomicMin(hdr + QH_BEST, (uint32_t)hi);
+    int no = 0, nm = 0;
+    for (int r = 0; r < R; ++r) {
+      if (s_H[r] > tmin) {
+        s_oH[no] = s_H[r];
+        s_oOff[no++] = r * ER;
+      }
+      if (s_H[r] < hi) {
+        s_mH[nm] = s_H[r];
+        s_mR[nm++] = r;
+      }
+    }
+    s_novr = no;
+    s_nroom = nm;
+  }
+  __syncthreads();
   if (valid) {
     const int64_t N = (int64_t)gridDim.x * blockDim.x;
     volatile uint32_t* best = hdr + QH_BEST;
-    for (int64_t tau = lo + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; tau < hi; tau += N) {
+    const int novr = s_novr, nroom = s_nroom;
+    for (int64_t tau = tmin + threadIdx.x; tau < hi; tau += N) {
       if (tau >= (int64_t)*best) break;
-      if (q_feasible(tau, s_T, s_H, s_ord, R, ER, B)) {
+      if (q_feasible((int32_t)tau, s_sT, s_oH, s_oOff, novr, s_mH, nroom, ER, B)) {
         atomicMin(hdr + QH_BEST, (uint32_t)tau);
         break;
       }
@@ -305,9 +361,8 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
   if (!s_last) return;
   __threadfence();
 
-  // ---- the plan at tau*, by the last CTA
-  const int cap = L.cap;
-  const int64_t tau = valid ? (int64_t)atomicAdd(hdr + QH_BEST, 0u) : -1;
+  // ---- the plan at tau*, by the last CTA, from shared memory
+  const int32_t tau = valid ? (int32_t)atomicAdd(hdr + QH_BEST, 0u) : -1;
   for (int x = threadIdx.x; x < E; x += blockDim.x) {
     s_rfirst[x] = 0;
     s_rcnt[x] = 0;
@@ -318,50 +373,103 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
     s_local = 0;
   }
   __syncthreads();
-  if (threadIdx.x == 0 && valid) {  // the walk at tau*, emitting one replica per piece
-    int n = 0, j = 0, pieces = 0;
-    while (j < R && s_H[j] >= tau) ++j;
-    int64_t room = j < R ? tau - s_H[j] : 0;
-    for (int r = 0; r < R; ++r) {
-      int64_t rem = (int64_t)s_H[r] - tau;
-      for (int i = 0; i < ER && rem > 0; ++i) {
-        const int e = s_ord[r * ER + i];
-        int64_t c = min((int64_t)s_T[e], rem);
-        if (c <= 0) break;
-        rem -= c;
-        s_rfirst[e] = n;
-        while (c > 0 && j < R && B > 0 && n < cap) {
-          const int64_t take = min(c, room);
-          plan[L.rep_expert + n] = e;
-          plan[L.rep_rank + n] = j;
-          plan[L.rep_count + n] = (int32_t)take;
-          ++n;
-          s_rcnt[e] += 1;
-          s_rnrep[j] += 1;
-          c -= take;
-          room -= take;
-          if (++pieces == B || room == 0) {
-            ++j;
-            while (j < R && s_H[j] >= tau) ++j;
-            room = j < R ? tau - s_H[j] : 0;
-            pieces = 0;
-          }
-        }
-      }
+  // chunks at tau*: each rank sheds H_r - tau* from its heaviest experts
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    const int32_t X = valid ? s_H[r] - tau : 0;
+    int m = 0;
+    for (int32_t acc = 0; m < ER && acc < X && s_sT[r * ER + m] > 0; ++m) acc += s_sT[r * ER + m];
+    s_rl[r] = m;  // (s_rl is free until the rank loads)
+  }
+  __syncthreads();
+  const int nch = block_scan_array(s_rl, R, warp_sums);
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    const int32_t X = valid ? s_H[r] - tau : 0;
+    const int m = (r + 1 < R ? s_rl[r + 1] : nch) - s_rl[r];
+    int32_t acc = 0;
+    for (int i = 0; i < m; ++i) {
+      const int32_t v = s_sT[r * ER + i];
+      s_chE[s_rl[r] + i] = s_ord[r * ER + i];
+      s_chN[s_rl[r] + i] = min(v, X - acc);
+      acc += v;
     }
-    s_nrep = n;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < nch; k += blockDim.x) s_chB[k] = s_chN[k];
+  __syncthreads();
+  const int32_t Xtot = block_scan_array(s_chB, nch, warp_sums);  // chunk starts
+  // room windows: room j takes [x, min(x + room, end of the B-th chunk from x));
+  // one thread runs the recurrence, with a forward pointer over the chunks
+  if (threadIdx.x == 0) {
+    int nw = 0, k = 0;
+    int32_t x = 0;
+    for (int j = 0; j < s_nroom && x < Xtot && B > 0; ++j) {
+      if (s_mH[j] >= tau) continue;
+      int32_t e = x + (tau - s_mH[j]);
+      if (k + B - 1 < nch) e = min(e, s_chB[k + B - 1] + s_chN[k + B - 1]);
+      e = min(e, Xtot);
+      s_wS[nw] = x;
+      s_wE[nw] = e;
+      s_wR[nw] = s_mR[j];
+      ++nw;
+      x = e;
+      while (k < nch && s_chB[k] + s_chN[k] <= x) ++k;
+    }
+    s_nwin = nw;
+  }
+  __syncthreads();
+  const int nw = s_nwin;
+  // pieces per window: the chunks it overlaps (binary searches over chunk starts)
+  for (int w = threadIdx.x; w < nw; w += blockDim.x) {
+    int a = 0, b = nch - 1;  // chunk holding position s_wS[w]: last start <= it
+    while (a < b) {
+      const int mid = (a + b + 1) >> 1;
+      if (s_chB[mid] <= s_wS[w]) a = mid; else b = mid - 1;
+    }
+    int c = a, d = nch - 1;  // chunk holding position s_wE[w] - 1
+    while (c < d) {
+      const int mid = (c + d + 1) >> 1;
+      if (s_chB[mid] <= s_wE[w] - 1) c = mid; else d = mid - 1;
+    }
+    s_wP[w] = c - a + 1;
+    s_rnrep[s_wR[w]] = c - a + 1;
+  }
+  __syncthreads();
+  const int n_pieces = block_scan_array(s_wP, nw, warp_sums);
+  // emit in match order: window by window, chunk by chunk
+  for (int w = threadIdx.x; w < nw; w += blockDim.x) {
+    int a = 0, b = nch - 1;
+    while (a < b) {
+      const int mid = (a + b + 1) >> 1;
+      if (s_chB[mid] <= s_wS[w]) a = mid; else b = mid - 1;
+    }
+    const int np = (w + 1 < nw ? s_wP[w + 1] : n_pieces) - s_wP[w];
+    for (int q = 0; q < np && s_wP[w] + q < cap; ++q) {
+      const int k = a + q, m = s_wP[w] + q;
+      const int32_t cb = s_chB[k], ce = cb + s_chN[k];
+      const int e = s_chE[k];
+      s_re[m] = e;
+      s_rr[m] = s_wR[w];
+      s_rc[m] = min(ce, s_wE[w]) - max(cb, s_wS[w]);
+      if (cb >= s_wS[w]) s_rfirst[e] = m;  // the chunk starts in this window
+      atomicAdd(&s_rcnt[e], 1);
+    }
+  }
+  for (int k = threadIdx.x; k < E; k += blockDim.x) plan[L.rep_experts + k] = k < nch ? s_chE[k] : -1;
+  if (threadIdx.x == 0) {
+    s_nrep = min(n_pieces, cap);
+    plan[L.n_chunks] = nch;
   }
   __syncthreads();
   const int n_rep = s_nrep;
-  for (int m = n_rep + threadIdx.x; m < cap; m += blockDim.x) {
-    plan[L.rep_expert + m] = -1;
-    plan[L.rep_rank + m] = -1;
-    plan[L.rep_count + m] = 0;
+  for (int m = threadIdx.x; m < cap; m += blockDim.x) {
+    const bool v = m < n_rep;
+    plan[L.rep_expert + m] = v ? s_re[m] : -1;
+    plan[L.rep_rank + m] = v ? s_rr[m] : -1;
+    plan[L.rep_count + m] = v ? s_rc[m] : 0;
   }
-  // home quotas, replica ranges per expert
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {  // home quotas
     int32_t q = valid ? s_T[x] : 0;
-    for (int k = 0; k < s_rcnt[x]; ++k) q -= plan[L.rep_count + s_rfirst[x] + k];
+    for (int k = 0; k < s_rcnt[x]; ++k) q -= s_rc[s_rfirst[x] + k];
     s_hq[x] = q;
     plan[L.home_quota + x] = q;
     plan[L.rep_first + x] = s_rfirst[x];
@@ -370,18 +478,45 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
   for (int r = threadIdx.x; r < R; r += blockDim.x) s_rrf[r] = s_rnrep[r];
   __syncthreads();
   block_scan_array(s_rrf, R, warp_sums);  // replicas received by lower ranks
-  // rank loads
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+  // local pairs of every instance: min(quota, pairs of e from the instance's
+  // rank); the prefix loads are independent, so they go out together
+  for (int i = threadIdx.x; i < E + n_rep; i += blockDim.x) {
+    const int e = i < E ? i : s_re[i - E];
+    const int r = i < E ? i / ER : s_rr[i - E];
+    const int32_t q = i < E ? s_hq[i] : s_rc[i - E];
+    const int32_t lpre = excl[(int64_t)r * tpr * E + e];
+    const int32_t lsrc = excl[(int64_t)(r + 1) * tpr * E + e] - lpre;
+    const int32_t loc = valid ? min(q, lsrc) : 0;
+    s_loc[i] = loc;
+    plan[L.inst_local + i] = loc;
+    plan[L.inst_lpre + i] = lpre;
+  }
+  __syncthreads();
+  // cumulative looked-up ranges in instance order (home, then replicas), and
+  // the running local count over e's replicas (match order = ascending rank)
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    int32_t cum = s_hq[x] - s_loc[x], inc = 0;
+    plan[L.inst_cum + x] = 0;
+    for (int k = 0; k < s_rcnt[x]; ++k) {
+      const int m = s_rfirst[x] + k;
+      plan[L.inst_cum + E + m] = cum;
+      cum += s_rc[m] - s_loc[E + m];
+      inc += s_loc[E + m];
+      plan[L.rep_local_incl + m] = inc;
+    }
+    atomicAdd(&s_local, s_loc[x] + inc);
+  }
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {  // rank loads
     int32_t l = 0;
     for (int x = r * ER; x < (r + 1) * ER; ++x) l += s_hq[x];
-    for (int k = 0; k < s_rnrep[r]; ++k) l += plan[L.rep_count + s_rrf[r] + k];
+    for (int k = 0; k < s_rnrep[r]; ++k) l += s_rc[s_rrf[r] + k];
     s_rl[r] = l;
     plan[L.rank_load + r] = l;
     plan[L.rank_nrep + r] = s_rnrep[r];
     plan[L.rank_rep_first + r] = s_rrf[r];
   }
   __syncthreads();
-  block_scan_array(s_rl, R, warp_sums);  // now the first row of each rank
+  block_scan_array(s_rl, R, warp_sums);  // first row of each rank
   // rows of every instance, rank by rank: home experts by id, then replicas
   for (int r = threadIdx.x; r < R; r += blockDim.x) {
     int32_t row = s_rl[r];
@@ -398,7 +533,7 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
       plan[L.inst_base + E + m] = row;
       const int slot = (r + 1) * ER + m;
       plan[L.slot_order + slot] = E + m;
-      row += plan[L.rep_count + m];
+      row += s_rc[m];
       plan[L.cu_seqlens + slot + 1] = row;
     }
   }
@@ -406,32 +541,12 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
     plan[L.slot_order + slot] = -1;
     plan[L.cu_seqlens + slot + 1] = valid ? (int32_t)P : 0;
   }
-  if (threadIdx.x == 0) plan[L.cu_seqlens] = 0;
-  // locality: instance i on rank r takes the first min(q_i, L[r][e]) pairs of
-  // e from source rank r; the rest of e's pairs fill the instances' remaining
-  // quotas in instance order (home, then replicas in match order)
-  const int64_t Eq = E;
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
-    int32_t cum = 0;
-    for (int k = 0; k <= s_rcnt[x]; ++k) {
-      const int i = k == 0 ? x : E + s_rfirst[x] + k - 1;
-      const int r = k == 0 ? x / ER : plan[L.rep_rank + s_rfirst[x] + k - 1];
-      const int32_t q = k == 0 ? s_hq[x] : plan[L.rep_count + s_rfirst[x] + k - 1];
-      const int32_t lpre = excl[(int64_t)r * tpr * Eq + x];
-      const int32_t lsrc = excl[(int64_t)(r + 1) * tpr * Eq + x] - lpre;
-      const int32_t loc = valid ? min(q, lsrc) : 0;
-      plan[L.inst_local + i] = loc;
-      plan[L.inst_cum + i] = cum;
-      plan[L.inst_lpre + i] = lpre;
-      cum += q - loc;
-      atomicAdd(&s_local, (unsigned long long)loc);
-    }
-  }
   __syncthreads();
   if (threadIdx.x == 0) {
-    plan[L.tau] = (int32_t)tau;
+    plan[L.cu_seqlens] = 0;
+    plan[L.tau] = tau;
     plan[L.n_rep] = n_rep;
-    plan[L.n_local] = (int32_t)s_local;
+    plan[L.n_local] = s_local;
     hdr[QH_TICKET_SEARCH] = 0;
   }
 }
@@ -443,8 +558,18 @@ __global__ void __launch_bounds__(SCAT_THREADS)
                const int32_t* __restrict__ excl, const int32_t* __restrict__ plan, EpQuotaLayout L,
                int32_t* __restrict__ pos, int32_t* __restrict__ src, int32_t* dev_status) {
   extern __shared__ int32_t sm[];
-  int32_t* s_ids = sm;              // [tile]
-  int32_t* s_whist = s_ids + tile;  // [SCAT_WARPS * E]
+  int32_t* s_ids = sm;                  // [tile]
+  int32_t* s_whist = s_ids + tile;      // [SCAT_WARPS * E]
+  int32_t* s_lpre = s_whist + SCAT_WARPS * E;  // [E] pairs of e from source ranks below this tile's
+  int32_t* s_oloc = s_lpre + E;         // [E] local pairs of e's instance on this rank (0: none)
+  int32_t* s_obase = s_oloc + E;        // [E] its first row
+  int32_t* s_locb = s_obase + E;        // [E] local pairs of e's instances on ranks <= this one
+  int32_t* s_rf = s_locb + E;           // [E]
+  int32_t* s_rc = s_rf + E;             // [E]
+  int32_t* s_rrank = s_rc + E;          // [cap] rep_rank
+  int32_t* s_icum = s_rrank + L.cap;    // [E + cap] cumulative start of instance i's looked-up range
+  int32_t* s_istart = s_icum + E + L.cap;  // [E + cap] its first looked-up row
+  int32_t* s_ispan = s_istart + E + L.cap; // [E + cap] its looked-up rows
   __shared__ int s_flags;
   const int64_t t = blockIdx.x;
   const int rs = (int)(t / tpr);
@@ -459,53 +584,64 @@ __global__ void __launch_bounds__(SCAT_THREADS)
     for (int i = threadIdx.x; i < n; i += blockDim.x) pos[p0 + i] = -1;
     return;
   }
-  const int32_t* lpre_src = excl + (int64_t)rs * tpr * E;  // pairs of e from source ranks below rs
-  auto emit = [&](int64_t p, int e, int32_t g) {
-    const int rf = __ldg(plan + L.rep_first + e), rc = __ldg(plan + L.rep_cnt + e);
-    // the instance of e on the pair's own source rank, if any (e's replicas
-    // sit on ascending ranks)
-    int inst = -1;
-    if (e / ER == rs) {
-      inst = e;
-    } else if (rc > 0) {
-      int a = rf, b = rf + rc - 1;
-      while (a < b) {
-        const int mid = (a + b) >> 1;
-        if (__ldg(plan + L.rep_rank + mid) < rs)
-          a = mid + 1;
-        else
-          b = mid;
-      }
-      if (__ldg(plan + L.rep_rank + a) == rs) inst = E + a;
+  const int n_rep = min(max(plan[L.n_rep], 0), L.cap);
+  for (int i = threadIdx.x; i < E + n_rep; i += blockDim.x) {
+    const int32_t q = i < E ? plan[L.home_quota + i] : plan[L.rep_count + i - E];
+    const int32_t loc = plan[L.inst_local + i];
+    s_icum[i] = plan[L.inst_cum + i];
+    s_istart[i] = plan[L.inst_base + i] + loc;
+    s_ispan[i] = q - loc;
+    if (i >= E) s_rrank[i - E] = plan[L.rep_rank + i - E];
+  }
+  __syncthreads();
+  // per-expert view from this tile's source rank (e's replicas sit on
+  // ascending ranks, so each lookup is a binary search)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int rf = plan[L.rep_first + e], rc = plan[L.rep_cnt + e];
+    s_rf[e] = rf;
+    s_rc[e] = rc;
+    s_lpre[e] = excl[(int64_t)rs * tpr * E + e];
+    int a = 0, b = rc;  // replicas of e on ranks < rs: the first a
+    while (a < b) {
+      const int mid = (a + b) >> 1;
+      if (s_rrank[rf + mid] < rs)
+        a = mid + 1;
+      else
+        b = mid;
     }
-    const int32_t ls = g - __ldg(lpre_src + e);
+    int own = -1, below = a;
+    if (e / ER == rs) {
+      own = e;
+    } else if (a < rc && s_rrank[rf + a] == rs) {
+      own = E + rf + a;
+      below = a + 1;
+    }
+    s_oloc[e] = own >= 0 ? plan[L.inst_local + own] : 0;
+    s_obase[e] = own >= 0 ? plan[L.inst_base + own] : 0;
+    s_locb[e] = (e / ER <= rs ? plan[L.inst_local + e] : 0) + (below > 0 ? plan[L.rep_local_incl + rf + below - 1] : 0);
+  }
+  // (tile_stable_ranks starts with a __syncthreads after its own loads)
+  auto emit = [&](int64_t p, int e, int32_t g) {
+    const int32_t ls = g - s_lpre[e];
     int32_t row = -1;
-    if (inst >= 0 && ls < __ldg(plan + L.inst_local + inst)) {
-      row = __ldg(plan + L.inst_base + inst) + ls;
+    if (ls < s_oloc[e]) {
+      row = s_obase[e] + ls;
     } else {
-      // rank among e's pairs that are not placed locally
-      int32_t j = g;
-      for (int k = 0; k <= rc; ++k) {
-        const int i = k == 0 ? e : E + rf + k - 1;
-        const int32_t d = g - __ldg(plan + L.inst_lpre + i);
-        const int32_t loc = __ldg(plan + L.inst_local + i);
-        j -= d <= 0 ? 0 : (d < loc ? d : loc);
-      }
-      // the last instance whose cumulative start is <= j
-      int a = 0, b = rc;
+      // rank among e's pairs not placed locally, then the last instance
+      // (home, replicas in match order) whose cumulative start is <= it
+      const int32_t j = g - s_locb[e];
+      const int rf = s_rf[e];
+      int a = 0, b = s_rc[e];
       while (a < b) {
         const int mid = (a + b + 1) >> 1;
-        const int i = mid == 0 ? e : E + rf + mid - 1;
-        if (__ldg(plan + L.inst_cum + i) <= j)
+        if (s_icum[E + rf + mid - 1] <= j)
           a = mid;
         else
           b = mid - 1;
       }
       const int i = a == 0 ? e : E + rf + a - 1;
-      const int32_t q = a == 0 ? __ldg(plan + L.home_quota + e) : __ldg(plan + L.rep_count + rf + a - 1);
-      const int32_t loc = __ldg(plan + L.inst_local + i);
-      const int32_t off = j - __ldg(plan + L.inst_cum + i);
-      if (off >= 0 && off < q - loc) row = __ldg(plan + L.inst_base + i) + loc + off;
+      const int32_t off = j - s_icum[i];
+      if (off >= 0 && off < s_ispan[i]) row = s_istart[i] + off;
     }
     if (row < 0 || row >= P) {
       atomicOr(&s_flags, EP_DEV_BAD_ROW);
@@ -559,20 +695,18 @@ extern "C" int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, 
   uint32_t* hdr = reinterpret_cast<uint32_t*>(base + w.hdr);
   int32_t* cnt = reinterpret_cast<int32_t*>(base + w.cnt);
   int32_t* excl = reinterpret_cast<int32_t*>(base + w.excl);
-  int32_t* H = reinterpret_cast<int32_t*>(base + w.H);
-  int32_t* ord = reinterpret_cast<int32_t*>(base + w.ord);
-
   k_q_count<<<(unsigned)std::max<int64_t>(q.ntiles, 1), SCAT_THREADS, sizeof(int32_t) * E, stream>>>(
       topk_ids, SK, E, q.tile, q.tpr, q.ntiles, cnt, hdr, dev_status);
-  const int scan_grid = (E + Q_SCAN_THREADS / 32 - 1) / (Q_SCAN_THREADS / 32);
-  k_q_scan<<<scan_grid, Q_SCAN_THREADS, sizeof(int32_t) * (E + R), stream>>>(cnt, q.ntiles, E, R, P, excl, loads, H,
-                                                                              ord, hdr);
-  const size_t search_smem = sizeof(int32_t) * (5 * (size_t)E + 4 * (size_t)R);
-  k_q_search<<<2 * num_sms(), Q_SEARCH_THREADS, search_smem, stream>>>(loads, H, ord, excl, q.tpr, E, R, B, P, hdr,
-                                                                       plan, L);
+  k_q_scan<<<(E + 31) / 32, Q_SCAN_THREADS, 0, stream>>>(cnt, q.ntiles, E, excl, loads);
+  const size_t search_smem = q_search_smem(E, R);
+  if (search_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_q_search, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)search_smem) != cudaSuccess)
+    return EP_ERR_CUDA;
+  k_q_search<<<2 * num_sms(), Q_SEARCH_THREADS, search_smem, stream>>>(loads, excl, q.tpr, E, R, B, P, hdr, plan, L);
   count_launch(3);
   if (q.ntiles > 0) {
-    const size_t smem = sizeof(int32_t) * ((size_t)q.tile + (size_t)SCAT_WARPS * E);
+    const size_t smem =
+        sizeof(int32_t) * ((size_t)q.tile + (size_t)SCAT_WARPS * E + 6 * (size_t)E + (size_t)L.cap + 3 * ((size_t)E + L.cap));
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(k_q_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return EP_ERR_CUDA;
