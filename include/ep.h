@@ -386,6 +386,96 @@ EP_API int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtyp
                            cudaStream_t stream);
 
 /*
+ * ---------------------------------------------------------------------------
+ * Rank-local form: the calls one rank makes when the R ranks are R processes
+ * (one GPU each) rather than R partitions of one buffer.  [GR] "Online
+ * planning, zero copy και στατικά σχήματα": tokens are written straight into
+ * their final expert-grouped rows on the remote ranks, and the application
+ * reads views of that communication buffer.  [JA] "その仕組みは高速な
+ * エキスパート複製に依存する": planning starts from the exact source-rank x
+ * expert load matrix after routing.  Flow on rank r:
+ *   1. ep_route_stats(topk_local [S, K], T = S) -> counts row r (its pairs per
+ *      expert) and, in ws, the per-tile prefixes ep_layout_rank reads;
+ *   2. the caller all-gathers the rows into counts [R, E] (one collective);
+ *   3. ep_plan_from_counts: the same plan on every rank, no further exchange;
+ *   4. ep_layout_rank: the global row of each local pair; a pair's rank in its
+ *      expert's list is (pairs of that expert on source ranks < r) + (its rank
+ *      among the local pairs), so no other coordination is needed;
+ *   5. ep_dispatch_peer / ep_combine_peer / ep_replica_grad_reduce_peer move
+ *      rows through a table of the R ranks' buffer base addresses.
+ * Every output equals, bit for bit, the slice of the one-buffer path's output
+ * that belongs to rank r.  Peer tables: device arrays of R uint64 device
+ * addresses (this GPU's own buffer or peers' buffers mapped into its address
+ * space, e.g. symmetric memory or IPC); each must be 16-byte aligned.  A zero
+ * or misaligned entry is never dereferenced: the rows it would serve are
+ * skipped and EP_DEV_BAD_ROW is set.  Global row g lives on rank
+ * g / rows_per_rank at local row g % rows_per_rank.
+ */
+
+/*
+ * The plan from the gathered load matrix: loads[e] = sum_r counts[r, e], then
+ * exactly ep_plan.  counts [R, E] int32 device; loads [E] int32 out (device) or
+ * NULL; plan as in ep_plan.  One CTA.
+ */
+EP_API int ep_plan_from_counts(const int32_t* counts, int R, int64_t S, int K, int E, int32_t* loads, int32_t* plan,
+                               size_t plan_words, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Rows of rank `rank`'s own pairs.  topk_local [S, K] int32; counts [R, E] from
+ * step 2; plan from ep_plan_from_counts; ws the scratch ep_route_stats filled
+ * for topk_local (T = S).  pos_local [S*K] int32 out: the global row of local
+ * pair i (= pos[rank*S*K + i] of the one-buffer layout).  pair_slot [S*K] out
+ * or NULL.  No src output: a receiving rank finds a row's expert from the plan's
+ * slot table (cu_seqlens, slot_order).
+ */
+EP_API int ep_layout_rank(const int32_t* topk_local, int64_t S, int K, int E, int R, int rank,
+                          const int32_t* counts, const int32_t* plan, size_t plan_words, const void* ws,
+                          size_t ws_bytes, int32_t* pos_local, int32_t* pair_slot, int32_t* dev_status,
+                          cudaStream_t stream);
+
+/*
+ * Dispatch of rank-local tokens: the row of x_local [S, H] bf16 of pair i goes
+ * to global row pos_local[i], i.e. to peer_bufs[g / rows_per_rank] at local row
+ * g % rows_per_rank (H bf16 per row).  One TMA bulk load per token row and K
+ * bulk stores, as ep_dispatch.
+ */
+EP_API int ep_dispatch_peer(const uint16_t* x_local, int64_t S, int K, int64_t H, const int32_t* pos_local,
+                            const uint64_t* peer_bufs, int R, int64_t rows_per_rank, int32_t* dev_status,
+                            cudaStream_t stream);
+
+/*
+ * Combine of rank-local tokens, reading the expert rows from the R rank
+ * buffers: out_local[t] = bf16_rn( sum_k w_local[t,k] * float(row pos_local[t*K+k]) ),
+ * fp32 in k order, as ep_combine.  w_local NULL: unit weights (the backward of
+ * dispatch, as ep_dispatch_backward).  1 <= K <= 8.
+ */
+EP_API int ep_combine_peer(const uint64_t* peer_bufs, int R, int64_t rows_per_rank, const float* w_local,
+                           const int32_t* pos_local, int64_t S, int K, int64_t H, uint16_t* out_local,
+                           int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Replica gradient reduction on the home rank.  [GR] "Τι συμβαίνει στους
+ * gradients κατά την εκπαίδευση": each rank views the R ranks' reduce buffers
+ * together and reads, over NVLink, the slots that hold its own experts'
+ * replica gradients, adds them into its local parameter gradient and clears
+ * the used slots.  Per element of each home expert e of `rank` with replicas:
+ *   g_home_local[e - rank*E/R] = ((g + rep(m1)) + rep(m2)) ...  (match order, fp32)
+ * where replica m's row is row (m - first replica rank d receives) of rank d's
+ * reduce buffer, d = the replica's receiving rank: the replicas a rank receives
+ * are consecutive in match order.
+ *   g_home_local [E/R, n] fp32 in/out; peer_g_rep: device table of R addresses
+ *   of [rep_rows, n] reduce buffers (fp32 or bf16 by rep_dtype), row j = the
+ *   j-th replica that rank receives; a replica with j >= rep_rows (no row) is
+ *   skipped and flagged EP_DEV_BAD_ROW (a rank receives at most E - E/R
+ *   replicas under any plan);
+ *   plan from ep_plan_from_counts; clear_replicas != 0 zeroes the rows used.
+ */
+EP_API int ep_replica_grad_reduce_peer(float* g_home_local, const uint64_t* peer_g_rep, int64_t rep_rows,
+                                       int rep_dtype, int64_t n, int E, int R, int rank, const int32_t* plan,
+                                       size_t plan_words, int clear_replicas, int32_t* dev_status,
+                                       cudaStream_t stream);
+
+/*
  * ep_route_stats without a scratch argument, for callers that cannot allocate
  * device memory for it: hosts that pass a kernel only its inputs and outputs at
  * enqueue time and forbid allocation there, or runtimes whose device memory is

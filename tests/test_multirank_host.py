@@ -48,3 +48,64 @@ def test_two_ranks_gloo():
     assert [r[1] for r in res] == [7, 1007]            # distinct seeds: independent layers
     assert all(r[2] == 15.0 for r in res)               # max over ranks on every rank
     assert all(r[3] == pytest.approx(2 * 196608 * 20 / 0.015) for r in res)
+
+
+def _gather_worker(rank, world, port, q):
+    """One rank of the rank-local form's exchange: its own expert counts, the
+    all-gather into [R, E] (gather_counts, gloo), and the list offsets a rank
+    derives from the gathered matrix."""
+    import datetime
+    import sys
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle as O
+        from gpu_path import case_inputs
+        from token_dispatch_histogram_b200.ranks import gather_counts
+        S, K, E = 300, 4, 8 * world
+        topk, _, _ = case_inputs(world, S, K, E, 0, seed=17, bias_scale=1.5)
+        own = topk[rank * S:(rank + 1) * S]
+        row = torch.from_numpy(np.bincount(own.reshape(-1), minlength=E).astype(np.int32))
+        counts = torch.full((world, E), -1, dtype=torch.int32)
+        gather_counts(row, counts)
+        C = counts.numpy()
+        # every pair of this rank: (pairs of its expert on lower source ranks)
+        # + (its stable rank among this rank's pairs of that expert) must be its
+        # rank among ALL pairs of that expert in global pair order
+        base = C[:rank].sum(axis=0)
+        flat_all = topk.reshape(-1)
+        ok = True
+        seen = np.zeros(E, dtype=np.int64)
+        for i, e in enumerate(own.reshape(-1)):
+            p = rank * S * K + i
+            g_rank = int(np.count_nonzero(flat_all[:p] == e))
+            ok &= int(base[e] + seen[e]) == g_rank
+            seen[e] += 1
+        loads, _, _ = O.route_stats(topk, E)
+        q.put((rank, C.tolist(), bool(ok), C.sum(axis=0).tolist() == loads.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_rank_local_count_exchange_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert all(r[1] == res[0][1] for r in res)          # the same matrix on every rank
+    assert all(r[2] for r in res)                        # source prefix + local rank = global rank
+    assert all(r[3] for r in res)                        # column sums = the oracle's loads

@@ -78,6 +78,11 @@ _SIGS = {
     "ep_combine_backward": (_I, [_V, _V, _V, _I64, _V, _I64, _I, _I64, _V, _V, _V, _V]),
     "ep_combine": (_I, [_V, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
     "ep_replica_grad_reduce": (_I, [_V, _V, _I, _I64, _I, _I, _V, _SZ, _I, _V, _V]),
+    "ep_plan_from_counts": (_I, [_V, _I, _I64, _I, _I, _V, _V, _SZ, _V, _V]),
+    "ep_layout_rank": (_I, [_V, _I64, _I, _I, _I, _I, _V, _V, _SZ, _V, _SZ, _V, _V, _V, _V]),
+    "ep_dispatch_peer": (_I, [_V, _I64, _I, _I64, _V, _V, _I, _I64, _V, _V]),
+    "ep_combine_peer": (_I, [_V, _I, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
+    "ep_replica_grad_reduce_peer": (_I, [_V, _V, _I64, _I, _I64, _I, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_status_read": (_I, [_V, _V, _V]),
     "ep_selftest_lookback_timeout": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
 }
@@ -319,6 +324,81 @@ def ep_quota_replica_grad_reduce(g_home, g_rep, E, R, plan, clear_replicas=False
     _check("ep_quota_replica_grad_reduce",
            lib().ep_quota_replica_grad_reduce(_p(g_home), _p(g_rep), dt, n, E, R, _p(plan), plan.numel(),
                                               int(bool(clear_replicas)), _p(dev_status), _s(stream)))
+
+
+# ---- rank-local form: one rank of R (one process per GPU), rows moved
+# through a device table of the R ranks' buffer addresses (see ep.h)
+
+def peer_table(tensors, device=None):
+    """Device int64 table of the base addresses of R buffers (this rank's own
+    and the peers' buffers mapped into this process).  The addresses are read
+    on the host from the tensors given; nothing is copied but the table."""
+    addrs = [int(t.data_ptr()) for t in tensors]
+    dev = device if device is not None else tensors[0].device
+    return torch.tensor(addrs, dtype=torch.int64, device=dev)
+
+
+def ep_plan_from_counts(counts, S, K, plan, loads=None, dev_status=None, stream=None):
+    """The plan from the gathered [R, E] load matrix (the same on every rank)."""
+    _dtype(counts, torch.int32)
+    _dtype(plan, torch.int32)
+    if loads is not None:
+        _dtype(loads, torch.int32)
+    R, E = counts.shape
+    _check("ep_plan_from_counts", lib().ep_plan_from_counts(_p(counts), R, S, K, E, _p(loads), _p(plan), plan.numel(),
+                                                            _p(dev_status), _s(stream)))
+
+
+def ep_layout_rank(topk_local, rank, counts, plan, ws, pos_local, pair_slot=None, dev_status=None, stream=None):
+    """Global rows of rank `rank`'s pairs; ws is the scratch ep_route_stats
+    filled for topk_local."""
+    for t in (topk_local, counts, plan, pos_local) + ((pair_slot,) if pair_slot is not None else ()):
+        _dtype(t, torch.int32)
+    S, K = topk_local.shape
+    R, E = counts.shape
+    _check("ep_layout_rank", lib().ep_layout_rank(_p(topk_local), S, K, E, R, rank, _p(counts), _p(plan), plan.numel(),
+                                                  _p(ws), ws.numel() * ws.element_size(), _p(pos_local),
+                                                  _p(pair_slot), _p(dev_status), _s(stream)))
+
+
+def ep_dispatch_peer(x_local, K, pos_local, peers, rows_per_rank, dev_status=None, stream=None):
+    """Rows of x_local [S, H] to their global rows in the R rank buffers."""
+    _dtype(x_local, torch.bfloat16, torch.int16, torch.uint16)
+    _dtype(pos_local, torch.int32)
+    _dtype(peers, torch.int64)
+    S, H = x_local.shape
+    _check("ep_dispatch_peer", lib().ep_dispatch_peer(_p(x_local), S, K, H, _p(pos_local), _p(peers), peers.numel(),
+                                                      rows_per_rank, _p(dev_status), _s(stream)))
+
+
+def ep_combine_peer(peers, rows_per_rank, w_local, pos_local, out_local, K=None, dev_status=None, stream=None):
+    """out_local[t] = sum_k w_local[t,k] * row pos_local[t*K+k] of the rank
+    buffers (w_local None: unit weights, the backward of dispatch; K given)."""
+    _dtype(pos_local, torch.int32)
+    _dtype(peers, torch.int64)
+    S, H = out_local.shape
+    if w_local is not None:
+        _dtype(w_local, torch.float32)
+        K = w_local.shape[1]
+    _check("ep_combine_peer", lib().ep_combine_peer(_p(peers), peers.numel(), rows_per_rank, _p(w_local),
+                                                    _p(pos_local), S, K, H, _p(out_local), _p(dev_status),
+                                                    _s(stream)))
+
+
+def ep_replica_grad_reduce_peer(g_home_local, peers, rep_rows, rep_dtype, E, rank, plan, clear_replicas=False,
+                                dev_status=None, stream=None):
+    """Home rank `rank` adds its experts' replica gradients, read through the
+    peer table of the R ranks' [rep_rows, n] reduce buffers, into
+    g_home_local [E/R, n]."""
+    _dtype(g_home_local, torch.float32)
+    _dtype(plan, torch.int32)
+    _dtype(peers, torch.int64)
+    dt = {torch.float32: EP_DTYPE_F32, torch.bfloat16: EP_DTYPE_BF16}[rep_dtype]
+    n = g_home_local.shape[1]
+    _check("ep_replica_grad_reduce_peer",
+           lib().ep_replica_grad_reduce_peer(_p(g_home_local), _p(peers), rep_rows, dt, n, E, peers.numel(), rank,
+                                             _p(plan), plan.numel(), int(bool(clear_replicas)), _p(dev_status),
+                                             _s(stream)))
 
 
 def ep_selftest_lookback_timeout(topk_ids, E, loads, max_vio, ws, dev_status, stream=None):

@@ -46,9 +46,9 @@ __device__ __forceinline__ void add_bf16x8(float (&a)[8], uint4 v) {
 // One 8-element vector of one replicated expert: home + replicas m0..m0+mc-1
 // in match order.  Up to GRAD_BATCH replica vectors are loaded before any add,
 // so their loads overlap; the adds still go in match order.
-template <bool BF16, bool CLEAR>
-__device__ __forceinline__ void reduce_vec8(float* __restrict__ home, void* __restrict__ g_rep, int64_t n, int64_t j,
-                                            int m0, int mc) {
+// rowp(m): base address of replica m's gradient row.
+template <bool BF16, bool CLEAR, class RowP>
+__device__ __forceinline__ void reduce_vec8(float* __restrict__ home, const RowP& rowp, int64_t j, int m0, int mc) {
   float a[8];
   const float4 h0 = *reinterpret_cast<const float4*>(home + j);
   const float4 h1 = *reinterpret_cast<const float4*>(home + j + 4);
@@ -60,9 +60,9 @@ __device__ __forceinline__ void reduce_vec8(float* __restrict__ home, void* __re
     for (int q = 0; q < GRAD_BATCH; ++q) {
       if (mb + q < m0 + mc) {
         if (BF16) {
-          r[q][0] = ld_stream_v4(static_cast<const uint16_t*>(g_rep) + (int64_t)(mb + q) * n + j);
+          r[q][0] = ld_stream_v4(reinterpret_cast<const uint16_t*>(rowp(mb + q)) + j);
         } else {
-          const float* rp = static_cast<const float*>(g_rep) + (int64_t)(mb + q) * n + j;
+          const float* rp = reinterpret_cast<const float*>(rowp(mb + q)) + j;
           r[q][0] = ld_stream_v4(rp);
           r[q][BF16 ? 0 : 1] = ld_stream_v4(rp + 4);
         }
@@ -77,9 +77,9 @@ __device__ __forceinline__ void reduce_vec8(float* __restrict__ home, void* __re
           add_f32x8(a, r[q][0], r[q][BF16 ? 0 : 1]);
         if (CLEAR) {
           if (BF16) {
-            st_v4(static_cast<uint16_t*>(g_rep) + (int64_t)(mb + q) * n + j, make_uint4(0, 0, 0, 0));
+            st_v4(reinterpret_cast<uint16_t*>(rowp(mb + q)) + j, make_uint4(0, 0, 0, 0));
           } else {
-            float* rp = static_cast<float*>(g_rep) + (int64_t)(mb + q) * n + j;
+            float* rp = reinterpret_cast<float*>(rowp(mb + q)) + j;
             st_v4(rp, make_uint4(0, 0, 0, 0));
             st_v4(rp + 4, make_uint4(0, 0, 0, 0));
           }
@@ -91,11 +91,18 @@ __device__ __forceinline__ void reduce_vec8(float* __restrict__ home, void* __re
   *reinterpret_cast<float4*>(home + j + 4) = make_float4(a[4], a[5], a[6], a[7]);
 }
 
-template <bool BF16, bool CLEAR>
+// PEER (rank-local form): only the experts homed on `rank` are reduced, into
+// g_home [E/R, n]; replica m's row is row m - rank_rep_first[d] of the buffer
+// at peers[d], d = rep_rank[m] (a rank's replicas are consecutive in match
+// order).  The unit's replica row addresses are staged in shared memory.
+template <bool BF16, bool CLEAR, bool PEER>
 __global__ void __launch_bounds__(GRAD_THREADS, 4)
     k_grad_reduce(float* __restrict__ g_home, void* __restrict__ g_rep, int64_t n, const int32_t* __restrict__ plan,
-                  EpPlanLayout L, int E, int32_t* dev_status) {
+                  EpPlanLayout L, int E, const uint64_t* __restrict__ peers, int R, int rank, int64_t rep_rows,
+                  int32_t* dev_status) {
   __shared__ int s_e, s_m0, s_mc;
+  __shared__ char* s_rows[PEER ? EP_MAX_RANKS : 1];
+  const int ER = E / R;
   const int nC = min(max(plan[L.n_chunks], 0), E);
   const int64_t units_per_expert = (n + GRAD_UNIT - 1) / GRAD_UNIT;
   const int64_t total = (int64_t)nC * units_per_expert;
@@ -111,9 +118,11 @@ __global__ void __launch_bounds__(GRAD_THREADS, 4)
         m0 = plan[L.copy_first + e];
         mc = plan[L.copy_cnt + e];
       }
-      if (e < 0 || e >= E || m0 < 0 || mc < 0 || m0 + mc > L.cap) {
+      if (e < 0 || e >= E || m0 < 0 || mc < 0 || m0 + mc > L.cap || (PEER && mc > EP_MAX_RANKS)) {
         flag(dev_status, EP_DEV_BAD_ROW);
         s_e = -1;
+      } else if (PEER && e / ER != rank) {
+        s_e = -1;  // another rank's expert
       } else {
         s_e = e;
         s_m0 = m0;
@@ -124,24 +133,46 @@ __global__ void __launch_bounds__(GRAD_THREADS, 4)
     const int e = s_e;
     if (e < 0) continue;
     const int m0 = s_m0, mc = s_mc;
-    float* home = g_home + (int64_t)e * n;
+    const int64_t esz = BF16 ? 2 : 4;
+    if (PEER) {
+      for (int q = threadIdx.x; q < mc; q += blockDim.x) {
+        const int m = m0 + q;
+        const int d = plan[L.rep_rank + m];
+        char* base = nullptr;
+        if (d >= 0 && d < R) {
+          const int64_t j = m - plan[L.rank_rep_first + d];
+          const uint64_t pb = __ldg(peers + d);
+          if (pb && !(pb & 15u) && j >= 0 && j < rep_rows) base = reinterpret_cast<char*>(pb) + j * n * esz;
+        }
+        if (!base) flag(dev_status, EP_DEV_BAD_ROW);
+        s_rows[PEER ? q : 0] = base;
+      }
+      __syncthreads();
+      bool ok = true;
+      for (int q = 0; q < mc; ++q) ok = ok && s_rows[PEER ? q : 0] != nullptr;
+      if (!ok) continue;  // every thread saw the same table: skip the unit together
+    }
+    auto rowp = [&](int m) -> char* {
+      return PEER ? s_rows[PEER ? m - m0 : 0] : static_cast<char*>(g_rep) + (int64_t)m * n * esz;
+    };
+    float* home = g_home + (int64_t)(PEER ? e - rank * ER : e) * n;
     if (vec) {
 #pragma unroll
       for (int vv = 0; vv < GRAD_VECS; ++vv) {
         const int64_t j = j0 + ((int64_t)vv * GRAD_THREADS + threadIdx.x) * 8;
         if (j >= n) break;
-        reduce_vec8<BF16, CLEAR>(home, g_rep, n, j, m0, mc);
+        reduce_vec8<BF16, CLEAR>(home, rowp, j, m0, mc);
       }
     } else {
       for (int64_t j = j0 + threadIdx.x; j < min(n, j0 + GRAD_UNIT); j += blockDim.x) {
         float a = home[j];
         for (int m = m0; m < m0 + mc; ++m) {
           if (!BF16) {
-            float* r = static_cast<float*>(g_rep) + (int64_t)m * n + j;
+            float* r = reinterpret_cast<float*>(rowp(m)) + j;
             a = __fadd_rn(a, *r);
             if (CLEAR) *r = 0.0f;
           } else {
-            uint16_t* r = static_cast<uint16_t*>(g_rep) + (int64_t)m * n + j;
+            uint16_t* r = reinterpret_cast<uint16_t*>(rowp(m)) + j;
             a = __fadd_rn(a, bf16_bits_to_f32(*r));
             if (CLEAR) *r = 0;
           }
@@ -163,18 +194,28 @@ void quota_layout(int E, int R, EpQuotaLayout* L);
 
 // The plan fields the reduction reads: replicated experts in match order, and
 // each expert's first replica and replica count.
+template <bool PEER>
+static const void* grad_fn(int rep_dtype, int clear) {
+  if (rep_dtype == EP_DTYPE_F32)
+    return clear ? (const void*)k_grad_reduce<false, true, PEER> : (const void*)k_grad_reduce<false, false, PEER>;
+  return clear ? (const void*)k_grad_reduce<true, true, PEER> : (const void*)k_grad_reduce<true, false, PEER>;
+}
+
+// peers == NULL: g_home [E, n], g_rep [cap, n] (row m = replica m).  Else the
+// rank-local form for `rank` (g_home [E/R, n], replica rows behind peers).
 static int run_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, const int32_t* plan,
-                           EpPlanLayout L, int clear_replicas, int32_t* dev_status, cudaStream_t stream) {
+                           EpPlanLayout L, int clear_replicas, const uint64_t* peers, int R, int rank,
+                           int64_t rep_rows, int32_t* dev_status, cudaStream_t stream) {
   if (n == 0) return EP_OK;
-  if (!g_home || !g_rep || !aligned16(g_home) || !aligned16(g_rep)) return EP_ERR_ARG;
+  if (!g_home || !aligned16(g_home)) return EP_ERR_ARG;
+  if (!peers && (!g_rep || !aligned16(g_rep))) return EP_ERR_ARG;
   const int64_t units = (int64_t)E * ((n + GRAD_UNIT - 1) / GRAD_UNIT);  // upper bound (n_chunks <= E)
   // 4 CTAs per SM measured best
-  const void* fn = rep_dtype == EP_DTYPE_F32
-                       ? (clear_replicas ? (const void*)k_grad_reduce<false, true> : (const void*)k_grad_reduce<false, false>)
-                       : (clear_replicas ? (const void*)k_grad_reduce<true, true> : (const void*)k_grad_reduce<true, false>);
+  const void* fn = peers ? grad_fn<true>(rep_dtype, clear_replicas) : grad_fn<false>(rep_dtype, clear_replicas);
   const int grid = occupancy_grid(fn, GRAD_THREADS, 0, units, 4);
   void* gr = const_cast<void*>(g_rep);
-  void* args[] = {(void*)&g_home, (void*)&gr, (void*)&n, (void*)&plan, (void*)&L, (void*)&E, (void*)&dev_status};
+  void* args[] = {(void*)&g_home, (void*)&gr,    (void*)&n, (void*)&plan, (void*)&L,         (void*)&E,
+                  (void*)&peers,  (void*)&R,     (void*)&rank, (void*)&rep_rows, (void*)&dev_status};
   if (cudaLaunchKernel(fn, dim3(grid), dim3(GRAD_THREADS), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
@@ -190,7 +231,23 @@ extern "C" int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_
   EpPlanLayout L;
   plan_layout(E, R, &L);
   if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
-  return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, dev_status, stream);
+  return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, nullptr, R, 0, 0, dev_status, stream);
+}
+
+extern "C" int ep_replica_grad_reduce_peer(float* g_home_local, const uint64_t* peer_g_rep, int64_t rep_rows,
+                                           int rep_dtype, int64_t n, int E, int R, int rank, const int32_t* plan,
+                                           size_t plan_words, int clear_replicas, int32_t* dev_status,
+                                           cudaStream_t stream) {
+  if (n < 0 || E < 1 || E > EP_MAX_EXPERTS || R < 1 || R > EP_MAX_RANKS || E % R || rank < 0 || rank >= R ||
+      rep_rows < 0)
+    return EP_ERR_ARG;
+  if (rep_dtype != EP_DTYPE_F32 && rep_dtype != EP_DTYPE_BF16) return EP_ERR_ARG;
+  if (!plan || !peer_g_rep) return EP_ERR_ARG;
+  EpPlanLayout L;
+  plan_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  return run_grad_reduce(g_home_local, nullptr, rep_dtype, n, E, plan, L, clear_replicas, peer_g_rep, R, rank,
+                         rep_rows, dev_status, stream);
 }
 
 extern "C" int ep_quota_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
@@ -209,5 +266,5 @@ extern "C" int ep_quota_replica_grad_reduce(float* g_home, const void* g_rep, in
   L.rep_experts = Q.rep_experts;
   L.copy_first = Q.rep_first;
   L.copy_cnt = Q.rep_cnt;
-  return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, dev_status, stream);
+  return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, nullptr, R, 0, 0, dev_status, stream);
 }

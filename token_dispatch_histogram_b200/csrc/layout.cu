@@ -24,8 +24,14 @@ namespace ep {
 int run_hist(const int32_t* topk, int64_t P, int E, void* ws, int32_t* loads, double* max_vio, int32_t* dev_status,
              cudaStream_t st);
 
+// base_counts == NULL: the pairs are the whole problem (rows in [0, P)).
+// Otherwise (rank-local form) they are source rank base_rank's pairs, counts
+// [R, E] is the gathered load matrix, each expert's list position is offset by
+// the pairs of that expert on lower source ranks, rows lie in [0, rows_total),
+// and src may be NULL.
 __global__ void __launch_bounds__(SCAT_THREADS)
     k_layout(const int32_t* __restrict__ topk, int64_t P, int E, int tile, const int32_t* __restrict__ tile_excl,
+             const int32_t* __restrict__ base_counts, int base_rank, int64_t rows_total,
              const int32_t* __restrict__ plan, EpPlanLayout L, int32_t* __restrict__ pos, int32_t* __restrict__ src,
              int32_t* __restrict__ pair_slot, int32_t* dev_status) {
   extern __shared__ int32_t sm[];
@@ -39,8 +45,18 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   int32_t* s_rb = s_cc + E;                       // [cap] rep_begin
   int32_t* s_rc = s_rb + cap;                     // [cap] rep_count
   int32_t* s_rbase = s_rc + cap;                  // [cap] rep_base
+  int32_t* s_excl = s_rbase + cap;                // [E] (rank-local form) list offset of the tile
   __shared__ int s_flags;
   if (threadIdx.x == 0) s_flags = 0;
+  const int32_t* excl_row = tile_excl + (int64_t)blockIdx.x * E;
+  if (base_counts) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int32_t b = excl_row[e];
+      for (int r = 0; r < base_rank; ++r) b += base_counts[(int64_t)r * E + e];
+      s_excl[e] = b;
+    }
+    excl_row = s_excl;  // read by tile_stable_ranks after its first barrier
+  }
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     s_hc[e] = plan[L.home_count + e];
     s_hb[e] = plan[L.home_base + e];
@@ -76,14 +92,14 @@ __global__ void __launch_bounds__(SCAT_THREADS)
         }
       }
     }
-    if (row < 0 || row >= P) {
+    if (row < 0 || row >= rows_total) {
       atomicOr(&s_flags, EP_DEV_BAD_ROW);
       pos[p] = -1;
       if (pair_slot) pair_slot[p] = -1;
       return;
     }
     pos[p] = row;
-    src[row] = (int32_t)p;
+    if (src) src[row] = (int32_t)p;
     if (pair_slot) pair_slot[p] = slot;
   };
   auto bad = [&](int64_t p) {
@@ -92,8 +108,7 @@ __global__ void __launch_bounds__(SCAT_THREADS)
     if (pair_slot) pair_slot[p] = -1;
   };
   const int64_t p0 = (int64_t)blockIdx.x * tile;
-  tile_stable_ranks(topk, E, tile, p0, (int)min((int64_t)tile, P - p0), tile_excl + (int64_t)blockIdx.x * E, s_ids,
-                    s_whist, emit, bad);
+  tile_stable_ranks(topk, E, tile, p0, (int)min((int64_t)tile, P - p0), excl_row, s_ids, s_whist, emit, bad);
   __syncthreads();
   if (threadIdx.x == 0 && s_flags) flag(dev_status, s_flags);
 }
@@ -159,6 +174,20 @@ __global__ void __launch_bounds__(SCAT_THREADS)
 
 size_t scatter_smem_base(int tile, int E) { return sizeof(int32_t) * ((size_t)tile + (size_t)SCAT_WARPS * E); }
 
+static int run_layout(const int32_t* topk, int64_t P, int E, int tile, int64_t nt, const int32_t* tile_excl,
+                      const int32_t* base_counts, int base_rank, int64_t rows_total, const int32_t* plan,
+                      const EpPlanLayout& L, int32_t* pos, int32_t* src, int32_t* pair_slot, int32_t* dev_status,
+                      cudaStream_t stream) {
+  const size_t smem = scatter_smem_base(tile, E) + sizeof(int32_t) * (5 * (size_t)E + 3 * (size_t)L.cap);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return EP_ERR_CUDA;
+  k_layout<<<(unsigned)nt, SCAT_THREADS, smem, stream>>>(topk, P, E, tile, tile_excl, base_counts, base_rank,
+                                                         rows_total, plan, L, pos, src, pair_slot, dev_status);
+  count_launch();
+  return launch_status();
+}
+
 }  // namespace ep
 
 using namespace ep;
@@ -178,16 +207,31 @@ extern "C" int ep_layout(const int32_t* topk_ids, int64_t T, int K, int E, int R
   if (P == 0) return EP_OK;
   const int tile = tile_pairs_for(P);
   const int64_t nt = num_tiles(P, tile);
-  const size_t smem = scatter_smem_base(tile, E) + sizeof(int32_t) * (4 * (size_t)E + 3 * (size_t)L.cap);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return EP_ERR_CUDA;
   const char* w = static_cast<const char*>(ws);
-  k_layout<<<(unsigned)nt, SCAT_THREADS, smem, stream>>>(topk_ids, P, E, tile,
-                                                         reinterpret_cast<const int32_t*>(w + wl.excl_off), plan, L,
-                                                         pos, src, pair_slot, dev_status);
-  count_launch();
-  return launch_status();
+  return run_layout(topk_ids, P, E, tile, nt, reinterpret_cast<const int32_t*>(w + wl.excl_off), nullptr, 0, P, plan, L,
+                    pos, src, pair_slot, dev_status, stream);
+}
+
+extern "C" int ep_layout_rank(const int32_t* topk_local, int64_t S, int K, int E, int R, int rank,
+                              const int32_t* counts, const int32_t* plan, size_t plan_words, const void* ws,
+                              size_t ws_bytes, int32_t* pos_local, int32_t* pair_slot, int32_t* dev_status,
+                              cudaStream_t stream) {
+  if (!valid_tke(S, K, E) || R < 1 || R > EP_MAX_RANKS || E % R || rank < 0 || rank >= R) return EP_ERR_ARG;
+  if ((int64_t)R * S * K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (!plan || !ws || !counts) return EP_ERR_ARG;
+  const int64_t P = S * K;
+  if (P > 0 && (!topk_local || !pos_local)) return EP_ERR_ARG;
+  EpPlanLayout L;
+  plan_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  const WsLayout wl = ws_layout(P, E);
+  if (ws_bytes < wl.bytes) return EP_ERR_CAPACITY;
+  if (P == 0) return EP_OK;
+  const int tile = tile_pairs_for(P);
+  const int64_t nt = num_tiles(P, tile);
+  const char* w = static_cast<const char*>(ws);
+  return run_layout(topk_local, P, E, tile, nt, reinterpret_cast<const int32_t*>(w + wl.excl_off), counts, rank,
+                    (int64_t)R * P, plan, L, pos_local, nullptr, pair_slot, dev_status, stream);
 }
 
 extern "C" int ep_align_sort(const int32_t* topk_ids, int64_t T, int K, int E, int block_m,

@@ -39,6 +39,31 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   plan_block(s_loads, R, SK, E, plan, L, work, dev_status);
 }
 
+// The plan from the gathered [R, E] load matrix (rank-local form): the column
+// sums are the loads, then the same block planner.  A column sum outside int32
+// range becomes -1, which the planner rejects as invalid loads.
+__global__ void __launch_bounds__(PLAN_THREADS)
+    k_plan_counts(const int32_t* __restrict__ counts, int R, int32_t SK, int E, int32_t* __restrict__ loads,
+                  int32_t* __restrict__ plan, EpPlanLayout L, int32_t* dev_status) {
+  extern __shared__ int32_t sm[];
+  int32_t* s_loads = sm;       // [E]
+  int32_t* work = sm + E;      // plan_work_words(E, R)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int64_t t = 0;
+    bool ok = true;
+    for (int r = 0; r < R; ++r) {
+      const int32_t c = counts[(int64_t)r * E + e];
+      ok = ok && c >= 0;
+      t += c;
+    }
+    const int32_t v = (ok && t <= INT32_MAX) ? (int32_t)t : -1;
+    s_loads[e] = v;
+    if (loads) loads[e] = v;
+  }
+  __syncthreads();
+  plan_block(s_loads, R, SK, E, plan, L, work, dev_status);
+}
+
 // Prefetch slots under a per-rank budget B: replica m is the j-th replica its
 // rank receives, j = m - rank_rep_first[rank] (replicas of a rank are
 // consecutive in match order); it gets weight row E + j while j < B, else -1
@@ -134,6 +159,23 @@ extern "C" int ep_plan(const int32_t* loads, int R, int64_t S, int K, int E, int
       cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EP_ERR_CUDA;
   k_plan<<<1, PLAN_THREADS, smem, stream>>>(loads, R, (int32_t)(S * K), E, plan, L, dev_status);
+  count_launch();
+  return launch_status();
+}
+
+extern "C" int ep_plan_from_counts(const int32_t* counts, int R, int64_t S, int K, int E, int32_t* loads,
+                                   int32_t* plan, size_t plan_words, int32_t* dev_status, cudaStream_t stream) {
+  if (!counts || !plan || R < 1 || R > EP_MAX_RANKS || E < 1 || E > EP_MAX_EXPERTS || E % R || K < 1 || S < 0)
+    return EP_ERR_ARG;
+  if ((int64_t)R * S * K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  EpPlanLayout L;
+  plan_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  const size_t smem = plan_smem_bytes(E, R);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_plan_counts, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return EP_ERR_CUDA;
+  k_plan_counts<<<1, PLAN_THREADS, smem, stream>>>(counts, R, (int32_t)(S * K), E, loads, plan, L, dev_status);
   count_launch();
   return launch_status();
 }

@@ -14,6 +14,12 @@
 // drain; the launch sizes stages x CTAs so about 32 KB of loads are in flight
 // per SM, which measured fastest.
 //
+// Rank-local form (PEER = true): the R ranks' buffers are separate allocations,
+// possibly on other GPUs, reached through a device table of R base pointers;
+// global row `row` lives at peers[row / rows_per_rank] + (row % rows_per_rank)
+// rows.  Dispatch then writes each row straight into the receiving rank's
+// buffer and combine reads it back from there; nothing else changes.
+//
 // Combine: out[t] = bf16_rn(sum_k w[t,k] * float(y[pos[t*K+k]])), fp32 in k
 // order, separate multiply and add roundings (no FMA).  One thread owns 8
 // consecutive bf16 of one output row (one 16-byte vector); it issues all K
@@ -36,9 +42,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
+template <bool PEER>
 __global__ void __launch_bounds__(32)
     k_dispatch(const uint8_t* __restrict__ x, int64_t T, int K, uint32_t row_bytes, const int32_t* __restrict__ pos,
-               int64_t buf_rows, uint8_t* __restrict__ buf, int stages, int32_t* dev_status) {
+               int64_t buf_rows, uint8_t* __restrict__ buf, const uint64_t* __restrict__ peers,
+               int64_t rows_per_rank, int stages, int32_t* dev_status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t stride_b = (row_bytes + 127u) & ~127u;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stride_b);
@@ -77,9 +85,22 @@ __global__ void __launch_bounds__(32)
     }
     if (lane < K) {
       const int32_t row = ring[s * K + lane];
-      if (row >= 0 && row < buf_rows)
-        bulk_store(buf + (int64_t)row * row_bytes, smem + (size_t)s * stride_b, row_bytes);
-      else
+      if (row >= 0 && row < buf_rows) {
+        uint8_t* dst;
+        if (PEER) {
+          const int64_t d = row / rows_per_rank;
+          const uint64_t base = __ldg(peers + d);
+          // a missing or misaligned rank buffer is reported, never written
+          dst = (base && !(base & 15u)) ? reinterpret_cast<uint8_t*>(base) + (row - d * rows_per_rank) * (int64_t)row_bytes
+                                        : nullptr;
+        } else {
+          dst = buf + (int64_t)row * row_bytes;
+        }
+        if (dst)
+          bulk_store(dst, smem + (size_t)s * stride_b, row_bytes);
+        else
+          bad = EP_DEV_BAD_ROW;
+      } else
         bad = EP_DEV_BAD_ROW;
     }
     bulk_commit();
@@ -144,14 +165,15 @@ __global__ void __launch_bounds__(256)
 // memory one iteration ahead (double buffer), so each thread's K 16-byte row
 // loads issue back to back without waiting on index loads, and registers stay
 // within 64 (four 256-thread CTAs per SM).
-template <int K>
+template <int K, bool PEER>
 __global__ void __launch_bounds__(256, 4)
     k_combine(const uint16_t* __restrict__ y, int64_t y_rows, const float* __restrict__ w,
               const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ out,
-              int32_t* dev_status) {
+              const uint64_t* __restrict__ peers, int64_t rows_per_rank, int32_t* dev_status) {
   constexpr int MAXT = 8;  // tokens per CTA iteration (rows narrower than 256 vectors)
   __shared__ int32_t s_rows[2][MAXT][K];
   __shared__ float s_w[2][MAXT][K];
+  __shared__ const uint16_t* s_ptr[PEER ? 2 : 1][PEER ? MAXT : 1][PEER ? K : 1];  // row bases (PEER)
   __shared__ int s_bad;
   const int64_t nvec = H / 8;
   const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);  // threads per token
@@ -175,6 +197,20 @@ __global__ void __launch_bounds__(256, 4)
       }
       s_rows[b][s][k] = r;
       s_w[b][s][k] = wk;
+      if constexpr (PEER) {
+        const uint16_t* base = nullptr;
+        if (r >= 0) {
+          const int64_t d = r / rows_per_rank;
+          const uint64_t pb = __ldg(peers + d);
+          if (pb && !(pb & 15u)) {
+            base = reinterpret_cast<const uint16_t*>(pb) + (r - d * rows_per_rank) * H;
+          } else {  // a missing or misaligned rank buffer is reported, never read
+            s_rows[b][s][k] = -1;
+            s_bad = 1;
+          }
+        }
+        s_ptr[PEER ? b : 0][PEER ? s : 0][PEER ? k : 0] = base;
+      }
     }
   };
   int64_t tb = (int64_t)blockIdx.x * tpc;
@@ -189,7 +225,11 @@ __global__ void __launch_bounds__(256, 4)
 #pragma unroll
         for (int k = 0; k < K; ++k) {
           const int32_t r = s_rows[b][sub][k];
-          in[k] = r >= 0 ? ld_stream_v4(y + (int64_t)r * H + v * 8) : make_uint4(0, 0, 0, 0);
+          if constexpr (PEER)
+            in[k] = r >= 0 ? ld_stream_v4(s_ptr[PEER ? b : 0][PEER ? sub : 0][PEER ? k : 0] + v * 8)
+                           : make_uint4(0, 0, 0, 0);
+          else
+            in[k] = r >= 0 ? ld_stream_v4(y + (int64_t)r * H + v * 8) : make_uint4(0, 0, 0, 0);
         }
         float acc[8];
 #pragma unroll
@@ -374,13 +414,13 @@ int occupancy_grid(const void* fn, int threads, size_t smem, int64_t work_items,
 
 using namespace ep;
 
-extern "C" int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
-                           int64_t buf_rows, int32_t* dev_status, cudaStream_t stream) {
-  if (T < 0 || K < 1 || K > 32 || H < 8 || H % 8 || buf_rows < 0) return EP_ERR_ARG;
-  if (H * 2 > (1 << 20)) return EP_ERR_ARG;  // one row per bulk copy, at most 1 MiB
-  if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
-  if (T == 0) return EP_OK;
-  if (!x || !pos || !buf || !aligned16(x) || !aligned16(buf)) return EP_ERR_ARG;
+namespace ep {
+
+// Dispatch launch shared by the one-buffer and the rank-local (peer) entry
+// points.  peers == NULL: rows go to buf[row]; else to the rank buffers.
+static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
+                        int64_t buf_rows, const uint64_t* peers, int64_t rows_per_rank, int32_t* dev_status,
+                        cudaStream_t stream) {
   const uint32_t row_bytes = (uint32_t)(H * 2);
   const uint32_t stride_b = (row_bytes + 127u) & ~127u;
   // Measured on B200: the scatter runs fastest with about 32 KB of row loads
@@ -393,14 +433,42 @@ extern "C" int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const
   const int per_sm = (int)std::min<uint32_t>(32, std::max<uint32_t>(1, (target + stages * stride_b - 1) / (stages * stride_b)));
   size_t smem = (size_t)stages * stride_b + DISPATCH_MAX_STAGES * 8 + (size_t)stages * K * 4;
   if (smem > 200 * 1024) return EP_ERR_ARG;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_dispatch, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  const void* fn = peers ? (const void*)k_dispatch<true> : (const void*)k_dispatch<false>;
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EP_ERR_CUDA;
-  const int grid = occupancy_grid((const void*)k_dispatch, 32, smem, T, per_sm);
-  k_dispatch<<<grid, 32, smem, stream>>>(reinterpret_cast<const uint8_t*>(x), T, K, row_bytes, pos, buf_rows,
-                                         reinterpret_cast<uint8_t*>(buf), stages, dev_status);
+  const int grid = occupancy_grid(fn, 32, smem, T, per_sm);
+  const uint8_t* xb = reinterpret_cast<const uint8_t*>(x);
+  uint8_t* bb = reinterpret_cast<uint8_t*>(buf);
+  void* args[] = {(void*)&xb,    (void*)&T,     (void*)&K,  (void*)&row_bytes,     (void*)&pos,
+                  (void*)&buf_rows, (void*)&bb, (void*)&peers, (void*)&rows_per_rank, (void*)&stages,
+                  (void*)&dev_status};
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(32), args, smem, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
+}
+
+}  // namespace ep
+
+extern "C" int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
+                           int64_t buf_rows, int32_t* dev_status, cudaStream_t stream) {
+  if (T < 0 || K < 1 || K > 32 || H < 8 || H % 8 || buf_rows < 0) return EP_ERR_ARG;
+  if (H * 2 > (1 << 20)) return EP_ERR_ARG;  // one row per bulk copy, at most 1 MiB
+  if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (T == 0) return EP_OK;
+  if (!x || !pos || !buf || !aligned16(x) || !aligned16(buf)) return EP_ERR_ARG;
+  return run_dispatch(x, T, K, H, pos, buf, buf_rows, nullptr, 0, dev_status, stream);
+}
+
+extern "C" int ep_dispatch_peer(const uint16_t* x_local, int64_t S, int K, int64_t H, const int32_t* pos_local,
+                                const uint64_t* peer_bufs, int R, int64_t rows_per_rank, int32_t* dev_status,
+                                cudaStream_t stream) {
+  if (S < 0 || K < 1 || K > 32 || H < 8 || H % 8 || R < 1 || R > EP_MAX_RANKS || rows_per_rank < 1) return EP_ERR_ARG;
+  if (H * 2 > (1 << 20)) return EP_ERR_ARG;
+  if (S * (int64_t)K >= ((int64_t)1 << 31) || (int64_t)R * rows_per_rank >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (S == 0) return EP_OK;
+  if (!x_local || !pos_local || !peer_bufs || !aligned16(x_local)) return EP_ERR_ARG;
+  return run_dispatch(x_local, S, K, H, pos_local, nullptr, (int64_t)R * rows_per_rank, peer_bufs, rows_per_rank,
+                      dev_status, stream);
 }
 
 extern "C" int ep_expert_scale(const uint16_t* buf, int64_t rows, int64_t H, const int32_t* src,
@@ -415,33 +483,61 @@ extern "C" int ep_expert_scale(const uint16_t* buf, int64_t rows, int64_t H, con
   return launch_status();
 }
 
+namespace ep {
+
+template <bool PEER>
+static const void* combine_fn(int K) {
+  switch (K) {
+    case 1: return (const void*)k_combine<1, PEER>;
+    case 2: return (const void*)k_combine<2, PEER>;
+    case 3: return (const void*)k_combine<3, PEER>;
+    case 4: return (const void*)k_combine<4, PEER>;
+    case 5: return (const void*)k_combine<5, PEER>;
+    case 6: return (const void*)k_combine<6, PEER>;
+    case 7: return (const void*)k_combine<7, PEER>;
+    case 8: return (const void*)k_combine<8, PEER>;
+    default: return nullptr;
+  }
+}
+
+}  // namespace ep
+
 extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* pos, int64_t T, int K,
                           int64_t H, uint16_t* out, int32_t* dev_status, cudaStream_t stream) {
   if (T < 0 || K < 1 || K > 32 || H < 8 || H % 8 || y_rows < 0) return EP_ERR_ARG;
   if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
   if (T == 0) return EP_OK;
   if (!y || !pos || !out || !aligned16(y) || !aligned16(out)) return EP_ERR_ARG;  // w == NULL: unit weights
-  const void* fn = nullptr;
-  switch (K) {
-    case 1: fn = (const void*)k_combine<1>; break;
-    case 2: fn = (const void*)k_combine<2>; break;
-    case 3: fn = (const void*)k_combine<3>; break;
-    case 4: fn = (const void*)k_combine<4>; break;
-    case 5: fn = (const void*)k_combine<5>; break;
-    case 6: fn = (const void*)k_combine<6>; break;
-    case 7: fn = (const void*)k_combine<7>; break;
-    case 8: fn = (const void*)k_combine<8>; break;
-    default: break;
-  }
+  const void* fn = combine_fn<false>(K);
   if (fn) {
     const int grid = occupancy_grid(fn, 256, 0, T, 4);
-    void* args[] = {(void*)&y, (void*)&y_rows, (void*)&w, (void*)&pos, (void*)&T, (void*)&H, (void*)&out,
-                    (void*)&dev_status};
+    const uint64_t* peers = nullptr;
+    int64_t rpr = 0;
+    void* args[] = {(void*)&y,   (void*)&y_rows, (void*)&w,     (void*)&pos, (void*)&T,
+                    (void*)&H,   (void*)&out,    (void*)&peers, (void*)&rpr, (void*)&dev_status};
     if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   } else {
     const int grid = occupancy_grid((const void*)k_combine_any, 256, 0, T * (H / 8) / 256 + 1, 8);
     k_combine_any<<<grid, 256, 0, stream>>>(y, y_rows, w, pos, T, K, H, out, dev_status);
   }
+  count_launch();
+  return launch_status();
+}
+
+extern "C" int ep_combine_peer(const uint64_t* peer_bufs, int R, int64_t rows_per_rank, const float* w_local,
+                               const int32_t* pos_local, int64_t S, int K, int64_t H, uint16_t* out_local,
+                               int32_t* dev_status, cudaStream_t stream) {
+  if (S < 0 || K < 1 || K > 8 || H < 8 || H % 8 || R < 1 || R > EP_MAX_RANKS || rows_per_rank < 1) return EP_ERR_ARG;
+  if (S * (int64_t)K >= ((int64_t)1 << 31) || (int64_t)R * rows_per_rank >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (S == 0) return EP_OK;
+  if (!peer_bufs || !pos_local || !out_local || !aligned16(out_local)) return EP_ERR_ARG;  // w NULL: unit weights
+  const void* fn = combine_fn<true>(K);
+  const int grid = occupancy_grid(fn, 256, 0, S, 4);
+  const uint16_t* y = nullptr;
+  int64_t y_rows = (int64_t)R * rows_per_rank;
+  void* args[] = {(void*)&y,         (void*)&y_rows,   (void*)&w_local,   (void*)&pos_local,     (void*)&S,
+                  (void*)&H,         (void*)&out_local, (void*)&peer_bufs, (void*)&rows_per_rank, (void*)&dev_status};
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }

@@ -1,0 +1,121 @@
+"""Rank-local form of the path: one rank of R, one process per GPU.
+
+The one-buffer path (EpLayer) holds all R ranks as partitions of one static
+buffer.  Here each rank holds only its own tokens and its own S*K-row receive
+buffer, and rows move through a device table of the R ranks' buffer addresses
+(this GPU's buffer and the peers' buffers mapped into this process, e.g. by
+symmetric memory or CUDA IPC).  The MoonEP page ("Online planning, zero copy
+και στατικά σχήματα") has tokens written straight into their final
+expert-grouped rows on the remote ranks; the UltraEP page ("その仕組みは高速な
+エキスパート複製に依存する") plans from the exact source-rank x expert load
+matrix.  One step on rank r:
+
+  count()           local histogram -> counts_row (ep_route_stats on S tokens)
+  gather            all ranks' rows -> counts [R, E] (the one collective)
+  plan_and_layout() ep_plan_from_counts + ep_layout_rank (no further exchange)
+  dispatch()        ep_dispatch_peer: rows into the receiving ranks' buffers
+  combine()         ep_combine_peer: expert rows back from those buffers
+  grad_reduce()     ep_replica_grad_reduce_peer: replica gradients home
+
+Every device step is one of libep.so's kernels; this module only allocates
+and sequences.  gather_counts is the collective, through torch.distributed.
+"""
+import torch
+import torch.distributed as dist
+
+from . import (ep_combine_peer, ep_dispatch_peer, ep_layout_rank, ep_plan_from_counts, ep_plan_layout,
+               ep_replica_grad_reduce_peer, ep_route_stats, ep_status_read, ep_workspace_size)
+
+
+def gather_counts(counts_row, counts, group=None):
+    """All-gather every rank's [E] expert counts into counts [R, E], row r =
+    rank r's, on every rank (NCCL on GPUs, gloo on CPU)."""
+    R = dist.get_world_size(group)
+    if counts.shape != (R, counts_row.numel()):
+        raise ValueError(f"counts must be [{R}, {counts_row.numel()}]")
+    parts = list(counts.unbind(0))
+    dist.all_gather(parts, counts_row.contiguous(), group=group)
+    return counts
+
+
+class EpRank:
+    """Static buffers of one rank of R: S tokens of top-K routing, H hidden.
+
+    buf is this rank's S*K-row receive buffer (expert-grouped: home experts in
+    id order, then received replicas in match order); peers must be set to the
+    R ranks' buffers (set_peers) before dispatch/combine.  With grad_n > 0,
+    g_home holds this rank's E/R home experts' gradients [E/R, grad_n] fp32 and
+    g_rep the gradients of the replicas it receives [rep_rows, grad_n], row j =
+    its j-th received replica (default E - E/R rows, enough for any plan;
+    grad_peers: the R ranks' g_rep, set_grad_peers)."""
+
+    def __init__(self, rank, R, S, K, E, H, device="cuda", grad_n=0, grad_dtype=torch.float32, rep_rows=None):
+        if E % R:
+            raise ValueError("E must be a multiple of R")
+        self.rank, self.R, self.S, self.K, self.E, self.H = rank, R, S, K, E, H
+        self.device = torch.device(device)
+        dev = self.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.SK = S * K
+        self.topk_local = torch.zeros((S, K), **i32)
+        self.w_local = torch.zeros((S, K), dtype=torch.float32, device=dev)
+        self.x_local = torch.zeros((S, H), dtype=torch.bfloat16, device=dev)
+        self.out_local = torch.zeros((S, H), dtype=torch.bfloat16, device=dev)
+        self.buf = torch.zeros((self.SK, H), dtype=torch.bfloat16, device=dev)
+        self.counts_row = torch.zeros(E, **i32)
+        self.counts = torch.zeros((R, E), **i32)
+        self.loads = torch.zeros(E, **i32)
+        self.max_vio_local = torch.zeros(1, dtype=torch.float64, device=dev)
+        self.plan_layout = ep_plan_layout(E, R)
+        self.plan = torch.zeros(self.plan_layout["words"], **i32)
+        self.pos_local = torch.zeros(self.SK, **i32)
+        self.ws = torch.zeros(ep_workspace_size(S, K, E), dtype=torch.uint8, device=dev)
+        self.dev_status = torch.zeros(1, **i32)
+        self.grad_n = grad_n
+        if grad_n:
+            self.g_home = torch.zeros((E // R, grad_n), dtype=torch.float32, device=dev)
+            # a rank receives at most E - E/R replicas (one per chunk of another rank's expert)
+            self.rep_rows = max(1, E - E // R) if rep_rows is None else rep_rows
+            self.g_rep = torch.zeros((self.rep_rows, grad_n), dtype=grad_dtype, device=dev)
+        self.peers = None
+        self.grad_peers = None
+
+    def set_peers(self, peers):
+        """peers: device int64 [R] table of the R ranks' buf addresses."""
+        if peers.numel() != self.R or peers.dtype != torch.int64:
+            raise ValueError("peers must be an int64 table of R addresses")
+        self.peers = peers
+
+    def set_grad_peers(self, grad_peers):
+        """grad_peers: device int64 [R] table of the R ranks' g_rep addresses."""
+        if grad_peers.numel() != self.R or grad_peers.dtype != torch.int64:
+            raise ValueError("grad_peers must be an int64 table of R addresses")
+        self.grad_peers = grad_peers
+
+    def count(self, stream=None):
+        ep_route_stats(self.topk_local, self.E, self.counts_row, self.max_vio_local, self.ws, self.dev_status, stream)
+
+    def plan_and_layout(self, stream=None):
+        ep_plan_from_counts(self.counts, self.S, self.K, self.plan, self.loads, self.dev_status, stream)
+        ep_layout_rank(self.topk_local, self.rank, self.counts, self.plan, self.ws, self.pos_local, None,
+                       self.dev_status, stream)
+
+    def route(self, group=None, stream=None):
+        """count -> all-gather of the counts (torch.distributed) -> plan and layout."""
+        self.count(stream)
+        gather_counts(self.counts_row, self.counts, group)
+        self.plan_and_layout(stream)
+
+    def dispatch(self, stream=None):
+        ep_dispatch_peer(self.x_local, self.K, self.pos_local, self.peers, self.SK, self.dev_status, stream)
+
+    def combine(self, stream=None):
+        ep_combine_peer(self.peers, self.SK, self.w_local, self.pos_local, self.out_local, None, self.dev_status,
+                        stream)
+
+    def grad_reduce(self, clear=False, stream=None):
+        ep_replica_grad_reduce_peer(self.g_home, self.grad_peers, self.rep_rows, self.g_rep.dtype, self.E, self.rank,
+                                    self.plan, clear, self.dev_status, stream)
+
+    def status(self, stream=None):
+        return ep_status_read(self.dev_status, stream)
