@@ -111,7 +111,12 @@ class EpLayer:
         is still arriving and slice i-1 is already going out (the host link is
         full duplex), so the transfers overlap each other and the kernels.
         Dispatch and combine of a token slice touch only that slice's pairs, so
-        the slices are independent.  The caller's stream waits for the last copy
+        the slices are independent.  The routing and gate weights go first on
+        the same copy stream as the token slices, ahead of them, so the route
+        never waits behind the hidden rows (copied on the compute stream
+        instead, they did so in every other step on B200, which then ran the
+        two copy directions one after the other: 4.97 against 3.32 ms for the
+        moderate EP8 workload).  The caller's stream waits for the last copy
         out before anything queued after this call."""
         main = stream if stream is not None else torch.cuda.current_stream(self.device)
         if chunks <= 1 or self.T < chunks:
@@ -128,10 +133,13 @@ class EpLayer:
         h2d, d2h = self._h2d, self._d2h
         h2d.wait_stream(main)  # buffers are free once the caller's earlier work is done
         d2h.wait_stream(main)
-        with torch.cuda.stream(main):
+        with torch.cuda.stream(h2d):
             self.topk_ids.copy_(topk_h, non_blocking=True)
             self.w.copy_(w_h, non_blocking=True)
-            self.route(main, fused)
+            routed = torch.cuda.Event()
+            routed.record(h2d)
+        main.wait_event(routed)
+        self.route(main, fused)
         bounds = [self.T * i // chunks for i in range(chunks + 1)]
         K = self.K
         for t0, t1 in zip(bounds[:-1], bounds[1:]):
