@@ -12,10 +12,9 @@
 //     never straddles two source ranks), so the load matrix L[s][e] and each
 //     pair's rank among the pairs of (source rank, expert) come out of one
 //     column scan.
-//  2. k_q_scan: one warp per expert scans its column of tile counts into
-//     exclusive per-tile prefixes (row ntiles holds T_e).  The last CTA to
-//     finish computes the rank loads H_r, each rank's experts heaviest first,
-//     and the threshold range [ceil(P/R), max(ceil(P/R), max H_r)].
+//  2. k_q_scan: every expert column of tile counts is scanned into
+//     exclusive per-tile prefixes (row ntiles holds T_e) by 128 threads, one
+//     short tile range each, 8 columns per CTA.
 //  3. k_q_search: every thread of the grid tests one threshold at a time, the
 //     smallest candidates first; a feasible one is folded into an atomicMin, so
 //     the result is the smallest feasible threshold whatever the order.  A
@@ -35,7 +34,7 @@ namespace ep {
 
 int num_sms();
 
-constexpr int Q_SCAN_THREADS = 512;
+constexpr int Q_SCAN_THREADS = 1024;
 constexpr int Q_SEARCH_THREADS = 256;
 
 // header words of the quota workspace
@@ -158,43 +157,61 @@ __global__ void __launch_bounds__(SCAT_THREADS)
 
 // ------------------------------------------------------------------- 2. scan
 
-constexpr int Q_SCAN_WARPS = Q_SCAN_THREADS / 32;
+constexpr int Q_SCAN_EXPERTS = 8;                              // expert columns per CTA
+constexpr int Q_SCAN_GROUPS = Q_SCAN_THREADS / Q_SCAN_EXPERTS;  // tile ranges per column
 
-// Lanes = 32 consecutive experts, warps = consecutive ranges of tiles: per-warp
-// sums, a scan over the warps, then each warp writes its exclusive prefixes.
-// Row ntiles of excl and loads get T_e.
+// Threads = (tile range g, expert j): 8 consecutive experts of one tile are 8
+// consecutive words, read by 8 consecutive threads.  Each thread sums its tile
+// range; warp j then scans column j's range sums (each lane four consecutive
+// ranges, one warp scan); each thread walks its range again writing the
+// exclusive prefixes.  Row ntiles of excl and loads get T_e.  Many CTAs with
+// one short range each keep the dependent load chains short.
 __global__ void __launch_bounds__(Q_SCAN_THREADS)
     k_q_scan(const int32_t* __restrict__ cnt, int64_t ntiles, int E, int32_t* __restrict__ excl,
              int32_t* __restrict__ loads) {
-  __shared__ int32_t s_part[Q_SCAN_WARPS][32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int e = blockIdx.x * 32 + lane;
-  const int64_t span = (ntiles + Q_SCAN_WARPS - 1) / Q_SCAN_WARPS;
-  const int64_t t0 = min(ntiles, warp * span), t1 = min(ntiles, t0 + span);
+  static_assert(Q_SCAN_GROUPS == 128 && Q_SCAN_EXPERTS <= Q_SCAN_THREADS / 32, "one warp scans 4 ranges per lane");
+  __shared__ int32_t s_part[Q_SCAN_GROUPS][Q_SCAN_EXPERTS];
+  const int j = threadIdx.x % Q_SCAN_EXPERTS, g = threadIdx.x / Q_SCAN_EXPERTS;
+  const int e = blockIdx.x * Q_SCAN_EXPERTS + j;
+  const int64_t span = (ntiles + Q_SCAN_GROUPS - 1) / Q_SCAN_GROUPS;
+  const int64_t t0 = min(ntiles, g * span), t1 = min(ntiles, t0 + span);
   int32_t sum = 0;
   if (e < E) {
-#pragma unroll 8
+#pragma unroll 4
     for (int64_t t = t0; t < t1; ++t) sum += cnt[t * E + e];
   }
-  s_part[warp][lane] = sum;
+  s_part[g][j] = sum;
   __syncthreads();
-  if (warp == 0) {
-    int32_t run = 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp < Q_SCAN_EXPERTS) {  // warp `warp` scans column `warp`: lane owns ranges 4*lane .. 4*lane+3
+    int32_t v[4], tot = 0;
 #pragma unroll
-    for (int w = 0; w < Q_SCAN_WARPS; ++w) {
-      const int32_t v = s_part[w][lane];
-      s_part[w][lane] = run;
-      run += v;
+    for (int q = 0; q < 4; ++q) {
+      v[q] = s_part[4 * lane + q][warp];
+      tot += v[q];
     }
-    if (e < E) {
-      excl[ntiles * E + e] = run;
-      loads[e] = run;
+    int32_t inc = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += y;
+    }
+    int32_t run = inc - tot;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      s_part[4 * lane + q][warp] = run;
+      run += v[q];
+    }
+    const int ew = blockIdx.x * Q_SCAN_EXPERTS + warp;
+    if (lane == 31 && ew < E) {
+      excl[ntiles * E + ew] = inc;
+      loads[ew] = inc;
     }
   }
   __syncthreads();
   if (e < E) {
-    int32_t run = s_part[warp][lane];
-#pragma unroll 8
+    int32_t run = s_part[g][j];
+#pragma unroll 4
     for (int64_t t = t0; t < t1; ++t) {
       const int32_t v = cnt[t * E + e];
       excl[t * E + e] = run;
@@ -697,7 +714,7 @@ extern "C" int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, 
   int32_t* excl = reinterpret_cast<int32_t*>(base + w.excl);
   k_q_count<<<(unsigned)std::max<int64_t>(q.ntiles, 1), SCAT_THREADS, sizeof(int32_t) * E, stream>>>(
       topk_ids, SK, E, q.tile, q.tpr, q.ntiles, cnt, hdr, dev_status);
-  k_q_scan<<<(E + 31) / 32, Q_SCAN_THREADS, 0, stream>>>(cnt, q.ntiles, E, excl, loads);
+  k_q_scan<<<(E + Q_SCAN_EXPERTS - 1) / Q_SCAN_EXPERTS, Q_SCAN_THREADS, 0, stream>>>(cnt, q.ntiles, E, excl, loads);
   const size_t search_smem = q_search_smem(E, R);
   if (search_smem > 48 * 1024 &&
       cudaFuncSetAttribute(k_q_search, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)search_smem) != cudaSuccess)

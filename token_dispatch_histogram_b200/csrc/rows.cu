@@ -294,64 +294,64 @@ __global__ void __launch_bounds__(256)
 // Backward of combine.  For every pair (t, k) with row r = pos[t*K+k]:
 //   dy[r]    = bf16_rn(w[t,k] * float(dout[t]))          (one fp32 multiply per element)
 //   dw[t,k]  = sum_h float(dout[t,h]) * float(y[r,h])     (fp32; any summation order)
-// A thread owns one 16-byte vector of the token's row: it loads the dout vector
-// and the K y vectors, writes the K scaled dy vectors and keeps K partial dot
-// products; those are reduced over the token's threads (warp shuffles, then
-// shared memory) once the row is done.
+// One group of G lanes owns one token (G = 32 for rows of 256+ elements, else
+// the power of two covering the row's 16-byte vectors, so a warp carries
+// 32 / G tokens).  Each lane walks every G-th vector of the row: it loads the
+// dout vector and the K y vectors, writes the K scaled dy vectors and keeps K
+// partial dot products, which a butterfly of shuffles inside the group adds
+// up at the end of the token.  No block-wide barrier: warps run independently,
+// and the next token's rows and weights are loaded while the current one runs.
+// Two CTAs per SM: about 124 registers at K = 6 without spills; bounds that
+// force 3 or 4 CTAs spill and measured 0-12% slower on B200.
 template <int K>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256, 2)
     k_combine_bwd(const uint16_t* __restrict__ dout, const float* __restrict__ w, const uint16_t* __restrict__ y,
                   int64_t y_rows, const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ dy,
                   float* __restrict__ dw, int32_t* dev_status) {
-  constexpr int MAXT = 8;
-  __shared__ int32_t s_rows[2][MAXT][K];
-  __shared__ float s_w[2][MAXT][K];
-  __shared__ float s_part[8][K];  // per warp partial dot products
-  __shared__ int s_bad;
   const int64_t nvec = H / 8;
-  const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);
-  const int tpc = 256 / tpr <= MAXT ? 256 / tpr : MAXT;
-  const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t step = (int64_t)gridDim.x * tpc;
-  if (threadIdx.x == 0) s_bad = 0;
-  auto stage = [&](int b, int64_t tb) {
-    if (threadIdx.x < tpc * K) {
-      const int s = threadIdx.x / K, k = threadIdx.x - s * K;
-      const int64_t t = tb + s;
-      int32_t r = -1;
-      float wk = 0.0f;
+  const int G = nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : (int)nvec);
+  const int lane = threadIdx.x & 31;
+  const int gpw = 32 / G;                  // tokens per warp
+  const int sub = lane / G, gl = lane % G;
+  const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  int32_t bad = 0;
+  auto rows_of = [&](int64_t t, int32_t (&r)[K], float (&wk)[K]) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      r[k] = -1;
+      wk[k] = 0.0f;
       if (t < T) {
-        r = __ldg(pos + t * K + k);
-        wk = __ldg(w + t * K + k);
-        if (r < 0 || r >= y_rows) {
-          r = -1;
-          s_bad = 1;
-        }
+        r[k] = __ldg(pos + t * K + k);
+        wk[k] = __ldg(w + t * K + k);
       }
-      s_rows[b][s][k] = r;
-      s_w[b][s][k] = wk;
     }
   };
-  int64_t tb = (int64_t)blockIdx.x * tpc;
-  stage(0, tb);
-  __syncthreads();
-  for (int b = 0; tb < T; tb += step, b ^= 1) {
-    stage(b ^ 1, tb + step);
+  int64_t tb = warp_id * gpw;
+  int32_t r[K];
+  float wk[K];
+  rows_of(tb + sub, r, wk);
+  for (; tb < T; tb += nwarps * gpw) {
     const int64_t t = tb + sub;
-    const bool live = sub < tpc && t < T;
+    int32_t rn[K];
+    float wn[K];
+    rows_of(tb + nwarps * gpw + sub, rn, wn);  // the next token's, ahead of use
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (t < T && (r[k] < 0 || r[k] >= y_rows)) {
+        r[k] = -1;
+        bad = EP_DEV_BAD_ROW;
+      }
     float part[K];
 #pragma unroll
     for (int k = 0; k < K; ++k) part[k] = 0.0f;
-    if (live) {
-      for (int64_t v = v0; v < nvec; v += tpr) {
+    if (t < T) {
+      for (int64_t v = gl; v < nvec; v += G) {
         const uint4 g = ld_stream_v4(dout + t * H + v * 8);
         uint4 in[K];
 #pragma unroll
-        for (int k = 0; k < K; ++k) {
-          const int32_t r = s_rows[b][sub][k];
-          in[k] = r >= 0 ? ld_stream_v4(y + (int64_t)r * H + v * 8) : make_uint4(0, 0, 0, 0);
-        }
+        for (int k = 0; k < K; ++k)
+          in[k] = r[k] >= 0 ? ld_stream_v4(y + (int64_t)r[k] * H + v * 8) : make_uint4(0, 0, 0, 0);
         const uint32_t gd[4] = {g.x, g.y, g.z, g.w};
         float gf[8];
 #pragma unroll
@@ -361,43 +361,35 @@ __global__ void __launch_bounds__(256, 4)
         }
 #pragma unroll
         for (int k = 0; k < K; ++k) {
-          const int32_t r = s_rows[b][sub][k];
-          if (r < 0) continue;
-          const float wk = s_w[b][sub][k];
+          if (r[k] < 0) continue;
           const uint32_t yd[4] = {in[k].x, in[k].y, in[k].z, in[k].w};
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            o[q] = f32_to_bf16_bits(__fmul_rn(wk, gf[2 * q])) | (f32_to_bf16_bits(__fmul_rn(wk, gf[2 * q + 1])) << 16);
+            o[q] = f32_to_bf16_bits(__fmul_rn(wk[k], gf[2 * q])) |
+                   (f32_to_bf16_bits(__fmul_rn(wk[k], gf[2 * q + 1])) << 16);
             part[k] = fmaf(gf[2 * q], bf16_bits_to_f32(yd[q] & 0xFFFFu), part[k]);
             part[k] = fmaf(gf[2 * q + 1], bf16_bits_to_f32(yd[q] >> 16), part[k]);
           }
-          st_v4(dy + (int64_t)r * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+          st_v4(dy + (int64_t)r[k] * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
     }
-    // reduce the K partial dot products over the token's threads
+    // add the group's partial products (every lane of the warp takes part)
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      for (int d = G >> 1; d; d >>= 1) part[k] += __shfl_xor_sync(0xffffffffu, part[k], d);
+    if (t < T && gl == 0) {
+#pragma unroll
+      for (int k = 0; k < K; ++k) dw[t * K + k] = r[k] >= 0 ? part[k] : 0.0f;
+    }
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-      float v = part[k];
-#pragma unroll
-      for (int d = 16; d; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
-      if (lane == 0) s_part[warp][k] = v;
+      r[k] = rn[k];
+      wk[k] = wn[k];
     }
-    __syncthreads();
-    const int wpt = tpr / 32;  // warps per token
-    if (threadIdx.x < tpc * K) {
-      const int s = threadIdx.x / K, k = threadIdx.x - s * K;
-      const int64_t tt = tb + s;
-      if (tt < T) {
-        float acc = 0.0f;
-        for (int i = 0; i < wpt; ++i) acc += s_part[s * wpt + i][k];
-        dw[tt * K + k] = s_rows[b][s][k] >= 0 ? acc : 0.0f;
-      }
-    }
-    __syncthreads();
   }
-  if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_ROW);
+  if (bad) flag(dev_status, bad);
 }
 
 int occupancy_grid(const void* fn, int threads, size_t smem, int64_t work_items, int cap_per_sm) {
@@ -566,7 +558,11 @@ extern "C" int ep_combine_backward(const uint16_t* dout, const float* w, const u
     case 7: fn = (const void*)k_combine_bwd<7>; break;
     default: fn = (const void*)k_combine_bwd<8>; break;
   }
-  const int grid = occupancy_grid(fn, 256, 0, T, 4);
+  // one token per group of lanes, 8 warps per CTA; as many CTAs as fit
+  const int64_t nvec = H / 8;
+  const int64_t G = nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : nvec);
+  const int64_t ctas = (T + 8 * (32 / G) - 1) / (8 * (32 / G));
+  const int grid = occupancy_grid(fn, 256, 0, ctas, 2);
   void* args[] = {(void*)&dout, (void*)&w, (void*)&y, (void*)&y_rows, (void*)&pos, (void*)&T, (void*)&H, (void*)&dy,
                   (void*)&dw, (void*)&dev_status};
   if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
