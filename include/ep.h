@@ -406,10 +406,14 @@ EP_API int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtyp
  * Every output equals, bit for bit, the slice of the one-buffer path's output
  * that belongs to rank r.  Peer tables: device arrays of R uint64 device
  * addresses (this GPU's own buffer or peers' buffers mapped into its address
- * space, e.g. symmetric memory or IPC); each must be 16-byte aligned.  A zero
- * or misaligned entry is never dereferenced: the rows it would serve are
- * skipped and EP_DEV_BAD_ROW is set.  Global row g lives on rank
- * g / rows_per_rank at local row g % rows_per_rank.
+ * space, e.g. symmetric memory or IPC); each must be 16-byte aligned.  Rows:
+ * pos_local holds global rows g in [0, total_rows).  With rank_first_row NULL
+ * every rank holds rows_per_rank rows and g lives on rank g / rows_per_rank
+ * (the exact-S*K plan: rows_per_rank = S*K); otherwise rank d's rows start at
+ * rank_first_row[d] (device int32 [R], ascending, from 0; a quota plan's
+ * rank_off) and its buffer holds rows_per_rank rows.  A zero or misaligned
+ * table entry, or a row past its rank's buffer, is never dereferenced: the
+ * rows it would serve are skipped and EP_DEV_BAD_ROW is set.
  */
 
 /*
@@ -435,13 +439,12 @@ EP_API int ep_layout_rank(const int32_t* topk_local, int64_t S, int K, int E, in
 
 /*
  * Dispatch of rank-local tokens: the row of x_local [S, H] bf16 of pair i goes
- * to global row pos_local[i], i.e. to peer_bufs[g / rows_per_rank] at local row
- * g % rows_per_rank (H bf16 per row).  One TMA bulk load per token row and K
- * bulk stores, as ep_dispatch.
+ * to global row pos_local[i] in the rank buffers (H bf16 per row).  One TMA
+ * bulk load per token row and K bulk stores, as ep_dispatch.
  */
 EP_API int ep_dispatch_peer(const uint16_t* x_local, int64_t S, int K, int64_t H, const int32_t* pos_local,
-                            const uint64_t* peer_bufs, int R, int64_t rows_per_rank, int32_t* dev_status,
-                            cudaStream_t stream);
+                            const uint64_t* peer_bufs, const int32_t* rank_first_row, int R, int64_t rows_per_rank,
+                            int64_t total_rows, int32_t* dev_status, cudaStream_t stream);
 
 /*
  * Combine of rank-local tokens, reading the expert rows from the R rank
@@ -449,9 +452,9 @@ EP_API int ep_dispatch_peer(const uint16_t* x_local, int64_t S, int K, int64_t H
  * fp32 in k order, as ep_combine.  w_local NULL: unit weights (the backward of
  * dispatch, as ep_dispatch_backward).  1 <= K <= 8.
  */
-EP_API int ep_combine_peer(const uint64_t* peer_bufs, int R, int64_t rows_per_rank, const float* w_local,
-                           const int32_t* pos_local, int64_t S, int K, int64_t H, uint16_t* out_local,
-                           int32_t* dev_status, cudaStream_t stream);
+EP_API int ep_combine_peer(const uint64_t* peer_bufs, const int32_t* rank_first_row, int R, int64_t rows_per_rank,
+                           int64_t total_rows, const float* w_local, const int32_t* pos_local, int64_t S, int K,
+                           int64_t H, uint16_t* out_local, int32_t* dev_status, cudaStream_t stream);
 
 /*
  * Replica gradient reduction on the home rank.  [GR] "Τι συμβαίνει στους
@@ -474,6 +477,44 @@ EP_API int ep_replica_grad_reduce_peer(float* g_home_local, const uint64_t* peer
                                        int rep_dtype, int64_t n, int E, int R, int rank, const int32_t* plan,
                                        size_t plan_words, int clear_replicas, int32_t* dev_status,
                                        cudaStream_t stream);
+
+/*
+ * The quota-driven planner (ep_quota_route) in rank-local form.  Flow on rank
+ * r: ep_route_stats(topk_local) -> counts row and per-tile prefixes in ws; the
+ * all-gather of the rows into counts [R, E] (exactly the source-rank x expert
+ * load matrix the planner starts from); ep_quota_plan_from_counts (the same
+ * plan on every rank); ep_quota_layout_rank (global rows of the rank's own
+ * pairs).  Then ep_dispatch_peer / ep_combine_peer with rank_first_row = the
+ * plan's rank_off array (rank r holds rank_load[r] <= tau* rows, so a buffer of
+ * rows_per_rank >= tau* rows per rank suffices; tau* <= max(ceil(P/R), max_r
+ * of the rank's home loads)), and ep_quota_replica_grad_reduce_peer.
+ */
+EP_API int ep_quota_counts_workspace_size(int E, int R, size_t* bytes /* host out */);
+
+/*
+ * counts [R, E] int32 device (gathered); loads [E] int32 out (T_e); plan as in
+ * ep_quota_route (EpQuotaLayout); ws device scratch of
+ * ep_quota_counts_workspace_size bytes.  Two launches.  Counts that do not add
+ * up to R*S*K (or are negative) give tau = -1 and no replica.
+ */
+EP_API int ep_quota_plan_from_counts(const int32_t* counts, int R, int64_t S, int K, int E, int B, int32_t* loads,
+                                     int32_t* plan, size_t plan_words, void* ws, size_t ws_bytes,
+                                     int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Rows of rank `rank`'s own pairs under a quota plan: pos_local[i] = pos[rank*S*K
+ * + i] of ep_quota_route for the whole problem.  ws is the scratch
+ * ep_route_stats filled for topk_local (T = S); counts the gathered matrix.
+ */
+EP_API int ep_quota_layout_rank(const int32_t* topk_local, int64_t S, int K, int E, int R, int rank,
+                                const int32_t* counts, const int32_t* plan, size_t plan_words, const void* ws,
+                                size_t ws_bytes, int32_t* pos_local, int32_t* dev_status, cudaStream_t stream);
+
+/* ep_replica_grad_reduce_peer for a plan from ep_quota_plan_from_counts. */
+EP_API int ep_quota_replica_grad_reduce_peer(float* g_home_local, const uint64_t* peer_g_rep, int64_t rep_rows,
+                                             int rep_dtype, int64_t n, int E, int R, int rank, const int32_t* plan,
+                                             size_t plan_words, int clear_replicas, int32_t* dev_status,
+                                             cudaStream_t stream);
 
 /*
  * ep_route_stats without a scratch argument, for callers that cannot allocate

@@ -128,7 +128,7 @@ def test_rank_local_path(case):
     want_dx = O.dispatch_backward(y, lo["pos"], T, K)
     for r, rk in enumerate(ranks):
         dx = torch.full((S, H), -1.0, dtype=torch.bfloat16, device="cuda")
-        tdh.ep_combine_peer(peers, SK, None, rk.pos_local, dx, K=K, dev_status=rk.dev_status)
+        tdh.ep_combine_peer(peers, SK, R * SK, None, rk.pos_local, dx, K=K, dev_status=rk.dev_status)
         np.testing.assert_array_equal(_u16(dx), want_dx[r * S:(r + 1) * S])
 
 
@@ -205,3 +205,129 @@ def test_rank_local_missing_peer_is_flagged():
             assert (got == _u16(torch.full((1,), -1.0, dtype=torch.bfloat16))[0]).all()  # untouched
         else:
             np.testing.assert_array_equal(got, buf[d * SK:(d + 1) * SK])
+
+
+# ---- the quota-driven planner in rank-local form
+
+QUOTA_CASES = [
+    # R, S, K, E, H, B, kind
+    (4, 64, 2, 16, 128, 1, "skew"),
+    (8, 700, 6, 64, 256, 2, "skew"),
+    (8, 512, 8, 64, 64, 8, "single"),
+    (16, 300, 4, 64, 64, 1, "uniform"),
+    (1, 500, 3, 8, 72, 2, "skew"),
+    (32, 96, 8, 256, 32, 3, "skew"),
+    (8, 512, 2, 8, 32, 0, "skew"),      # B = 0: no replica, the unplanned loads
+]
+
+
+def _quota_ranks(R, S, K, E, H, B, topk, w, x, buf_rows, grad_n=0):
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    from token_dispatch_histogram_b200.ranks import EpRank
+    dev = torch.device("cuda")
+    ranks = []
+    for r in range(R):
+        rk = EpRank(r, R, S, K, E, H, device=dev, grad_n=grad_n, planner="quota", B=B, buf_rows=buf_rows)
+        rk.topk_local.copy_(_t(torch, topk[r * S:(r + 1) * S], dev))
+        rk.w_local.copy_(_t(torch, w[r * S:(r + 1) * S], dev))
+        rk.x_local.copy_(_t(torch, x[r * S:(r + 1) * S], dev))
+        rk.buf.fill_(-1.0)
+        rk.pos_local.fill_(-7)
+        ranks.append(rk)
+    for rk in ranks:
+        rk.count()
+    counts = torch.stack([rk.counts_row for rk in ranks])  # the all-gather
+    for rk in ranks:
+        rk.counts.copy_(counts)
+        rk.plan_and_layout()
+    peers = tdh.peer_table([rk.buf for rk in ranks])
+    for rk in ranks:
+        rk.set_peers(peers)
+        rk.dispatch()
+    torch.cuda.synchronize()
+    return ranks, peers
+
+
+@pytest.mark.parametrize("case", QUOTA_CASES, ids=lambda c: "R{}_S{}_K{}_E{}_H{}_B{}_{}".format(*c))
+def test_rank_local_quota_path(case):
+    import torch
+    R, S, K, E, H, B, kind = case
+    topk, w, x = case_inputs(R, S, K, E, H, seed=R * 17 + S + B, kind=kind, bias_scale=1.5)
+    T, SK = R * S, S * K
+    loads, _, _ = O.route_stats(topk, E)
+    qp = O.quota_plan(loads, R, S, K, E, B)
+    lo = O.quota_layout(topk, qp, R, S, K, E)
+    n = qp["n_rep"]
+    buf_rows = max(int(lo["rank_load"].max()), 1)  # tau*: every rank's rows fit
+    ranks, peers = _quota_ranks(R, S, K, E, H, B, topk, w, x, buf_rows)
+    buf = O.dispatch(x, lo["pos"], K, T * K)
+    off = np.concatenate([[0], np.cumsum(lo["rank_load"])[:-1]]).astype(np.int64)
+    L = ranks[0].plan_layout
+
+    def field(plan, name, cnt):
+        return plan[L[name]:L[name] + cnt]
+
+    for r, rk in enumerate(ranks):
+        assert rk.status() == 0
+        plan = rk.plan.cpu().numpy()
+        assert int(field(plan, "tau", 1)[0]) == qp["tau"]
+        assert int(field(plan, "n_rep", 1)[0]) == n
+        assert int(field(plan, "n_local", 1)[0]) == lo["n_local"]
+        np.testing.assert_array_equal(field(plan, "rep_expert", n), qp["rep_expert"])
+        np.testing.assert_array_equal(field(plan, "rep_rank", n), qp["rep_rank"])
+        np.testing.assert_array_equal(field(plan, "rep_count", n), qp["rep_count"])
+        np.testing.assert_array_equal(field(plan, "home_quota", E), qp["home_quota"])
+        np.testing.assert_array_equal(field(plan, "rank_load", R), lo["rank_load"])
+        np.testing.assert_array_equal(field(plan, "rank_off", R), off)
+        np.testing.assert_array_equal(field(plan, "cu_seqlens", E + n + 1), lo["cu_seqlens"])
+        np.testing.assert_array_equal(rk.pos_local.cpu().numpy(), lo["pos"][r * SK:(r + 1) * SK])
+    for d, rk in enumerate(ranks):  # rank d's rows [off_d, off_d + load_d) of the one buffer
+        ld = int(lo["rank_load"][d])
+        got = _u16(rk.buf)
+        np.testing.assert_array_equal(got[:ld], buf[off[d]:off[d] + ld])
+    # combine through the peers (rows = the dispatched rows, no expert in between)
+    want = O.combine(buf, w, lo["pos"], K)
+    for rk in ranks:
+        rk.out_local.fill_(-1.0)
+        rk.combine()
+    torch.cuda.synchronize()
+    for r, rk in enumerate(ranks):
+        assert rk.status() == 0
+        np.testing.assert_array_equal(_u16(rk.out_local), want[r * S:(r + 1) * S])
+
+
+def test_rank_local_quota_grad_reduce():
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    R, S, K, E, H, B = 8, 512, 6, 64, 16, 2
+    topk, w, x = case_inputs(R, S, K, E, H, seed=93, bias_scale=1.5)
+    loads, _, _ = O.route_stats(topk, E)
+    qp = O.quota_plan(loads, R, S, K, E, B)
+    lo = O.quota_layout(topk, qp, R, S, K, E)
+    n_rep = qp["n_rep"]
+    assert n_rep > 0
+    ER, cap = E // R, E + R - 1
+    nrep_r = np.bincount(qp["rep_rank"], minlength=R)
+    first = np.concatenate([[0], np.cumsum(nrep_r)[:-1]])
+    n = 4096 + 8
+    g_home = W.grad_rows(3, W.STREAM_GHOME, n, E)
+    g_rep = W.grad_rows(4, W.STREAM_GREP, n, cap)
+    ranks, _ = _quota_ranks(R, S, K, E, H, B, topk, w, x, max(int(lo["rank_load"].max()), 1), grad_n=n)
+    for r, rk in enumerate(ranks):
+        rk.g_home.copy_(_t(torch, g_home[r * ER:(r + 1) * ER], "cuda"))
+        rk.g_rep.zero_()
+        c = int(nrep_r[r])
+        if c:
+            rk.g_rep[:c].copy_(_t(torch, g_rep[first[r]:first[r] + c], "cuda"))
+    gpeers = tdh.peer_table([rk.g_rep for rk in ranks])
+    for rk in ranks:
+        rk.set_grad_peers(gpeers)
+        rk.grad_reduce(True)
+    torch.cuda.synchronize()
+    gh, gr = O.grad_reduce(g_home, g_rep, qp["rep_expert"], True)
+    for r, rk in enumerate(ranks):
+        assert rk.status() == 0
+        np.testing.assert_array_equal(rk.g_home.cpu().numpy(), gh[r * ER:(r + 1) * ER])
+        c = int(nrep_r[r])
+        np.testing.assert_array_equal(rk.g_rep[:c].cpu().numpy(), gr[first[r]:first[r] + c])

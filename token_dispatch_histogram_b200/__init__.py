@@ -80,8 +80,12 @@ _SIGS = {
     "ep_replica_grad_reduce": (_I, [_V, _V, _I, _I64, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_plan_from_counts": (_I, [_V, _I, _I64, _I, _I, _V, _V, _SZ, _V, _V]),
     "ep_layout_rank": (_I, [_V, _I64, _I, _I, _I, _I, _V, _V, _SZ, _V, _SZ, _V, _V, _V, _V]),
-    "ep_dispatch_peer": (_I, [_V, _I64, _I, _I64, _V, _V, _I, _I64, _V, _V]),
-    "ep_combine_peer": (_I, [_V, _I, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
+    "ep_dispatch_peer": (_I, [_V, _I64, _I, _I64, _V, _V, _V, _I, _I64, _I64, _V, _V]),
+    "ep_combine_peer": (_I, [_V, _V, _I, _I64, _I64, _V, _V, _I64, _I, _I64, _V, _V, _V]),
+    "ep_quota_counts_workspace_size": (_I, [_I, _I, _V]),
+    "ep_quota_plan_from_counts": (_I, [_V, _I, _I64, _I, _I, _I, _V, _V, _SZ, _V, _SZ, _V, _V]),
+    "ep_quota_layout_rank": (_I, [_V, _I64, _I, _I, _I, _I, _V, _V, _SZ, _V, _SZ, _V, _V, _V]),
+    "ep_quota_replica_grad_reduce_peer": (_I, [_V, _V, _I64, _I, _I64, _I, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_replica_grad_reduce_peer": (_I, [_V, _V, _I64, _I, _I64, _I, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_status_read": (_I, [_V, _V, _V]),
     "ep_selftest_lookback_timeout": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
@@ -361,28 +365,65 @@ def ep_layout_rank(topk_local, rank, counts, plan, ws, pos_local, pair_slot=None
                                                   _p(pair_slot), _p(dev_status), _s(stream)))
 
 
-def ep_dispatch_peer(x_local, K, pos_local, peers, rows_per_rank, dev_status=None, stream=None):
-    """Rows of x_local [S, H] to their global rows in the R rank buffers."""
+def ep_dispatch_peer(x_local, K, pos_local, peers, rows_per_rank, total_rows, rank_first_row=None, dev_status=None,
+                     stream=None):
+    """Rows of x_local [S, H] to their global rows in the R rank buffers (rank
+    of a row: row // rows_per_rank, or by rank_first_row when given)."""
     _dtype(x_local, torch.bfloat16, torch.int16, torch.uint16)
     _dtype(pos_local, torch.int32)
     _dtype(peers, torch.int64)
+    if rank_first_row is not None:
+        _dtype(rank_first_row, torch.int32)
     S, H = x_local.shape
-    _check("ep_dispatch_peer", lib().ep_dispatch_peer(_p(x_local), S, K, H, _p(pos_local), _p(peers), peers.numel(),
-                                                      rows_per_rank, _p(dev_status), _s(stream)))
+    _check("ep_dispatch_peer", lib().ep_dispatch_peer(_p(x_local), S, K, H, _p(pos_local), _p(peers), _p(rank_first_row),
+                                                      peers.numel(), rows_per_rank, total_rows, _p(dev_status),
+                                                      _s(stream)))
 
 
-def ep_combine_peer(peers, rows_per_rank, w_local, pos_local, out_local, K=None, dev_status=None, stream=None):
+def ep_combine_peer(peers, rows_per_rank, total_rows, w_local, pos_local, out_local, K=None, rank_first_row=None,
+                    dev_status=None, stream=None):
     """out_local[t] = sum_k w_local[t,k] * row pos_local[t*K+k] of the rank
     buffers (w_local None: unit weights, the backward of dispatch; K given)."""
     _dtype(pos_local, torch.int32)
     _dtype(peers, torch.int64)
+    if rank_first_row is not None:
+        _dtype(rank_first_row, torch.int32)
     S, H = out_local.shape
     if w_local is not None:
         _dtype(w_local, torch.float32)
         K = w_local.shape[1]
-    _check("ep_combine_peer", lib().ep_combine_peer(_p(peers), peers.numel(), rows_per_rank, _p(w_local),
-                                                    _p(pos_local), S, K, H, _p(out_local), _p(dev_status),
-                                                    _s(stream)))
+    _check("ep_combine_peer", lib().ep_combine_peer(_p(peers), _p(rank_first_row), peers.numel(), rows_per_rank,
+                                                    total_rows, _p(w_local), _p(pos_local), S, K, H, _p(out_local),
+                                                    _p(dev_status), _s(stream)))
+
+
+def ep_quota_counts_workspace_size(E, R):
+    n = ctypes.c_size_t(0)
+    _check("ep_quota_counts_workspace_size", lib().ep_quota_counts_workspace_size(E, R, ctypes.byref(n)))
+    return int(n.value)
+
+
+def ep_quota_plan_from_counts(counts, S, K, B, loads, plan, ws, dev_status=None, stream=None):
+    """The quota-driven plan (budget B replicas per rank) from the gathered
+    [R, E] load matrix; the same on every rank."""
+    for t in (counts, loads, plan):
+        _dtype(t, torch.int32)
+    R, E = counts.shape
+    _check("ep_quota_plan_from_counts",
+           lib().ep_quota_plan_from_counts(_p(counts), R, S, K, E, B, _p(loads), _p(plan), plan.numel(), _p(ws),
+                                           ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
+
+
+def ep_quota_layout_rank(topk_local, rank, counts, plan, ws, pos_local, dev_status=None, stream=None):
+    """Global rows of rank `rank`'s pairs under a quota plan; ws is the scratch
+    ep_route_stats filled for topk_local."""
+    for t in (topk_local, counts, plan, pos_local):
+        _dtype(t, torch.int32)
+    S, K = topk_local.shape
+    R, E = counts.shape
+    _check("ep_quota_layout_rank",
+           lib().ep_quota_layout_rank(_p(topk_local), S, K, E, R, rank, _p(counts), _p(plan), plan.numel(), _p(ws),
+                                      ws.numel() * ws.element_size(), _p(pos_local), _p(dev_status), _s(stream)))
 
 
 def ep_replica_grad_reduce_peer(g_home_local, peers, rep_rows, rep_dtype, E, rank, plan, clear_replicas=False,
@@ -399,6 +440,20 @@ def ep_replica_grad_reduce_peer(g_home_local, peers, rep_rows, rep_dtype, E, ran
            lib().ep_replica_grad_reduce_peer(_p(g_home_local), _p(peers), rep_rows, dt, n, E, peers.numel(), rank,
                                              _p(plan), plan.numel(), int(bool(clear_replicas)), _p(dev_status),
                                              _s(stream)))
+
+
+def ep_quota_replica_grad_reduce_peer(g_home_local, peers, rep_rows, rep_dtype, E, rank, plan, clear_replicas=False,
+                                      dev_status=None, stream=None):
+    """ep_replica_grad_reduce_peer for a plan from ep_quota_plan_from_counts."""
+    _dtype(g_home_local, torch.float32)
+    _dtype(plan, torch.int32)
+    _dtype(peers, torch.int64)
+    dt = {torch.float32: EP_DTYPE_F32, torch.bfloat16: EP_DTYPE_BF16}[rep_dtype]
+    n = g_home_local.shape[1]
+    _check("ep_quota_replica_grad_reduce_peer",
+           lib().ep_quota_replica_grad_reduce_peer(_p(g_home_local), _p(peers), rep_rows, dt, n, E, peers.numel(), rank,
+                                                   _p(plan), plan.numel(), int(bool(clear_replicas)), _p(dev_status),
+                                                   _s(stream)))
 
 
 def ep_selftest_lookback_timeout(topk_ids, E, loads, max_vio, ws, dev_status, stream=None):

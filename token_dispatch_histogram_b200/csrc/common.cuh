@@ -189,6 +189,35 @@ __device__ __forceinline__ void bulk_wait_read() {
 
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Rank-local form: address of global row g in the R ranks' buffers.  Ranks
+// hold rows_per_rank rows each (rank_first == NULL: rank g / rows_per_rank), or
+// rank r's rows start at rank_first[r] (ascending, rank_first[0] = 0) and fit
+// in its buffer of rows_per_rank rows.  nullptr when the rank's table entry is
+// zero or not 16-byte aligned, or the row falls past its rank's buffer.
+__device__ __forceinline__ char* peer_row(const uint64_t* __restrict__ peers, const int32_t* __restrict__ rank_first,
+                                          int R, int64_t rows_per_rank, int64_t g, int64_t row_bytes) {
+  int64_t d, lr;
+  if (rank_first) {
+    int lo = 0, hi = R - 1;  // last rank whose first row is <= g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(rank_first + mid) <= g)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    d = lo;
+    lr = g - __ldg(rank_first + lo);
+  } else {
+    d = g / rows_per_rank;
+    lr = g - d * rows_per_rank;
+  }
+  if (d < 0 || d >= R || lr < 0 || lr >= rows_per_rank) return nullptr;
+  const uint64_t base = __ldg(peers + d);
+  if (!base || (base & 15u)) return nullptr;
+  return reinterpret_cast<char*>(base) + lr * row_bytes;
+}
+
 // 16-byte global loads that skip L1 allocation (streamed once)
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 v;

@@ -201,6 +201,21 @@ static const void* grad_fn(int rep_dtype, int clear) {
   return clear ? (const void*)k_grad_reduce<true, true, PEER> : (const void*)k_grad_reduce<true, false, PEER>;
 }
 
+// The fields of a quota plan the reduction reads, under the names of the
+// exact-S*K plan's layout.
+static EpPlanLayout grad_view(const EpQuotaLayout& Q) {
+  EpPlanLayout L{};
+  L.words = Q.words;
+  L.cap = Q.cap;
+  L.n_chunks = Q.n_chunks;
+  L.rep_experts = Q.rep_experts;
+  L.copy_first = Q.rep_first;
+  L.copy_cnt = Q.rep_cnt;
+  L.rep_rank = Q.rep_rank;
+  L.rank_rep_first = Q.rank_rep_first;
+  return L;
+}
+
 // peers == NULL: g_home [E, n], g_rep [cap, n] (row m = replica m).  Else the
 // rank-local form for `rank` (g_home [E/R, n], replica rows behind peers).
 static int run_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, const int32_t* plan,
@@ -250,6 +265,23 @@ extern "C" int ep_replica_grad_reduce_peer(float* g_home_local, const uint64_t* 
                          rep_rows, dev_status, stream);
 }
 
+extern "C" int ep_quota_replica_grad_reduce_peer(float* g_home_local, const uint64_t* peer_g_rep, int64_t rep_rows,
+                                                 int rep_dtype, int64_t n, int E, int R, int rank, const int32_t* plan,
+                                                 size_t plan_words, int clear_replicas, int32_t* dev_status,
+                                                 cudaStream_t stream) {
+  if (n < 0 || E < 1 || E > EP_MAX_EXPERTS || R < 1 || R > EP_MAX_RANKS || E % R || rank < 0 || rank >= R ||
+      rep_rows < 0)
+    return EP_ERR_ARG;
+  if (rep_dtype != EP_DTYPE_F32 && rep_dtype != EP_DTYPE_BF16) return EP_ERR_ARG;
+  if (!plan || !peer_g_rep) return EP_ERR_ARG;
+  EpQuotaLayout Q;
+  quota_layout(E, R, &Q);
+  if ((int64_t)plan_words < Q.words) return EP_ERR_CAPACITY;
+  const EpPlanLayout L = grad_view(Q);
+  return run_grad_reduce(g_home_local, nullptr, rep_dtype, n, E, plan, L, clear_replicas, peer_g_rep, R, rank,
+                         rep_rows, dev_status, stream);
+}
+
 extern "C" int ep_quota_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int64_t n, int E, int R,
                                             const int32_t* plan, size_t plan_words, int clear_replicas,
                                             int32_t* dev_status, cudaStream_t stream) {
@@ -259,12 +291,6 @@ extern "C" int ep_quota_replica_grad_reduce(float* g_home, const void* g_rep, in
   EpQuotaLayout Q;
   quota_layout(E, R, &Q);
   if ((int64_t)plan_words < Q.words) return EP_ERR_CAPACITY;
-  EpPlanLayout L{};
-  L.words = Q.words;
-  L.cap = Q.cap;
-  L.n_chunks = Q.n_chunks;
-  L.rep_experts = Q.rep_experts;
-  L.copy_first = Q.rep_first;
-  L.copy_cnt = Q.rep_cnt;
+  const EpPlanLayout L = grad_view(Q);
   return run_grad_reduce(g_home, g_rep, rep_dtype, n, E, plan, L, clear_replicas, nullptr, R, 0, 0, dev_status, stream);
 }

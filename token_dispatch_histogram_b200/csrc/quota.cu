@@ -220,6 +220,36 @@ __global__ void __launch_bounds__(Q_SCAN_THREADS)
   }
 }
 
+// Rank-local form: the gathered load matrix counts [R, E] (row s = source rank
+// s's pairs per expert) as the per-rank prefixes the search reads with one
+// "tile" per rank: pre[s][e] = sum_{s' < s} counts[s'][e], pre[R][e] = T_e =
+// loads[e].  A column with a negative entry or a sum past int32 gets -1, so
+// the loads do not add up and the search writes no plan.  Also resets the
+// search's ticket and best threshold.
+__global__ void __launch_bounds__(256)
+    k_q_counts_prefix(const int32_t* __restrict__ counts, int R, int E, int32_t* __restrict__ pre,
+                      int32_t* __restrict__ loads, uint32_t* __restrict__ hdr) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    hdr[QH_TICKET_SEARCH] = 0;
+    hdr[QH_BEST] = 0xffffffffu;
+  }
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  int64_t run = 0;
+  bool ok = true;
+  for (int r = 0; r < R; ++r) {
+    const int32_t c = counts[(int64_t)r * E + e];
+    pre[(int64_t)r * E + e] = (int32_t)run;
+    ok = ok && c >= 0;
+    run += c;
+    ok = ok && run <= INT32_MAX;
+    if (!ok) run = 0;
+  }
+  const int32_t tot = ok ? (int32_t)run : -1;
+  pre[(int64_t)R * E + e] = tot;
+  loads[e] = tot;
+}
+
 // --------------------------------------------------------- 3. search + build
 
 // Whether every chunk finds room at threshold tau: the chunk/room walk over
@@ -570,10 +600,17 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
 
 // ----------------------------------------------------------------- 4. layout
 
+// base_counts == NULL: the pairs of all R source ranks, rank-aligned tiles,
+// excl the global per-tile prefixes.  Otherwise (rank-local form) the pairs of
+// source rank base_rank only: excl holds the per-tile prefixes of those pairs
+// alone (tpr = its tile count), base_counts [R, E] is the gathered load matrix
+// that gives the pairs of each expert on lower source ranks, pos is indexed by
+// the rank's own pairs and src may be NULL.
 __global__ void __launch_bounds__(SCAT_THREADS)
     k_q_layout(const int32_t* __restrict__ topk, int64_t SK, int E, int R, int tile, int tpr,
-               const int32_t* __restrict__ excl, const int32_t* __restrict__ plan, EpQuotaLayout L,
-               int32_t* __restrict__ pos, int32_t* __restrict__ src, int32_t* dev_status) {
+               const int32_t* __restrict__ excl, const int32_t* __restrict__ base_counts, int base_rank,
+               const int32_t* __restrict__ plan, EpQuotaLayout L, int32_t* __restrict__ pos,
+               int32_t* __restrict__ src, int32_t* dev_status) {
   extern __shared__ int32_t sm[];
   int32_t* s_ids = sm;                  // [tile]
   int32_t* s_whist = s_ids + tile;      // [SCAT_WARPS * E]
@@ -587,11 +624,13 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   int32_t* s_icum = s_rrank + L.cap;    // [E + cap] cumulative start of instance i's looked-up range
   int32_t* s_istart = s_icum + E + L.cap;  // [E + cap] its first looked-up row
   int32_t* s_ispan = s_istart + E + L.cap; // [E + cap] its looked-up rows
+  int32_t* s_excl = s_ispan + E + L.cap;   // [E] (rank-local form) this tile's list offsets
   __shared__ int s_flags;
   const int64_t t = blockIdx.x;
-  const int rs = (int)(t / tpr);
-  const int64_t lt = t % tpr;
-  const int64_t p0 = (int64_t)rs * SK + lt * tile;
+  const bool local = base_counts != nullptr;
+  const int rs = local ? base_rank : (int)(t / tpr);
+  const int64_t lt = local ? t : t % tpr;
+  const int64_t p0 = (local ? 0 : (int64_t)rs * SK) + lt * tile;
   const int n = (int)min((int64_t)tile, SK - lt * tile);
   const int ER = E / R;
   const int64_t P = (int64_t)R * SK;
@@ -617,7 +656,14 @@ __global__ void __launch_bounds__(SCAT_THREADS)
     const int rf = plan[L.rep_first + e], rc = plan[L.rep_cnt + e];
     s_rf[e] = rf;
     s_rc[e] = rc;
-    s_lpre[e] = excl[(int64_t)rs * tpr * E + e];
+    if (local) {
+      int32_t b = 0;
+      for (int r = 0; r < rs; ++r) b += base_counts[(int64_t)r * E + e];
+      s_lpre[e] = b;
+      s_excl[e] = excl[t * E + e] + b;
+    } else {
+      s_lpre[e] = excl[(int64_t)rs * tpr * E + e];
+    }
     int a = 0, b = rc;  // replicas of e on ranks < rs: the first a
     while (a < b) {
       const int mid = (a + b) >> 1;
@@ -666,15 +712,41 @@ __global__ void __launch_bounds__(SCAT_THREADS)
       return;
     }
     pos[p] = row;
-    src[row] = (int32_t)p;
+    if (src) src[row] = (int32_t)p;
   };
   auto bad = [&](int64_t p) {
     atomicOr(&s_flags, EP_DEV_BAD_EXPERT_ID);
     pos[p] = -1;
   };
-  tile_stable_ranks(topk, E, tile, p0, n, excl + t * E, s_ids, s_whist, emit, bad);
+  tile_stable_ranks(topk, E, tile, p0, n, local ? s_excl : excl + t * E, s_ids, s_whist, emit, bad);
   __syncthreads();
   if (threadIdx.x == 0 && s_flags) flag(dev_status, s_flags);
+}
+
+struct QCountsWs {
+  size_t hdr, pre, bytes;
+};
+inline QCountsWs q_counts_ws(int E, int R) {
+  QCountsWs w;
+  w.hdr = 0;
+  w.pre = 256;
+  w.bytes = (w.pre + sizeof(int32_t) * (size_t)E * (size_t)(R + 1) + 255) & ~(size_t)255;
+  return w;
+}
+
+static int run_q_layout(const int32_t* topk, int64_t SK, int E, int R, int tile, int tpr, int64_t ntiles,
+                        const int32_t* excl, const int32_t* base_counts, int base_rank, const int32_t* plan,
+                        const EpQuotaLayout& L, int32_t* pos, int32_t* src, int32_t* dev_status,
+                        cudaStream_t stream) {
+  const size_t smem = sizeof(int32_t) * ((size_t)tile + (size_t)SCAT_WARPS * E + 7 * (size_t)E + (size_t)L.cap +
+                                         3 * ((size_t)E + L.cap));
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_q_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return EP_ERR_CUDA;
+  k_q_layout<<<(unsigned)ntiles, SCAT_THREADS, smem, stream>>>(topk, SK, E, R, tile, tpr, excl, base_counts,
+                                                               base_rank, plan, L, pos, src, dev_status);
+  count_launch();
+  return launch_status();
 }
 
 }  // namespace ep
@@ -722,14 +794,63 @@ extern "C" int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, 
   k_q_search<<<2 * num_sms(), Q_SEARCH_THREADS, search_smem, stream>>>(loads, excl, q.tpr, E, R, B, P, hdr, plan, L);
   count_launch(3);
   if (q.ntiles > 0) {
-    const size_t smem =
-        sizeof(int32_t) * ((size_t)q.tile + (size_t)SCAT_WARPS * E + 6 * (size_t)E + (size_t)L.cap + 3 * ((size_t)E + L.cap));
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(k_q_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return EP_ERR_CUDA;
-    k_q_layout<<<(unsigned)q.ntiles, SCAT_THREADS, smem, stream>>>(topk_ids, SK, E, R, q.tile, q.tpr, excl, plan, L,
-                                                                   pos, src, dev_status);
-    count_launch();
+    const int rc = run_q_layout(topk_ids, SK, E, R, q.tile, q.tpr, q.ntiles, excl, nullptr, 0, plan, L, pos, src,
+                                dev_status, stream);
+    if (rc != EP_OK) return rc;
   }
   return launch_status();
+}
+
+extern "C" int ep_quota_counts_workspace_size(int E, int R, size_t* bytes) {
+  if (!bytes || E < 1 || E > EP_MAX_EXPERTS || R < 1 || R > EP_MAX_RANKS || E % R) return EP_ERR_ARG;
+  *bytes = q_counts_ws(E, R).bytes;
+  return EP_OK;
+}
+
+extern "C" int ep_quota_plan_from_counts(const int32_t* counts, int R, int64_t S, int K, int E, int B, int32_t* loads,
+                                         int32_t* plan, size_t plan_words, void* ws, size_t ws_bytes,
+                                         int32_t* dev_status, cudaStream_t stream) {
+  if (!counts || !loads || !plan || !ws || R < 1 || R > EP_MAX_RANKS || E < 1 || E > EP_MAX_EXPERTS || E % R ||
+      K < 1 || K > E || S < 0 || B < 0)
+    return EP_ERR_ARG;
+  if ((int64_t)R * S * K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  EpQuotaLayout L;
+  quota_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  const QCountsWs w = q_counts_ws(E, R);
+  if (ws_bytes < w.bytes) return EP_ERR_CAPACITY;
+  char* base = static_cast<char*>(ws);
+  uint32_t* hdr = reinterpret_cast<uint32_t*>(base + w.hdr);
+  int32_t* pre = reinterpret_cast<int32_t*>(base + w.pre);
+  k_q_counts_prefix<<<(E + 255) / 256, 256, 0, stream>>>(counts, R, E, pre, loads, hdr);
+  const size_t search_smem = q_search_smem(E, R);
+  if (search_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_q_search, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)search_smem) != cudaSuccess)
+    return EP_ERR_CUDA;
+  const int64_t P = (int64_t)R * S * K;
+  k_q_search<<<2 * num_sms(), Q_SEARCH_THREADS, search_smem, stream>>>(loads, pre, 1, E, R, B, P, hdr, plan, L);
+  count_launch(2);
+  (void)dev_status;  // invalid counts show as tau = -1 in the plan
+  return launch_status();
+}
+
+extern "C" int ep_quota_layout_rank(const int32_t* topk_local, int64_t S, int K, int E, int R, int rank,
+                                    const int32_t* counts, const int32_t* plan, size_t plan_words, const void* ws,
+                                    size_t ws_bytes, int32_t* pos_local, int32_t* dev_status, cudaStream_t stream) {
+  if (!valid_tke(S, K, E) || R < 1 || R > EP_MAX_RANKS || E % R || rank < 0 || rank >= R) return EP_ERR_ARG;
+  if ((int64_t)R * S * K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (!plan || !ws || !counts) return EP_ERR_ARG;
+  const int64_t SK = S * K;
+  if (SK > 0 && (!topk_local || !pos_local)) return EP_ERR_ARG;
+  EpQuotaLayout L;
+  quota_layout(E, R, &L);
+  if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
+  const WsLayout wl = ws_layout(SK, E);  // the scratch ep_route_stats filled for topk_local
+  if (ws_bytes < wl.bytes) return EP_ERR_CAPACITY;
+  if (SK == 0) return EP_OK;
+  const int tile = tile_pairs_for(SK);
+  const int64_t nt = num_tiles(SK, tile);
+  const int32_t* excl = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + wl.excl_off);
+  return run_q_layout(topk_local, SK, E, R, tile, (int)nt, nt, excl, counts, rank, plan, L, pos_local, nullptr,
+                      dev_status, stream);
 }

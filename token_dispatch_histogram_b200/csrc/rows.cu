@@ -46,7 +46,8 @@ template <bool PEER>
 __global__ void __launch_bounds__(32)
     k_dispatch(const uint8_t* __restrict__ x, int64_t T, int K, uint32_t row_bytes, const int32_t* __restrict__ pos,
                int64_t buf_rows, uint8_t* __restrict__ buf, const uint64_t* __restrict__ peers,
-               int64_t rows_per_rank, int stages, int32_t* dev_status) {
+               const int32_t* __restrict__ rank_first, int R, int64_t rows_per_rank, int stages,
+               int32_t* dev_status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t stride_b = (row_bytes + 127u) & ~127u;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stride_b);
@@ -87,12 +88,8 @@ __global__ void __launch_bounds__(32)
       const int32_t row = ring[s * K + lane];
       if (row >= 0 && row < buf_rows) {
         uint8_t* dst;
-        if (PEER) {
-          const int64_t d = row / rows_per_rank;
-          const uint64_t base = __ldg(peers + d);
-          // a missing or misaligned rank buffer is reported, never written
-          dst = (base && !(base & 15u)) ? reinterpret_cast<uint8_t*>(base) + (row - d * rows_per_rank) * (int64_t)row_bytes
-                                        : nullptr;
+        if (PEER) {  // a missing or misaligned rank buffer, or a row past it, is reported, never written
+          dst = reinterpret_cast<uint8_t*>(peer_row(peers, rank_first, R, rows_per_rank, row, row_bytes));
         } else {
           dst = buf + (int64_t)row * row_bytes;
         }
@@ -169,7 +166,8 @@ template <int K, bool PEER>
 __global__ void __launch_bounds__(256, 4)
     k_combine(const uint16_t* __restrict__ y, int64_t y_rows, const float* __restrict__ w,
               const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ out,
-              const uint64_t* __restrict__ peers, int64_t rows_per_rank, int32_t* dev_status) {
+              const uint64_t* __restrict__ peers, const int32_t* __restrict__ rank_first, int R,
+              int64_t rows_per_rank, int32_t* dev_status) {
   constexpr int MAXT = 8;  // tokens per CTA iteration (rows narrower than 256 vectors)
   __shared__ int32_t s_rows[2][MAXT][K];
   __shared__ float s_w[2][MAXT][K];
@@ -200,11 +198,8 @@ __global__ void __launch_bounds__(256, 4)
       if constexpr (PEER) {
         const uint16_t* base = nullptr;
         if (r >= 0) {
-          const int64_t d = r / rows_per_rank;
-          const uint64_t pb = __ldg(peers + d);
-          if (pb && !(pb & 15u)) {
-            base = reinterpret_cast<const uint16_t*>(pb) + (r - d * rows_per_rank) * H;
-          } else {  // a missing or misaligned rank buffer is reported, never read
+          base = reinterpret_cast<const uint16_t*>(peer_row(peers, rank_first, R, rows_per_rank, r, H * 2));
+          if (!base) {  // a missing or misaligned rank buffer, or a row past it, is reported, never read
             s_rows[b][s][k] = -1;
             s_bad = 1;
           }
@@ -411,8 +406,8 @@ namespace ep {
 // Dispatch launch shared by the one-buffer and the rank-local (peer) entry
 // points.  peers == NULL: rows go to buf[row]; else to the rank buffers.
 static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
-                        int64_t buf_rows, const uint64_t* peers, int64_t rows_per_rank, int32_t* dev_status,
-                        cudaStream_t stream) {
+                        int64_t buf_rows, const uint64_t* peers, const int32_t* rank_first, int R,
+                        int64_t rows_per_rank, int32_t* dev_status, cudaStream_t stream) {
   const uint32_t row_bytes = (uint32_t)(H * 2);
   const uint32_t stride_b = (row_bytes + 127u) & ~127u;
   // Measured on B200: the scatter runs fastest with about 32 KB of row loads
@@ -431,9 +426,9 @@ static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const in
   const int grid = occupancy_grid(fn, 32, smem, T, per_sm);
   const uint8_t* xb = reinterpret_cast<const uint8_t*>(x);
   uint8_t* bb = reinterpret_cast<uint8_t*>(buf);
-  void* args[] = {(void*)&xb,    (void*)&T,     (void*)&K,  (void*)&row_bytes,     (void*)&pos,
-                  (void*)&buf_rows, (void*)&bb, (void*)&peers, (void*)&rows_per_rank, (void*)&stages,
-                  (void*)&dev_status};
+  void* args[] = {(void*)&xb,    (void*)&T,          (void*)&K, (void*)&row_bytes,     (void*)&pos,
+                  (void*)&buf_rows, (void*)&bb,      (void*)&peers, (void*)&rank_first, (void*)&R,
+                  (void*)&rows_per_rank, (void*)&stages, (void*)&dev_status};
   if (cudaLaunchKernel(fn, dim3(grid), dim3(32), args, smem, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
@@ -448,18 +443,20 @@ extern "C" int ep_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const
   if (T * (int64_t)K >= ((int64_t)1 << 31)) return EP_ERR_ARG;
   if (T == 0) return EP_OK;
   if (!x || !pos || !buf || !aligned16(x) || !aligned16(buf)) return EP_ERR_ARG;
-  return run_dispatch(x, T, K, H, pos, buf, buf_rows, nullptr, 0, dev_status, stream);
+  return run_dispatch(x, T, K, H, pos, buf, buf_rows, nullptr, nullptr, 1, 0, dev_status, stream);
 }
 
 extern "C" int ep_dispatch_peer(const uint16_t* x_local, int64_t S, int K, int64_t H, const int32_t* pos_local,
-                                const uint64_t* peer_bufs, int R, int64_t rows_per_rank, int32_t* dev_status,
+                                const uint64_t* peer_bufs, const int32_t* rank_first_row, int R,
+                                int64_t rows_per_rank, int64_t total_rows, int32_t* dev_status,
                                 cudaStream_t stream) {
-  if (S < 0 || K < 1 || K > 32 || H < 8 || H % 8 || R < 1 || R > EP_MAX_RANKS || rows_per_rank < 1) return EP_ERR_ARG;
+  if (S < 0 || K < 1 || K > 32 || H < 8 || H % 8 || R < 1 || R > EP_MAX_RANKS || rows_per_rank < 1 || total_rows < 0)
+    return EP_ERR_ARG;
   if (H * 2 > (1 << 20)) return EP_ERR_ARG;
-  if (S * (int64_t)K >= ((int64_t)1 << 31) || (int64_t)R * rows_per_rank >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (S * (int64_t)K >= ((int64_t)1 << 31) || total_rows >= ((int64_t)1 << 31)) return EP_ERR_ARG;
   if (S == 0) return EP_OK;
   if (!x_local || !pos_local || !peer_bufs || !aligned16(x_local)) return EP_ERR_ARG;
-  return run_dispatch(x_local, S, K, H, pos_local, nullptr, (int64_t)R * rows_per_rank, peer_bufs, rows_per_rank,
+  return run_dispatch(x_local, S, K, H, pos_local, nullptr, total_rows, peer_bufs, rank_first_row, R, rows_per_rank,
                       dev_status, stream);
 }
 
@@ -504,9 +501,11 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
   if (fn) {
     const int grid = occupancy_grid(fn, 256, 0, T, 4);
     const uint64_t* peers = nullptr;
+    const int32_t* rank_first = nullptr;
+    int R = 1;
     int64_t rpr = 0;
-    void* args[] = {(void*)&y,   (void*)&y_rows, (void*)&w,     (void*)&pos, (void*)&T,
-                    (void*)&H,   (void*)&out,    (void*)&peers, (void*)&rpr, (void*)&dev_status};
+    void* args[] = {(void*)&y,     (void*)&y_rows,     (void*)&w, (void*)&pos, (void*)&T,          (void*)&H,
+                    (void*)&out,   (void*)&peers, (void*)&rank_first, (void*)&R, (void*)&rpr, (void*)&dev_status};
     if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   } else {
     const int grid = occupancy_grid((const void*)k_combine_any, 256, 0, T * (H / 8) / 256 + 1, 8);
@@ -516,19 +515,21 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
   return launch_status();
 }
 
-extern "C" int ep_combine_peer(const uint64_t* peer_bufs, int R, int64_t rows_per_rank, const float* w_local,
+extern "C" int ep_combine_peer(const uint64_t* peer_bufs, const int32_t* rank_first_row, int R,
+                               int64_t rows_per_rank, int64_t total_rows, const float* w_local,
                                const int32_t* pos_local, int64_t S, int K, int64_t H, uint16_t* out_local,
                                int32_t* dev_status, cudaStream_t stream) {
-  if (S < 0 || K < 1 || K > 8 || H < 8 || H % 8 || R < 1 || R > EP_MAX_RANKS || rows_per_rank < 1) return EP_ERR_ARG;
-  if (S * (int64_t)K >= ((int64_t)1 << 31) || (int64_t)R * rows_per_rank >= ((int64_t)1 << 31)) return EP_ERR_ARG;
+  if (S < 0 || K < 1 || K > 8 || H < 8 || H % 8 || R < 1 || R > EP_MAX_RANKS || rows_per_rank < 1 || total_rows < 0)
+    return EP_ERR_ARG;
+  if (S * (int64_t)K >= ((int64_t)1 << 31) || total_rows >= ((int64_t)1 << 31)) return EP_ERR_ARG;
   if (S == 0) return EP_OK;
   if (!peer_bufs || !pos_local || !out_local || !aligned16(out_local)) return EP_ERR_ARG;  // w NULL: unit weights
   const void* fn = combine_fn<true>(K);
   const int grid = occupancy_grid(fn, 256, 0, S, 4);
   const uint16_t* y = nullptr;
-  int64_t y_rows = (int64_t)R * rows_per_rank;
-  void* args[] = {(void*)&y,         (void*)&y_rows,   (void*)&w_local,   (void*)&pos_local,     (void*)&S,
-                  (void*)&H,         (void*)&out_local, (void*)&peer_bufs, (void*)&rows_per_rank, (void*)&dev_status};
+  void* args[] = {(void*)&y,          (void*)&total_rows, (void*)&w_local,        (void*)&pos_local,
+                  (void*)&S,          (void*)&H,          (void*)&out_local,      (void*)&peer_bufs,
+                  (void*)&rank_first_row, (void*)&R,      (void*)&rows_per_rank,  (void*)&dev_status};
   if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();

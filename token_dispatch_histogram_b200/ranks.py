@@ -12,7 +12,8 @@ matrix.  One step on rank r:
 
   count()           local histogram -> counts_row (ep_route_stats on S tokens)
   gather            all ranks' rows -> counts [R, E] (the one collective)
-  plan_and_layout() ep_plan_from_counts + ep_layout_rank (no further exchange)
+  plan_and_layout() ep_plan_from_counts + ep_layout_rank, or the quota-driven
+                    ep_quota_plan_from_counts + ep_quota_layout_rank (no further exchange)
   dispatch()        ep_dispatch_peer: rows into the receiving ranks' buffers
   combine()         ep_combine_peer: expert rows back from those buffers
   grad_reduce()     ep_replica_grad_reduce_peer: replica gradients home
@@ -24,7 +25,9 @@ import torch
 import torch.distributed as dist
 
 from . import (ep_combine_peer, ep_dispatch_peer, ep_layout_rank, ep_plan_from_counts, ep_plan_layout,
-               ep_replica_grad_reduce_peer, ep_route_stats, ep_status_read, ep_workspace_size)
+               ep_quota_counts_workspace_size, ep_quota_layout_rank, ep_quota_plan_from_counts,
+               ep_quota_plan_layout, ep_quota_replica_grad_reduce_peer, ep_replica_grad_reduce_peer,
+               ep_route_stats, ep_status_read, ep_workspace_size)
 
 
 def gather_counts(counts_row, counts, group=None):
@@ -41,33 +44,50 @@ def gather_counts(counts_row, counts, group=None):
 class EpRank:
     """Static buffers of one rank of R: S tokens of top-K routing, H hidden.
 
-    buf is this rank's S*K-row receive buffer (expert-grouped: home experts in
-    id order, then received replicas in match order); peers must be set to the
-    R ranks' buffers (set_peers) before dispatch/combine.  With grad_n > 0,
-    g_home holds this rank's E/R home experts' gradients [E/R, grad_n] fp32 and
-    g_rep the gradients of the replicas it receives [rep_rows, grad_n], row j =
-    its j-th received replica (default E - E/R rows, enough for any plan;
-    grad_peers: the R ranks' g_rep, set_grad_peers)."""
+    planner "exact": the exact-S*K replica plan (every rank receives S*K rows);
+    "quota": the quota-driven plan with at most B replicas per rank (rank r
+    receives rank_load[r] <= tau* rows).  buf is this rank's receive buffer of
+    buf_rows rows (default S*K; a quota plan needs tau*, and rows past the
+    buffer are skipped and flagged), expert-grouped: home experts in id order,
+    then received replicas in match order.  peers must be set to the R ranks'
+    buffers (set_peers) before dispatch/combine.  With grad_n > 0, g_home holds
+    this rank's E/R home experts' gradients [E/R, grad_n] fp32 and g_rep the
+    gradients of the replicas it receives [rep_rows, grad_n], row j = its j-th
+    received replica (default E - E/R rows, enough for any plan; grad_peers:
+    the R ranks' g_rep, set_grad_peers)."""
 
-    def __init__(self, rank, R, S, K, E, H, device="cuda", grad_n=0, grad_dtype=torch.float32, rep_rows=None):
+    def __init__(self, rank, R, S, K, E, H, device="cuda", grad_n=0, grad_dtype=torch.float32, rep_rows=None,
+                 planner="exact", B=0, buf_rows=None):
         if E % R:
             raise ValueError("E must be a multiple of R")
+        if planner not in ("exact", "quota"):
+            raise ValueError(planner)
         self.rank, self.R, self.S, self.K, self.E, self.H = rank, R, S, K, E, H
+        self.planner, self.B = planner, B
         self.device = torch.device(device)
         dev = self.device
         i32 = dict(dtype=torch.int32, device=dev)
         self.SK = S * K
+        self.buf_rows = self.SK if buf_rows is None else buf_rows
         self.topk_local = torch.zeros((S, K), **i32)
         self.w_local = torch.zeros((S, K), dtype=torch.float32, device=dev)
         self.x_local = torch.zeros((S, H), dtype=torch.bfloat16, device=dev)
         self.out_local = torch.zeros((S, H), dtype=torch.bfloat16, device=dev)
-        self.buf = torch.zeros((self.SK, H), dtype=torch.bfloat16, device=dev)
+        self.buf = torch.zeros((self.buf_rows, H), dtype=torch.bfloat16, device=dev)
         self.counts_row = torch.zeros(E, **i32)
         self.counts = torch.zeros((R, E), **i32)
         self.loads = torch.zeros(E, **i32)
         self.max_vio_local = torch.zeros(1, dtype=torch.float64, device=dev)
-        self.plan_layout = ep_plan_layout(E, R)
+        if planner == "exact":
+            self.plan_layout = ep_plan_layout(E, R)
+            self.rank_first = None
+        else:
+            self.plan_layout = ep_quota_plan_layout(E, R)
+            self.ws_q = torch.zeros(ep_quota_counts_workspace_size(E, R), dtype=torch.uint8, device=dev)
         self.plan = torch.zeros(self.plan_layout["words"], **i32)
+        if planner == "quota":  # a view of the plan: each rank's first global row
+            off = self.plan_layout["rank_off"]
+            self.rank_first = self.plan[off:off + R]
         self.pos_local = torch.zeros(self.SK, **i32)
         self.ws = torch.zeros(ep_workspace_size(S, K, E), dtype=torch.uint8, device=dev)
         self.dev_status = torch.zeros(1, **i32)
@@ -96,9 +116,15 @@ class EpRank:
         ep_route_stats(self.topk_local, self.E, self.counts_row, self.max_vio_local, self.ws, self.dev_status, stream)
 
     def plan_and_layout(self, stream=None):
-        ep_plan_from_counts(self.counts, self.S, self.K, self.plan, self.loads, self.dev_status, stream)
-        ep_layout_rank(self.topk_local, self.rank, self.counts, self.plan, self.ws, self.pos_local, None,
-                       self.dev_status, stream)
+        if self.planner == "exact":
+            ep_plan_from_counts(self.counts, self.S, self.K, self.plan, self.loads, self.dev_status, stream)
+            ep_layout_rank(self.topk_local, self.rank, self.counts, self.plan, self.ws, self.pos_local, None,
+                           self.dev_status, stream)
+        else:
+            ep_quota_plan_from_counts(self.counts, self.S, self.K, self.B, self.loads, self.plan, self.ws_q,
+                                      self.dev_status, stream)
+            ep_quota_layout_rank(self.topk_local, self.rank, self.counts, self.plan, self.ws, self.pos_local,
+                                 self.dev_status, stream)
 
     def route(self, group=None, stream=None):
         """count -> all-gather of the counts (torch.distributed) -> plan and layout."""
@@ -107,15 +133,17 @@ class EpRank:
         self.plan_and_layout(stream)
 
     def dispatch(self, stream=None):
-        ep_dispatch_peer(self.x_local, self.K, self.pos_local, self.peers, self.SK, self.dev_status, stream)
+        ep_dispatch_peer(self.x_local, self.K, self.pos_local, self.peers, self.buf_rows, self.R * self.SK,
+                         self.rank_first, self.dev_status, stream)
 
     def combine(self, stream=None):
-        ep_combine_peer(self.peers, self.SK, self.w_local, self.pos_local, self.out_local, None, self.dev_status,
-                        stream)
+        ep_combine_peer(self.peers, self.buf_rows, self.R * self.SK, self.w_local, self.pos_local, self.out_local,
+                        None, self.rank_first, self.dev_status, stream)
 
     def grad_reduce(self, clear=False, stream=None):
-        ep_replica_grad_reduce_peer(self.g_home, self.grad_peers, self.rep_rows, self.g_rep.dtype, self.E, self.rank,
-                                    self.plan, clear, self.dev_status, stream)
+        fn = ep_replica_grad_reduce_peer if self.planner == "exact" else ep_quota_replica_grad_reduce_peer
+        fn(self.g_home, self.grad_peers, self.rep_rows, self.g_rep.dtype, self.E, self.rank, self.plan, clear,
+           self.dev_status, stream)
 
     def status(self, stream=None):
         return ep_status_read(self.dev_status, stream)
