@@ -13,6 +13,7 @@ token's top-1 on one expert, an expert with no pair, T = 0.
 import numpy as np
 import pytest
 
+import oracle as O
 import oracle_pins as PINS
 import workload as W
 from gpu_path import (bf16_ulp_diff, case_inputs, expected_plan_tables, plan_field, run_cuda, run_oracle)
@@ -145,6 +146,54 @@ def test_dispatch_expert_combine(case):
     # combine against the layout-free closed form too
     cf = __import__("oracle").combine_closed(x, w, topk, scale)
     assert bf16_ulp_diff(cu["out"], cf).max() <= 1
+
+
+def test_bf16_rounding_edges():
+    """The row kernels round fp32 to bf16 with the hardware pair conversion.
+    Through the stand-in expert (one fp32 multiply, one rounding) and combine
+    (K = 1, unit weight), crafted values hit every class: exact ties to even,
+    overflow to Inf, subnormal results, signed zeros, Inf in; each must equal
+    the oracle's rounding bit for bit, and NaN in must give NaN out."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    rng = np.random.default_rng(11)
+    specials = np.array([0x7F7F, 0xFF7F, 0x0001, 0x8001, 0x0080, 0x007F, 0x0000, 0x8000, 0x7F80, 0xFF80,
+                         0x3F81, 0x3FC1, 0x4001, 0xBF81, 0x3C01, 0x0100], dtype=np.uint16)
+    H, E = 64, 4
+    rows = 64
+    x = rng.integers(0, 0x10000, size=(rows, H), dtype=np.uint16)
+    x[(x & 0x7F80) == 0x7F80] = 0x3F80  # no NaN/Inf at random
+    x[:, :len(specials)] = specials
+    scale = np.array([1.5, 2.0 ** -10, 1.0 + 2.0 ** -8, 1.0 + 2.0 ** -23], dtype=np.float32)
+    topk = (np.arange(rows) % E).astype(np.int32).reshape(rows, 1)
+    src = np.arange(rows, dtype=np.int32)
+    want = O.expert_standin(x, src, topk, scale)
+    dev = "cuda"
+    t_x = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    y = torch.empty_like(t_x)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    tdh.ep_expert_scale(t_x, torch.from_numpy(src).to(dev), torch.from_numpy(topk).to(dev),
+                        torch.from_numpy(scale).to(dev), y, st)
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert tdh.ep_status_read(st) == 0
+    np.testing.assert_array_equal(got, want)
+    assert np.any(got == 0x7F80) and np.any(got == 0xFF80)   # overflow to +-Inf happened
+    assert np.any((got & 0x7F80) == 0) and np.any((got & 0x7FFF) != 0)  # subnormal results happened
+    # combine of one unit-weight row per token: the row, except that -0 comes
+    # out +0 (the accumulator starts at +0 and +0 + -0 = +0), as in the oracle
+    out = torch.empty_like(y)
+    w1 = torch.ones((rows, 1), dtype=torch.float32, device=dev)
+    tdh.ep_combine(y, w1, torch.from_numpy(src).to(dev), out, st)
+    got_c = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got_c, O.combine(got, np.ones((rows, 1), np.float32), src, 1))
+    np.testing.assert_array_equal(got_c, np.where(got == 0x8000, 0, got))
+    # NaN in, NaN out (the hardware writes the canonical NaN; the oracle keeps the payload)
+    xn = x.copy()
+    xn[:, 0] = 0x7FC1
+    t_xn = torch.from_numpy(xn.view(np.int16)).to(dev).view(torch.bfloat16)
+    tdh.ep_expert_scale(t_xn, torch.from_numpy(src).to(dev), torch.from_numpy(topk).to(dev),
+                        torch.from_numpy(scale).to(dev), y, st)
+    assert torch.isnan(y[:, 0].float()).all()
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

@@ -189,6 +189,17 @@ __device__ __forceinline__ void bulk_wait_read() {
 
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Two fp32 values to one packed bf16x2 word (lo in bits 0-15, hi in 16-31),
+// each rounded to nearest, ties to even, by the hardware conversion (one
+// instruction for both).  For every non-NaN input this equals
+// f32_to_bf16_bits (Inf and subnormals included); a NaN comes out as the
+// canonical bf16 NaN instead of keeping its payload bits.
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Rank-local form: address of global row g in the R ranks' buffers.  Ranks
 // hold rows_per_rank rows each (rank_first == NULL: rank g / rows_per_rank), or
 // rank r's rows start at rank_first[r] (ascending, rank_first[0] = 0) and fit

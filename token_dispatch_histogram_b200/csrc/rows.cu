@@ -148,9 +148,8 @@ __global__ void __launch_bounds__(256)
       uint32_t o[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint32_t lo = f32_to_bf16_bits(__fmul_rn(bf16_bits_to_f32(w[q] & 0xFFFFu), s));
-        const uint32_t hi = f32_to_bf16_bits(__fmul_rn(bf16_bits_to_f32(w[q] >> 16), s));
-        o[q] = lo | (hi << 16);
+        o[q] = f32x2_to_bf16x2(__fmul_rn(bf16_bits_to_f32(w[q] & 0xFFFFu), s),
+                               __fmul_rn(bf16_bits_to_f32(w[q] >> 16), s));
       }
       st_v4(y + r * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
     }
@@ -242,7 +241,7 @@ __global__ void __launch_bounds__(256, 4)
         }
         uint32_t o[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) o[q] = f32_to_bf16_bits(acc[2 * q]) | (f32_to_bf16_bits(acc[2 * q + 1]) << 16);
+        for (int q = 0; q < 4; ++q) o[q] = f32x2_to_bf16x2(acc[2 * q], acc[2 * q + 1]);
         st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
@@ -280,7 +279,7 @@ __global__ void __launch_bounds__(256)
     }
     uint32_t o[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) o[q] = f32_to_bf16_bits(acc[2 * q]) | (f32_to_bf16_bits(acc[2 * q + 1]) << 16);
+    for (int q = 0; q < 4; ++q) o[q] = f32x2_to_bf16x2(acc[2 * q], acc[2 * q + 1]);
     st_v4(out + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
   }
   if (bad) flag(dev_status, bad);
@@ -361,8 +360,7 @@ __global__ void __launch_bounds__(256, 2)
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            o[q] = f32_to_bf16_bits(__fmul_rn(wk[k], gf[2 * q])) |
-                   (f32_to_bf16_bits(__fmul_rn(wk[k], gf[2 * q + 1])) << 16);
+            o[q] = f32x2_to_bf16x2(__fmul_rn(wk[k], gf[2 * q]), __fmul_rn(wk[k], gf[2 * q + 1]));
             part[k] = fmaf(gf[2 * q], bf16_bits_to_f32(yd[q] & 0xFFFFu), part[k]);
             part[k] = fmaf(gf[2 * q + 1], bf16_bits_to_f32(yd[q] >> 16), part[k]);
           }
