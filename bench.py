@@ -385,6 +385,26 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device status {st:#x} in the backward timing")
         del dy, dx, dw
 
+    def replay_ms(fn, flush_between):
+        """Mean ms of fn captured as one CUDA graph and replayed args.steps
+        times (L2 flushed before each replay when asked), max over ranks."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i in range(args.steps):
+            if flush_between:
+                flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            g.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        del g
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / args.steps
+
     # ---- the quota-driven planner (a per-rank replica budget B) in place of
     # the exact-S*K plan: the same step (route, dispatch, combine, replica
     # gradients) and the route alone, each as one captured graph, replayed
@@ -411,24 +431,6 @@ def run_ours(args, rank, world, local_rank):
         def q_routes(B):
             for li, ly in enumerate(layers):
                 q_route(B, li, ly)
-
-        def replay_ms(fn, flush_between):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                fn()
-            g.replay()
-            torch.cuda.synchronize()
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-            for i in range(args.steps):
-                if flush_between:
-                    flush.fill_(i & 0xFF)
-                ev[i][0].record(stream)
-                g.replay()
-                ev[i][1].record(stream)
-            torch.cuda.synchronize()
-            del g
-            return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / args.steps
 
         try:
             for B in sorted({1, 3, E // R}):
@@ -460,6 +462,40 @@ def run_ours(args, rank, world, local_rank):
                 raise
             print(f"graph capture unavailable: {exc}", file=sys.stderr)
         del q_plans, q_pos, q_src, q_ws
+
+    # ---- the metric exactly as named (plan + dispatch + combine): the route
+    # without the align-sort walk, dispatch and combine, as one graph; and the
+    # align-sort and the replica gradient reduction alone.  `value` above is
+    # the whole step (all of them), so it is the lower of the two numbers.
+    as_named = None
+    if not args.no_graph:
+        def pdc():
+            for ly in layers:
+                tdh.ep_route_fused(ly.topk_ids, E, R, S, ly.loads, ly.max_vio, ly.plan, ly.pos, ly.src, ly.ws,
+                                   ly.pair_slot, 0, None, None, None, ly.dev_status)
+                tdh.ep_dispatch(ly.x, K, ly.pos, ly.buf, ly.dev_status)
+                tdh.ep_combine(ly.buf, ly.w, ly.pos, ly.out, ly.dev_status)
+
+        def align_only():
+            for ly in layers:
+                tdh.ep_align_sort(ly.topk_ids, E, ly.block_m, ly.sorted_token_ids, ly.expert_ids,
+                                  ly.num_tokens_post_pad, ly.ws, ly.dev_status)
+
+        def grads_only():
+            for ly in layers:
+                if ly.grad_n:
+                    ly.grad_reduce(False)
+
+        pdc_ms = replay_ms(pdc, True)
+        as_named = {"value": job_throughput(world, nl * P, 1, pdc_ms), "unit": UNIT, "ms_per_step": round(pdc_ms, 5),
+                    "what": "route without align-sort + dispatch + combine, one graph, L2 flushed",
+                    "align_sort_us": round(replay_ms(align_only, True) * 1e3 / nl, 2)}
+        if any(ly.grad_n for ly in layers):
+            as_named["grad_reduce_us"] = round(replay_ms(grads_only, True) * 1e3 / nl, 2)
+        for ly in layers:
+            st = ly.status(stream)
+            if st:
+                raise RuntimeError(f"device status {st:#x} in the plan+dispatch+combine timing")
 
     # ---- prefetch slots under a per-rank budget B (one small launch, timed
     # apart as device time: 20 launches in one captured graph, replayed):
@@ -575,6 +611,7 @@ def run_ours(args, rank, world, local_rank):
         "backward": backward,
         "prefetch_slots": prefetch,
         "quota_planner": quota,
+        "plan_dispatch_combine": as_named,
         "layers_per_step": nl,
         "route_path": args.route,
     }
