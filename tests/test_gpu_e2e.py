@@ -10,7 +10,7 @@ import workload as W
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("chunks", [1, 3, 8])
+@pytest.mark.parametrize("chunks", [1, 3, 8, 11])
 def test_run_host_matches_oracle(chunks):
     import torch
     import token_dispatch_histogram_b200 as tdh
