@@ -72,14 +72,6 @@ __device__ __forceinline__ void flag(int32_t* dev_status, int32_t bits) {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 
-// fp32 -> bf16 bits, round to nearest even; NaN kept quiet.
-__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (u >> 16) | 0x40u;
-  u += 0x7FFFu + ((u >> 16) & 1u);
-  return u >> 16;
-}
-
 __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
   uint64_t v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -191,9 +183,9 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 
 // Two fp32 values to one packed bf16x2 word (lo in bits 0-15, hi in 16-31),
 // each rounded to nearest, ties to even, by the hardware conversion (one
-// instruction for both).  For every non-NaN input this equals
-// f32_to_bf16_bits (Inf and subnormals included); a NaN comes out as the
-// canonical bf16 NaN instead of keeping its payload bits.
+// instruction for both).  For every non-NaN input this is the IEEE rounding
+// (overflow to Inf, subnormals kept); a NaN comes out as the canonical bf16
+// NaN (a quiet NaN with its payload bits dropped).
 __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
