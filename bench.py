@@ -497,6 +497,54 @@ def run_ours(args, rank, world, local_rank):
             if st:
                 raise RuntimeError(f"device status {st:#x} in the plan+dispatch+combine timing")
 
+    # ---- the rank-local form emulated on this GPU: R rank buffers reached
+    # through the peer table, each rank's dispatch and combine launched in
+    # turn (one graph), against the one-buffer dispatch + combine above
+    rank_local = None
+    if not args.no_graph and nl == 1 and 2 * P * H <= (4 << 30):
+        from token_dispatch_histogram_b200.ranks import EpRank
+        rks = [EpRank(r, R, S, K, E, H, device=dev) for r in range(R)]
+        for r, rk in enumerate(rks):
+            rk.topk_local.copy_(layer.topk_ids[r * S:(r + 1) * S])
+            rk.w_local.copy_(layer.w[r * S:(r + 1) * S])
+            rk.x_local.copy_(layer.x[r * S:(r + 1) * S])
+            rk.count()
+        counts = torch.stack([rk.counts_row for rk in rks])  # the all-gather, emulated
+        peers = tdh.peer_table([rk.buf for rk in rks])
+        for rk in rks:
+            rk.counts.copy_(counts)
+            rk.plan_and_layout()
+            rk.set_peers(peers)
+
+        side = [torch.cuda.Stream(dev) for _ in rks]
+
+        def rank_rows():  # the ranks run side by side, as on R GPUs; combine after every dispatch
+            cur = torch.cuda.current_stream(dev)
+            for phase in ("dispatch", "combine"):
+                for rk, s2 in zip(rks, side):
+                    s2.wait_stream(cur)
+                    with torch.cuda.stream(s2):
+                        getattr(rk, phase)(s2)
+                for s2 in side:
+                    cur.wait_stream(s2)
+
+        def one_buffer_rows():
+            for ly in layers:
+                tdh.ep_dispatch(ly.x, K, ly.pos, ly.buf, ly.dev_status)
+                tdh.ep_combine(ly.buf, ly.w, ly.pos, ly.out, ly.dev_status)
+
+        rl_ms = replay_ms(rank_rows, True)
+        ob_ms = replay_ms(one_buffer_rows, True)
+        same = all(torch.equal(rk.out_local, layer.out[r * S:(r + 1) * S]) for r, rk in enumerate(rks))
+        st = max(rk.status(stream) for rk in rks)
+        if st or not same:
+            raise RuntimeError(f"rank-local rows differ from the one-buffer rows (status {st:#x})")
+        rank_local = {"dispatch_combine_ms": round(rl_ms, 5), "one_buffer_ms": round(ob_ms, 5),
+                      "launches": 2 * R,
+                      "what": "R ranks' dispatch_peer, then their combine_peer, each rank on its own stream, one graph, "
+                              "L2 flushed"}
+        del rks, peers, side
+
     # ---- prefetch slots under a per-rank budget B (one small launch, timed
     # apart as device time: 20 launches in one captured graph, replayed):
     # replicas whose weights are read from the home rank, and the rank loads if
@@ -612,6 +660,7 @@ def run_ours(args, rank, world, local_rank):
         "prefetch_slots": prefetch,
         "quota_planner": quota,
         "plan_dispatch_combine": as_named,
+        "rank_local": rank_local,
         "layers_per_step": nl,
         "route_path": args.route,
     }

@@ -331,3 +331,68 @@ def test_rank_local_quota_grad_reduce():
         np.testing.assert_array_equal(rk.g_home.cpu().numpy(), gh[r * ER:(r + 1) * ER])
         c = int(nrep_r[r])
         np.testing.assert_array_equal(rk.g_rep[:c].cpu().numpy(), gr[first[r]:first[r] + c])
+
+
+def _nccl_one_rank(port, q):
+    """Child process: EpRank.route() through a real NCCL process group of one
+    rank (the all-gather of the counts is a genuine NCCL call), then dispatch
+    and combine through the peer table; results back through the queue."""
+    import datetime
+    import os
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from gpu_path import case_inputs
+    import token_dispatch_histogram_b200 as tdh
+    from token_dispatch_histogram_b200.ranks import EpRank
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        S, K, E, H = 1000, 4, 16, 256
+        topk, w, x = case_inputs(1, S, K, E, H, seed=8, bias_scale=1.5)
+        rk = EpRank(0, 1, S, K, E, H, device="cuda")
+        rk.topk_local.copy_(torch.from_numpy(topk))
+        rk.w_local.copy_(torch.from_numpy(w))
+        rk.x_local.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
+        rk.route()
+        rk.set_peers(tdh.peer_table([rk.buf]))
+        rk.dispatch()
+        rk.combine()
+        torch.cuda.synchronize()
+        q.put(dict(status=rk.status(), counts=rk.counts.cpu().numpy(), pos=rk.pos_local.cpu().numpy(),
+                   out=rk.out_local.view(torch.int16).cpu().numpy().view(np.uint16)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_local_route_through_nccl():
+    import socket
+    import torch.multiprocessing as mp
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_nccl_one_rank, args=(port, q))
+    p.start()
+    res = q.get(timeout=240)
+    p.join(60)
+    assert p.exitcode == 0
+    S, K, E, H = 1000, 4, 16, 256
+    topk, w, x = case_inputs(1, S, K, E, H, seed=8, bias_scale=1.5)
+    loads, _, _ = O.route_stats(topk, E)
+    pl = O.plan(loads, 1, S, K, E)
+    lo = O.layout(topk, pl, 1, S, E)
+    assert res["status"] == 0
+    np.testing.assert_array_equal(res["counts"][0], loads)
+    np.testing.assert_array_equal(res["pos"], lo["pos"])
+    buf = O.dispatch(x, lo["pos"], K, S * K)
+    np.testing.assert_array_equal(res["out"], O.combine(buf, w, lo["pos"], K))
