@@ -6,16 +6,16 @@
 // so on B200 it is bound by latency chains, not HBM: launch gaps, the serial
 // look-back, one CTA planning while the GPU idles.  Here all CTAs stay resident
 // (cooperative launch) and meet at grid barriers instead:
-//   1. each CTA counts its tile per warp (__match_any_sync aggregation) and
-//      writes the tile's per-expert counts, column-major [E][tiles];
+//   1. each CTA counts its tile per warp (warp-match aggregation), writes the
+//      tile's per-expert counts, column-major [E][tiles], and adds them into
+//      the totals T_e (integer atomics: the sums do not depend on order);
 //   -- grid barrier --
-//   2. the per-expert columns are scanned in parallel (one CTA per expert
-//      column): exclusive tile prefixes, and the column totals are T_e;
-//   -- grid barrier --
-//   3. one extra CTA with no tile runs the planner (plan_block.cuh) and
-//      max_vio and raises a flag; meanwhile every tile CTA walks its tile once
-//      for the align-sort ranks (which need only T_e), writing sorted ids,
-//      padding and block experts;
+//   2. one extra CTA with no tile reads T_e and runs the planner
+//      (plan_block.cuh) and max_vio at once, then raises a flag; meanwhile the
+//      tile CTAs scan the per-expert columns in parallel (exclusive tile
+//      prefixes), meet at a second barrier of their own, and walk their tiles
+//      once for the align-sort ranks (which need only T_e), writing sorted
+//      ids, padding and block experts;
 //   4. after the flag, every CTA walks its tile again for the layout ranks and
 //      writes pos / src / pair_slot from the plan.
 // A pair's stable rank within its expert = (its tile's prefix) + (earlier warps
@@ -42,8 +42,9 @@ struct FusedArgs {
   int E, R;
   int32_t SK;
   int tile, ntiles;
-  uint32_t* sync;  // [0] barrier arrivals, [1] plan-ready flag
+  uint32_t* sync;  // [0] barrier arrivals, [1] plan-ready flag (zeroed by the host)
   int32_t* counts; // [E][ntiles] tile counts, then exclusive tile prefixes
+  int32_t* tot;    // [E] T_e, summed by atomics (zeroed by the host)
   int32_t* loads;
   double* max_vio;
   int32_t* plan;
@@ -201,23 +202,31 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
         run += c;
       }
       a.counts[(int64_t)e * NT + t] = run;
+      if (run) atomicAdd(a.tot + e, run);
     }
   }
   grid_barrier(a.sync, (uint32_t)G, a.dev_status);
 
-  // ---- 2. exclusive scan of every expert column over the tiles; totals = T_e
-  for (int e = t; e < E; e += G) {
-    const int32_t total = block_scan_inplace(a.counts + (int64_t)e * NT, NT, warp_sums);
-    if (tid == 0) a.loads[e] = total;
+  // ---- 2. the planner CTA plans from T_e at once; the tile CTAs scan every
+  // expert column over the tiles (exclusive prefixes; totals = T_e again) and
+  // meet at a barrier of their own
+  if (planner) {
+    for (int e = tid; e < E; e += FUSED_THREADS) s_loads[e] = __ldcg(a.tot + e);
+    __syncthreads();
+  } else {
+    for (int e = t; e < E; e += NT) {
+      const int32_t total = block_scan_inplace(a.counts + (int64_t)e * NT, NT, warp_sums);
+      if (tid == 0) a.loads[e] = total;
+    }
+    grid_barrier(a.sync, (uint32_t)(G + NT), a.dev_status);
+    for (int e = tid; e < E; e += FUSED_THREADS) {
+      s_loads[e] = __ldcg(a.loads + e);
+      s_excl[e] = __ldcg(a.counts + (int64_t)e * NT + t);
+    }
+    __syncthreads();
   }
-  grid_barrier(a.sync, 2u * G, a.dev_status);
 
-  // ---- 3. planner on CTA 0; align-sort ranks everywhere
-  for (int e = tid; e < E; e += FUSED_THREADS) {
-    s_loads[e] = __ldcg(a.loads + e);
-    s_excl[e] = has_tile ? __ldcg(a.counts + (int64_t)e * NT + t) : 0;
-  }
-  __syncthreads();
+  // ---- 3. planner on the last CTA; align-sort ranks on the tile CTAs
   if (planner) {
     int32_t m = 0;
     for (int e = tid; e < E; e += FUSED_THREADS) m = max(m, s_loads[e]);
@@ -381,7 +390,7 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   const WsLayout wl = ws_layout(P, E);
   if (ws_bytes < wl.bytes) return EP_ERR_CAPACITY;
 
-  // grid: at most two resident CTAs per SM, tiles a multiple of 512 pairs
+  // grid: one or two resident CTAs per SM, tiles a multiple of 512 pairs
   const size_t smem = fused_smem_bytes(E, R);
   int occ = 0;
   if (P > 0 && smem <= 227 * 1024) {
@@ -391,22 +400,35 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_route_fused, FUSED_THREADS, smem) != cudaSuccess)
       occ = 0;
   }
-  const int64_t resident = (int64_t)num_sms() * std::min(occ, 2);
+  // One CTA per SM while that keeps tiles at 2048 pairs or fewer: the planner
+  // CTA then has an SM to itself (measured on B200 at 196,608 pairs: kernel span
+  // 17.9 -> 15.9 us); larger problems keep two per SM (one per SM measured
+  // slower there: the longer tile walks outweigh the faster plan).
+  int per_sm = std::min(occ, 2);
+  if (per_sm == 2 && num_sms() > 1) {
+    const int64_t t1 = ((P + num_sms() - 2) / (num_sms() - 1) + 511) / 512 * 512;
+    if (t1 <= 2048) per_sm = 1;
+  }
+  const int64_t resident = (int64_t)num_sms() * per_sm;
   int64_t tile = 0, ntiles = 0;
   if (resident > 1) {  // one CTA per tile plus the planner CTA
     tile = (P + resident - 2) / (resident - 1);
     tile = std::max<int64_t>(512, (tile + 511) / 512 * 512);
     ntiles = (P + tile - 1) / tile;
   }
-  // the [E][tiles] counts must fit where the separate path keeps its look-back words
+  // the [E][tiles] counts must fit below T_e (the separate path's regions are unused here)
   const bool fits = resident > 1 && ntiles + 1 <= resident && tile <= (1 << 20) &&
-                    256 + (size_t)E * ntiles * 4 <= wl.excl_off;
+                    (size_t)E * ntiles * 4 <= wl.loads_off;
   if (!fits)
     return fused_route_separate(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot,
                                 block_m, sorted_token_ids, sorted_cap, expert_ids, expert_ids_cap,
                                 num_tokens_post_pad, ws, ws_bytes, dev_status, stream);
+  // workspace: counts [E][tiles] from byte 0; T_e [E] where ep_align_sort
+  // keeps its histogram, then the two sync words (in the slack after it);
+  // one memset zeroes T_e and the sync words
   char* w = static_cast<char*>(ws);
-  if (cudaMemsetAsync(w, 0, 256, stream) != cudaSuccess) return EP_ERR_CUDA;
+  const size_t tot_bytes = ((size_t)E * 4 + 15) & ~(size_t)15;
+  if (cudaMemsetAsync(w + wl.loads_off, 0, tot_bytes + 16, stream) != cudaSuccess) return EP_ERR_CUDA;
   FusedArgs args;
   args.topk = topk_ids;
   args.P = P;
@@ -415,8 +437,9 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   args.SK = (int32_t)(S * K);
   args.tile = (int)tile;
   args.ntiles = (int)ntiles;
-  args.sync = reinterpret_cast<uint32_t*>(w);
-  args.counts = reinterpret_cast<int32_t*>(w + 256);
+  args.sync = reinterpret_cast<uint32_t*>(w + wl.loads_off + tot_bytes);
+  args.counts = reinterpret_cast<int32_t*>(w);
+  args.tot = reinterpret_cast<int32_t*>(w + wl.loads_off);
   args.loads = loads;
   args.max_vio = max_vio;
   args.plan = plan;
