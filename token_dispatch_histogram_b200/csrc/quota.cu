@@ -38,7 +38,7 @@ constexpr int Q_SCAN_THREADS = 1024;
 constexpr int Q_SEARCH_THREADS = 256;
 
 // header words of the quota workspace
-enum : int { QH_TICKET_SEARCH = 0, QH_BEST = 1 };
+enum : int { QH_TICKET_SEARCH = 0, QH_BEST = 1, QH_BARRIER = 2, QH_FLAG = 3 };
 
 struct QTiles {
   int tile;       // pairs per tile, a multiple of 512
@@ -62,14 +62,18 @@ inline QTiles q_tiles(int64_t SK, int R) {
   return q;
 }
 
+// Workspace: header words, T_e (the one-launch route's atomic sums; the
+// header and T_e are zeroed together), tile counts [ntiles][E], exclusive
+// tile prefixes [ntiles + 1][E].
 struct QWs {
-  size_t hdr, cnt, excl, bytes;
+  size_t hdr, tot, cnt, excl, bytes;
 };
 inline QWs q_ws(int64_t ntiles, int E, int R) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   QWs w;
   w.hdr = 0;
-  w.cnt = 256;
+  w.tot = 256;
+  w.cnt = al(w.tot + sizeof(int32_t) * (size_t)E);
   w.excl = al(w.cnt + sizeof(int32_t) * (size_t)E * (size_t)std::max<int64_t>(ntiles, 1));
   w.bytes = al(w.excl + sizeof(int32_t) * (size_t)E * (size_t)(ntiles + 1));
   return w;
@@ -111,48 +115,62 @@ void quota_layout(int E, int R, EpQuotaLayout* L) {
 
 // ------------------------------------------------------------------ 1. count
 
-constexpr int Q_ITEMS = 16;  // keys per thread: tiles of up to 512 * 16 = 8192 pairs
+constexpr int Q_ITEMS = 16;  // keys per thread per round: 512 * 16 = 8192 pairs
 
-// Counts are order-free, so plain shared-memory adds do (no warp aggregation).
+// Per-expert counts of tile t (rank-aligned): cnt[t*E + e]; with tot != NULL
+// also added into tot[e] (integer atomics, so the sums do not depend on
+// order).  Counts are order-free, so plain shared-memory adds do.  s_hist: [E].
+__device__ void q_count_tile(const int32_t* __restrict__ topk, int64_t SK, int E, int tile, int tpr, int64_t t,
+                             int32_t* __restrict__ cnt, int32_t* __restrict__ tot, int32_t* s_hist,
+                             int32_t* dev_status) {
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  const int64_t r = t / tpr, lt = t % tpr;
+  const int64_t p0 = r * SK + lt * tile;
+  const int n = (int)min((int64_t)tile, SK - lt * tile);
+  __syncthreads();
+  bool bad = false;
+  for (int c0 = 0; c0 < n; c0 += Q_ITEMS * SCAT_THREADS) {
+    int key[Q_ITEMS];
+#pragma unroll
+    for (int k = 0; k < Q_ITEMS; ++k) {  // every load issued before the first add
+      const int i = c0 + k * SCAT_THREADS + threadIdx.x;
+      key[k] = i < n ? __ldg(topk + p0 + i) : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < Q_ITEMS; ++k) {
+      const int i = c0 + k * SCAT_THREADS + threadIdx.x;
+      if (i < n) {
+        const int e = key[k];
+        if (e >= 0 && e < E)
+          atomicAdd(&s_hist[e], 1);
+        else
+          bad = true;
+      }
+    }
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t v = s_hist[e];
+    cnt[t * E + e] = v;
+    if (tot && v) atomicAdd(tot + e, v);
+  }
+  if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_EXPERT_ID);
+}
+
 __global__ void __launch_bounds__(SCAT_THREADS)
     k_q_count(const int32_t* __restrict__ topk, int64_t SK, int E, int tile, int tpr, int64_t ntiles,
               int32_t* __restrict__ cnt, uint32_t* __restrict__ hdr, int32_t* dev_status) {
   extern __shared__ int32_t s_hist[];  // [E]
-  __shared__ int s_bad;
   const int64_t t = blockIdx.x;
   if (t == 0 && threadIdx.x == 0) {
     hdr[QH_TICKET_SEARCH] = 0;
     hdr[QH_BEST] = 0xffffffffu;
   }
   if (t >= ntiles) return;
-  if (threadIdx.x == 0) s_bad = 0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
-  const int64_t r = t / tpr, lt = t % tpr;
-  const int64_t p0 = r * SK + lt * tile;
-  const int n = (int)min((int64_t)tile, SK - lt * tile);
-  int key[Q_ITEMS];
-#pragma unroll
-  for (int k = 0; k < Q_ITEMS; ++k) {  // every load issued before the first add
-    const int i = k * SCAT_THREADS + threadIdx.x;
-    key[k] = i < n ? __ldg(topk + p0 + i) : 0;
-  }
-  __syncthreads();
-  bool bad = false;
-#pragma unroll
-  for (int k = 0; k < Q_ITEMS; ++k) {
-    const int i = k * SCAT_THREADS + threadIdx.x;
-    if (i < n) {
-      const int e = key[k];
-      if (e >= 0 && e < E)
-        atomicAdd(&s_hist[e], 1);
-      else
-        bad = true;
-    }
-  }
-  if (bad) s_bad = 1;
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[t * E + e] = s_hist[e];
-  if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_EXPERT_ID);
+  q_count_tile(topk, SK, E, tile, tpr, t, cnt, nullptr, s_hist, dev_status);
 }
 
 // ------------------------------------------------------------------- 2. scan
@@ -297,10 +315,15 @@ inline size_t q_search_smem(int E, int R) {
   return sizeof(int32_t) * (9 * (size_t)E + 12 * (size_t)R + 3 * cap + ((size_t)E + cap));
 }
 
-__global__ void __launch_bounds__(Q_SEARCH_THREADS)
-    k_q_search(const int32_t* __restrict__ loads, const int32_t* __restrict__ excl, int tpr, int E, int R, int B,
-               int64_t P, uint32_t* hdr, int32_t* __restrict__ plan, EpQuotaLayout L) {
-  extern __shared__ int32_t sm[];
+// What a call of q_search_build does: the threshold search (every CTA: its
+// own view of the loads, then its candidates), the plan at tau* (one CTA,
+// from the view it built in an earlier Q_SEARCH call), or both with a ticket
+// between them (the last CTA to finish builds).
+enum QPhase : int { Q_SEARCH = 1, Q_BUILD = 2, Q_ALL = 3 };
+
+__device__ void q_search_build(const int32_t* __restrict__ loads, const int32_t* __restrict__ excl, int tpr, int E,
+                               int R, int B, int64_t P, uint32_t* hdr, int32_t* __restrict__ plan,
+                               const EpQuotaLayout& L, int32_t* sm, int phase) {
   const int cap = L.cap;
   int32_t* s_T = sm;                // [E]
   int32_t* s_sT = s_T + E;          // [E] each rank's loads, heaviest first
@@ -331,6 +354,8 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t s_total, s_local;
   const int ER = E / R;
+  const int64_t lo = (P + R - 1) / R;
+  if (phase & Q_SEARCH) {
   // every CTA derives the rank loads, each rank's order and the range itself
   if (threadIdx.x == 0) {
     s_total = 0;
@@ -341,7 +366,7 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
   {
     int32_t part = 0;  // loads count valid pairs only, so every sum stays below 2^31
     for (int x = threadIdx.x; x < E; x += blockDim.x) {
-      const int32_t v = loads[x];
+      const int32_t v = __ldcg(loads + x);  // (written by atomics in the one-launch route)
       s_T[x] = v;
       part += v;
       atomicAdd(&s_H[x / ER], v);
@@ -350,7 +375,6 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
     if ((threadIdx.x & 31) == 0) atomicAdd(&s_total, part);
   }
   __syncthreads();
-  const int64_t lo = (P + R - 1) / R;
   for (int x = threadIdx.x; x < E; x += blockDim.x) {  // heaviest first, ties to the lower id
     const int r = x / ER;
     if (s_H[r] <= lo) {  // never sheds: the order is not needed
@@ -369,9 +393,11 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
   }
   for (int r = threadIdx.x; r < R; r += blockDim.x) atomicMax(&s_maxH, s_H[r]);
   __syncthreads();
+  }
   const bool valid = (int64_t)s_total == P;
   const int64_t hi = (int64_t)s_maxH > lo ? (int64_t)s_maxH : lo;
   const int64_t tmin = lo + (int64_t)blockIdx.x * blockDim.x;  // this CTA's smallest candidate
+  if (phase & Q_SEARCH) {
   if (threadIdx.x == 0) {
     if (valid && blockIdx.x == 0) atomicMin(hdr + QH_BEST, (uint32_t)hi);
     int no = 0, nm = 0;
@@ -401,12 +427,16 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
       }
     }
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&hdr[QH_TICKET_SEARCH], 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  }
+  if (!(phase & Q_BUILD)) return;
+  if (phase & Q_SEARCH) {  // both: the last CTA to finish its candidates builds
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&hdr[QH_TICKET_SEARCH], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+  }
 
   // ---- the plan at tau*, by the last CTA, from shared memory
   const int32_t tau = valid ? (int32_t)atomicAdd(hdr + QH_BEST, 0u) : -1;
@@ -531,8 +561,8 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
     const int e = i < E ? i : s_re[i - E];
     const int r = i < E ? i / ER : s_rr[i - E];
     const int32_t q = i < E ? s_hq[i] : s_rc[i - E];
-    const int32_t lpre = excl[(int64_t)r * tpr * E + e];
-    const int32_t lsrc = excl[(int64_t)(r + 1) * tpr * E + e] - lpre;
+    const int32_t lpre = __ldcg(excl + (int64_t)r * tpr * E + e);
+    const int32_t lsrc = __ldcg(excl + (int64_t)(r + 1) * tpr * E + e) - lpre;
     const int32_t loc = valid ? min(q, lsrc) : 0;
     s_loc[i] = loc;
     plan[L.inst_local + i] = loc;
@@ -594,8 +624,15 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
     plan[L.tau] = tau;
     plan[L.n_rep] = n_rep;
     plan[L.n_local] = s_local;
-    hdr[QH_TICKET_SEARCH] = 0;
+    if (phase & Q_SEARCH) hdr[QH_TICKET_SEARCH] = 0;
   }
+}
+
+__global__ void __launch_bounds__(Q_SEARCH_THREADS)
+    k_q_search(const int32_t* __restrict__ loads, const int32_t* __restrict__ excl, int tpr, int E, int R, int B,
+               int64_t P, uint32_t* hdr, int32_t* __restrict__ plan, EpQuotaLayout L) {
+  extern __shared__ int32_t sm[];
+  q_search_build(loads, excl, tpr, E, R, B, P, hdr, plan, L, sm, Q_ALL);
 }
 
 // ----------------------------------------------------------------- 4. layout
@@ -606,12 +643,14 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
 // alone (tpr = its tile count), base_counts [R, E] is the gathered load matrix
 // that gives the pairs of each expert on lower source ranks, pos is indexed by
 // the rank's own pairs and src may be NULL.
-__global__ void __launch_bounds__(SCAT_THREADS)
-    k_q_layout(const int32_t* __restrict__ topk, int64_t SK, int E, int R, int tile, int tpr,
-               const int32_t* __restrict__ excl, const int32_t* __restrict__ base_counts, int base_rank,
-               const int32_t* __restrict__ plan, EpQuotaLayout L, int32_t* __restrict__ pos,
-               int32_t* __restrict__ src, int32_t* dev_status) {
-  extern __shared__ int32_t sm[];
+// Tile t of the layout; sm: the layout's shared memory (q_layout_smem).  The
+// plan and the prefixes are read past L1 (in the one-launch route other CTAs
+// of the same launch wrote them).
+__device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int E, int R, int tile, int tpr,
+                              const int32_t* __restrict__ excl, const int32_t* __restrict__ base_counts,
+                              int base_rank, const int32_t* __restrict__ plan, const EpQuotaLayout& L,
+                              int32_t* __restrict__ pos, int32_t* __restrict__ src, int32_t* dev_status, int64_t t,
+                              int32_t* sm) {
   int32_t* s_ids = sm;                  // [tile]
   int32_t* s_whist = s_ids + tile;      // [SCAT_WARPS * E]
   int32_t* s_lpre = s_whist + SCAT_WARPS * E;  // [E] pairs of e from source ranks below this tile's
@@ -626,7 +665,6 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   int32_t* s_ispan = s_istart + E + L.cap; // [E + cap] its looked-up rows
   int32_t* s_excl = s_ispan + E + L.cap;   // [E] (rank-local form) this tile's list offsets
   __shared__ int s_flags;
-  const int64_t t = blockIdx.x;
   const bool local = base_counts != nullptr;
   const int rs = local ? base_rank : (int)(t / tpr);
   const int64_t lt = local ? t : t % tpr;
@@ -634,35 +672,35 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   const int n = (int)min((int64_t)tile, SK - lt * tile);
   const int ER = E / R;
   const int64_t P = (int64_t)R * SK;
-  const int32_t tau = plan[L.tau];
+  const int32_t tau = __ldcg(plan + L.tau);
   if (threadIdx.x == 0) s_flags = 0;
   if (tau < 0) {  // no plan (bad input): nothing is placed
     for (int i = threadIdx.x; i < n; i += blockDim.x) pos[p0 + i] = -1;
     return;
   }
-  const int n_rep = min(max(plan[L.n_rep], 0), L.cap);
+  const int n_rep = min(max(__ldcg(plan + L.n_rep), 0), L.cap);
   for (int i = threadIdx.x; i < E + n_rep; i += blockDim.x) {
-    const int32_t q = i < E ? plan[L.home_quota + i] : plan[L.rep_count + i - E];
-    const int32_t loc = plan[L.inst_local + i];
-    s_icum[i] = plan[L.inst_cum + i];
-    s_istart[i] = plan[L.inst_base + i] + loc;
+    const int32_t q = i < E ? __ldcg(plan + L.home_quota + i) : __ldcg(plan + L.rep_count + i - E);
+    const int32_t loc = __ldcg(plan + L.inst_local + i);
+    s_icum[i] = __ldcg(plan + L.inst_cum + i);
+    s_istart[i] = __ldcg(plan + L.inst_base + i) + loc;
     s_ispan[i] = q - loc;
-    if (i >= E) s_rrank[i - E] = plan[L.rep_rank + i - E];
+    if (i >= E) s_rrank[i - E] = __ldcg(plan + L.rep_rank + i - E);
   }
   __syncthreads();
   // per-expert view from this tile's source rank (e's replicas sit on
   // ascending ranks, so each lookup is a binary search)
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int rf = plan[L.rep_first + e], rc = plan[L.rep_cnt + e];
+    const int rf = __ldcg(plan + L.rep_first + e), rc = __ldcg(plan + L.rep_cnt + e);
     s_rf[e] = rf;
     s_rc[e] = rc;
     if (local) {
       int32_t b = 0;
       for (int r = 0; r < rs; ++r) b += base_counts[(int64_t)r * E + e];
       s_lpre[e] = b;
-      s_excl[e] = excl[t * E + e] + b;
+      s_excl[e] = __ldcg(excl + t * E + e) + b;
     } else {
-      s_lpre[e] = excl[(int64_t)rs * tpr * E + e];
+      s_lpre[e] = __ldcg(excl + (int64_t)rs * tpr * E + e);
     }
     int a = 0, b = rc;  // replicas of e on ranks < rs: the first a
     while (a < b) {
@@ -679,9 +717,10 @@ __global__ void __launch_bounds__(SCAT_THREADS)
       own = E + rf + a;
       below = a + 1;
     }
-    s_oloc[e] = own >= 0 ? plan[L.inst_local + own] : 0;
-    s_obase[e] = own >= 0 ? plan[L.inst_base + own] : 0;
-    s_locb[e] = (e / ER <= rs ? plan[L.inst_local + e] : 0) + (below > 0 ? plan[L.rep_local_incl + rf + below - 1] : 0);
+    s_oloc[e] = own >= 0 ? __ldcg(plan + L.inst_local + own) : 0;
+    s_obase[e] = own >= 0 ? __ldcg(plan + L.inst_base + own) : 0;
+    s_locb[e] = (e / ER <= rs ? __ldcg(plan + L.inst_local + e) : 0) +
+               (below > 0 ? __ldcg(plan + L.rep_local_incl + rf + below - 1) : 0);
   }
   // (tile_stable_ranks starts with a __syncthreads after its own loads)
   auto emit = [&](int64_t p, int e, int32_t g) {
@@ -723,6 +762,21 @@ __global__ void __launch_bounds__(SCAT_THREADS)
   if (threadIdx.x == 0 && s_flags) flag(dev_status, s_flags);
 }
 
+inline size_t q_layout_smem(int tile, int E, int cap) {
+  return sizeof(int32_t) *
+         ((size_t)tile + (size_t)SCAT_WARPS * E + 7 * (size_t)E + (size_t)cap + 3 * ((size_t)E + cap));
+}
+
+__global__ void __launch_bounds__(SCAT_THREADS)
+    k_q_layout(const int32_t* __restrict__ topk, int64_t SK, int E, int R, int tile, int tpr,
+               const int32_t* __restrict__ excl, const int32_t* __restrict__ base_counts, int base_rank,
+               const int32_t* __restrict__ plan, EpQuotaLayout L, int32_t* __restrict__ pos,
+               int32_t* __restrict__ src, int32_t* dev_status) {
+  extern __shared__ int32_t sm[];
+  q_layout_tile(topk, SK, E, R, tile, tpr, excl, base_counts, base_rank, plan, L, pos, src, dev_status, blockIdx.x,
+                sm);
+}
+
 struct QCountsWs {
   size_t hdr, pre, bytes;
 };
@@ -738,8 +792,7 @@ static int run_q_layout(const int32_t* topk, int64_t SK, int E, int R, int tile,
                         const int32_t* excl, const int32_t* base_counts, int base_rank, const int32_t* plan,
                         const EpQuotaLayout& L, int32_t* pos, int32_t* src, int32_t* dev_status,
                         cudaStream_t stream) {
-  const size_t smem = sizeof(int32_t) * ((size_t)tile + (size_t)SCAT_WARPS * E + 7 * (size_t)E + (size_t)L.cap +
-                                         3 * ((size_t)E + L.cap));
+  const size_t smem = q_layout_smem(tile, E, L.cap);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(k_q_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EP_ERR_CUDA;

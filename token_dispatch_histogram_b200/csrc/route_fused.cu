@@ -23,6 +23,7 @@
 // integer adds only, so nothing depends on scheduling.  Every wait is bounded.
 #include <algorithm>
 
+#include "grid_sync.cuh"
 #include "plan_block.cuh"
 
 namespace ep {
@@ -60,41 +61,6 @@ struct FusedArgs {
   int32_t* ntpp;
   int32_t* dev_status;
 };
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Thread 0 waits (bounded) until *ctr >= target; the block follows.
-__device__ void wait_at_least(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
-  if (threadIdx.x == 0 && ld_acquire_u32(ctr) < target) {
-    const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_u32(ctr) < target) {
-      __nanosleep(32);
-      if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
-        flag(dev_status, EP_DEV_LOOKBACK_TIMEOUT);
-        break;
-      }
-    }
-  }
-  __syncthreads();
-}
-
-// Barrier over all CTAs of the cooperative grid (they are co-resident).
-__device__ void grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1u);
-  }
-  wait_at_least(ctr, target, dev_status);
-}
 
 constexpr int WALK_UNROLL = 8;  // tile loads each lane keeps in flight during a walk
 
