@@ -19,7 +19,7 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
 }
 
 // Thread 0 waits (bounded) until *ctr >= target; the block follows.
-__device__ void wait_at_least(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
+static __device__ void wait_at_least(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
   if (threadIdx.x == 0 && ld_acquire_u32(ctr) < target) {
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire_u32(ctr) < target) {
@@ -34,7 +34,7 @@ __device__ void wait_at_least(uint32_t* ctr, uint32_t target, int32_t* dev_statu
 }
 
 // Barrier over all CTAs of the cooperative grid (they are co-resident).
-__device__ void grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
+static __device__ void grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_status) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();

@@ -28,6 +28,7 @@
 //     looked-up range holds its rank among the non-local pairs of the expert.
 #include <algorithm>
 
+#include "grid_sync.cuh"
 #include "tile_ranks.cuh"
 
 namespace ep {
@@ -645,12 +646,14 @@ __global__ void __launch_bounds__(Q_SEARCH_THREADS)
 // the rank's own pairs and src may be NULL.
 // Tile t of the layout; sm: the layout's shared memory (q_layout_smem).  The
 // plan and the prefixes are read past L1 (in the one-launch route other CTAs
-// of the same launch wrote them).
+// of the same launch wrote them).  stage & 1: load the tile's ids and its
+// per-warp first ranks (needs only the prefixes); stage & 2: read the plan and
+// place every pair (needs the plan, and stage 1 done on the same sm).
 __device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int E, int R, int tile, int tpr,
                               const int32_t* __restrict__ excl, const int32_t* __restrict__ base_counts,
                               int base_rank, const int32_t* __restrict__ plan, const EpQuotaLayout& L,
                               int32_t* __restrict__ pos, int32_t* __restrict__ src, int32_t* dev_status, int64_t t,
-                              int32_t* sm) {
+                              int32_t* sm, int stage) {
   int32_t* s_ids = sm;                  // [tile]
   int32_t* s_whist = s_ids + tile;      // [SCAT_WARPS * E]
   int32_t* s_lpre = s_whist + SCAT_WARPS * E;  // [E] pairs of e from source ranks below this tile's
@@ -663,7 +666,7 @@ __device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int 
   int32_t* s_icum = s_rrank + L.cap;    // [E + cap] cumulative start of instance i's looked-up range
   int32_t* s_istart = s_icum + E + L.cap;  // [E + cap] its first looked-up row
   int32_t* s_ispan = s_istart + E + L.cap; // [E + cap] its looked-up rows
-  int32_t* s_excl = s_ispan + E + L.cap;   // [E] (rank-local form) this tile's list offsets
+  int32_t* s_excl = s_ispan + E + L.cap;   // [E] this tile's list offsets
   __shared__ int s_flags;
   const bool local = base_counts != nullptr;
   const int rs = local ? base_rank : (int)(t / tpr);
@@ -672,6 +675,17 @@ __device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int 
   const int n = (int)min((int64_t)tile, SK - lt * tile);
   const int ER = E / R;
   const int64_t P = (int64_t)R * SK;
+  if (stage & 1) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int32_t b = 0;
+      if (local)
+        for (int r = 0; r < rs; ++r) b += base_counts[(int64_t)r * E + e];
+      s_excl[e] = __ldcg(excl + t * E + e) + b;
+    }
+    // (tile_ranks_prepare reads s_excl after its own barriers)
+    tile_ranks_prepare(topk, E, tile, p0, n, s_excl, s_ids, s_whist);
+  }
+  if (!(stage & 2)) return;
   const int32_t tau = __ldcg(plan + L.tau);
   if (threadIdx.x == 0) s_flags = 0;
   if (tau < 0) {  // no plan (bad input): nothing is placed
@@ -698,7 +712,6 @@ __device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int 
       int32_t b = 0;
       for (int r = 0; r < rs; ++r) b += base_counts[(int64_t)r * E + e];
       s_lpre[e] = b;
-      s_excl[e] = __ldcg(excl + t * E + e) + b;
     } else {
       s_lpre[e] = __ldcg(excl + (int64_t)rs * tpr * E + e);
     }
@@ -722,7 +735,7 @@ __device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int 
     s_locb[e] = (e / ER <= rs ? __ldcg(plan + L.inst_local + e) : 0) +
                (below > 0 ? __ldcg(plan + L.rep_local_incl + rf + below - 1) : 0);
   }
-  // (tile_stable_ranks starts with a __syncthreads after its own loads)
+  __syncthreads();
   auto emit = [&](int64_t p, int e, int32_t g) {
     const int32_t ls = g - s_lpre[e];
     int32_t row = -1;
@@ -757,7 +770,7 @@ __device__ void q_layout_tile(const int32_t* __restrict__ topk, int64_t SK, int 
     atomicOr(&s_flags, EP_DEV_BAD_EXPERT_ID);
     pos[p] = -1;
   };
-  tile_stable_ranks(topk, E, tile, p0, n, local ? s_excl : excl + t * E, s_ids, s_whist, emit, bad);
+  tile_ranks_walk(E, tile, p0, n, s_ids, s_whist, emit, bad);
   __syncthreads();
   if (threadIdx.x == 0 && s_flags) flag(dev_status, s_flags);
 }
@@ -774,7 +787,140 @@ __global__ void __launch_bounds__(SCAT_THREADS)
                int32_t* __restrict__ src, int32_t* dev_status) {
   extern __shared__ int32_t sm[];
   q_layout_tile(topk, SK, E, R, tile, tpr, excl, base_counts, base_rank, plan, L, pos, src, dev_status, blockIdx.x,
-                sm);
+                sm, 3);
+}
+
+// ------------------------------------------------------- the one-launch route
+
+// The four steps in one cooperative launch (all CTAs co-resident), every CTA
+// owning one rank-aligned tile:
+//   1. tile counts, added into T_e by integer atomics;  -- grid barrier --
+//   2. every CTA tests its threshold candidates from T_e (its own view of the
+//      loads, as k_q_search) while the CTAs scan the tile columns into the
+//      exclusive prefixes;  -- grid barrier --
+//   3. CTA 0 builds the plan at tau* from its view and raises a flag, while
+//      the others load their tiles and count them per warp;
+//   4. every CTA places its tile's pairs once the flag is up.
+// Same outputs as the four launches, bit for bit; every wait is bounded.
+struct QFusedArgs {
+  const int32_t* topk;
+  int64_t SK, P;
+  int E, R, B, tile, tpr, ntiles;
+  uint32_t* hdr;
+  int32_t* tot;
+  int32_t* cnt;
+  int32_t* excl;
+  int32_t* loads;
+  int32_t* plan;
+  EpQuotaLayout L;
+  int32_t* pos;
+  int32_t* src;
+  int32_t* dev_status;
+};
+
+__global__ void __launch_bounds__(SCAT_THREADS) k_q_fused(QFusedArgs a) {
+  extern __shared__ int32_t sm[];
+  __shared__ int32_t warp_sums[32];
+  const int G = gridDim.x, t = blockIdx.x, tid = threadIdx.x, E = a.E;
+  if (t == 0 && tid == 0) a.hdr[QH_BEST] = 0xffffffffu;  // read by no CTA before the first barrier
+  q_count_tile(a.topk, a.SK, E, a.tile, a.tpr, t, a.cnt, a.tot, sm, a.dev_status);
+  grid_barrier(a.hdr + QH_BARRIER, (uint32_t)G, a.dev_status);
+
+  q_search_build(a.tot, a.excl, a.tpr, E, a.R, a.B, a.P, a.hdr, a.plan, a.L, sm, Q_SEARCH);
+  for (int e = t; e < E; e += G) {  // column e over the G tiles (G <= blockDim)
+    const int32_t v = tid < G ? __ldcg(a.cnt + (int64_t)tid * E + e) : 0;
+    int32_t total;
+    const int32_t ex = block_exclusive_scan(v, warp_sums, &total);
+    if (tid < G) a.excl[(int64_t)tid * E + e] = ex;
+    if (tid == 0) {
+      a.excl[(int64_t)G * E + e] = total;
+      a.loads[e] = total;
+    }
+  }
+  grid_barrier(a.hdr + QH_BARRIER, 2u * G, a.dev_status);
+
+  if (t == 0) {
+    q_search_build(a.tot, a.excl, a.tpr, E, a.R, a.B, a.P, a.hdr, a.plan, a.L, sm, Q_BUILD);
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release_u32(a.hdr + QH_FLAG, 1u);
+    }
+  }
+  // the plan-free half of the layout while CTA 0 builds (its search state is
+  // dead once the build is done), then the rest once the plan is out
+  q_layout_tile(a.topk, a.SK, E, a.R, a.tile, a.tpr, a.excl, nullptr, 0, a.plan, a.L, a.pos, a.src, a.dev_status,
+                t, sm, 1);
+  wait_at_least(a.hdr + QH_FLAG, 1u, a.dev_status);
+  q_layout_tile(a.topk, a.SK, E, a.R, a.tile, a.tpr, a.excl, nullptr, 0, a.plan, a.L, a.pos, a.src, a.dev_status,
+                t, sm, 2);
+}
+
+// Launches the one-launch route when its grid can be co-resident within the
+// workspace's tile regions; returns false (nothing launched) otherwise.
+static bool q_fused_launch(const int32_t* topk, int64_t SK, int E, int R, int B, int32_t* loads, int32_t* plan,
+                           const EpQuotaLayout& L, int32_t* pos, int32_t* src, char* ws, const QWs& w,
+                           int64_t ws_tiles, int32_t* dev_status, cudaStream_t stream, int* rc) {
+  *rc = EP_OK;
+  if (SK <= 0) return false;
+  const size_t base = std::max(q_search_smem(E, R), sizeof(int32_t) * (size_t)E);
+  for (int per_sm = 2; per_sm >= 1; --per_sm) {
+    const int64_t resident = (int64_t)num_sms() * per_sm;
+    if (R > resident) continue;
+    const int64_t tpr0 = std::min<int64_t>(resident / R, SCAT_THREADS / R > 0 ? SCAT_THREADS / R : 1);
+    if (tpr0 < 1) continue;
+    int64_t tile = ((SK + tpr0 - 1) / tpr0 + 511) / 512 * 512;
+    const int64_t tpr = (SK + tile - 1) / tile;
+    const int64_t nt = (int64_t)R * tpr;
+    if (nt > resident || nt > SCAT_THREADS || nt > ws_tiles || tile > (1 << 20)) continue;
+    const size_t smem = std::max(base, q_layout_smem((int)tile, E, L.cap));
+    if (smem > 227 * 1024) continue;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_q_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      continue;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_q_fused, SCAT_THREADS, smem) != cudaSuccess ||
+        occ < per_sm)
+      continue;
+    if (cudaMemsetAsync(ws, 0, w.cnt, stream) != cudaSuccess) {  // header words and T_e
+      *rc = EP_ERR_CUDA;
+      return true;
+    }
+    QFusedArgs args;
+    args.topk = topk;
+    args.SK = SK;
+    args.P = (int64_t)R * SK;
+    args.E = E;
+    args.R = R;
+    args.B = B;
+    args.tile = (int)tile;
+    args.tpr = (int)tpr;
+    args.ntiles = (int)nt;
+    args.hdr = reinterpret_cast<uint32_t*>(ws + w.hdr);
+    args.tot = reinterpret_cast<int32_t*>(ws + w.tot);
+    args.cnt = reinterpret_cast<int32_t*>(ws + w.cnt);
+    args.excl = reinterpret_cast<int32_t*>(ws + w.excl);
+    args.loads = loads;
+    args.plan = plan;
+    args.L = L;
+    args.pos = pos;
+    args.src = src;
+    args.dev_status = dev_status;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nt);
+    cfg.blockDim = dim3(SCAT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    *rc = cudaLaunchKernelEx(&cfg, k_q_fused, args) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    if (*rc == EP_OK) count_launch();
+    return true;
+  }
+  return false;
 }
 
 struct QCountsWs {
@@ -834,6 +980,9 @@ extern "C" int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, 
   const QWs w = q_ws(q.ntiles, E, R);
   if (ws_bytes < w.bytes) return EP_ERR_CAPACITY;
   char* base = static_cast<char*>(ws);
+  int frc = EP_OK;
+  if (q_fused_launch(topk_ids, SK, E, R, B, loads, plan, L, pos, src, base, w, q.ntiles, dev_status, stream, &frc))
+    return frc == EP_OK ? launch_status() : frc;
   uint32_t* hdr = reinterpret_cast<uint32_t*>(base + w.hdr);
   int32_t* cnt = reinterpret_cast<int32_t*>(base + w.cnt);
   int32_t* excl = reinterpret_cast<int32_t*>(base + w.excl);

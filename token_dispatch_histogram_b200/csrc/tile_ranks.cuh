@@ -17,11 +17,13 @@ constexpr int SCAT_WARPS = SCAT_THREADS / 32;
 // multiple of 32 * SCAT_WARPS); excl_row[e] = pairs of e before p0.  Calls
 // emit(p, e, g) for every valid pair (g = rank of p among all pairs of expert
 // e) and bad(p) for pairs whose id is outside [0, E).  s_ids: [tile] ints,
-// s_whist: [SCAT_WARPS][E] ints.
-template <class Emit, class Bad>
-__device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ topk, int E, int tile, int64_t p0, int n,
-                                                  const int32_t* __restrict__ excl_row, int32_t* s_ids,
-                                                  int32_t* s_whist, Emit emit, Bad bad) {
+// s_whist: [SCAT_WARPS][E] ints.  Two halves: tile_ranks_prepare (loads the
+// ids, counts them per warp and turns the counts into each warp's first rank
+// per expert) and tile_ranks_walk (the ranks themselves, emitted in order),
+// so a caller can run the first before the data emit needs is ready.
+__device__ __forceinline__ void tile_ranks_prepare(const int32_t* __restrict__ topk, int E, int tile, int64_t p0,
+                                                   int n, const int32_t* __restrict__ excl_row, int32_t* s_ids,
+                                                   int32_t* s_whist) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < tile; i += blockDim.x) {
     int e = -1;
@@ -54,6 +56,15 @@ __device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ to
     }
   }
   __syncthreads();
+}
+
+template <class Emit, class Bad>
+__device__ __forceinline__ void tile_ranks_walk(int E, int tile, int64_t p0, int n, const int32_t* s_ids,
+                                                int32_t* s_whist, Emit emit, Bad bad) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = tile / SCAT_WARPS;
+  const int nbits = key_bits(E + 2);
+  int32_t* my = s_whist + warp * E;
   const uint32_t lt = lanemask_lt();
   for (int c = 0; c < sub; c += 32) {
     const int i = warp * sub + c + lane;
@@ -71,6 +82,14 @@ __device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ to
         bad(p0 + i);
     }
   }
+}
+
+template <class Emit, class Bad>
+__device__ __forceinline__ void tile_stable_ranks(const int32_t* __restrict__ topk, int E, int tile, int64_t p0, int n,
+                                                  const int32_t* __restrict__ excl_row, int32_t* s_ids,
+                                                  int32_t* s_whist, Emit emit, Bad bad) {
+  tile_ranks_prepare(topk, E, tile, p0, n, excl_row, s_ids, s_whist);
+  tile_ranks_walk(E, tile, p0, n, s_ids, s_whist, emit, bad);
 }
 
 }  // namespace ep
