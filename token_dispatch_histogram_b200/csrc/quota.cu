@@ -357,77 +357,77 @@ __device__ void q_search_build(const int32_t* __restrict__ loads, const int32_t*
   const int ER = E / R;
   const int64_t lo = (P + R - 1) / R;
   if (phase & Q_SEARCH) {
-  // every CTA derives the rank loads, each rank's order and the range itself
-  if (threadIdx.x == 0) {
-    s_total = 0;
-    s_maxH = 0;
-  }
-  for (int r = threadIdx.x; r < R; r += blockDim.x) s_H[r] = 0;
-  __syncthreads();
-  {
-    int32_t part = 0;  // loads count valid pairs only, so every sum stays below 2^31
-    for (int x = threadIdx.x; x < E; x += blockDim.x) {
-      const int32_t v = __ldcg(loads + x);  // (written by atomics in the one-launch route)
-      s_T[x] = v;
-      part += v;
-      atomicAdd(&s_H[x / ER], v);
+    // every CTA derives the rank loads, each rank's order and the range itself
+    if (threadIdx.x == 0) {
+      s_total = 0;
+      s_maxH = 0;
     }
-    for (int d = 16; d > 0; d >>= 1) part += __shfl_down_sync(0xffffffffu, part, d);
-    if ((threadIdx.x & 31) == 0) atomicAdd(&s_total, part);
-  }
-  __syncthreads();
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {  // heaviest first, ties to the lower id
-    const int r = x / ER;
-    if (s_H[r] <= lo) {  // never sheds: the order is not needed
-      s_sT[x] = s_T[x];
-      s_ord[x] = x;
-      continue;
+    for (int r = threadIdx.x; r < R; r += blockDim.x) s_H[r] = 0;
+    __syncthreads();
+    {
+      int32_t part = 0;  // loads count valid pairs only, so every sum stays below 2^31
+      for (int x = threadIdx.x; x < E; x += blockDim.x) {
+        const int32_t v = __ldcg(loads + x);  // (written by atomics in the one-launch route)
+        s_T[x] = v;
+        part += v;
+        atomicAdd(&s_H[x / ER], v);
+      }
+      for (int d = 16; d > 0; d >>= 1) part += __shfl_down_sync(0xffffffffu, part, d);
+      if ((threadIdx.x & 31) == 0) atomicAdd(&s_total, part);
     }
-    const int32_t v = s_T[x];
-    int k = 0;
-    for (int y = r * ER; y < (r + 1) * ER; ++y) {
-      const int32_t w = s_T[y];
-      k += (w > v) || (w == v && y < x);
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {  // heaviest first, ties to the lower id
+      const int r = x / ER;
+      if (s_H[r] <= lo) {  // never sheds: the order is not needed
+        s_sT[x] = s_T[x];
+        s_ord[x] = x;
+        continue;
+      }
+      const int32_t v = s_T[x];
+      int k = 0;
+      for (int y = r * ER; y < (r + 1) * ER; ++y) {
+        const int32_t w = s_T[y];
+        k += (w > v) || (w == v && y < x);
+      }
+      s_sT[r * ER + k] = v;
+      s_ord[r * ER + k] = x;
     }
-    s_sT[r * ER + k] = v;
-    s_ord[r * ER + k] = x;
-  }
-  for (int r = threadIdx.x; r < R; r += blockDim.x) atomicMax(&s_maxH, s_H[r]);
-  __syncthreads();
+    for (int r = threadIdx.x; r < R; r += blockDim.x) atomicMax(&s_maxH, s_H[r]);
+    __syncthreads();
   }
   const bool valid = (int64_t)s_total == P;
   const int64_t hi = (int64_t)s_maxH > lo ? (int64_t)s_maxH : lo;
   const int64_t tmin = lo + (int64_t)blockIdx.x * blockDim.x;  // this CTA's smallest candidate
   if (phase & Q_SEARCH) {
-  if (threadIdx.x == 0) {
-    if (valid && blockIdx.x == 0) atomicMin(hdr + QH_BEST, (uint32_t)hi);
-    int no = 0, nm = 0;
-    for (int r = 0; r < R; ++r) {
-      if (s_H[r] > tmin) {
-        s_oH[no] = s_H[r];
-        s_oOff[no++] = r * ER;
+    if (threadIdx.x == 0) {
+      if (valid && blockIdx.x == 0) atomicMin(hdr + QH_BEST, (uint32_t)hi);
+      int no = 0, nm = 0;
+      for (int r = 0; r < R; ++r) {
+        if (s_H[r] > tmin) {
+          s_oH[no] = s_H[r];
+          s_oOff[no++] = r * ER;
+        }
+        if (s_H[r] < hi) {
+          s_mH[nm] = s_H[r];
+          s_mR[nm++] = r;
+        }
       }
-      if (s_H[r] < hi) {
-        s_mH[nm] = s_H[r];
-        s_mR[nm++] = r;
+      s_novr = no;
+      s_nroom = nm;
+    }
+    __syncthreads();
+    if (valid) {
+      const int64_t N = (int64_t)gridDim.x * blockDim.x;
+      volatile uint32_t* best = hdr + QH_BEST;
+      const int novr = s_novr, nroom = s_nroom;
+      for (int64_t tau = tmin + threadIdx.x; tau < hi; tau += N) {
+        if (tau >= (int64_t)*best) break;
+        if (q_feasible((int32_t)tau, s_sT, s_oH, s_oOff, novr, s_mH, nroom, ER, B)) {
+          atomicMin(hdr + QH_BEST, (uint32_t)tau);
+          break;
+        }
       }
     }
-    s_novr = no;
-    s_nroom = nm;
-  }
-  __syncthreads();
-  if (valid) {
-    const int64_t N = (int64_t)gridDim.x * blockDim.x;
-    volatile uint32_t* best = hdr + QH_BEST;
-    const int novr = s_novr, nroom = s_nroom;
-    for (int64_t tau = tmin + threadIdx.x; tau < hi; tau += N) {
-      if (tau >= (int64_t)*best) break;
-      if (q_feasible((int32_t)tau, s_sT, s_oH, s_oOff, novr, s_mH, nroom, ER, B)) {
-        atomicMin(hdr + QH_BEST, (uint32_t)tau);
-        break;
-      }
-    }
-  }
   }
   if (!(phase & Q_BUILD)) return;
   if (phase & Q_SEARCH) {  // both: the last CTA to finish its candidates builds
