@@ -276,6 +276,8 @@ def run_ours(args, rank, world, local_rank):
     n_rep = [int(ly.plan_view("n_rep", 1).item()) for ly in layers]
     n_chunks = [int(ly.plan_view("n_chunks", 1).item()) for ly in layers]
     max_vio = [float(ly.max_vio.item()) for ly in layers]
+    top_share = [round(float(ly.loads.max().item()) / P, 5) for ly in layers]  # hottest expert's share of the pairs
+    max_rep_rank = [int(ly.plan_view("rank_nrep", R).max().item()) for ly in layers]
 
     # ---- device-resident timed region: per-op CUDA events on the launching stream
     marks = []  # per step: list of (op, event)
@@ -339,8 +341,10 @@ def run_ours(args, rank, world, local_rank):
             torch.cuda.synchronize()
             barrier()
             clk_g = clocks_g.stop()
-            g_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(gs, ge)), world, dev)
-            graph = {"ms": g_ms, "launches": int(per_replay * args.steps), "clocks": clk_g}
+            per_step = sorted(a.elapsed_time(b) for a, b in zip(gs, ge))
+            g_ms = max_over_ranks(sum(per_step), world, dev)
+            graph = {"ms": g_ms, "launches": int(per_replay * args.steps), "clocks": clk_g,
+                     "step_ms_median": per_step[len(per_step) // 2], "step_ms_min": per_step[0]}
             del g
             for ly in layers:
                 st = ly.status(stream)
@@ -647,6 +651,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": graph["clocks"] if graph else clk,
         "timing": ("one captured CUDA graph per step, replayed; CUDA events around each replay"
                    if graph else "eager launches; CUDA events around each step"),
+        "step_ms_median": round(graph["step_ms_median"], 5) if graph else None,
+        "step_ms_min": round(graph["step_ms_min"], 5) if graph else None,
         "eager": eager,
         "breakdown": breakdown,
         "step_hbm": {"bytes": step_bytes, "GB_s": round(step_bytes / (timed_ms / args.steps / 1e3) / 1e9, 1),
@@ -655,7 +661,9 @@ def run_ours(args, rank, world, local_rank):
                              "GB_s": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9, 1),
                              "frac": round((ab["dispatch"] + ab["combine"]) / (d_c_ms / 1e3) / 1e9 / peak, 4)},
         "routing": {"max_vio": max_vio if nl > 1 else max_vio[0], "n_rep": n_rep if nl > 1 else n_rep[0],
-                    "replicated_experts": n_chunks if nl > 1 else n_chunks[0]},
+                    "replicated_experts": n_chunks if nl > 1 else n_chunks[0],
+                    "top_expert_share": top_share if nl > 1 else top_share[0],
+                    "max_replicas_per_rank": max_rep_rank if nl > 1 else max_rep_rank[0]},
         "backward": backward,
         "prefetch_slots": prefetch,
         "quota_planner": quota,
@@ -710,13 +718,21 @@ def time_oracle(c, seed, steps, topk=None, w=None, x=None, budget_s=None):
         x = W.hidden(c["T"], c["H"], seed)
     gh, gr, local = oracle_inputs(c, seed, topk)
     times = []
-    t_begin = time.perf_counter()
-    for i in range(steps):
-        t0 = time.perf_counter()
-        oracle_step(c, topk, w, x, gh, gr, local)
-        times.append(time.perf_counter() - t0)
-        if budget_s is not None and time.perf_counter() - t_begin > budget_s:
-            break
+    # one host core, as the oracle is single-threaded (restored afterwards)
+    prev = os.sched_getaffinity(0) if hasattr(os, "sched_getaffinity") else None
+    if prev:
+        os.sched_setaffinity(0, {min(prev)})
+    try:
+        t_begin = time.perf_counter()
+        for i in range(steps):
+            t0 = time.perf_counter()
+            oracle_step(c, topk, w, x, gh, gr, local)
+            times.append(time.perf_counter() - t0)
+            if budget_s is not None and time.perf_counter() - t_begin > budget_s:
+                break
+    finally:
+        if prev:
+            os.sched_setaffinity(0, prev)
     return times
 
 
