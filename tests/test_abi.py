@@ -96,3 +96,59 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         tdh.ep_route_stats(t, 8, torch.zeros(8, dtype=torch.int32), torch.zeros(1, dtype=torch.float64),
                            torch.zeros(64, dtype=torch.uint8))
+
+
+def test_rank_local_and_quota_argument_errors():
+    """The rank-local and quota entry points refuse bad shapes and short
+    buffers on the host, before anything is enqueued (no GPU needed)."""
+    import token_dispatch_histogram_b200 as tdh
+    L = tdh.lib()
+    fake = ctypes.c_void_p(0x1000)
+    n = ctypes.c_size_t()
+    # plan from the gathered matrix: E % R, plan buffer too small
+    assert L.ep_plan_from_counts(fake, 3, 4, 2, 8, None, fake, 1 << 20, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_plan_from_counts(fake, 4, 4, 2, 8, None, fake, 3, None, None) == tdh.EP_ERR_CAPACITY
+    # rank-local layout: rank outside [0, R), missing counts, short workspace
+    assert L.ep_layout_rank(fake, 16, 2, 8, 4, 4, fake, fake, 1 << 20, fake, 1 << 20, fake, None, None,
+                            None) == tdh.EP_ERR_ARG
+    assert L.ep_layout_rank(fake, 16, 2, 8, 4, 0, None, fake, 1 << 20, fake, 1 << 20, fake, None, None,
+                            None) == tdh.EP_ERR_ARG
+    assert L.ep_layout_rank(fake, 16, 2, 8, 4, 0, fake, fake, 1 << 20, fake, 8, fake, None, None,
+                            None) == tdh.EP_ERR_CAPACITY
+    # peer dispatch / combine: H not a multiple of 8, no peer table, K > 8 for combine, misaligned rows
+    assert L.ep_dispatch_peer(fake, 16, 2, 12, fake, fake, None, 4, 32, 128, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_dispatch_peer(fake, 16, 2, 16, fake, None, None, 4, 32, 128, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_dispatch_peer(ctypes.c_void_p(0x1008), 16, 2, 16, fake, fake, None, 4, 32, 128, None,
+                              None) == tdh.EP_ERR_ARG
+    assert L.ep_combine_peer(fake, None, 4, 32, 128, fake, fake, 16, 9, 16, fake, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_combine_peer(None, None, 4, 32, 128, fake, fake, 16, 2, 16, fake, None, None) == tdh.EP_ERR_ARG
+    assert L.ep_dispatch_peer(None, 0, 2, 16, None, fake, None, 4, 32, 0, None, None) == tdh.EP_OK
+    # peer replica gradients: rank outside [0, R), negative rows, bad dtype, plan too small
+    assert L.ep_replica_grad_reduce_peer(fake, fake, 8, 0, 16, 8, 4, 4, fake, 1 << 20, 0, None,
+                                         None) == tdh.EP_ERR_ARG
+    assert L.ep_replica_grad_reduce_peer(fake, fake, -1, 0, 16, 8, 4, 0, fake, 1 << 20, 0, None,
+                                         None) == tdh.EP_ERR_ARG
+    assert L.ep_replica_grad_reduce_peer(fake, fake, 8, 5, 16, 8, 4, 0, fake, 1 << 20, 0, None,
+                                         None) == tdh.EP_ERR_ARG
+    assert L.ep_replica_grad_reduce_peer(fake, fake, 8, 0, 16, 8, 4, 0, fake, 3, 0, None,
+                                         None) == tdh.EP_ERR_CAPACITY
+    # quota planner from the gathered matrix: B < 0, short workspace, plan too small
+    assert L.ep_quota_counts_workspace_size(8, 4, ctypes.byref(n)) == tdh.EP_OK and n.value > 0
+    assert L.ep_quota_counts_workspace_size(10, 4, ctypes.byref(n)) == tdh.EP_ERR_ARG
+    assert L.ep_quota_plan_from_counts(fake, 4, 4, 2, 8, -1, fake, fake, 1 << 20, fake, 1 << 20, None,
+                                       None) == tdh.EP_ERR_ARG
+    assert L.ep_quota_plan_from_counts(fake, 4, 4, 2, 8, 1, fake, fake, 1 << 20, fake, 16, None,
+                                       None) == tdh.EP_ERR_CAPACITY
+    assert L.ep_quota_plan_from_counts(fake, 4, 4, 2, 8, 1, fake, fake, 3, fake, 1 << 20, None,
+                                       None) == tdh.EP_ERR_CAPACITY
+    assert L.ep_quota_layout_rank(fake, 16, 2, 8, 4, -1, fake, fake, 1 << 20, fake, 1 << 20, fake, None,
+                                  None) == tdh.EP_ERR_ARG
+    assert L.ep_quota_replica_grad_reduce_peer(fake, fake, 8, 0, 16, 8, 4, 0, fake, 3, 0, None,
+                                               None) == tdh.EP_ERR_CAPACITY
+    # quota route: T not R*S, B < 0, workspace too small
+    assert L.ep_quota_route(fake, 17, 2, 8, 4, 4, 1, fake, fake, 1 << 20, fake, fake, fake, 1 << 20, None,
+                            None) == tdh.EP_ERR_ARG
+    assert L.ep_quota_route(fake, 16, 2, 8, 4, 4, -1, fake, fake, 1 << 20, fake, fake, fake, 1 << 20, None,
+                            None) == tdh.EP_ERR_ARG
+    assert L.ep_quota_route(fake, 16, 2, 8, 4, 4, 1, fake, fake, 1 << 20, fake, fake, fake, 16, None,
+                            None) == tdh.EP_ERR_CAPACITY
