@@ -324,6 +324,8 @@ EP_API int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int 
  * written in place into the expert-grouped buffer, no intermediate copy.
  *   x   [T, H] bf16; buf [buf_rows, H] bf16 out; buf[pos[p]] = x[p / K] bitwise.
  *   Rows whose pos is outside [0, buf_rows) are skipped and flagged.
+ *   Rows up to about 100 KB (two shared-memory stages of one row each within
+ *   200 KB: H <= 51,136 at K <= 8); wider rows get EP_ERR_ARG.
  * Each token row is read once (TMA bulk copy into shared memory) and written to
  * its K rows by bulk stores.
  */

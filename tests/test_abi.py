@@ -84,6 +84,8 @@ def test_argument_errors_return_before_any_launch():
     # grad reduce: bad dtype, plan too small
     assert L.ep_replica_grad_reduce(fake, fake, 7, 8, 8, 4, fake, 1 << 20, 0, None, None) == tdh.EP_ERR_ARG
     assert L.ep_replica_grad_reduce(fake, fake, 0, 8, 8, 4, fake, 3, 0, None, None) == tdh.EP_ERR_CAPACITY
+    # a row wider than two shared-memory stages (about 100 KB) is refused
+    assert L.ep_dispatch(fake, 16, 2, 51200, fake, fake, 32, None, None) == tdh.EP_ERR_ARG
     # zero-size work is a no-op that succeeds without touching the device
     assert L.ep_dispatch(None, 0, 2, 16, None, None, 0, None, None) == tdh.EP_OK
     assert L.ep_combine(None, 0, None, None, 0, 2, 16, None, None, None) == tdh.EP_OK

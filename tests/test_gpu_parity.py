@@ -122,6 +122,8 @@ ROW_CASES = [
     (16, 64, 8, 256, 4096, "uniform"),
     (2, 40, 12, 16, 64, "skew"),       # K > 8: the generic combine kernel
     (8, 512, 8, 64, 7168, "single"),   # K = 8, wide rows, a dominant expert
+    (2, 64, 4, 8, 16384, "skew"),      # 32 KB rows
+    (4, 100, 3, 8, 8, "skew"),         # the narrowest row, one 16-byte vector
 ]
 
 
