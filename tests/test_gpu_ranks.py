@@ -396,3 +396,46 @@ def test_rank_local_route_through_nccl():
     np.testing.assert_array_equal(res["pos"], lo["pos"])
     buf = O.dispatch(x, lo["pos"], K, S * K)
     np.testing.assert_array_equal(res["out"], O.combine(buf, w, lo["pos"], K))
+
+
+def test_rank_local_fuzz():
+    """Random shapes through the rank-local form, both planners: every rank's
+    rows, receive buffer and combine equal its slice of the oracle's."""
+    import torch
+    rng = np.random.default_rng(4242)
+    for it in range(20):
+        R = int(rng.choice([1, 2, 3, 4, 6, 8, 16, 24]))
+        E = R * int(rng.integers(1, 7))
+        K = int(rng.integers(1, min(8, E) + 1))
+        S = int(rng.integers(1, 400))
+        H = 8 * int(rng.integers(1, 40))
+        planner = "quota" if it % 2 else "exact"
+        B = int(rng.integers(0, 4))
+        topk, w, x = case_inputs(R, S, K, E, H, seed=1000 + it, bias_scale=float(rng.uniform(0.5, 3.0)))
+        T, SK = R * S, S * K
+        loads, _, _ = O.route_stats(topk, E)
+        if planner == "exact":
+            pl = O.plan(loads, R, S, K, E)
+            lo = O.layout(topk, pl, R, S, E)
+            off = np.arange(R, dtype=np.int64) * SK
+            rl = np.full(R, SK)
+            ranks, _ = _ranks(R, S, K, E, H, topk, w, x)
+        else:
+            qp = O.quota_plan(loads, R, S, K, E, B)
+            lo = O.quota_layout(topk, qp, R, S, K, E)
+            rl = lo["rank_load"]
+            off = np.concatenate([[0], np.cumsum(rl)[:-1]]).astype(np.int64)
+            ranks, _ = _quota_ranks(R, S, K, E, H, B, topk, w, x, max(int(rl.max()), 1))
+        buf = O.dispatch(x, lo["pos"], K, T * K)
+        want = O.combine(buf, w, lo["pos"], K)
+        for rk in ranks:
+            rk.out_local.fill_(-1.0)
+            rk.combine()
+        torch.cuda.synchronize()
+        for r, rk in enumerate(ranks):
+            msg = f"it {it} {planner} R={R} S={S} K={K} E={E} H={H} B={B} rank {r}"
+            assert rk.status() == 0, msg
+            np.testing.assert_array_equal(rk.pos_local.cpu().numpy(), lo["pos"][r * SK:(r + 1) * SK], err_msg=msg)
+            ld = int(rl[r])
+            np.testing.assert_array_equal(_u16(rk.buf)[:ld], buf[off[r]:off[r] + ld], err_msg=msg)
+            np.testing.assert_array_equal(_u16(rk.out_local), want[r * S:(r + 1) * S], err_msg=msg)
