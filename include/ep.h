@@ -8,6 +8,15 @@
  *   ep_route_stats -> ep_plan -> ep_layout -> ep_dispatch -> (expert) -> ep_combine
  *   ep_align_sort (block-aligned expert sort for a grouped GEMM)
  *   ep_replica_grad_reduce (backward: replica gradients into the home expert)
+ *   ep_route_fused (stats, plan, layout and align-sort in one launch)
+ *   ep_dispatch_backward, ep_combine_backward (gradients of the row movers)
+ *   ep_prefetch_slots (a per-rank replica slot budget B applied to a plan)
+ *   ep_quota_route, ep_quota_replica_grad_reduce (the quota-driven planner:
+ *       a searched load threshold with at most B replicas per rank)
+ *   rank-local form, one rank per process (ep_plan_from_counts,
+ *       ep_layout_rank, ep_dispatch_peer, ep_combine_peer,
+ *       ep_replica_grad_reduce_peer and their quota-planner counterparts)
+ *   ep_route_stats_noalloc (ep_route_stats with the library's own scratch)
  *
  * Sources, cited by page title and section:
  *  [GR] "MoonEP: πώς η εξισορρόπηση των AI experts αλλάζει την υποδομή των MoE
