@@ -12,7 +12,9 @@
 // lanes 0..K-1 each issue one bulk store (shared->global) of that row to one
 // destination.  Loads for the next stages are in flight while the stores
 // drain; the launch sizes stages x CTAs so about 32 KB of loads are in flight
-// per SM, which measured fastest.
+// per SM, which measured fastest.  The stores carry an L2 evict-first policy:
+// each buffer row is written once.  On B200 that measured 1-2% faster for
+// 15-17 GB dispatch buffers and the same for a 0.8 GB one.
 //
 // Rank-local form (PEER = true): the R ranks' buffers are separate allocations,
 // possibly on other GPUs, reached through a device table of R base pointers;
@@ -53,6 +55,7 @@ __global__ void __launch_bounds__(32)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stride_b);
   int32_t* ring = reinterpret_cast<int32_t*>(bars + DISPATCH_MAX_STAGES);  // [stages][K] destination rows
   const int lane = threadIdx.x;
+  const uint64_t evict_first = l2_evict_first_policy();  // each buffer row is written once
   if (lane == 0)
     for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
   fence_mbar_init();
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(32)
           dst = buf + (int64_t)row * row_bytes;
         }
         if (dst)
-          bulk_store(dst, smem + (size_t)s * stride_b, row_bytes);
+          bulk_store_hint(dst, smem + (size_t)s * stride_b, row_bytes, evict_first);
         else
           bad = EP_DEV_BAD_ROW;
       } else
