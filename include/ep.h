@@ -47,6 +47,9 @@
  *    are then defined but unspecified, and no write goes out of bounds.
  *  - Limits: 1 <= K <= min(E, 32), E <= EP_MAX_EXPERTS, R <= EP_MAX_RANKS,
  *    E % R == 0, H % 8 == 0, P < 2^31.
+ *  - A workspace (ws) holds the counters and grid-barrier words of the call
+ *    that uses it: calls in flight at the same time (on different streams)
+ *    need workspaces of their own.  Calls on one stream may share one.
  *  - The dispatch buffer and the combine input are views that the next dispatch
  *    or combine overwrites ([GR] "Ένα ρεαλιστικό πλαίσιο αξιολόγησης πριν από
  *    την υιοθέτηση": zero-copy views must not be kept past the next dispatch or
