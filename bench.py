@@ -501,6 +501,29 @@ def run_ours(args, rank, world, local_rank):
             if st:
                 raise RuntimeError(f"device status {st:#x} in the plan+dispatch+combine timing")
 
+    # ---- fused layout + dispatch: the route (with align-sort) and dispatch in
+    # one cooperative launch, against ep_route_fused followed by ep_dispatch
+    route_dispatch = None
+    if not args.no_graph:
+        def rd_separate():
+            for ly in layers:
+                ly.route()
+                tdh.ep_dispatch(ly.x, K, ly.pos, ly.buf, ly.dev_status)
+
+        def rd_fused():
+            for ly in layers:
+                ly.route_dispatch()
+
+        sep_ms = replay_ms(rd_separate, True)
+        fus_ms = replay_ms(rd_fused, True)
+        route_dispatch = {"fused_ms": round(fus_ms, 5), "separate_ms": round(sep_ms, 5),
+                          "what": "route (stats, plan, layout, align-sort) + dispatch per layer: ep_route_dispatch_fused "
+                                  "(one launch) against ep_route_fused then ep_dispatch; one graph each, L2 flushed"}
+        for ly in layers:
+            st = ly.status(stream)
+            if st:
+                raise RuntimeError(f"device status {st:#x} in the fused route + dispatch timing")
+
     # ---- the rank-local form emulated on this GPU: R rank buffers reached
     # through the peer table, each rank's dispatch and combine launched in
     # turn (one graph), against the one-buffer dispatch + combine above
@@ -668,6 +691,7 @@ def run_ours(args, rank, world, local_rank):
         "prefetch_slots": prefetch,
         "quota_planner": quota,
         "plan_dispatch_combine": as_named,
+        "route_dispatch": route_dispatch,
         "rank_local": rank_local,
         "layers_per_step": nl,
         "route_path": args.route,

@@ -9,6 +9,7 @@
  *   ep_align_sort (block-aligned expert sort for a grouped GEMM)
  *   ep_replica_grad_reduce (backward: replica gradients into the home expert)
  *   ep_route_fused (stats, plan, layout and align-sort in one launch)
+ *   ep_route_dispatch_fused (the same, with dispatch, in one launch)
  *   ep_dispatch_backward, ep_combine_backward (gradients of the row movers)
  *   ep_prefetch_slots (a per-rank replica slot budget B applied to a plan)
  *   ep_quota_route, ep_quota_replica_grad_reduce (the quota-driven planner:
@@ -330,6 +331,30 @@ EP_API int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int 
                           int32_t* pair_slot, int block_m, int32_t* sorted_token_ids, int64_t sorted_cap,
                           int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad, void* ws,
                           size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Fused layout + dispatch: ep_route_fused followed by ep_dispatch(x, T, K, H,
+ * pos, buf, buf_rows) in one cooperative launch, same outputs bit for bit
+ * (every route output, and buf[pos[p]] = x[p / K] for every pair).  [GR]
+ * "Online planning, zero copy και στατικά σχήματα": the rows go straight to
+ * their final expert-grouped position; here each tile CTA copies the token
+ * rows of its own pairs as soon as it has placed them, with no launch or
+ * grid-wide wait between layout and dispatch.  Token rows whose pairs fall in
+ * two tiles are read twice (at most one extra row per tile).
+ *   x    [T, H] bf16 in (non-NULL when T > 0), buf [buf_rows, H] bf16 out, H as in
+ *        ep_dispatch (H % 8 == 0, 8 <= H, 2H <= 1 MiB); both 16-byte aligned.
+ * Other arguments as in ep_route_fused.  When the grid with its row stages
+ * cannot be co-resident it runs ep_route_fused's fallback and ep_dispatch.
+ * Errors: as ep_route_fused and ep_dispatch (EP_DEV_BAD_ROW for a pair whose
+ * row is outside the buffer, EP_DEV_COPY_TIMEOUT for a copy that did not land).
+ */
+EP_API int ep_route_dispatch_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S,
+                                   int32_t* loads, double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos,
+                                   int32_t* src, int32_t* pair_slot, int block_m, int32_t* sorted_token_ids,
+                                   int64_t sorted_cap, int32_t* expert_ids, int64_t expert_ids_cap,
+                                   int32_t* num_tokens_post_pad, const uint16_t* x, int64_t H, uint16_t* buf,
+                                   int64_t buf_rows, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                   cudaStream_t stream);
 
 /*
  * a5. Dispatch.  [GR] "Online planning, zero copy και στατικά σχήματα": rows are

@@ -15,7 +15,9 @@ def _torch():
 def run_cuda(topk, w, x, R, S, E, block_m, scale=None, g_home=None, g_rep=None, clear=False, with_y=True,
              fused=False):
     """All outputs of one pass: stats, plan, layout, align-sort, dispatch,
-    stand-in expert, combine, grad-reduce.  x: uint16 [T,H] (or None)."""
+    stand-in expert, combine, grad-reduce.  x: uint16 [T,H] (or None).
+    fused: False (the separate route calls), True (ep_route_fused) or
+    "dispatch" (ep_route_dispatch_fused: route and dispatch in one launch)."""
     torch = _torch()
     import token_dispatch_histogram_b200 as tdh
     T, K = topk.shape
@@ -36,7 +38,13 @@ def run_cuda(topk, w, x, R, S, E, block_m, scale=None, g_home=None, g_rep=None, 
     sids = torch.full((cap,), -7, dtype=torch.int32, device=dev)
     eids = torch.full((capb,), -7, dtype=torch.int32, device=dev)
     ntpp = torch.full((1,), -7, dtype=torch.int32, device=dev)
-    if fused:
+    if fused == "dispatch":  # route and dispatch in one launch
+        H = x.shape[1]
+        t_x = torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).to(dev)
+        buf = torch.full((P, H), -1, dtype=torch.int16, device=dev).view(torch.bfloat16)
+        tdh.ep_route_dispatch_fused(t_topk, E, R, S, loads, mv, plan, pos, src, ws, t_x, buf, slot, block_m, sids,
+                                    eids, ntpp, status)
+    elif fused:
         tdh.ep_route_fused(t_topk, E, R, S, loads, mv, plan, pos, src, ws, slot, block_m, sids, eids, ntpp, status)
     else:
         tdh.ep_route_stats(t_topk, E, loads, mv, ws, status)
@@ -48,9 +56,10 @@ def run_cuda(topk, w, x, R, S, E, block_m, scale=None, g_home=None, g_rep=None, 
                sorted_ids=sids.cpu().numpy(), expert_ids=eids.cpu().numpy(), ntpp=int(ntpp.cpu().numpy()[0]))
     if x is not None:
         H = x.shape[1]
-        t_x = torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).to(dev)
-        buf = torch.full((P, H), -1, dtype=torch.int16, device=dev).view(torch.bfloat16)
-        tdh.ep_dispatch(t_x, K, pos, buf, status)
+        if fused != "dispatch":
+            t_x = torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).to(dev)
+            buf = torch.full((P, H), -1, dtype=torch.int16, device=dev).view(torch.bfloat16)
+            tdh.ep_dispatch(t_x, K, pos, buf, status)
         out["buf"] = buf.view(torch.int16).cpu().numpy().view(np.uint16)
         if with_y:
             t_scale = torch.from_numpy(np.ascontiguousarray(scale, dtype=np.float32)).to(dev)
@@ -142,3 +151,33 @@ def case_inputs(R, S, K, E, H, seed, kind="skew", bias_scale=1.0):
         topk, w = W.routing_from(T, E, K, seed=seed, bias_e=rng.normal(0, bias_scale, E))
     x = W.hidden(T, H, seed=seed + 1000) if H else None
     return topk, w, x
+
+
+def assert_route_parity(cu, orc, R, S, K, E):
+    """Every route output of run_cuda equals the oracle's, bit for bit."""
+    assert cu["status"] == 0
+    np.testing.assert_array_equal(cu["loads"], orc["loads"])
+    assert cu["max_vio"] == orc["max_vio"]  # fp64, same expression on both sides
+    pl = orc["plan"]
+    n = pl["n_rep"]
+    assert plan_field(cu, "n_rep", 1)[0] == n
+    np.testing.assert_array_equal(plan_field(cu, "rep_expert", n), pl["rep_expert"])
+    np.testing.assert_array_equal(plan_field(cu, "rep_rank", n), pl["rep_rank"])
+    np.testing.assert_array_equal(plan_field(cu, "rep_count", n), pl["rep_count"])
+    np.testing.assert_array_equal(plan_field(cu, "home_count", E), pl["home_count"])
+    lo = orc["layout"]
+    np.testing.assert_array_equal(plan_field(cu, "slot_order", E + n), lo["slot_order"])
+    np.testing.assert_array_equal(plan_field(cu, "cu_seqlens", E + n + 1), lo["cu_seqlens"])
+    exp = expected_plan_tables(pl, lo, R, S, K, E)
+    for name in ("home_base", "copy_cnt", "rank_nrep", "rank_rep_first"):
+        np.testing.assert_array_equal(plan_field(cu, name, len(exp[name])), exp[name], err_msg=name)
+    for name in ("rep_base", "rep_begin"):
+        np.testing.assert_array_equal(plan_field(cu, name, n), exp[name], err_msg=name)
+    has = exp["copy_cnt"] > 0
+    np.testing.assert_array_equal(plan_field(cu, "copy_first", E)[has], exp["copy_first"][has])
+    np.testing.assert_array_equal(cu["pos"], lo["pos"])
+    np.testing.assert_array_equal(cu["src"], lo["src"])
+    np.testing.assert_array_equal(cu["pair_slot"], lo["pair_slot"])
+    np.testing.assert_array_equal(cu["sorted_ids"], orc["sorted_ids"])
+    np.testing.assert_array_equal(cu["expert_ids"], orc["expert_ids"])
+    assert cu["ntpp"] == orc["ntpp"]

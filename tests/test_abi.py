@@ -86,6 +86,15 @@ def test_argument_errors_return_before_any_launch():
     assert L.ep_replica_grad_reduce(fake, fake, 0, 8, 8, 4, fake, 3, 0, None, None) == tdh.EP_ERR_CAPACITY
     # a row wider than two shared-memory stages (about 100 KB) is refused
     assert L.ep_dispatch(fake, 16, 2, 51200, fake, fake, 32, None, None) == tdh.EP_ERR_ARG
+    # fused layout + dispatch: the route's checks, then the dispatch's (before anything is enqueued)
+    def rdf(x, H, R=4, S=4):
+        return L.ep_route_dispatch_fused(fake, R * S, 2, 8, R, S, fake, fake, fake, 1 << 20, fake, fake, None, 4,
+                                         None, 0, None, 0, None, x, H, fake, 32, fake, 1 << 20, None, None)
+    assert rdf(None, 16) == tdh.EP_ERR_ARG                       # no x
+    assert rdf(fake, 12) == tdh.EP_ERR_ARG                       # H % 8
+    assert rdf(fake, 51200) == tdh.EP_ERR_ARG                    # rows the dispatch kernel refuses
+    assert rdf(ctypes.c_void_p(0x1008), 16) == tdh.EP_ERR_ARG    # misaligned x
+    assert rdf(fake, 16, R=3) == tdh.EP_ERR_ARG                  # E % R
     # zero-size work is a no-op that succeeds without touching the device
     assert L.ep_dispatch(None, 0, 2, 16, None, None, 0, None, None) == tdh.EP_OK
     assert L.ep_combine(None, 0, None, None, 0, 2, 16, None, None, None) == tdh.EP_OK

@@ -16,38 +16,9 @@ import pytest
 import oracle as O
 import oracle_pins as PINS
 import workload as W
-from gpu_path import (bf16_ulp_diff, case_inputs, expected_plan_tables, plan_field, run_cuda, run_oracle)
+from gpu_path import assert_route_parity, bf16_ulp_diff, case_inputs, plan_field, run_cuda, run_oracle
 
 pytestmark = pytest.mark.gpu
-
-
-def _assert_route_parity(cu, orc, R, S, K, E):
-    assert cu["status"] == 0
-    np.testing.assert_array_equal(cu["loads"], orc["loads"])
-    assert cu["max_vio"] == orc["max_vio"]  # fp64, same expression on both sides
-    pl = orc["plan"]
-    n = pl["n_rep"]
-    assert plan_field(cu, "n_rep", 1)[0] == n
-    np.testing.assert_array_equal(plan_field(cu, "rep_expert", n), pl["rep_expert"])
-    np.testing.assert_array_equal(plan_field(cu, "rep_rank", n), pl["rep_rank"])
-    np.testing.assert_array_equal(plan_field(cu, "rep_count", n), pl["rep_count"])
-    np.testing.assert_array_equal(plan_field(cu, "home_count", E), pl["home_count"])
-    lo = orc["layout"]
-    np.testing.assert_array_equal(plan_field(cu, "slot_order", E + n), lo["slot_order"])
-    np.testing.assert_array_equal(plan_field(cu, "cu_seqlens", E + n + 1), lo["cu_seqlens"])
-    exp = expected_plan_tables(pl, lo, R, S, K, E)
-    for name in ("home_base", "copy_cnt", "rank_nrep", "rank_rep_first"):
-        np.testing.assert_array_equal(plan_field(cu, name, len(exp[name])), exp[name], err_msg=name)
-    for name in ("rep_base", "rep_begin"):
-        np.testing.assert_array_equal(plan_field(cu, name, n), exp[name], err_msg=name)
-    has = exp["copy_cnt"] > 0
-    np.testing.assert_array_equal(plan_field(cu, "copy_first", E)[has], exp["copy_first"][has])
-    np.testing.assert_array_equal(cu["pos"], lo["pos"])
-    np.testing.assert_array_equal(cu["src"], lo["src"])
-    np.testing.assert_array_equal(cu["pair_slot"], lo["pair_slot"])
-    np.testing.assert_array_equal(cu["sorted_ids"], orc["sorted_ids"])
-    np.testing.assert_array_equal(cu["expert_ids"], orc["expert_ids"])
-    assert cu["ntpp"] == orc["ntpp"]
 
 
 @pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
@@ -92,7 +63,7 @@ def test_route_plan_layout_align(case, fused):
         topk, w, _ = case_inputs(R, S, K, E, 0, seed=R * 131 + S, kind=kind, bias_scale=1.5)
     cu = run_cuda(topk, None, None, R, S, E, bm, fused=fused)
     orc = run_oracle(topk, None, None, R, S, E, bm)
-    _assert_route_parity(cu, orc, R, S, K, E)
+    assert_route_parity(cu, orc, R, S, K, E)
 
 
 @pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
@@ -109,7 +80,7 @@ def test_route_fuzz(fused):
         topk, w, _ = case_inputs(R, S, K, E, 0, seed=it, kind=kind, bias_scale=float(rng.uniform(0.2, 3)))
         cu = run_cuda(topk, None, None, R, S, E, bm, fused=fused)
         orc = run_oracle(topk, None, None, R, S, E, bm)
-        _assert_route_parity(cu, orc, R, S, K, E)
+        assert_route_parity(cu, orc, R, S, K, E)
 
 
 ROW_CASES = [

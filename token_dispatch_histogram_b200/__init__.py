@@ -72,6 +72,8 @@ _SIGS = {
     "ep_align_sort": (_I, [_V, _I64, _I, _I, _I, _V, _I64, _V, _I64, _V, _V, _SZ, _V, _V]),
     "ep_route_fused": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _V, _V, _SZ, _V, _V, _V, _I, _V, _I64, _V, _I64, _V,
                             _V, _SZ, _V, _V]),
+    "ep_route_dispatch_fused": (_I, [_V, _I64, _I, _I, _I, _I64, _V, _V, _V, _SZ, _V, _V, _V, _I, _V, _I64, _V,
+                                     _I64, _V, _V, _I64, _V, _I64, _V, _SZ, _V, _V]),
     "ep_dispatch": (_I, [_V, _I64, _I, _I64, _V, _V, _I64, _V, _V]),
     "ep_expert_scale": (_I, [_V, _I64, _I64, _V, _V, _I64, _V, _I, _V, _V, _V]),
     "ep_dispatch_backward": (_I, [_V, _I64, _V, _I64, _I, _I64, _V, _V, _V]),
@@ -252,6 +254,28 @@ def ep_route_fused(topk_ids, E, R, S, loads, max_vio, plan, pos, src, ws, pair_s
         _p(pair_slot), block_m, _p(sorted_token_ids), sorted_token_ids.numel() if align else 0,
         _p(expert_ids), expert_ids.numel() if align else 0, _p(num_tokens_post_pad), _p(ws),
         ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
+
+
+def ep_route_dispatch_fused(topk_ids, E, R, S, loads, max_vio, plan, pos, src, ws, x, buf, pair_slot=None,
+                            block_m=0, sorted_token_ids=None, expert_ids=None, num_tokens_post_pad=None,
+                            dev_status=None, stream=None):
+    """ep_route_fused followed by ep_dispatch(x, K, pos, buf), in one
+    cooperative launch (the rows are copied as each tile is placed)."""
+    for t in (topk_ids, loads, plan, pos, src):
+        _dtype(t, torch.int32)
+    _dtype(max_vio, torch.float64)
+    _dtype(x, torch.bfloat16, torch.int16, torch.uint16)
+    _dtype(buf, torch.bfloat16, torch.int16, torch.uint16)
+    T, K = topk_ids.shape
+    H = x.shape[1]
+    if x.shape[0] != T or buf.shape[1] != H:
+        raise EpError("ep_route_dispatch_fused", EP_ERR_ARG)
+    align = sorted_token_ids is not None
+    _check("ep_route_dispatch_fused", lib().ep_route_dispatch_fused(
+        _p(topk_ids), T, K, E, R, S, _p(loads), _p(max_vio), _p(plan), plan.numel(), _p(pos), _p(src),
+        _p(pair_slot), block_m, _p(sorted_token_ids), sorted_token_ids.numel() if align else 0,
+        _p(expert_ids), expert_ids.numel() if align else 0, _p(num_tokens_post_pad), _p(x), H, _p(buf),
+        buf.shape[0], _p(ws), ws.numel() * ws.element_size(), _p(dev_status), _s(stream)))
 
 
 def align_sort_capacity(P, E, block_m):

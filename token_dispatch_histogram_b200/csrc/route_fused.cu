@@ -21,6 +21,15 @@
 // A pair's stable rank within its expert = (its tile's prefix) + (earlier warps
 // of the tile) + (earlier chunks of its warp) + popc(peers & lanemask_lt):
 // integer adds only, so nothing depends on scheduling.  Every wait is bounded.
+//
+// Fused layout + dispatch (ep_route_dispatch_fused, DISPATCH = true): once a
+// tile CTA has written its pairs' rows (step 4), it copies the hidden rows of
+// the tokens its tile touches straight to those rows -- the dispatch kernel's
+// scheme (one TMA bulk load per token row into a shared-memory stage, one bulk
+// store per pair) run by a few warps of the CTA, with the pair rows read back
+// from pos.  A token whose pairs straddle two tiles is loaded by both CTAs,
+// each storing only its own pairs.  Same outputs as ep_route_fused followed by
+// ep_dispatch, bit for bit; no launch and no grid-wide wait between them.
 #include <algorithm>
 
 #include "grid_sync.cuh"
@@ -33,6 +42,7 @@ int fused_route_separate(const int32_t* topk_ids, int64_t T, int K, int E, int R
                          int32_t* pair_slot, int block_m, int32_t* sorted_ids, int64_t sorted_cap,
                          int32_t* expert_ids, int64_t expert_ids_cap, int32_t* ntpp, void* ws, size_t ws_bytes,
                          int32_t* dev_status, cudaStream_t stream);
+bool dispatch_shape_ok(int64_t H, int K);  // rows.cu
 
 constexpr int FUSED_THREADS = 512;
 constexpr int FUSED_WARPS = FUSED_THREADS / 32;
@@ -60,6 +70,15 @@ struct FusedArgs {
   int64_t expert_ids_cap;
   int32_t* ntpp;
   int32_t* dev_status;
+  // fused dispatch (DISPATCH = true only)
+  const uint8_t* x;     // [T, row_bytes] token rows
+  uint8_t* buf;         // [buf_rows, row_bytes]
+  int64_t buf_rows;
+  uint32_t row_bytes;
+  int K;
+  int copy_warps;       // warps of each tile CTA that copy rows
+  int copy_stages;      // shared-memory row stages per copying warp
+  uint32_t copy_off;    // byte offset of the copy region in dynamic shared memory
 };
 
 constexpr int WALK_UNROLL = 8;  // tile loads each lane keeps in flight during a walk
@@ -103,8 +122,87 @@ __device__ __forceinline__ void walk_warp(const int32_t* __restrict__ topk, int6
   }
 }
 
+// Copy the rows of the tokens that pairs [pb, pe) belong to: buf[pos[p]] =
+// x[p / K] for every p in [pb, pe).  Warps 0 .. copy_warps-1 take the tokens in
+// turn, each with a ring of copy_stages row stages (TMA bulk load of the token
+// row, completion on an mbarrier; one bulk store per pair of the range, with
+// an L2 evict-first policy as in the dispatch kernel).  pos is read back with
+// L2 loads: this CTA wrote it, before a block barrier.  Rows outside
+// [0, buf_rows) (pos = -1 for an invalid id) are reported, never written.
+__device__ void route_copy_rows(const FusedArgs& a, int64_t pb, int64_t pe, uint8_t* cs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp >= a.copy_warps || pe <= pb) return;
+  const int K = a.K, stages = a.copy_stages, nw = a.copy_warps;
+  const uint32_t row_bytes = a.row_bytes;
+  const uint32_t stride_b = (row_bytes + 127u) & ~127u;
+  uint8_t* st0 = cs + (size_t)warp * stages * stride_b;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cs + (size_t)nw * stages * stride_b) + (size_t)warp * stages;
+  int32_t* ring = reinterpret_cast<int32_t*>(cs + (size_t)nw * stages * (stride_b + 8)) + (size_t)warp * stages * K;
+  const uint64_t evict_first = l2_evict_first_policy();
+  if (lane == 0)
+    for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
+  fence_mbar_init();
+  __syncwarp();
+
+  constexpr int32_t NOT_MINE = INT32_MIN;  // a pair of the token outside [pb, pe)
+  const int64_t t_lo = pb / K, t_hi = (pe - 1) / K + 1;
+  const int64_t first = t_lo + warp;
+  const int64_t njobs = first < t_hi ? (t_hi - first + nw - 1) / nw : 0;
+  auto issue = [&](int64_t j) {
+    const int s = (int)(j % stages);
+    const int64_t t = first + j * nw;
+    if (lane < K) {
+      const int64_t p = t * K + lane;
+      ring[s * K + lane] = (p >= pb && p < pe) ? __ldcg(a.pos + p) : NOT_MINE;
+    }
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[s], row_bytes);
+      bulk_load(st0 + (size_t)s * stride_b, a.x + t * (int64_t)row_bytes, row_bytes, &bars[s]);
+    }
+  };
+  const int64_t pro = njobs < stages ? njobs : (int64_t)stages;
+  for (int64_t j = 0; j < pro; ++j) issue(j);
+  int64_t issued = pro;
+
+  int32_t bad = 0;
+  bool ok = true;
+  int64_t j = 0;
+  for (; j < njobs; ++j) {
+    const int s = (int)(j % stages);
+    const uint32_t parity = (uint32_t)((j / stages) & 1);
+    const bool landed = mbar_wait_bounded(&bars[s], parity);
+    if (!__all_sync(0xffffffffu, landed)) {
+      ok = false;
+      break;
+    }
+    if (lane < K) {
+      const int32_t row = ring[s * K + lane];
+      if (row != NOT_MINE) {
+        if (row >= 0 && row < a.buf_rows)
+          bulk_store_hint(a.buf + (int64_t)row * row_bytes, st0 + (size_t)s * stride_b, row_bytes, evict_first);
+        else
+          bad = EP_DEV_BAD_ROW;
+      }
+    }
+    bulk_commit();
+    if (j >= 1 && issued < njobs) {  // refill the previous job's stage once its stores have read it
+      bulk_wait_read<1>();
+      __syncwarp();
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (!ok) {  // a row did not land in time: report, and give the loads in flight a bounded chance to land
+    if (lane == 0) flag(a.dev_status, EP_DEV_COPY_TIMEOUT);
+    for (int64_t q = j; q < issued; ++q) mbar_wait_bounded(&bars[(int)(q % stages)], (uint32_t)((q / stages) & 1));
+  }
+  bulk_wait_all();
+  if (bad) flag(a.dev_status, bad);
+}
+
+template <bool DISPATCH>
 __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
-  extern __shared__ int32_t sm[];
+  extern __shared__ __align__(128) int32_t sm[];
   // CTAs 0..NT-1 own one tile each; the last CTA (NT) owns none and runs the
   // planner, so the plan overlaps the align-sort walks of the others.
   const int E = a.E, tile = a.tile, G = gridDim.x, NT = a.ntiles, t = blockIdx.x, tid = threadIdx.x;
@@ -321,6 +419,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
     if (s_bad) flag(a.dev_status, EP_DEV_BAD_EXPERT_ID);
     if (s_badrow) flag(a.dev_status, EP_DEV_BAD_ROW);
   }
+  if constexpr (DISPATCH) {
+    __syncthreads();  // every pos of this tile is written (the walk and the fix-up above)
+    route_copy_rows(a, p0, min(p0 + (int64_t)tile, P), reinterpret_cast<uint8_t*>(sm) + a.copy_off);
+  }
 }
 
 size_t fused_smem_bytes(int E, int R) {
@@ -334,11 +436,37 @@ size_t fused_smem_bytes(int E, int R) {
 
 using namespace ep;
 
-extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
-                              double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
-                              int32_t* pair_slot, int block_m, int32_t* sorted_token_ids, int64_t sorted_cap,
-                              int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad, void* ws,
-                              size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
+namespace ep {
+
+// Rows in flight for the fused copy, as the dispatch kernel sizes them: about
+// 32 KB of row loads per SM (4 stages per warp for rows up to 1 KB, else 2),
+// split over the CTAs of an SM.
+struct CopyShape {
+  int warps = 0, stages = 0;
+  size_t bytes = 0;
+};
+
+static CopyShape copy_shape(uint32_t row_bytes, int K, int per_sm) {
+  const uint32_t stride_b = (row_bytes + 127u) & ~127u;
+  const uint32_t target = 32u * 1024u;
+  const int stages = stride_b * 2u * 16u <= target ? 4 : 2;
+  const int ctas = (int)std::min<uint32_t>(32, std::max<uint32_t>(1, (target + stages * stride_b - 1) / (stages * stride_b)));
+  const int rows_cta = std::max(1, stages * ctas / std::max(1, per_sm));
+  CopyShape c;
+  c.stages = std::min(stages, rows_cta);
+  c.warps = std::min(FUSED_WARPS, std::max(1, rows_cta / c.stages));
+  c.bytes = (size_t)c.warps * c.stages * (stride_b + 8 + 4 * (size_t)K);
+  return c;
+}
+
+// ep_route_fused, and with x != nullptr the dispatch of x into buf in the
+// same launch (ep_route_dispatch_fused).
+static int route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
+                       double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
+                       int32_t* pair_slot, int block_m, int32_t* sorted_token_ids, int64_t sorted_cap,
+                       int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad,
+                       const uint16_t* x, int64_t H, uint16_t* buf, int64_t buf_rows, void* ws, size_t ws_bytes,
+                       int32_t* dev_status, cudaStream_t stream) {
   if (!valid_tke(T, K, E) || R < 1 || R > EP_MAX_RANKS || E % R || S < 0 || (int64_t)R * S != T) return EP_ERR_ARG;
   if (!loads || !max_vio || !plan || !ws) return EP_ERR_ARG;
   const int64_t P = T * K;
@@ -350,31 +478,48 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
     if (need >= ((int64_t)1 << 31)) return EP_ERR_ARG;
     if (sorted_cap < need || expert_ids_cap < (sorted_cap + block_m - 1) / block_m) return EP_ERR_CAPACITY;
   }
+  const bool dispatch = x != nullptr;
+  if (dispatch) {  // as ep_dispatch (its fallback must accept the same rows)
+    if (!dispatch_shape_ok(H, K) || buf_rows < 0) return EP_ERR_ARG;
+    if (T > 0 && (!buf || !aligned16(x) || !aligned16(buf))) return EP_ERR_ARG;
+  }
   EpPlanLayout L;
   plan_layout(E, R, &L);
   if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
   const WsLayout wl = ws_layout(P, E);
   if (ws_bytes < wl.bytes) return EP_ERR_CAPACITY;
 
-  // grid: one or two resident CTAs per SM, tiles a multiple of 512 pairs
-  const size_t smem = fused_smem_bytes(E, R);
-  int occ = 0;
-  if (P > 0 && smem <= 227 * 1024) {
+  // grid: one or two resident CTAs per SM, tiles a multiple of 512 pairs; the
+  // fused copy adds its row stages to each CTA's shared memory
+  const void* fn = dispatch ? (const void*)k_route_fused<true> : (const void*)k_route_fused<false>;
+  const uint32_t row_bytes = dispatch ? (uint32_t)(H * 2) : 0u;
+  const size_t route_smem = (fused_smem_bytes(E, R) + 127) & ~(size_t)127;
+  auto smem_for = [&](int ps) { return route_smem + (dispatch ? copy_shape(row_bytes, K, ps).bytes : 0); };
+  auto resident_ok = [&](int ps, size_t smem) {
+    if (smem > 227 * 1024) return false;
     if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(k_route_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return EP_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_route_fused, FUSED_THREADS, smem) != cudaSuccess)
-      occ = 0;
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return false;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, FUSED_THREADS, smem) != cudaSuccess) return false;
+    return occ >= ps;
+  };
+  int per_sm = 0;
+  if (P > 0) {
+    if (resident_ok(2, smem_for(2)))
+      per_sm = 2;
+    else if (resident_ok(1, smem_for(1)))
+      per_sm = 1;
   }
   // One CTA per SM while that keeps tiles at 2048 pairs or fewer: the planner
   // CTA then has an SM to itself (measured on B200 at 196,608 pairs: kernel span
   // 17.9 -> 15.9 us); larger problems keep two per SM (one per SM measured
   // slower there: the longer tile walks outweigh the faster plan).
-  int per_sm = std::min(occ, 2);
   if (per_sm == 2 && num_sms() > 1) {
     const int64_t t1 = ((P + num_sms() - 2) / (num_sms() - 1) + 511) / 512 * 512;
-    if (t1 <= 2048) per_sm = 1;
+    if (t1 <= 2048 && resident_ok(1, smem_for(1))) per_sm = 1;
   }
+  const size_t smem = per_sm ? smem_for(per_sm) : 0;
   const int64_t resident = (int64_t)num_sms() * per_sm;
   int64_t tile = 0, ntiles = 0;
   if (resident > 1) {  // one CTA per tile plus the planner CTA
@@ -385,17 +530,20 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   // the [E][tiles] counts must fit below T_e (the separate path's regions are unused here)
   const bool fits = resident > 1 && ntiles + 1 <= resident && tile <= (1 << 20) &&
                     (size_t)E * ntiles * 4 <= wl.loads_off;
-  if (!fits)
-    return fused_route_separate(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot,
-                                block_m, sorted_token_ids, sorted_cap, expert_ids, expert_ids_cap,
-                                num_tokens_post_pad, ws, ws_bytes, dev_status, stream);
+  if (!fits) {
+    int rc = fused_route_separate(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot,
+                                  block_m, sorted_token_ids, sorted_cap, expert_ids, expert_ids_cap,
+                                  num_tokens_post_pad, ws, ws_bytes, dev_status, stream);
+    if (rc == EP_OK && dispatch) rc = ep_dispatch(x, T, K, H, pos, buf, buf_rows, dev_status, stream);
+    return rc;
+  }
   // workspace: counts [E][tiles] from byte 0; T_e [E] where ep_align_sort
   // keeps its histogram, then the two sync words (in the slack after it);
   // one memset zeroes T_e and the sync words
   char* w = static_cast<char*>(ws);
   const size_t tot_bytes = ((size_t)E * 4 + 15) & ~(size_t)15;
   if (cudaMemsetAsync(w + wl.loads_off, 0, tot_bytes + 16, stream) != cudaSuccess) return EP_ERR_CUDA;
-  FusedArgs args;
+  FusedArgs args = {};
   args.topk = topk_ids;
   args.P = P;
   args.E = E;
@@ -420,6 +568,17 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   args.expert_ids_cap = expert_ids_cap;
   args.ntpp = num_tokens_post_pad;
   args.dev_status = dev_status;
+  if (dispatch) {
+    const CopyShape c = copy_shape(row_bytes, K, per_sm);
+    args.x = reinterpret_cast<const uint8_t*>(x);
+    args.buf = reinterpret_cast<uint8_t*>(buf);
+    args.buf_rows = buf_rows;
+    args.row_bytes = row_bytes;
+    args.K = K;
+    args.copy_warps = c.warps;
+    args.copy_stages = c.stages;
+    args.copy_off = (uint32_t)route_smem;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ntiles + 1);
   cfg.blockDim = dim3(FUSED_THREADS);
@@ -430,9 +589,36 @@ extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k_route_fused, args) != cudaSuccess) return EP_ERR_CUDA;
+  const cudaError_t err = dispatch ? cudaLaunchKernelEx(&cfg, k_route_fused<true>, args)
+                                   : cudaLaunchKernelEx(&cfg, k_route_fused<false>, args);
+  if (err != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
+}
+
+}  // namespace ep
+
+extern "C" int ep_route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S, int32_t* loads,
+                              double* max_vio, int32_t* plan, size_t plan_words, int32_t* pos, int32_t* src,
+                              int32_t* pair_slot, int block_m, int32_t* sorted_token_ids, int64_t sorted_cap,
+                              int32_t* expert_ids, int64_t expert_ids_cap, int32_t* num_tokens_post_pad, void* ws,
+                              size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
+  return route_fused(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot, block_m,
+                     sorted_token_ids, sorted_cap, expert_ids, expert_ids_cap, num_tokens_post_pad, nullptr, 0,
+                     nullptr, 0, ws, ws_bytes, dev_status, stream);
+}
+
+extern "C" int ep_route_dispatch_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, int64_t S,
+                                       int32_t* loads, double* max_vio, int32_t* plan, size_t plan_words,
+                                       int32_t* pos, int32_t* src, int32_t* pair_slot, int block_m,
+                                       int32_t* sorted_token_ids, int64_t sorted_cap, int32_t* expert_ids,
+                                       int64_t expert_ids_cap, int32_t* num_tokens_post_pad, const uint16_t* x,
+                                       int64_t H, uint16_t* buf, int64_t buf_rows, void* ws, size_t ws_bytes,
+                                       int32_t* dev_status, cudaStream_t stream) {
+  if (!x && T > 0) return EP_ERR_ARG;  // (T = 0: nothing to copy, x may be NULL)
+  return route_fused(topk_ids, T, K, E, R, S, loads, max_vio, plan, plan_words, pos, src, pair_slot, block_m,
+                     sorted_token_ids, sorted_cap, expert_ids, expert_ids_cap, num_tokens_post_pad, x, H, buf,
+                     buf_rows, ws, ws_bytes, dev_status, stream);
 }
 
 namespace ep {

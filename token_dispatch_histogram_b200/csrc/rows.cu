@@ -35,15 +35,6 @@ namespace ep {
 
 constexpr int DISPATCH_MAX_STAGES = 8;
 
-// Wait (bounded by WAIT_LIMIT_NS) for phase `parity` of an mbarrier.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
-  return true;
-}
-
 template <bool PEER>
 __global__ void __launch_bounds__(32)
     k_dispatch(const uint8_t* __restrict__ x, int64_t T, int K, uint32_t row_bytes, const int32_t* __restrict__ pos,
@@ -406,6 +397,19 @@ namespace ep {
 
 // Dispatch launch shared by the one-buffer and the rank-local (peer) entry
 // points.  peers == NULL: rows go to buf[row]; else to the rank buffers.
+// Shared-memory stages of one dispatch CTA for rows of H bf16 values (the
+// launch below): 4 stages for rows up to 1 KB, else 2.
+static size_t dispatch_smem(int64_t H, int K) {
+  const uint32_t stride_b = ((uint32_t)(H * 2) + 127u) & ~127u;
+  const int stages = stride_b * 2u * 16u <= 32u * 1024u ? 4 : 2;
+  return (size_t)stages * stride_b + DISPATCH_MAX_STAGES * 8 + (size_t)stages * K * 4;
+}
+
+// Whether ep_dispatch accepts rows of H values at top-K = K (its stages fit).
+bool dispatch_shape_ok(int64_t H, int K) {
+  return K >= 1 && K <= 32 && H >= 8 && H % 8 == 0 && H * 2 <= (1 << 20) && dispatch_smem(H, K) <= 200 * 1024;
+}
+
 static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
                         int64_t buf_rows, const uint64_t* peers, const int32_t* rank_first, int R,
                         int64_t rows_per_rank, int32_t* dev_status, cudaStream_t stream) {
@@ -419,7 +423,7 @@ static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const in
   const uint32_t target = 32u * 1024u;
   const int stages = stride_b * 2u * 16u <= target ? 4 : 2;
   const int per_sm = (int)std::min<uint32_t>(32, std::max<uint32_t>(1, (target + stages * stride_b - 1) / (stages * stride_b)));
-  size_t smem = (size_t)stages * stride_b + DISPATCH_MAX_STAGES * 8 + (size_t)stages * K * 4;
+  const size_t smem = dispatch_smem(H, K);
   if (smem > 200 * 1024) return EP_ERR_ARG;
   const void* fn = peers ? (const void*)k_dispatch<true> : (const void*)k_dispatch<false>;
   if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -16,7 +16,8 @@ Plumbing only: every computation happens in the library's kernels.
 import torch
 
 from . import (align_sort_capacity, ep_align_sort, ep_combine, ep_dispatch, ep_expert_scale, ep_layout,
-               ep_plan, ep_plan_layout, ep_replica_grad_reduce, ep_route_fused, ep_route_stats, ep_status_read,
+               ep_plan, ep_plan_layout, ep_replica_grad_reduce, ep_route_dispatch_fused, ep_route_fused, ep_route_stats,
+               ep_status_read,
                ep_workspace_size)
 
 
@@ -97,6 +98,14 @@ class EpLayer:
                   self.dev_status, stream)
         ep_align_sort(self.topk_ids, self.E, self.block_m, self.sorted_token_ids, self.expert_ids,
                       self.num_tokens_post_pad, self.ws, self.dev_status, stream)
+
+    def route_dispatch(self, stream=None):
+        """route() and dispatch() in one cooperative launch: each tile's rows
+        are copied as soon as the tile is placed (same outputs)."""
+        ep_route_dispatch_fused(self.topk_ids, self.E, self.R, self.S, self.loads, self.max_vio, self.plan, self.pos,
+                                self.src, self.ws, self.x, self.buf, self.pair_slot, self.block_m,
+                                self.sorted_token_ids, self.expert_ids, self.num_tokens_post_pad, self.dev_status,
+                                stream)
 
     def dispatch(self, stream=None):
         ep_dispatch(self.x, self.K, self.pos, self.buf, self.dev_status, stream)
