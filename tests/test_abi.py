@@ -163,3 +163,21 @@ def test_rank_local_and_quota_argument_errors():
                             None) == tdh.EP_ERR_ARG
     assert L.ep_quota_route(fake, 16, 2, 8, 4, 4, 1, fake, fake, 1 << 20, fake, fake, fake, 16, None,
                             None) == tdh.EP_ERR_CAPACITY
+
+
+def test_missing_library_fails_loudly_and_build_does_not_need_it():
+    """Without libep.so the package does not import (no CPU fallback), and the
+    build entry point reaches its build script without importing the package."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    hide = ("import os; real = os.path.exists; "
+            "os.path.exists = lambda p: False if str(p).endswith('libep.so') else real(p); ")
+    r = subprocess.run([sys.executable, "-c", hide + "import token_dispatch_histogram_b200"], cwd=root,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "not built" in r.stderr
+    probe = (hide + "import sys, __graft_entry__ as g; "
+             "b = g._load_by_path('_b', os.path.join(g.ROOT, 'token_dispatch_histogram_b200', 'build.py')); "
+             "assert callable(b.build) and 'token_dispatch_histogram_b200' not in sys.modules; print('ok')")
+    r = subprocess.run([sys.executable, "-c", probe], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
