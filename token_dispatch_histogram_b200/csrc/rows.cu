@@ -6,15 +6,21 @@
 // buf[pos[t*K + k]] = x[t] for k < K.  Minimal traffic: each x row is read once
 // (T*H*2 bytes) and each buffer row written once (P*H*2 bytes).
 //
-// B200 design: a persistent grid of one-warp CTAs, each with a ring of shared
-// memory stages.  Lane 0 brings a whole row in with one TMA bulk copy
-// (cp.async.bulk global->shared, completion on an mbarrier); once it lands,
-// lanes 0..K-1 each issue one bulk store (shared->global) of that row to one
-// destination.  Loads for the next stages are in flight while the stores
-// drain; the launch sizes stages x CTAs so about 32 KB of loads are in flight
-// per SM, which measured fastest.  The stores carry an L2 evict-first policy:
-// each buffer row is written once.  On B200 that measured 1-2% faster for
-// 15-17 GB dispatch buffers and the same for a 0.8 GB one.
+// B200 design: one-warp CTAs, each owning DISPATCH_TOKENS_PER_CTA consecutive
+// tokens, with a ring of shared-memory stages.  Lane 0 brings a whole row in
+// with one TMA bulk copy (cp.async.bulk global->shared, completion on an
+// mbarrier); once it lands, lanes 0..K-1 each issue one bulk store
+// (shared->global) of that row to one destination.  The grid has one CTA per
+// pair of tokens (not a persistent grid), and each CTA reserves enough shared
+// memory that only as many fit an SM as keep about 32 KB of row loads in flight
+// per SM, which measured fastest.  Measured on B200 against a persistent
+// grid-stride grid of the same residency: 5-14% faster alone (the block
+// scheduler keeps the tokens in flight close together and balances the tail),
+// and it shares the GPU gracefully: next to an unrelated kernel on another
+// stream, the persistent grid took 2-4x its time (its late-starting CTAs still
+// owned a full share of tokens), this one the sum of the two.  The stores carry
+// an L2 evict-first policy: each buffer row is written once (1-2% faster for
+// 15-17 GB dispatch buffers, the same for a 0.8 GB one).
 //
 // Rank-local form (PEER = true): the R ranks' buffers are separate allocations,
 // possibly on other GPUs, reached through a device table of R base pointers;
@@ -34,6 +40,8 @@
 namespace ep {
 
 constexpr int DISPATCH_MAX_STAGES = 8;
+constexpr int DISPATCH_TOKENS_PER_CTA = 2;  // 1, 4 and 8 measured slower on B200
+constexpr int COMBINE_ITERS = 4;  // token iterations per combine CTA (1-3 measured slower at 0.9 GB)
 
 template <bool PEER>
 __global__ void __launch_bounds__(32)
@@ -52,11 +60,11 @@ __global__ void __launch_bounds__(32)
   fence_mbar_init();
   __syncwarp();
 
-  const int64_t first = blockIdx.x, step = gridDim.x;
-  const int64_t njobs = first < T ? (T - first + step - 1) / step : 0;
+  const int64_t first = (int64_t)blockIdx.x * DISPATCH_TOKENS_PER_CTA;
+  const int64_t njobs = first < T ? min((int64_t)DISPATCH_TOKENS_PER_CTA, T - first) : 0;
   auto issue = [&](int64_t j) {
     const int s = (int)(j % stages);
-    const int64_t t = first + j * step;
+    const int64_t t = first + j;
     if (lane < K) ring[s * K + lane] = __ldg(pos + t * K + lane);
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars[s], row_bytes);
@@ -154,7 +162,10 @@ __global__ void __launch_bounds__(256)
 // Combine with the indices and gate weights of a CTA's tokens staged in shared
 // memory one iteration ahead (double buffer), so each thread's K 16-byte row
 // loads issue back to back without waiting on index loads, and registers stay
-// within 64 (four 256-thread CTAs per SM).
+// within 64 (four 256-thread CTAs per SM).  Each CTA owns COMBINE_ITERS
+// iterations of consecutive tokens (not a persistent grid): on B200 the same
+// time as a persistent grid-stride grid at 0.9 GB, 4-6% faster at 17-19 GB
+// (the block scheduler keeps the tokens in flight close together).
 template <int K, bool PEER>
 __global__ void __launch_bounds__(256, 4)
     k_combine(const uint16_t* __restrict__ y, int64_t y_rows, const float* __restrict__ w,
@@ -170,7 +181,9 @@ __global__ void __launch_bounds__(256, 4)
   const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);  // threads per token
   const int tpc = 256 / tpr <= MAXT ? 256 / tpr : MAXT;                // tokens per CTA iteration
   const int sub = threadIdx.x / tpr, v0 = threadIdx.x % tpr;
-  const int64_t step = (int64_t)gridDim.x * tpc;
+  const int64_t step = tpc;
+  const int64_t t_begin = (int64_t)blockIdx.x * tpc * COMBINE_ITERS;
+  const int64_t t_end = min(T, t_begin + (int64_t)tpc * COMBINE_ITERS);
   if (threadIdx.x == 0) s_bad = 0;
   auto stage = [&](int b, int64_t tb) {
     if (threadIdx.x < tpc * K) {
@@ -201,11 +214,11 @@ __global__ void __launch_bounds__(256, 4)
       }
     }
   };
-  int64_t tb = (int64_t)blockIdx.x * tpc;
+  int64_t tb = t_begin;
   stage(0, tb);
   __syncthreads();
-  for (int b = 0; tb < T; tb += step, b ^= 1) {
-    stage(b ^ 1, tb + step);
+  for (int b = 0; tb < t_end; tb += step, b ^= 1) {
+    if (tb + step < t_end) stage(b ^ 1, tb + step);
     const int64_t t = tb + sub;
     if (sub < tpc && t < T) {
       for (int64_t v = v0; v < nvec; v += tpr) {
@@ -379,6 +392,16 @@ __global__ void __launch_bounds__(256, 2)
   if (bad) flag(dev_status, bad);
 }
 
+// Grid of k_combine<K, *> for T tokens of H values: one CTA per
+// COMBINE_ITERS iterations of its tokens-per-iteration (the kernel's tpc).
+static int combine_grid(int64_t T, int64_t H) {
+  const int64_t nvec = H / 8;
+  const int tpr = (int)(nvec >= 256 ? 256 : (nvec + 31) / 32 * 32);
+  const int tpc = 256 / tpr <= 8 ? 256 / tpr : 8;
+  const int64_t per_cta = (int64_t)tpc * COMBINE_ITERS;
+  return (int)std::min<int64_t>((T + per_cta - 1) / per_cta, 0x7fffffff);
+}
+
 int occupancy_grid(const void* fn, int threads, size_t smem, int64_t work_items, int cap_per_sm) {
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess || per_sm < 1)
@@ -395,8 +418,6 @@ using namespace ep;
 
 namespace ep {
 
-// Dispatch launch shared by the one-buffer and the rank-local (peer) entry
-// points.  peers == NULL: rows go to buf[row]; else to the rank buffers.
 // Shared-memory stages of one dispatch CTA for rows of H bf16 values (the
 // launch below): 4 stages for rows up to 1 KB, else 2.
 static size_t dispatch_smem(int64_t H, int K) {
@@ -410,6 +431,8 @@ bool dispatch_shape_ok(int64_t H, int K) {
   return K >= 1 && K <= 32 && H >= 8 && H % 8 == 0 && H * 2 <= (1 << 20) && dispatch_smem(H, K) <= 200 * 1024;
 }
 
+// Dispatch launch shared by the one-buffer and the rank-local (peer) entry
+// points.  peers == NULL: rows go to buf[row]; else to the rank buffers.
 static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const int32_t* pos, uint16_t* buf,
                         int64_t buf_rows, const uint64_t* peers, const int32_t* rank_first, int R,
                         int64_t rows_per_rank, int32_t* dev_status, cudaStream_t stream) {
@@ -423,12 +446,21 @@ static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const in
   const uint32_t target = 32u * 1024u;
   const int stages = stride_b * 2u * 16u <= target ? 4 : 2;
   const int per_sm = (int)std::min<uint32_t>(32, std::max<uint32_t>(1, (target + stages * stride_b - 1) / (stages * stride_b)));
-  const size_t smem = dispatch_smem(H, K);
-  if (smem > 200 * 1024) return EP_ERR_ARG;
+  const size_t need = dispatch_smem(H, K);
+  if (need > 200 * 1024) return EP_ERR_ARG;
+  // the same rows in flight per SM as per_sm CTAs of `stages` rows each: a CTA
+  // holds DISPATCH_TOKENS_PER_CTA rows, so per_sm * stages / that many CTAs
+  // may be resident; the shared memory each reserves caps them (228 KB per SM,
+  // 1 KB of it per CTA; at most 32 CTAs)
+  static_assert(DISPATCH_TOKENS_PER_CTA <= 2, "stages (2 or 4) must cover a CTA's tokens");
+  const int resident = std::min(32, per_sm * stages / DISPATCH_TOKENS_PER_CTA);
+  const size_t smem = std::max(need, (size_t)(220 * 1024) / resident);
   const void* fn = peers ? (const void*)k_dispatch<true> : (const void*)k_dispatch<false>;
   if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EP_ERR_CUDA;
-  const int grid = occupancy_grid(fn, 32, smem, T, per_sm);
+  const int64_t blocks = (T + DISPATCH_TOKENS_PER_CTA - 1) / DISPATCH_TOKENS_PER_CTA;
+  if (blocks > 0x7fffffff) return EP_ERR_ARG;
+  const int grid = (int)blocks;
   const uint8_t* xb = reinterpret_cast<const uint8_t*>(x);
   uint8_t* bb = reinterpret_cast<uint8_t*>(buf);
   void* args[] = {(void*)&xb,    (void*)&T,          (void*)&K, (void*)&row_bytes,     (void*)&pos,
@@ -504,7 +536,7 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
   if (!y || !pos || !out || !aligned16(y) || !aligned16(out)) return EP_ERR_ARG;  // w == NULL: unit weights
   const void* fn = combine_fn<false>(K);
   if (fn) {
-    const int grid = occupancy_grid(fn, 256, 0, T, 4);
+    const int grid = combine_grid(T, H);
     const uint64_t* peers = nullptr;
     const int32_t* rank_first = nullptr;
     int R = 1;
@@ -530,7 +562,7 @@ extern "C" int ep_combine_peer(const uint64_t* peer_bufs, const int32_t* rank_fi
   if (S == 0) return EP_OK;
   if (!peer_bufs || !pos_local || !out_local || !aligned16(out_local)) return EP_ERR_ARG;  // w NULL: unit weights
   const void* fn = combine_fn<true>(K);
-  const int grid = occupancy_grid(fn, 256, 0, S, 4);
+  const int grid = combine_grid(S, H);
   const uint16_t* y = nullptr;
   void* args[] = {(void*)&y,          (void*)&total_rows, (void*)&w_local,        (void*)&pos_local,
                   (void*)&S,          (void*)&H,          (void*)&out_local,      (void*)&peer_bufs,
