@@ -9,7 +9,8 @@
 //
 // Work = (replicated expert, 4096-element unit) items; the replicated experts
 // and each one's replica range come from the plan on the device (no host sync),
-// read once per unit into shared memory.  Each thread owns two 8-element
+// read into shared memory once per CTA (one-buffer form) or once per unit
+// (rank-local form, which also stages the unit's replica row addresses).  Each thread owns two 8-element
 // vectors of a unit and loads up to four replica vectors before adding them in
 // match order, so several 32-byte loads are in flight per thread.
 #include <algorithm>
@@ -91,6 +92,37 @@ __device__ __forceinline__ void reduce_vec8(float* __restrict__ home, const RowP
   *reinterpret_cast<float4*>(home + j + 4) = make_float4(a[4], a[5], a[6], a[7]);
 }
 
+// One unit (GRAD_UNIT elements from j0) of one replicated expert: home row
+// `home`, replicas m0 .. m0+mc-1 (rowp(m): replica m's row), in match order.
+template <bool BF16, bool CLEAR, class RowP>
+__device__ __forceinline__ void reduce_unit(float* __restrict__ home, const RowP& rowp, int64_t n, int64_t j0, int m0,
+                                            int mc, bool vec) {
+  if (vec) {
+#pragma unroll
+    for (int vv = 0; vv < GRAD_VECS; ++vv) {
+      const int64_t j = j0 + ((int64_t)vv * GRAD_THREADS + threadIdx.x) * 8;
+      if (j >= n) break;
+      reduce_vec8<BF16, CLEAR>(home, rowp, j, m0, mc);
+    }
+    return;
+  }
+  for (int64_t j = j0 + threadIdx.x; j < min(n, j0 + GRAD_UNIT); j += blockDim.x) {
+    float a = home[j];
+    for (int m = m0; m < m0 + mc; ++m) {
+      if (!BF16) {
+        float* r = reinterpret_cast<float*>(rowp(m)) + j;
+        a = __fadd_rn(a, *r);
+        if (CLEAR) *r = 0.0f;
+      } else {
+        uint16_t* r = reinterpret_cast<uint16_t*>(rowp(m)) + j;
+        a = __fadd_rn(a, bf16_bits_to_f32(*r));
+        if (CLEAR) *r = 0;
+      }
+    }
+    home[j] = a;
+  }
+}
+
 // PEER (rank-local form): only the experts homed on `rank` are reduced, into
 // g_home [E/R, n]; replica m's row is row m - rank_rep_first[d] of the buffer
 // at peers[d], d = rep_rank[m] (a rank's replicas are consecutive in match
@@ -107,78 +139,93 @@ __global__ void __launch_bounds__(GRAD_THREADS, 4)
   const int64_t units_per_expert = (n + GRAD_UNIT - 1) / GRAD_UNIT;
   const int64_t total = (int64_t)nC * units_per_expert;
   const bool vec = (n % 8) == 0;
-  for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
-    const int c = (int)(u / units_per_expert);
-    const int64_t j0 = (u - (int64_t)c * units_per_expert) * GRAD_UNIT;
-    __syncthreads();  // the previous unit is done with s_e, s_m0, s_mc
-    if (threadIdx.x == 0) {
+  if (!PEER && vec) {
+    // one-buffer form, rows of 8-element vectors: every replicated expert's
+    // (e, first replica, replica count) read once into shared memory, so a
+    // unit starts without a dependent plan lookup or a block barrier (on B200:
+    // 1% faster with fp32 replica rows, 4% with bf16 ones, than looking them
+    // up per unit)
+    __shared__ int s_tab[PEER ? 1 : 3 * EP_MAX_EXPERTS];
+    for (int c = threadIdx.x; c < nC; c += blockDim.x) {
       const int e = plan[L.rep_experts + c];
       int m0 = 0, mc = 0;
       if (e >= 0 && e < E) {
         m0 = plan[L.copy_first + e];
         mc = plan[L.copy_cnt + e];
       }
-      if (e < 0 || e >= E || m0 < 0 || mc < 0 || m0 + mc > L.cap || (PEER && mc > EP_MAX_RANKS)) {
-        flag(dev_status, EP_DEV_BAD_ROW);
-        s_e = -1;
-      } else if (PEER && e / ER != rank) {
-        s_e = -1;  // another rank's expert
-      } else {
-        s_e = e;
-        s_m0 = m0;
-        s_mc = mc;
-      }
+      const bool bad = e < 0 || e >= E || m0 < 0 || mc < 0 || m0 + mc > L.cap;
+      if (bad) flag(dev_status, EP_DEV_BAD_ROW);
+      s_tab[3 * c] = bad ? -1 : e;
+      s_tab[3 * c + 1] = m0;
+      s_tab[3 * c + 2] = mc;
     }
     __syncthreads();
-    const int e = s_e;
-    if (e < 0) continue;
-    const int m0 = s_m0, mc = s_mc;
     const int64_t esz = BF16 ? 2 : 4;
-    if (PEER) {
-      for (int q = threadIdx.x; q < mc; q += blockDim.x) {
-        const int m = m0 + q;
-        const int d = plan[L.rep_rank + m];
-        char* base = nullptr;
-        if (d >= 0 && d < R) {
-          const int64_t j = m - plan[L.rank_rep_first + d];
-          const uint64_t pb = __ldg(peers + d);
-          if (pb && !(pb & 15u) && j >= 0 && j < rep_rows) base = reinterpret_cast<char*>(pb) + j * n * esz;
-        }
-        if (!base) flag(dev_status, EP_DEV_BAD_ROW);
-        s_rows[PEER ? q : 0] = base;
-      }
-      __syncthreads();
-      bool ok = true;
-      for (int q = 0; q < mc; ++q) ok = ok && s_rows[PEER ? q : 0] != nullptr;
-      if (!ok) continue;  // every thread saw the same table: skip the unit together
-    }
-    auto rowp = [&](int m) -> char* {
-      return PEER ? s_rows[PEER ? m - m0 : 0] : static_cast<char*>(g_rep) + (int64_t)m * n * esz;
-    };
-    float* home = g_home + (int64_t)(PEER ? e - rank * ER : e) * n;
-    if (vec) {
+    auto rowp = [&](int m) -> char* { return static_cast<char*>(g_rep) + (int64_t)m * n * esz; };
+    for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+      const int c = (int)(u / units_per_expert);
+      const int64_t j0 = (u - (int64_t)c * units_per_expert) * GRAD_UNIT;
+      const int e = s_tab[3 * c];
+      if (e < 0) continue;
+      float* home = g_home + (int64_t)e * n;
+      const int m0 = s_tab[3 * c + 1], mc = s_tab[3 * c + 2];
 #pragma unroll
       for (int vv = 0; vv < GRAD_VECS; ++vv) {
         const int64_t j = j0 + ((int64_t)vv * GRAD_THREADS + threadIdx.x) * 8;
         if (j >= n) break;
         reduce_vec8<BF16, CLEAR>(home, rowp, j, m0, mc);
       }
-    } else {
-      for (int64_t j = j0 + threadIdx.x; j < min(n, j0 + GRAD_UNIT); j += blockDim.x) {
-        float a = home[j];
-        for (int m = m0; m < m0 + mc; ++m) {
-          if (!BF16) {
-            float* r = reinterpret_cast<float*>(rowp(m)) + j;
-            a = __fadd_rn(a, *r);
-            if (CLEAR) *r = 0.0f;
-          } else {
-            uint16_t* r = reinterpret_cast<uint16_t*>(rowp(m)) + j;
-            a = __fadd_rn(a, bf16_bits_to_f32(*r));
-            if (CLEAR) *r = 0;
-          }
+    }
+  } else {
+    for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+      const int c = (int)(u / units_per_expert);
+      const int64_t j0 = (u - (int64_t)c * units_per_expert) * GRAD_UNIT;
+      __syncthreads();  // the previous unit is done with s_e, s_m0, s_mc
+      if (threadIdx.x == 0) {
+        const int e = plan[L.rep_experts + c];
+        int m0 = 0, mc = 0;
+        if (e >= 0 && e < E) {
+          m0 = plan[L.copy_first + e];
+          mc = plan[L.copy_cnt + e];
         }
-        home[j] = a;
+        if (e < 0 || e >= E || m0 < 0 || mc < 0 || m0 + mc > L.cap || (PEER && mc > EP_MAX_RANKS)) {
+          flag(dev_status, EP_DEV_BAD_ROW);
+          s_e = -1;
+        } else if (PEER && e / ER != rank) {
+          s_e = -1;  // another rank's expert
+        } else {
+          s_e = e;
+          s_m0 = m0;
+          s_mc = mc;
+        }
       }
+      __syncthreads();
+      const int e = s_e;
+      if (e < 0) continue;
+      const int m0 = s_m0, mc = s_mc;
+      const int64_t esz = BF16 ? 2 : 4;
+      if (PEER) {
+        for (int q = threadIdx.x; q < mc; q += blockDim.x) {
+          const int m = m0 + q;
+          const int d = plan[L.rep_rank + m];
+          char* base = nullptr;
+          if (d >= 0 && d < R) {
+            const int64_t j = m - plan[L.rank_rep_first + d];
+            const uint64_t pb = __ldg(peers + d);
+            if (pb && !(pb & 15u) && j >= 0 && j < rep_rows) base = reinterpret_cast<char*>(pb) + j * n * esz;
+          }
+          if (!base) flag(dev_status, EP_DEV_BAD_ROW);
+          s_rows[PEER ? q : 0] = base;
+        }
+        __syncthreads();
+        bool ok = true;
+        for (int q = 0; q < mc; ++q) ok = ok && s_rows[PEER ? q : 0] != nullptr;
+        if (!ok) continue;  // every thread saw the same table: skip the unit together
+      }
+      auto rowp = [&](int m) -> char* {
+        return PEER ? s_rows[PEER ? m - m0 : 0] : static_cast<char*>(g_rep) + (int64_t)m * n * esz;
+      };
+      reduce_unit<BF16, CLEAR>(g_home + (int64_t)(PEER ? e - rank * ER : e) * n, rowp, n, j0, m0, mc, vec);
     }
   }
 }
