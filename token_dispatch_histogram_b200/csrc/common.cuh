@@ -20,6 +20,24 @@ inline int launch_status() { return cudaGetLastError() == cudaSuccess ? EP_OK : 
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch with programmatic dependent launch allowed: the kernel may be
+// scheduled while its predecessor in the stream finishes, and must call
+// wait_for_predecessor() before touching memory the predecessor writes or
+// reads (the row movers do so first thing).
+inline cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, void** args, size_t smem, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 int num_sms();  // cached per device
 
 // Pairs per tile of the histogram / rank scatter passes.  The largest of
@@ -154,6 +172,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+
+// Block until the preceding kernel in the stream has completed and its memory
+// is visible (a no-op for a kernel not launched by launch_pdl).
+__device__ __forceinline__ void wait_for_predecessor() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Wait (bounded by WAIT_LIMIT_NS) for phase `parity` of an mbarrier.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {

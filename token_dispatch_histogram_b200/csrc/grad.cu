@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(GRAD_THREADS, 4)
                   int32_t* dev_status) {
   __shared__ int s_e, s_m0, s_mc;
   __shared__ char* s_rows[PEER ? EP_MAX_RANKS : 1];
+  wait_for_predecessor();
   const int ER = E / R;
   const int nC = min(max(plan[L.n_chunks], 0), E);
   const int64_t units_per_expert = (n + GRAD_UNIT - 1) / GRAD_UNIT;
@@ -278,7 +279,7 @@ static int run_grad_reduce(float* g_home, const void* g_rep, int rep_dtype, int6
   void* gr = const_cast<void*>(g_rep);
   void* args[] = {(void*)&g_home, (void*)&gr,    (void*)&n, (void*)&plan, (void*)&L,         (void*)&E,
                   (void*)&peers,  (void*)&R,     (void*)&rank, (void*)&rep_rows, (void*)&dev_status};
-  if (cudaLaunchKernel(fn, dim3(grid), dim3(GRAD_THREADS), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (launch_pdl(fn, dim3(grid), dim3(GRAD_THREADS), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }

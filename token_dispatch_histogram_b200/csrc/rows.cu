@@ -50,6 +50,7 @@ __global__ void __launch_bounds__(32)
                const int32_t* __restrict__ rank_first, int R, int64_t rows_per_rank, int stages,
                int32_t* dev_status) {
   extern __shared__ __align__(128) uint8_t smem[];
+  wait_for_predecessor();
   const uint32_t stride_b = (row_bytes + 127u) & ~127u;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stride_b);
   int32_t* ring = reinterpret_cast<int32_t*>(bars + DISPATCH_MAX_STAGES);  // [stages][K] destination rows
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(256, 4)
               const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ out,
               const uint64_t* __restrict__ peers, const int32_t* __restrict__ rank_first, int R,
               int64_t rows_per_rank, int32_t* dev_status) {
+  wait_for_predecessor();
   constexpr int MAXT = 8;  // tokens per CTA iteration (rows narrower than 256 vectors)
   __shared__ int32_t s_rows[2][MAXT][K];
   __shared__ float s_w[2][MAXT][K];
@@ -466,7 +468,7 @@ static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const in
   void* args[] = {(void*)&xb,    (void*)&T,          (void*)&K, (void*)&row_bytes,     (void*)&pos,
                   (void*)&buf_rows, (void*)&bb,      (void*)&peers, (void*)&rank_first, (void*)&R,
                   (void*)&rows_per_rank, (void*)&stages, (void*)&dev_status};
-  if (cudaLaunchKernel(fn, dim3(grid), dim3(32), args, smem, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (launch_pdl(fn, dim3(grid), dim3(32), args, smem, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }
@@ -543,7 +545,7 @@ extern "C" int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, con
     int64_t rpr = 0;
     void* args[] = {(void*)&y,     (void*)&y_rows,     (void*)&w, (void*)&pos, (void*)&T,          (void*)&H,
                     (void*)&out,   (void*)&peers, (void*)&rank_first, (void*)&R, (void*)&rpr, (void*)&dev_status};
-    if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+    if (launch_pdl(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   } else {
     const int grid = occupancy_grid((const void*)k_combine_any, 256, 0, T * (H / 8) / 256 + 1, 8);
     k_combine_any<<<grid, 256, 0, stream>>>(y, y_rows, w, pos, T, K, H, out, dev_status);
@@ -567,7 +569,7 @@ extern "C" int ep_combine_peer(const uint64_t* peer_bufs, const int32_t* rank_fi
   void* args[] = {(void*)&y,          (void*)&total_rows, (void*)&w_local,        (void*)&pos_local,
                   (void*)&S,          (void*)&H,          (void*)&out_local,      (void*)&peer_bufs,
                   (void*)&rank_first_row, (void*)&R,      (void*)&rows_per_rank,  (void*)&dev_status};
-  if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (launch_pdl(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }
