@@ -48,10 +48,11 @@
  *    are then defined but unspecified, and no write goes out of bounds.
  *  - Limits: 1 <= K <= min(E, 32), E <= EP_MAX_EXPERTS, R <= EP_MAX_RANKS,
  *    E % R == 0, H % 8 == 0, P < 2^31.
- *  - Dispatch, combine (and their backward of dispatch) and the replica
- *    gradient reduction are launched with programmatic dependent launch: the
- *    GPU may schedule them while the preceding kernel in the stream finishes,
- *    and each waits for that kernel's completion before touching memory, so
+ *  - The row movers (dispatch; combine, which also serves as the backward of
+ *    dispatch; the replica gradient reduction; one-buffer and rank-local
+ *    forms) are launched with programmatic dependent launch: the GPU may
+ *    schedule them while the preceding kernel in the stream finishes, and
+ *    each waits for that kernel's completion before touching memory, so
  *    stream order holds as for any launch.
  *  - A workspace (ws) holds the counters and grid-barrier words of the call
  *    that uses it: calls in flight at the same time (on different streams)
