@@ -310,7 +310,7 @@ template <int K>
 __global__ void __launch_bounds__(256, 2)
     k_combine_bwd(const uint16_t* __restrict__ dout, const float* __restrict__ w, const uint16_t* __restrict__ y,
                   int64_t y_rows, const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ dy,
-                  float* __restrict__ dw, int32_t* dev_status) {
+                  float* __restrict__ dw, int64_t iters, int32_t* dev_status) {
   const int64_t nvec = H / 8;
   const int G = nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : (int)nvec);
   const int lane = threadIdx.x & 31;
@@ -330,15 +330,19 @@ __global__ void __launch_bounds__(256, 2)
       }
     }
   };
-  int64_t tb = warp_id * gpw;
+  // iters > 0: each warp owns `iters` consecutive groups of tokens (a
+  // non-persistent grid); else a persistent grid-stride loop
+  const int64_t tstep = iters > 0 ? gpw : nwarps * gpw;
+  int64_t tb = iters > 0 ? warp_id * gpw * iters : warp_id * gpw;
+  const int64_t tend = iters > 0 ? min(T, tb + gpw * iters) : T;
   int32_t r[K];
   float wk[K];
   rows_of(tb + sub, r, wk);
-  for (; tb < T; tb += nwarps * gpw) {
+  for (; tb < tend; tb += tstep) {
     const int64_t t = tb + sub;
     int32_t rn[K];
     float wn[K];
-    rows_of(tb + nwarps * gpw + sub, rn, wn);  // the next token's, ahead of use
+    rows_of(tb + tstep + sub, rn, wn);  // the next token's, ahead of use
 #pragma unroll
     for (int k = 0; k < K; ++k)
       if (t < T && (r[k] < 0 || r[k] >= y_rows)) {
@@ -602,9 +606,13 @@ extern "C" int ep_combine_backward(const uint16_t* dout, const float* w, const u
   const int64_t nvec = H / 8;
   const int64_t G = nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : nvec);
   const int64_t ctas = (T + 8 * (32 / G) - 1) / (8 * (32 / G));
-  const int grid = occupancy_grid(fn, 256, 0, ctas, 2);
+  // Measured on B200: a persistent grid is fastest at 0.9 GB of rows (2% ahead
+  // of short CTAs), CTAs of two token groups per warp at 17-19 GB (4% ahead).
+  const int64_t iters = T * H >= ((int64_t)1 << 28) ? 2 : 0;
+  const int grid = iters > 0 ? (int)std::min<int64_t>((ctas + iters - 1) / iters, 0x7fffffff)
+                             : occupancy_grid(fn, 256, 0, ctas, 2);
   void* args[] = {(void*)&dout, (void*)&w, (void*)&y, (void*)&y_rows, (void*)&pos, (void*)&T, (void*)&H, (void*)&dy,
-                  (void*)&dw, (void*)&dev_status};
+                  (void*)&dw, (void*)&iters, (void*)&dev_status};
   if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
