@@ -1,6 +1,8 @@
 // Library-wide entry points of libep.so: version, launch counter, status read,
 // and the per-device SM count used to size persistent grids.
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 
@@ -20,6 +22,23 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, never lowering it: two host threads launching the same
+// kernel with different sizes cannot undo each other's setting between a
+// set and a launch.
+bool raise_smem_limit(const void* fn, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> limits;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& cur = limits[std::make_pair(dev, fn)];
+  if (bytes <= cur) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
+  cur = bytes;
+  return true;
 }
 
 }  // namespace ep

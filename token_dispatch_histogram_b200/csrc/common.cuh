@@ -39,6 +39,7 @@ inline cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, void** args
 }
 
 int num_sms();  // cached per device
+bool raise_smem_limit(const void* fn, size_t bytes);  // never lowers; thread-safe
 
 // Pairs per tile of the histogram / rank scatter passes.  The largest of
 // 2048, 4096, 8192 that still gives two tiles per SM (so small problems spread

@@ -180,7 +180,7 @@ static int run_layout(const int32_t* topk, int64_t P, int E, int tile, int64_t n
                       cudaStream_t stream) {
   const size_t smem = scatter_smem_base(tile, E) + sizeof(int32_t) * (5 * (size_t)E + 3 * (size_t)L.cap);
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_layout, smem))
     return EP_ERR_CUDA;
   k_layout<<<(unsigned)nt, SCAT_THREADS, smem, stream>>>(topk, P, E, tile, tile_excl, base_counts, base_rank,
                                                          rows_total, plan, L, pos, src, pair_slot, dev_status);
@@ -256,7 +256,7 @@ extern "C" int ep_align_sort(const int32_t* topk_ids, int64_t T, int K, int E, i
   int grid = (int)std::max<int64_t>(nt, 2 * num_sms());
   const size_t smem = scatter_smem_base(tile, E) + sizeof(int32_t) * (2 * (size_t)E + 1);
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_align_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_align_scatter, smem))
     return EP_ERR_CUDA;
   k_align_scatter<<<grid, SCAT_THREADS, smem, stream>>>(topk_ids, P, E, tile,
                                                         reinterpret_cast<const int32_t*>(w + wl.excl_off), counts,

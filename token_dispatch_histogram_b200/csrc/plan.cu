@@ -156,7 +156,7 @@ extern "C" int ep_plan(const int32_t* loads, int R, int64_t S, int K, int E, int
   if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
   const size_t smem = plan_smem_bytes(E, R);  // <= 61 KB at the limits
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_plan, smem))
     return EP_ERR_CUDA;
   k_plan<<<1, PLAN_THREADS, smem, stream>>>(loads, R, (int32_t)(S * K), E, plan, L, dev_status);
   count_launch();
@@ -173,7 +173,7 @@ extern "C" int ep_plan_from_counts(const int32_t* counts, int R, int64_t S, int 
   if ((int64_t)plan_words < L.words) return EP_ERR_CAPACITY;
   const size_t smem = plan_smem_bytes(E, R);
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_plan_counts, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_plan_counts, smem))
     return EP_ERR_CUDA;
   k_plan_counts<<<1, PLAN_THREADS, smem, stream>>>(counts, R, (int32_t)(S * K), E, loads, plan, L, dev_status);
   count_launch();

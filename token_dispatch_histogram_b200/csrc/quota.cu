@@ -876,7 +876,7 @@ static bool q_fused_launch(const int32_t* topk, int64_t SK, int E, int R, int B,
     const size_t smem = std::max(base, q_layout_smem((int)tile, E, L.cap));
     if (smem > 227 * 1024) continue;
     if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(k_q_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        !raise_smem_limit((const void*)k_q_fused, smem))
       continue;
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_q_fused, SCAT_THREADS, smem) != cudaSuccess ||
@@ -940,7 +940,7 @@ static int run_q_layout(const int32_t* topk, int64_t SK, int E, int R, int tile,
                         cudaStream_t stream) {
   const size_t smem = q_layout_smem(tile, E, L.cap);
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_q_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_q_layout, smem))
     return EP_ERR_CUDA;
   k_q_layout<<<(unsigned)ntiles, SCAT_THREADS, smem, stream>>>(topk, SK, E, R, tile, tpr, excl, base_counts,
                                                                base_rank, plan, L, pos, src, dev_status);
@@ -991,7 +991,7 @@ extern "C" int ep_quota_route(const int32_t* topk_ids, int64_t T, int K, int E, 
   k_q_scan<<<(E + Q_SCAN_EXPERTS - 1) / Q_SCAN_EXPERTS, Q_SCAN_THREADS, 0, stream>>>(cnt, q.ntiles, E, excl, loads);
   const size_t search_smem = q_search_smem(E, R);
   if (search_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_q_search, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)search_smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_q_search, search_smem))
     return EP_ERR_CUDA;
   k_q_search<<<2 * num_sms(), Q_SEARCH_THREADS, search_smem, stream>>>(loads, excl, q.tpr, E, R, B, P, hdr, plan, L);
   count_launch(3);
@@ -1027,7 +1027,7 @@ extern "C" int ep_quota_plan_from_counts(const int32_t* counts, int R, int64_t S
   k_q_counts_prefix<<<(E + 255) / 256, 256, 0, stream>>>(counts, R, E, pre, loads, hdr);
   const size_t search_smem = q_search_smem(E, R);
   if (search_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_q_search, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)search_smem) != cudaSuccess)
+      !raise_smem_limit((const void*)k_q_search, search_smem))
     return EP_ERR_CUDA;
   const int64_t P = (int64_t)R * S * K;
   k_q_search<<<2 * num_sms(), Q_SEARCH_THREADS, search_smem, stream>>>(loads, pre, 1, E, R, B, P, hdr, plan, L);

@@ -498,7 +498,7 @@ static int route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, 
   auto resident_ok = [&](int ps, size_t smem) {
     if (smem > 227 * 1024) return false;
     if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        !raise_smem_limit(fn, smem))
       return false;
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, FUSED_THREADS, smem) != cudaSuccess) return false;

@@ -462,7 +462,7 @@ static int run_dispatch(const uint16_t* x, int64_t T, int K, int64_t H, const in
   const int resident = std::min(32, per_sm * stages / DISPATCH_TOKENS_PER_CTA);
   const size_t smem = std::max(need, (size_t)(220 * 1024) / resident);
   const void* fn = peers ? (const void*)k_dispatch<true> : (const void*)k_dispatch<false>;
-  if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (smem > 48 * 1024 && !raise_smem_limit(fn, smem))
     return EP_ERR_CUDA;
   const int64_t blocks = (T + DISPATCH_TOKENS_PER_CTA - 1) / DISPATCH_TOKENS_PER_CTA;
   if (blocks > 0x7fffffff) return EP_ERR_ARG;
