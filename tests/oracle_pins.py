@@ -687,6 +687,77 @@ def pin_quota_invariants(L):
             assert rest.tolist() == mine
 
 
+def unit_quota_plan(loads, R, E, tau, B):
+    """Independent statement of the quota rule at threshold tau, one pair at a
+    time: every rank above tau lists its excess pairs (ranks ascending; within a
+    rank its home experts heaviest first, ties to the lower id, each giving up to
+    what is still in excess); the ranks below tau are rooms (ascending) of
+    tau - H_r pairs and at most B pieces.  Each pair goes to the current room;
+    a pair that would open a new piece (another expert's chunk, or a new room)
+    moves on to the next room when the current one is full or holds B pieces.
+    Returns [expert, room rank, pairs] per piece in walk order, or None when
+    the rooms run out first."""
+    ER = E // R
+    H = [int(sum(int(loads[e]) for e in range(r * ER, (r + 1) * ER))) for r in range(R)]
+    units = []  # (chunk id, expert)
+    for r in range(R):
+        rem = H[r] - tau
+        if rem <= 0:
+            continue
+        for e in sorted(range(r * ER, (r + 1) * ER), key=lambda x: (-int(loads[x]), x)):
+            take = min(int(loads[e]), rem)
+            units += [((r, e), e)] * take
+            rem -= take
+            if rem == 0:
+                break
+    rooms = [r for r in range(R) if H[r] < tau]
+    j, left, pieces, reps, last = 0, (tau - H[rooms[0]] if rooms else 0), 0, [], None
+    for chunk, e in units:
+        new_piece = last != (chunk, j)
+        while j < len(rooms) and (left == 0 or (new_piece and pieces == B)):
+            j += 1
+            left = tau - H[rooms[j]] if j < len(rooms) else 0
+            pieces, new_piece = 0, True
+        if j >= len(rooms):
+            return None
+        if new_piece:
+            reps.append([e, rooms[j], 0])
+            pieces += 1
+        reps[-1][2] += 1
+        left -= 1
+        last = (chunk, j)
+    return reps
+
+
+def pin_quota_unit_restatement(L):
+    """The oracle's threshold and plan against unit_quota_plan: tau* is the
+    smallest tau from ceil(P/R) up at which every excess pair finds a room
+    (the largest H_r always does), and the replicas, in match order, and the
+    home quotas are those of the pair-by-pair walk at tau*."""
+    rng = np.random.default_rng(34)
+    for it in range(400):
+        R = int(rng.choice([1, 2, 3, 4, 5, 8]))
+        ER = int(rng.integers(1, 6))
+        E = R * ER
+        SK = int(rng.integers(1, 30))
+        loads = _rand_loads(rng, R, ER, SK) if it % 2 else rng.multinomial(
+            R * SK, rng.dirichlet(np.full(E, rng.uniform(0.1, 3.0)))).astype(np.int32)
+        P = R * SK
+        B = int(rng.choice([0, 1, 2, 3, E]))
+        H = loads.reshape(R, ER).sum(axis=1)
+        lo, hi = -(-P // R), max(-(-P // R), int(H.max()))
+        want_tau = next(t for t in range(lo, hi + 1) if t == hi or unit_quota_plan(loads, R, E, t, B) is not None)
+        qp = O.quota_plan(loads, R, SK, 1, E, B, L=L)
+        assert qp["tau"] == want_tau, (loads.tolist(), R, B, qp["tau"], want_tau)
+        want = unit_quota_plan(loads, R, E, want_tau, B) or []
+        got = [[int(a), int(b), int(c)] for a, b, c in zip(qp["rep_expert"], qp["rep_rank"], qp["rep_count"])]
+        assert got == want, (loads.tolist(), R, B, want_tau, got, want)
+        hq = loads.astype(np.int64).copy()
+        for e, _, c in want:
+            hq[e] -= c
+        assert qp["home_quota"].tolist() == hq.tolist()
+
+
 def pin_quota_no_replica_is_a_sort(L):
     """B = 0: no copy, so the layout is a stable sort by (expert, pair not from
     the expert's home rank) -- numpy's lexsort."""
@@ -709,4 +780,5 @@ def pin_quota_no_replica_is_a_sort(L):
 ALL_PINS = [pin_hand_example, pin_max_vio_closed_forms, pin_plan_unit_restatement, pin_layout_brute_force,
             pin_layout_library_reductions, pin_layout_invariants, pin_align_sort, pin_dispatch, pin_combine,
             pin_grad_reduce, pin_dispatch_backward, pin_combine_backward, pin_prefetch_slots, pin_quota_hand_example,
-            pin_quota_threshold_closed_forms, pin_quota_invariants, pin_quota_no_replica_is_a_sort]
+            pin_quota_threshold_closed_forms, pin_quota_invariants, pin_quota_no_replica_is_a_sort,
+            pin_quota_unit_restatement]

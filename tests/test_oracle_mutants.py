@@ -59,6 +59,10 @@ MUTANTS = [
     ("quota_descending_id_chunks", "if (!used[e] && (best < 0 || loads[e] > loads[best])) best = e;",
      "if (!used[e] && (best < 0 || e > best)) best = e;"),
     ("quota_no_slot_budget", "if (left_r == 0 || pieces == B) {", "if (left_r == 0) {"),
+    ("quota_rooms_descending", "  for (int r = 0; r < R; ++r) {\n    if (tau - H[r] > 0) {",
+     "  for (int r = R - 1; r >= 0; --r) {\n    if (tau - H[r] > 0) {"),
+    ("quota_pieces_not_reset", "      ++j;\n      pieces = 0;", "      ++j;\n      pieces = pieces;"),
+    ("quota_chunk_whole_expert", "int64_t take = loads[best] < rem ? loads[best] : rem;", "int64_t take = loads[best];"),
     ("quota_zero_rooms", "if (tau - H[r] > 0) {\n      rm_r[nrm] = r;", "if (tau - H[r] >= 0) {\n      rm_r[nrm] = r;"),
     ("quota_scan_from_above", "int64_t tau = (P + R - 1) / R;", "int64_t tau = (P + R - 1) / R + 1;"),
     ("quota_no_locality", "if (i >= 0 && ls < il[i]) {", "if (i >= 0 && ls < 0) {"),
