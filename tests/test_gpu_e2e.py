@@ -6,6 +6,7 @@ import pytest
 
 import oracle as O
 import workload as W
+from gpu_path import case_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -35,3 +36,28 @@ def test_run_host_matches_oracle(chunks):
     ref = O.combine(buf, w, lo["pos"], K)
     np.testing.assert_array_equal(out_h.view(torch.int16).numpy().view(np.uint16), ref)
     _ = (S, T)
+
+
+def test_overlapped_step_matches_the_sequential_one():
+    """EpLayer.step(overlap=True) runs the replica gradient reduction on a
+    second stream beside combine: the same outputs, bit for bit."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    R, S, K, E, H, n = 8, 300, 6, 64, 256, 4096 * 3 + 8
+    topk, w, x = case_inputs(R, S, K, E, H, seed=11, bias_scale=1.5)
+    lay = tdh.EpLayer(R, S, K, E, H, 16, device="cuda", grad_n=n)
+    lay.topk_ids.copy_(torch.from_numpy(topk))
+    lay.w.copy_(torch.from_numpy(w))
+    lay.x.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
+    g0 = torch.randn((E, n), device="cuda")
+    W.fill_device(lay.g_rep, 3, W.STREAM_GREP)
+    outs = []
+    for overlap in (False, True):
+        lay.g_home.copy_(g0)
+        lay.out.zero_()
+        lay.step(overlap=overlap)
+        torch.cuda.synchronize()
+        outs.append((lay.out.clone(), lay.g_home.clone()))
+    assert lay.status() == 0
+    assert int(lay.plan_view("n_rep", 1).item()) > 0
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])

