@@ -40,9 +40,11 @@ def test_algorithmic_bytes_of_the_moderate_workload():
     # the committed ncu traffic records use the same per-launch figures
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     rec = json.load(open(os.path.join(root, "profiles", "traffic.json")))
-    assert rec["k_dispatch"]["algorithmic_bytes_per_launch"] == ab["dispatch"]
-    assert rec["k_combine"]["algorithmic_bytes_per_launch"] == ab["combine"]
-    assert rec["k_grad_reduce"]["algorithmic_bytes_per_launch"] == ab["grad_reduce"]
+    assert rec["k_dispatch@moderate_ep8"]["algorithmic_bytes_per_launch"] == ab["dispatch"]
+    assert rec["k_combine@moderate_ep8"]["algorithmic_bytes_per_launch"] == ab["combine"]
+    assert rec["k_grad_reduce@moderate_ep8"]["algorithmic_bytes_per_launch"] == ab["grad_reduce"]
+    for k, r in rec.items():  # every record names the pairs of the launch it was captured on
+        assert k.split("@")[1] == r["workload"] and r["pairs_per_launch"] > 0
 
 
 def test_clock_sampler_parses_reasons_and_median():
@@ -59,15 +61,64 @@ def test_clock_sampler_parses_reasons_and_median():
 
 
 def test_traffic_record_only_for_the_captured_source(tmp_path, monkeypatch):
+    """A record is used only at the source it was captured on, and only for
+    its own workload shape, scaled by pairs per launch."""
     import bench
     src = tmp_path / "k.cu"
     src.write_text("kernel source\n")
     sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
     (tmp_path / "profiles").mkdir()
-    rec = {"k_x": {"dram_bytes_per_launch": 123, "source": "k.cu", "source_sha": sha}}
+    rec = {"k_x@fine": {"dram_bytes_per_launch": 1000, "source": "k.cu", "source_sha": sha, "capture": "cap",
+                        "pairs_per_launch": 100, "workload": "fine"}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.traffic_record("k_x")["dram_bytes_per_launch"] == 123
-    assert bench.traffic_record("k_y") is None
+    got = bench.traffic_record("k_x", {"name": "fine", "P": 1600})
+    assert got["dram_bytes_per_launch"] == 16000 and got["scaled_by"] == 16.0
+    assert bench.traffic_record("k_x", {"name": "other", "P": 1600}) is None
+    assert bench.traffic_record("k_y", {"name": "fine", "P": 1600}) is None
     src.write_text("kernel source, changed\n")
-    assert bench.traffic_record("k_x") is None
+    assert bench.traffic_record("k_x", {"name": "fine", "P": 1600}) is None
+
+
+def test_both_arms_print_the_same_config():
+    """The reference arm and ours describe the workload with one function of
+    the workload alone (nothing about the timing method in it)."""
+    import bench
+    for cfg in (1, 2, 3, 4, 5):
+        c = bench.workload_shape(cfg)
+        a, b = bench.config_obj(c), bench.config_obj(bench.workload_shape(cfg))
+        assert a == b and "l2" not in a
+        assert a["pairs_per_step"] == c["P"] * c["layers"]
+    c4 = bench.workload_shape(4)
+    assert (c4["R"], c4["S"], c4["E"], c4["K"], c4["H"], c4["layers"]) == (64, 8192, 384, 8, 7168, 8)
+    assert bench.parse([]).config == 4          # the largest single-GPU workload is the default
+
+
+def test_smaller_case_overrides():
+    import bench
+    c = bench.workload_shape(4, tokens_per_rank=512, layers=1)
+    assert (c["S"], c["T"], c["P"], c["layers"]) == (512, 64 * 512, 64 * 512 * 8, 1)
+    assert c["name"] == "fine_grained_ep64_8layers"
+
+
+def test_oracle_sample_extrapolation():
+    """The CPU baseline's layer time: the route ran over the whole layer, the
+    rows over Ts tokens, the gradients over nc columns; each phase's time per
+    unit times the layer's units."""
+    import bench
+    c = bench.workload_shape(3)
+    Ts, nc = bench.sample_tokens(c), bench.sample_cols(c)
+    assert Ts * c["K"] * c["H"] <= (1 << 28) < (Ts + 1) * c["K"] * c["H"]
+    assert nc == 1 << 22
+    s = bench.layer_seconds(c, 0.5, 2.0, 1.0, Ts, nc)
+    assert s == pytest.approx(0.5 + 2.0 * c["T"] / Ts + 1.0 * c["grad_n"] / nc)
+    c1 = bench.workload_shape(1)
+    assert bench.sample_tokens(c1) == c1["T"] and bench.sample_cols(c1) == c1["grad_n"]
+    assert bench.layer_seconds(c1, 0.5, 2.0, 1.0, c1["T"], c1["grad_n"]) == pytest.approx(3.5)
+
+
+def test_side_measurement_replays():
+    import bench
+    assert bench.side_steps(20, 0.4) == 20          # short steps: all of them
+    assert bench.side_steps(20, 163.0) == 15        # 2.5 s of replays
+    assert bench.side_steps(20, 5000.0) == 3        # at least three

@@ -101,16 +101,16 @@ def _ptr(a):
     return ctypes.c_void_p(a.ctypes.data)
 
 
-def normal_f32(seed, stream, offset, n):
+def normal_f32(seed, stream, offset, n, threads=None):
     out = np.empty(n, dtype=np.float32)
-    lib().gen_fill_normal_f32(seed, stream, offset, n, _ptr(out), nthreads())
+    lib().gen_fill_normal_f32(seed, stream, offset, n, _ptr(out), threads or nthreads())
     return out
 
 
-def normal_bf16(seed, stream, offset, n):
+def normal_bf16(seed, stream, offset, n, threads=None):
     """bf16 bit patterns (uint16)."""
     out = np.empty(n, dtype=np.uint16)
-    lib().gen_fill_normal_bf16(seed, stream, offset, n, _ptr(out), nthreads())
+    lib().gen_fill_normal_bf16(seed, stream, offset, n, _ptr(out), threads or nthreads())
     return out
 
 
@@ -165,9 +165,9 @@ def routing_from(T, E, K, seed, bias_e=None, stream=STREAM_LOGITS, uniform=False
     return topk, w
 
 
-def hidden(T, H, seed, layer=0, t0=0):
+def hidden(T, H, seed, layer=0, t0=0, threads=None):
     """x rows [t0, t0+T) of a [*, H] bf16 hidden matrix, as uint16 bits."""
-    return normal_bf16(seed, STREAM_X + layer, t0 * H, T * H).reshape(T, H)
+    return normal_bf16(seed, STREAM_X + layer, t0 * H, T * H, threads).reshape(T, H)
 
 
 def hidden_rows(H, seed, layer, tokens):
