@@ -73,6 +73,8 @@ def parse(argv=None):
     ap.add_argument("--tokens-per-rank", type=int, default=None,
                     help="override S (a smaller case of the same shape, e.g. for a profiler capture)")
     ap.add_argument("--layers", type=int, default=None, help="override the number of layers per step")
+    ap.add_argument("--hidden", type=int, default=None,
+                    help="override H (e.g. a full-size route with small rows, for a profiler capture of the route)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the backward of dispatch and combine")
@@ -92,7 +94,7 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
-def workload_shape(cfg, tokens_per_rank=None, layers=None):
+def workload_shape(cfg, tokens_per_rank=None, layers=None, hidden=None):
     """The workload's shape dict, with the optional smaller-case overrides."""
     import workload as W
     c = dict(W.CONFIGS[cfg])
@@ -100,6 +102,8 @@ def workload_shape(cfg, tokens_per_rank=None, layers=None):
         c["S"] = int(tokens_per_rank)
     if layers:
         c["layers"] = int(layers)
+    if hidden:
+        c["H"] = int(hidden)
     c = W.shape(c)
     c["cfg"] = cfg
     return c
@@ -270,7 +274,8 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     over = cfg == args.config
-    c = workload_shape(cfg, args.tokens_per_rank if over else None, args.layers if over else None)
+    c = workload_shape(cfg, args.tokens_per_rank if over else None, args.layers if over else None,
+                       args.hidden if over else None)
     seed = rank_seed(args.seed, rank)
     R, S, E, K, H, T, P = c["R"], c["S"], c["E"], c["K"], c["H"], c["T"], c["P"]
     nl = c["layers"]
@@ -439,7 +444,8 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
 
     # ---- backward of combine and of dispatch (timed apart from the step)
     backward = None
-    if side and not args.no_backward and 2 * P * H <= (20 << 30):
+    bwd_bytes = 2 * P * H + 2 * T * H + 4 * T * K  # dy, dx, dw
+    if not args.no_graph and not args.no_backward and bwd_bytes + (2 << 30) <= torch.cuda.mem_get_info(dev)[0]:
         dy = torch.empty_like(layer.buf)
         dx = torch.empty_like(layer.x)
         dw = torch.empty((T, K), dtype=torch.float32, device=dev)
@@ -776,9 +782,10 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
                     "max_replicas_per_rank": max_rep_rank[0] if one else max_rep_rank},
         "layers_per_step": nl,
         "route_path": args.route,
+        "backward": backward,
     }
     if full:
-        res.update({"backward": backward, "prefetch_slots": prefetch, "quota_planner": quota,
+        res.update({"prefetch_slots": prefetch, "quota_planner": quota,
                     "plan_dispatch_combine": as_named, "route_dispatch": route_dispatch, "rank_local": rank_local})
     del layers, layer, flush
     torch.cuda.synchronize()
@@ -803,7 +810,7 @@ def run_rank_local(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    c = workload_shape(args.config, args.tokens_per_rank, args.layers)
+    c = workload_shape(args.config, args.tokens_per_rank, args.layers, args.hidden)
     R, S, E, K, H, T, P = c["R"], c["S"], c["E"], c["K"], c["H"], c["T"], c["P"]
     nl = c["layers"]
     if R % world:
@@ -873,8 +880,9 @@ def run_rank_local(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Philox4x32-10 router logits with a per-workload expert bias, hidden rows ~ normal)",
-        "config": config_obj(c), "l2": L2_NOTE, "form": f"rank-local: {R} ranks over {world} processes, "
-                                                         f"{R // world} per GPU, peers by CUDA IPC",
+        "config": config_obj(c), "l2": L2_NOTE,
+        "form": f"rank-local: {R} ranks over {world} processes, {R // world} per GPU, "
+                + ("other processes' buffers mapped by CUDA IPC" if world > 1 else "every peer buffer local"),
         "e2e": None, "gpu_launches": int(launches), "clocks": clk,
         "timing": "CUDA events around each eager step (host fences inside), max over ranks",
     }
@@ -887,7 +895,7 @@ def workload_summary(res):
     """The keys of a non-headline workload's result kept in the JSON line."""
     keep = ("value", "unit", "ms_per_step", "step_ms_median", "step_ms_min", "steps", "dispatch_combine", "step_hbm",
             "roofline", "breakdown", "route_us_per_layer", "routing", "e2e", "clocks", "gpu_launches",
-            "layers_per_step")
+            "layers_per_step", "backward")
     out = {k: res[k] for k in keep if k in res}
     out["workload"] = res["config"]["workload"]
     return out
@@ -1012,7 +1020,7 @@ def cpu_model():
 
 def run_reference(args):
     import workload as W
-    c = workload_shape(args.config, args.tokens_per_rank, args.layers)
+    c = workload_shape(args.config, args.tokens_per_rank, args.layers, args.hidden)
     nl = c["layers"]
     routes = [W.routing(c, args.seed, i) for i in range(nl)]
     time_oracle(c, args.seed, routes, args.warmup)

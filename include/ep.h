@@ -16,7 +16,9 @@
  *       a searched load threshold with at most B replicas per rank)
  *   rank-local form, one rank per process (ep_plan_from_counts,
  *       ep_layout_rank, ep_dispatch_peer, ep_combine_peer,
- *       ep_replica_grad_reduce_peer and their quota-planner counterparts)
+ *       ep_replica_grad_reduce_peer and their quota-planner counterparts;
+ *       ep_ipc_export / ep_ipc_open / ep_ipc_close map peer buffers across
+ *       processes)
  *   ep_route_stats_noalloc (ep_route_stats with the library's own scratch)
  *
  * Sources, cited by page title and section:
@@ -462,6 +464,32 @@ EP_API int ep_replica_grad_reduce(float* g_home, const void* g_rep, int rep_dtyp
  */
 
 /*
+ * Peer buffers across processes (host calls, no stream; set-up, not part of a
+ * step).  [GR] "Online planning, zero copy και στατικά σχήματα": a sending rank
+ * writes rows straight into the receiving rank's buffer, so that buffer must
+ * be mapped into the sender's address space.  With one process per rank this
+ * is done with CUDA IPC handles:
+ *   ep_ipc_export: dev_ptr (device, a buffer from cudaMalloc or a caching
+ *     allocator built on it; not VMM/cuMemMap memory) -> *handle (host,
+ *     EP_IPC_HANDLE_BYTES opaque bytes naming the allocation that holds
+ *     dev_ptr) and *offset (host, dev_ptr's byte offset in that allocation).
+ *   ep_ipc_open (in another process): *base = the allocation mapped here,
+ *     *dev_ptr = *base + offset, usable in a peer table.  Opening a handle
+ *     exported by the same process fails (EP_ERR_CUDA): a rank uses its own
+ *     pointer for itself.  Peer access to another GPU is enabled by the driver.
+ *   ep_ipc_close(base): unmaps (every process that opened a handle closes it
+ *     before the owner frees the buffer).
+ * Returns EP_OK, EP_ERR_ARG (null argument, or dev_ptr not device memory) or
+ * EP_ERR_CUDA.  The handles carry no synchronisation: the caller orders the
+ * ranks' kernels (e.g. every rank's dispatch done before any rank's combine).
+ */
+#define EP_IPC_HANDLE_BYTES 64
+EP_API int ep_ipc_export(const void* dev_ptr, void* handle /* host out */, uint64_t* offset /* host out */);
+EP_API int ep_ipc_open(const void* handle /* host */, uint64_t offset, void** base /* host out */,
+                       void** dev_ptr /* host out */);
+EP_API int ep_ipc_close(void* base);
+
+/*
  * The plan from the gathered load matrix: loads[e] = sum_r counts[r, e], then
  * exactly ep_plan.  counts [R, E] int32 device; loads [E] int32 out (device) or
  * NULL; plan as in ep_plan.  One CTA.
@@ -572,10 +600,13 @@ EP_API int ep_quota_replica_grad_reduce_peer(float* g_home_local, const uint64_t
  *   must fit: about 12 * ceil(T*K / tile) * E + 4*E + 512 bytes, tile = 2048,
  *   4096 or 8192 pairs (as ep_workspace_size reports for the same T, K, E);
  *   larger problems get EP_ERR_CAPACITY and nothing is enqueued.
- *   The first call on a device (with that device current) looks the array's
- *   device address up with cudaGetSymbolAddress; make that first call before
- *   any stream capture.  No call allocates (no cudaMalloc, cudaFree or
- *   allocating library routine).
+ *   The first call in a CUDA context (with that context's device current)
+ *   looks the array's device address up with cudaGetSymbolAddress and caches
+ *   it with the context's unique id; a later call under a different context of
+ *   the same device (after cudaDeviceReset, or a context the caller created)
+ *   looks it up again.  Make the first call in each context before any stream
+ *   capture.  No call allocates (no cudaMalloc, cudaFree or allocating library
+ *   routine).
  *   All calls share the one array and it keeps the previous call's contents:
  *   calls whose work overlaps on the GPU (other streams, other threads) race
  *   on it and must be serialised by the caller.  ep_layout cannot use this

@@ -1,22 +1,35 @@
 """Parity at the full workload sizes (-m gpu), in the launch configuration the
-benchmark uses (the same binding and EpLayer buffers).
+benchmark uses (the same binding and EpLayer buffers), every output compared
+in full:
 
   * loads, max_vio, plan, layout (pos, src, pair_slot), cu_seqlens, align-sort:
-    compared in full, bit-exact, against the CPU oracle;
-  * dispatch: sampled buffer rows (every slot's first and last row plus random
-    rows) must equal the hidden row of their pair's token, bitwise, with x
-    regenerated on the host from the counter-based generator;
-  * combine (after the stand-in expert): sampled tokens against the layout-free
-    closed form, within 1 bf16 ulp (and checked identical);
-  * replica gradient reduction: sampled columns of every expert row, fp32 adds
-    in match order, within 1e-6 relative (and checked identical).
+    bit-exact against the CPU oracle;
+  * dispatch: every row of the dispatch buffer, bitwise.  The tokens are taken
+    in chunks; a chunk's rows are gathered from the device buffer in row order
+    and compared with the oracle's dispatch of that chunk (its hidden rows
+    regenerated on the host from the counter-based generator, its pairs placed
+    at their rank among the chunk's rows), so the whole buffer is covered
+    without a host copy of it;
+  * combine (after the stand-in expert): every output token against the
+    oracle's layout-free closed form, within 1 bf16 ulp (and checked
+    identical);
+  * replica gradient reduction: every element of every replicated expert's
+    home row against the oracle's reduction (fp32 adds in match order), within
+    1e-6 relative (and checked identical); every other home row unchanged.
+
+The host checks of a chunk run on a thread pool (the oracle and the generator
+are C calls that release the interpreter lock; each oracle call is still one
+single-threaded pass over its chunk).
 
 Workloads: moderate EP8 (R=8, S=4096, E=64, K=6, H=2048), DeepSeek-V3-shaped
 (R=32, S=4096, E=256, K=8, H=7168, bf16 replica grads), fine-grained 8-layer
-(R=64, S=8192, E=384, K=8, H=7168, bias redrawn per layer), adversarial
-prefill (R=16, S=16384, E=256, K=8, H=4096) with its uniform and single-expert
-companions.
+(R=64, S=8192, E=384, K=8, H=7168, bias redrawn per layer; rows of layers 0
+and 7), adversarial prefill (R=16, S=16384, E=256, K=8, H=4096) with its
+uniform and single-expert companions.
 """
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 
@@ -25,6 +38,9 @@ import workload as W
 from gpu_path import bf16_ulp_diff
 
 pytestmark = pytest.mark.gpu
+
+WORKERS = max(2, min(32, os.cpu_count() or 2))
+CHUNK_ELEMS = 1 << 26  # row elements per checked chunk (128 MB of bf16 rows)
 
 
 def _layer(c, dev, grads=False):
@@ -59,27 +75,62 @@ def _check_route(layer, c, topk):
     return pl, lo, mv
 
 
-def _check_rows(layer, c, topk, w, lo, seed, layer_id, rng):
+def _token_chunks(c):
+    ch = max(1, min(c["T"], CHUNK_ELEMS // (c["K"] * c["H"])))
+    return [(t0, min(c["T"], t0 + ch)) for t0 in range(0, c["T"], ch)]
+
+
+def _drain(futs, keep):
+    """Wait until at most `keep` checks are in flight; raise the first failure."""
+    while len(futs) > keep:
+        futs.pop(0).result()
+
+
+def _dispatch_chunk_ok(got, local, t0, t1, seed, layer_id, K, H):
+    x = W.hidden(t1 - t0, H, seed, layer_id, t0, threads=1)
+    want = O.dispatch(x, local, K, local.size)
+    assert np.array_equal(got, want), f"dispatch rows of tokens [{t0}, {t1}) differ"
+
+
+def _combine_chunk_ok(got, t0, t1, seed, layer_id, H, w, topk, scale):
+    x = W.hidden(t1 - t0, H, seed, layer_id, t0, threads=1)
+    want = O.combine_closed(x, w[t0:t1], topk[t0:t1], scale)
+    ulp = bf16_ulp_diff(got, want)
+    assert ulp.max() <= 1, f"combine of tokens [{t0}, {t1}): {ulp.max()} ulp"
+    assert np.count_nonzero(ulp) == 0, f"combine of tokens [{t0}, {t1}) not identical"
+
+
+def _check_rows(layer, c, topk, w, lo, seed, layer_id):
     import torch
     K, H, T, P = c["K"], c["H"], c["T"], c["P"]
-    cu = lo["cu_seqlens"].astype(np.int64)
-    edge = np.concatenate([cu[:-1][np.diff(cu) > 0], cu[1:][np.diff(cu) > 0] - 1])
-    rows = np.unique(np.concatenate([edge, rng.integers(0, P, 2048)]))
-    src = lo["src"].astype(np.int64)
-    toks = src[rows] // K
-    got = layer.buf.index_select(0, torch.from_numpy(rows).to(layer.buf.device)).view(torch.int16).cpu().numpy()
-    want = W.hidden_rows(H, seed, layer_id, toks)
-    assert np.array_equal(got.view(np.uint16), want), "dispatch rows differ"
-    # stand-in expert, then combine; sampled tokens against the closed form
+    dev = layer.buf.device
+    pos = lo["pos"].astype(np.int64)
+    covered = np.zeros(P, dtype=bool)
+    with ThreadPoolExecutor(WORKERS) as ex:
+        futs = []
+        for t0, t1 in _token_chunks(c):
+            pc = pos[t0 * K:t1 * K]
+            order = np.argsort(pc, kind="stable")
+            rows = pc[order]
+            local = np.empty(pc.size, dtype=np.int32)
+            local[order] = np.arange(pc.size, dtype=np.int32)  # the pair's rank among the chunk's rows
+            covered[rows] = True
+            got = layer.buf.index_select(0, torch.from_numpy(rows).to(dev)).view(torch.int16).cpu().numpy()
+            futs.append(ex.submit(_dispatch_chunk_ok, got.view(np.uint16), local, t0, t1, seed, layer_id, K, H))
+            _drain(futs, 2 * WORKERS)
+        _drain(futs, 0)
+    assert covered.all(), "some buffer rows belong to no pair"
+    # stand-in expert, then combine; every token against the closed form
     scale = W.expert_scale(c["E"])
-    layer.expert_standin(torch.from_numpy(scale).to(layer.buf.device))
+    layer.expert_standin(torch.from_numpy(scale).to(dev))
     layer.combine()
-    tok = np.unique(np.concatenate([rng.integers(0, T, 1024), toks[:512], [0, T - 1]]))
-    got = layer.out.index_select(0, torch.from_numpy(tok).to(layer.out.device)).view(torch.int16).cpu().numpy()
-    want = O.combine_closed(W.hidden_rows(H, seed, layer_id, tok), w[tok], topk[tok], scale)
-    ulp = bf16_ulp_diff(got.view(np.uint16), want)
-    assert ulp.max() <= 1
-    assert np.count_nonzero(ulp) == 0
+    with ThreadPoolExecutor(WORKERS) as ex:
+        futs = []
+        for t0, t1 in _token_chunks(c):
+            got = layer.out[t0:t1].view(torch.int16).cpu().numpy().view(np.uint16)
+            futs.append(ex.submit(_combine_chunk_ok, got, t0, t1, seed, layer_id, H, w, topk, scale))
+            _drain(futs, 2 * WORKERS)
+        _drain(futs, 0)
 
 
 def _run_layer(cfg, seed, layer_id=0, variant="default", rows=True, grads=False, fused=True):
@@ -98,9 +149,24 @@ def _run_layer(cfg, seed, layer_id=0, variant="default", rows=True, grads=False,
     assert layer.status() == 0
     pl, lo, mv = _check_route(layer, c, topk)
     if rows:
-        _check_rows(layer, c, topk, w, lo, seed, layer_id, np.random.default_rng(seed * 31 + layer_id))
+        _check_rows(layer, c, topk, w, lo, seed, layer_id)
     assert layer.status() == 0
     return layer, c, pl, lo, mv
+
+
+def test_device_generator_matches_host():
+    """The full-size checks regenerate the device-filled inputs on the host:
+    both generators give the same bits (fp32 and bf16, at offsets that are not
+    multiples of the generator's four-value block)."""
+    import torch
+    t32 = torch.empty(100003, dtype=torch.float32, device="cuda")
+    t16 = torch.empty(100003, dtype=torch.bfloat16, device="cuda")
+    for off in (0, 1, 7, 123457):
+        W.fill_device(t32, 5, W.STREAM_GHOME, off)
+        W.fill_device(t16, 5, W.STREAM_X + 3, off)
+        assert np.array_equal(t32.cpu().numpy(), W.normal_f32(5, W.STREAM_GHOME, off, t32.numel()))
+        assert np.array_equal(t16.view(torch.int16).cpu().numpy().view(np.uint16),
+                              W.normal_bf16(5, W.STREAM_X + 3, off, t16.numel()))
 
 
 @pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
@@ -129,28 +195,40 @@ def test_full_size_adversarial_companions():
     del layer
 
 
+def _grad_row_ok(got, e, ms, seed, n, dt):
+    home = W.normal_f32(seed, W.STREAM_GHOME, e * n, n, threads=1)[None]
+    gen = W.normal_f32 if dt == "f32" else W.normal_bf16
+    reps = np.stack([gen(seed, W.STREAM_GREP, int(m) * n, n, threads=1) for m in ms])
+    want, _ = O.grad_reduce(home, reps, np.zeros(len(ms), dtype=np.int32))  # home first, then match order
+    want = want[0]
+    rel = np.abs(got - want) / np.maximum(np.abs(want), 1e-30)
+    assert rel.max() <= 1e-6, f"expert {e}: relative error {rel.max()}"
+    assert np.array_equal(got, want), f"expert {e}: not identical"
+
+
 @pytest.mark.parametrize("cfg", [2, 3, 5])
 def test_full_size_grad_reduce(cfg):
     import torch
     seed = 0
     layer, c, pl, lo, mv = _run_layer(cfg, seed, rows=False, grads=True)
-    n, E = c["grad_n"], c["E"]
+    n, E, dt = c["grad_n"], c["E"], c["grad_dtype"]
     W.fill_device(layer.g_home, seed, W.STREAM_GHOME)
     W.fill_device(layer.g_rep, seed, W.STREAM_GREP)
     layer.grad_reduce(clear=False)
     assert layer.status() == 0
-    rng = np.random.default_rng(cfg)
-    cols = np.unique(np.concatenate([rng.integers(0, n, 96), [0, 1, n - 1]]))
-    got = layer.g_home.index_select(1, torch.from_numpy(cols).to(layer.g_home.device)).cpu().numpy()
-    home0 = np.stack([W.grad_elements(seed, W.STREAM_GHOME, n, e, cols) for e in range(E)])
     reps = pl["rep_expert"]
-    dt = c["grad_dtype"]
-    rep0 = [W.grad_elements(seed, W.STREAM_GREP, n, m, cols, dt) for m in range(len(reps))]
-    want = home0.copy()
-    for m, e in enumerate(reps):  # home first, then replicas in match order
-        r = rep0[m] if dt == "f32" else O.bf16_to_f32(rep0[m])
-        want[e] = (want[e] + r).astype(np.float32)
-    rel = np.abs(got - want) / np.maximum(np.abs(want), 1e-30)
-    assert rel.max() <= 1e-6
-    assert np.array_equal(got, want)
+    replicated = sorted(set(reps.tolist()))
+    assert replicated
+    with ThreadPoolExecutor(WORKERS) as ex:
+        futs = []
+        for e in replicated:
+            got = layer.g_home[e].cpu().numpy()
+            futs.append(ex.submit(_grad_row_ok, got, e, np.nonzero(reps == e)[0], seed, n, dt))
+            _drain(futs, WORKERS)
+        _drain(futs, 0)
+    # every other home row is its input, unchanged (regenerated on the device)
+    fresh = torch.empty(n, dtype=torch.float32, device=layer.g_home.device)
+    for e in sorted(set(range(E)) - set(replicated)):
+        W.fill_device(fresh, seed, W.STREAM_GHOME, e * n)
+        assert torch.equal(fresh, layer.g_home[e]), f"expert {e} has no replica but its row changed"
     del layer

@@ -109,3 +109,66 @@ def test_rank_local_count_exchange_gloo(world):
     assert all(r[1] == res[0][1] for r in res)          # the same matrix on every rank
     assert all(r[2] for r in res)                        # source prefix + local rank = global rank
     assert all(r[3] for r in res)                        # column sums = the oracle's loads
+
+
+def _exchange_worker(rank, world, port, R, q):
+    """One process of the rank-local job's handle exchange, with stand-ins for
+    the IPC export and open (no GPU): every process ends with the same R
+    addresses, its own ranks' buffers by their own address and every other
+    rank's through the opener, given that rank's own handle and offset."""
+    import datetime
+    import sys
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from token_dispatch_histogram_b200.ranks import EP_IPC_HANDLE_BYTES, exchange_addresses
+        n = R // world
+        local = {rank * n + i: torch.zeros(16) for i in range(n)}
+
+        def exporter(t):
+            r = next(k for k, v in local.items() if v is t)
+            h = bytes([r % 251]) * EP_IPC_HANDLE_BYTES
+            return h, 16 * r
+
+        opened_args = []
+
+        def opener(h, off):
+            opened_args.append((h[0], off))
+            return 1000 + off, 0x7000_0000 + off
+
+        addrs, opened = exchange_addresses(local, R, exporter=exporter, opener=opener)
+        ok_local = all(addrs[r] == t.data_ptr() for r, t in local.items())
+        ok_remote = all(addrs[r] == 0x7000_0000 + 16 * r for r in range(R) if r not in local)
+        ok_args = sorted(opened_args) == sorted((r % 251, 16 * r) for r in range(R) if r not in local)
+        q.put((rank, bool(ok_local), bool(ok_remote), bool(ok_args), len(opened)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,R", [(2, 2), (2, 8), (3, 6)])
+def test_rank_local_handle_exchange_gloo(world, R):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_exchange_worker, args=(r, world, port, R, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert all(r[1] and r[2] and r[3] for r in res)
+    assert all(r[4] == R - R // world for r in res)       # every other process's ranks opened once
+
+
+def test_export_record_round_trip():
+    from token_dispatch_histogram_b200.ranks import RECORD_BYTES, pack_export, unpack_export
+    h = bytes(range(64))
+    rec = pack_export(37, h, 123456789012, 4242)
+    assert rec.size == RECORD_BYTES
+    assert unpack_export(rec) == (37, 123456789012, 4242, h)

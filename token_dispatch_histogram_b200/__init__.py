@@ -25,6 +25,7 @@ EP_DEV_COPY_TIMEOUT = 0x10
 EP_MAX_EXPERTS = 1024
 EP_MAX_RANKS = 1024
 EP_DTYPE_F32, EP_DTYPE_BF16 = 0, 1
+EP_IPC_HANDLE_BYTES = 64
 
 
 class EpError(RuntimeError):
@@ -89,6 +90,9 @@ _SIGS = {
     "ep_quota_layout_rank": (_I, [_V, _I64, _I, _I, _I, _I, _V, _V, _SZ, _V, _SZ, _V, _V, _V]),
     "ep_quota_replica_grad_reduce_peer": (_I, [_V, _V, _I64, _I, _I64, _I, _I, _I, _V, _SZ, _I, _V, _V]),
     "ep_replica_grad_reduce_peer": (_I, [_V, _V, _I64, _I, _I64, _I, _I, _I, _V, _SZ, _I, _V, _V]),
+    "ep_ipc_export": (_I, [_V, _V, _V]),
+    "ep_ipc_open": (_I, [_V, ctypes.c_uint64, _V, _V]),
+    "ep_ipc_close": (_I, [_V]),
     "ep_status_read": (_I, [_V, _V, _V]),
     "ep_selftest_lookback_timeout": (_I, [_V, _I64, _I, _I, _V, _V, _V, _SZ, _V, _V]),
 }
@@ -364,6 +368,30 @@ def peer_table(tensors, device=None):
     addrs = [int(t.data_ptr()) for t in tensors]
     dev = device if device is not None else tensors[0].device
     return torch.tensor(addrs, dtype=torch.int64, device=dev)
+
+
+def ep_ipc_export(tensor):
+    """(handle bytes, byte offset) naming `tensor`'s device memory for another
+    process (ep_ipc_open there)."""
+    h = (ctypes.c_uint8 * EP_IPC_HANDLE_BYTES)()
+    off = ctypes.c_uint64(0)
+    _check("ep_ipc_export", lib().ep_ipc_export(_p(tensor), ctypes.byref(h), ctypes.byref(off)))
+    return bytes(h), int(off.value)
+
+
+def ep_ipc_open(handle, offset):
+    """Map another process's exported buffer here: (base, device address);
+    base is what ep_ipc_close takes."""
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle must be EP_IPC_HANDLE_BYTES bytes")
+    h = (ctypes.c_uint8 * EP_IPC_HANDLE_BYTES).from_buffer_copy(handle)
+    base, ptr = ctypes.c_void_p(0), ctypes.c_void_p(0)
+    _check("ep_ipc_open", lib().ep_ipc_open(ctypes.byref(h), int(offset), ctypes.byref(base), ctypes.byref(ptr)))
+    return int(base.value), int(ptr.value)
+
+
+def ep_ipc_close(base):
+    _check("ep_ipc_close", lib().ep_ipc_close(ctypes.c_void_p(int(base))))
 
 
 def ep_plan_from_counts(counts, S, K, plan, loads=None, dev_status=None, stream=None):

@@ -20,14 +20,40 @@ matrix.  One step on rank r:
 
 Every device step is one of libep.so's kernels; this module only allocates
 and sequences.  gather_counts is the collective, through torch.distributed.
+
+RankLocalJob runs the R ranks over the processes of a torch.distributed group,
+R / world ranks per process (one process per GPU; world = R is one rank per
+GPU), with the peer tables built from CUDA IPC handles exchanged over the
+group (ep_ipc_export / ep_ipc_open) and a host fence between the ranks'
+dispatch and their combine.
 """
+import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import (ep_combine_peer, ep_dispatch_peer, ep_layout_rank, ep_plan_from_counts, ep_plan_layout,
-               ep_quota_counts_workspace_size, ep_quota_layout_rank, ep_quota_plan_from_counts,
-               ep_quota_plan_layout, ep_quota_replica_grad_reduce_peer, ep_replica_grad_reduce_peer,
-               ep_route_stats, ep_status_read, ep_workspace_size)
+from . import (EP_IPC_HANDLE_BYTES, ep_combine_peer, ep_dispatch_peer, ep_ipc_close, ep_ipc_export, ep_ipc_open,
+               ep_layout_rank, ep_plan_from_counts, ep_plan_layout, ep_quota_counts_workspace_size,
+               ep_quota_layout_rank, ep_quota_plan_from_counts, ep_quota_plan_layout,
+               ep_quota_replica_grad_reduce_peer, ep_replica_grad_reduce_peer, ep_route_stats, ep_status_read,
+               ep_workspace_size)
+
+
+def _on_backend(t, group=None):
+    """`t` on the device the group's backend exchanges (CPU for gloo)."""
+    backend = dist.get_backend(group)
+    if backend == "gloo":
+        return t.cpu()
+    return t
+
+
+def all_gather_rows(rows, group=None):
+    """Concatenate every process's [n, ...] block (the same n everywhere) in
+    process order, on every process; returned on rows' device."""
+    world = dist.get_world_size(group)
+    mine = _on_backend(rows.contiguous(), group)
+    parts = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(parts, mine, group=group)
+    return torch.cat(parts).to(rows.device)
 
 
 def gather_counts(counts_row, counts, group=None):
@@ -36,9 +62,157 @@ def gather_counts(counts_row, counts, group=None):
     R = dist.get_world_size(group)
     if counts.shape != (R, counts_row.numel()):
         raise ValueError(f"counts must be [{R}, {counts_row.numel()}]")
+    if dist.get_backend(group) == "gloo" and counts.is_cuda:
+        counts.copy_(all_gather_rows(counts_row.view(1, -1), group))
+        return counts
     parts = list(counts.unbind(0))
     dist.all_gather(parts, counts_row.contiguous(), group=group)
     return counts
+
+
+def pack_export(rank, handle, offset, pid):
+    """One exchanged record: [rank, offset, pid] int64 then the handle bytes."""
+    head = np.array([rank, offset, pid], dtype=np.int64).view(np.uint8)
+    return np.concatenate([head, np.frombuffer(handle, dtype=np.uint8)])
+
+
+def unpack_export(rec):
+    rec = np.ascontiguousarray(rec, dtype=np.uint8)
+    rank, offset, pid = (int(v) for v in rec[:24].view(np.int64))
+    return rank, offset, pid, bytes(rec[24:24 + EP_IPC_HANDLE_BYTES])
+
+
+RECORD_BYTES = 24 + EP_IPC_HANDLE_BYTES
+
+
+def exchange_addresses(local, R, group=None, exporter=None, opener=None):
+    """Addresses of all R ranks' buffers in this process.
+
+    local: {rank: tensor} for the ranks this process holds (every process
+    holds the same number).  Each process exports its buffers (CUDA IPC
+    handles), the records are all-gathered over the group, and the other
+    processes' buffers are opened here.  Returns (addrs [R] ints, opened
+    bases to close).  exporter/opener stand in for ep_ipc_export/ep_ipc_open
+    (tests of the exchange without a GPU)."""
+    import os
+    exporter = exporter or ep_ipc_export
+    opener = opener or ep_ipc_open
+    pid = os.getpid()
+    recs = []
+    for r in sorted(local):
+        h, off = exporter(local[r])
+        recs.append(pack_export(r, h, off, pid))
+    mine = torch.from_numpy(np.stack(recs))
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    every = all_gather_rows(mine, group).numpy() if world > 1 else mine.numpy()
+    addrs = [0] * R
+    opened = []
+    seen = set()
+    for rec in every:
+        r, off, owner, h = unpack_export(rec)
+        if not 0 <= r < R or r in seen:
+            raise ValueError(f"rank {r} exported twice or out of range")
+        seen.add(r)
+        if owner == pid and r in local:
+            addrs[r] = int(local[r].data_ptr())
+        else:
+            base, ptr = opener(h, off)
+            opened.append(base)
+            addrs[r] = int(ptr)
+    if len(seen) != R:
+        raise ValueError(f"{R - len(seen)} ranks exported no buffer")
+    return addrs, opened
+
+
+class RankLocalJob:
+    """The rank-local form over the processes of a torch.distributed group
+    (or this process alone): R ranks, R / world of them in each process
+    (ranks [p*n, (p+1)*n) in process p), one EpRank each, on this process's
+    GPU.  open_peers() must run once (collectively) before dispatch;
+    close() (collectively) before the buffers are freed.
+
+    One step: route() (counts of every local rank, one all-gather of the
+    [n, E] blocks, plan and layout per rank), dispatch(), fence() (every
+    rank's rows are written before any rank reads them: a stream
+    synchronisation and a barrier), combine(), and with gradients
+    grad_reduce() after a fence of its own."""
+
+    def __init__(self, R, S, K, E, H, group=None, device="cuda", grad_n=0, grad_dtype=torch.float32):
+        self.group = group
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.me = dist.get_rank(group) if dist.is_initialized() else 0
+        if R % self.world:
+            raise ValueError(f"R={R} ranks do not divide over {self.world} processes")
+        self.R, self.S, self.K, self.E, self.H = R, S, K, E, H
+        self.n = R // self.world
+        self.device = torch.device(device)
+        first = self.me * self.n
+        self.ranks = [EpRank(first + i, R, S, K, E, H, device=self.device, grad_n=grad_n, grad_dtype=grad_dtype)
+                      for i in range(self.n)]
+        self.counts = torch.zeros((R, E), dtype=torch.int32, device=self.device)
+        self._opened = []
+
+    def open_peers(self):
+        """Peer tables of all R ranks' receive buffers (and replica gradient
+        buffers) in this process: own buffers by address, the other
+        processes' through their IPC handles."""
+        addrs, opened = exchange_addresses({rk.rank: rk.buf for rk in self.ranks}, self.R, self.group)
+        self._opened += opened
+        peers = torch.tensor(addrs, dtype=torch.int64, device=self.device)
+        for rk in self.ranks:
+            rk.set_peers(peers)
+        if self.ranks[0].grad_n:
+            gaddrs, gopened = exchange_addresses({rk.rank: rk.g_rep for rk in self.ranks}, self.R, self.group)
+            self._opened += gopened
+            gpeers = torch.tensor(gaddrs, dtype=torch.int64, device=self.device)
+            for rk in self.ranks:
+                rk.set_grad_peers(gpeers)
+
+    def route(self, stream=None):
+        for rk in self.ranks:
+            rk.count(stream)
+        rows = torch.stack([rk.counts_row for rk in self.ranks])
+        if self.world > 1:
+            rows = all_gather_rows(rows, self.group)
+        self.counts.copy_(rows)
+        for rk in self.ranks:
+            rk.counts.copy_(self.counts)
+            rk.plan_and_layout(stream)
+
+    def dispatch(self, stream=None):
+        for rk in self.ranks:
+            rk.dispatch(stream)
+
+    def combine(self, stream=None):
+        for rk in self.ranks:
+            rk.combine(stream)
+
+    def grad_reduce(self, clear=False, stream=None):
+        for rk in self.ranks:
+            rk.grad_reduce(clear, stream)
+
+    def fence(self):
+        """Every process's queued work done, then a barrier: rows another
+        process wrote into this one's buffers (or will read) are in place."""
+        torch.cuda.synchronize(self.device)
+        if self.world > 1:
+            dist.barrier(group=self.group)
+
+    def status(self, stream=None):
+        st = 0
+        for rk in self.ranks:
+            st |= rk.status(stream)
+        return st
+
+    def close(self):
+        """Unmap the other processes' buffers (after a fence, so no process
+        still reads or writes them)."""
+        self.fence()
+        for base in self._opened:
+            ep_ipc_close(base)
+        self._opened = []
+        if self.world > 1:
+            dist.barrier(group=self.group)
 
 
 class EpRank:
