@@ -3,17 +3,20 @@ allocate device scratch (hosts that hand a kernel only its inputs and outputs
 at enqueue time, runtimes whose memory is planned in advance).  It keeps its
 scratch in a fixed array inside libep.so instead of a caller workspace.
 
-Checked through the C ABI against ep_route_stats (which takes a workspace):
-loads and max_vio must agree exactly (integer counts, and max_vio is the same
-fp64 expression), on several calls in a row that reuse the shared array, and a
-problem larger than the array must be refused before anything is enqueued.
-This file is collected last on purpose, and each test also runs on its own.
+Checked through the C ABI against ep_route_stats (which takes a workspace)
+and against the CPU oracle: loads and max_vio must agree exactly (integer
+counts, and max_vio is the same fp64 expression), on several calls in a row
+that reuse the shared array; after the first call no further call changes the
+device's free memory; and a problem larger than the array must be refused
+before anything is enqueued.  This file is collected last on purpose, and
+each test also runs on its own.
 """
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle as O
 import workload as W
 
 pytestmark = pytest.mark.gpu
@@ -53,7 +56,40 @@ def test_noalloc_matches_route_stats_on_consecutive_calls():
         (la, ma), (lb, mb) = _call_both(topk, c["E"])
         np.testing.assert_array_equal(la, lb)
         assert ma == mb
-        np.testing.assert_array_equal(la, np.bincount(topk.ravel(), minlength=c["E"]))
+        lo, mo, bad = O.route_stats(topk, c["E"])
+        assert bad == 0
+        np.testing.assert_array_equal(la, lo)
+        assert ma == mo
+
+
+def test_noalloc_calls_leave_free_memory_unchanged():
+    """Once the first call has run, further calls allocate nothing: the
+    device's free memory (cudaMemGetInfo) is the same after twenty calls."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    L = tdh.lib()
+    c = W.shape(5)
+    topk_np, _ = W.routing(5, 0)
+    dev = torch.device("cuda")
+    topk = torch.from_numpy(topk_np).to(dev)
+    loads = torch.zeros(c["E"], dtype=torch.int32, device=dev)
+    mv = torch.zeros(1, dtype=torch.float64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    args = (ctypes.c_void_p(topk.data_ptr()), c["T"], c["K"], c["E"], ctypes.c_void_p(loads.data_ptr()),
+            ctypes.c_void_p(mv.data_ptr()), ctypes.c_void_p(status.data_ptr()), stream)
+    assert L.ep_route_stats_noalloc(*args) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(20):
+        assert L.ep_route_stats_noalloc(*args) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert int(status.item()) == 0
+    lo, mo, _ = O.route_stats(topk_np, c["E"])
+    np.testing.assert_array_equal(loads.cpu().numpy(), lo)
+    assert float(mv.item()) == mo
 
 
 def test_noalloc_refuses_problems_larger_than_its_array():

@@ -16,6 +16,8 @@
 //    (tile, expert), every wait bounded,
 //  - the last tile's inclusive prefix is T_e; it also reduces max_e T_e.
 // Only integer adds feed the outputs, so they do not depend on scheduling.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -195,29 +197,70 @@ extern "C" int ep_route_stats(const int32_t* topk_ids, int64_t T, int K, int E, 
 // allocation there (plugin-style interfaces), or runtimes whose device memory is
 // planned once up front.  For them ep_route_stats_noalloc keeps its scratch in
 // the fixed array below, which exists on every GPU that loads this library
-// until the process exits.  Its device address is looked up once per device
-// (cudaGetSymbolAddress) on the first call made with that device current.  All
-// calls share the array and it keeps the last call's contents; the part that
-// must start at zero (the look-back words and the tile counter) is cleared on
-// the call's stream, so calls must not overlap on the GPU: two calls running at
-// the same time race on the array.
+// until the process exits.  Its device address is looked up (cudaGetSymbolAddress)
+// on the first call made in a CUDA context, with that context's device current,
+// and cached per device together with the context's unique id; a call made in
+// another context of the same device (after cudaDeviceReset, or under a context
+// the caller created) looks it up again.  All calls share the array and it keeps
+// the last call's contents; the part that must start at zero (the look-back
+// words and the tile counter) is cleared on the call's stream, so calls must
+// not overlap on the GPU: two calls running at the same time race on the array.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[EP_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64] = {nullptr};
+struct NoallocEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+NoallocEntry g_noalloc[64] = {};
+
+// The driver's cuCtxGetCurrent / cuCtxGetId, reached through the runtime's
+// entry-point query (so the library needs no link against the driver library).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+int current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || !f1)
+      return EP_ERR_CUDA;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || !f2)
+      return EP_ERR_CUDA;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return EP_ERR_CUDA;
+  *id = 0;  // no context current yet
+  if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return EP_ERR_CUDA;
+  return EP_OK;
+}
 
 int noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
   if (dev < 0 || dev >= 64) return EP_ERR_ARG;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
+  unsigned long long id = 0;
+  int rc = current_context_id(&id);
+  if (rc != EP_OK) return rc;
+  NoallocEntry& ent = g_noalloc[dev];
+  if (!ent.addr || id == 0 || ent.ctx_id != id) {
+    void* p = nullptr;  // the lookup makes the device's context current if none was
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return EP_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
+    rc = current_context_id(&id);
+    if (rc != EP_OK) return rc;
+    ent.addr = p;
+    ent.ctx_id = id;
   }
-  *out = g_noalloc_addr[dev];
+  *out = ent.addr;
   return EP_OK;
 }
 }  // namespace
