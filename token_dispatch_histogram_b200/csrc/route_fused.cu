@@ -6,18 +6,19 @@
 // so on B200 it is bound by latency chains, not HBM: launch gaps, the serial
 // look-back, one CTA planning while the GPU idles.  Here all CTAs stay resident
 // (cooperative launch) and meet at grid barriers instead:
-//   1. each CTA counts its tile per warp (warp-match aggregation), writes the
-//      tile's per-expert counts, column-major [E][tiles], and adds them into
-//      the totals T_e (integer atomics: the sums do not depend on order);
+//   1. each CTA counts its tile per warp (shared-memory integer atomics into
+//      the warp's own row), writes the tile's per-expert counts, column-major
+//      [E][tiles], and adds them into the totals T_e (integer atomics: the
+//      sums do not depend on order);
 //   -- grid barrier --
 //   2. one extra CTA with no tile reads T_e and runs the planner
 //      (plan_block.cuh) and max_vio at once, then raises a flag; meanwhile the
 //      tile CTAs scan the per-expert columns in parallel (exclusive tile
-//      prefixes), meet at a second barrier of their own, and walk their tiles
-//      once for the align-sort ranks (which need only T_e), writing sorted
-//      ids, padding and block experts;
-//   4. after the flag, every CTA walks its tile again for the layout ranks and
-//      writes pos / src / pair_slot from the plan.
+//      prefixes), meet at a second barrier of their own, and write what the
+//      align-sort needs no rank for (group offsets, padding, block experts);
+//   4. after the flag, every CTA walks its tile once: each pair's stable rank
+//      within its expert gives both its align-sort slot (sorted ids) and its
+//      layout row (pos / src / pair_slot from the plan).
 // A pair's stable rank within its expert = (its tile's prefix) + (earlier warps
 // of the tile) + (earlier chunks of its warp) + popc(peers & lanemask_lt):
 // integer adds only, so nothing depends on scheduling.  Every wait is bounded.
@@ -237,23 +238,19 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   for (int i = tid; i < FUSED_WARPS * E; i += FUSED_THREADS) s_wb[i] = 0;
   __syncthreads();
   if (has_tile) {
+    // counts only: shared-memory integer atomics into the warp's own row (the
+    // sum does not depend on the order the lanes are served in)
     int32_t* my = s_wb + warp * E;
-    const int nbits1 = key_bits(E + 1);
     for (int c0 = 0; c0 < sub; c0 += 32 * WALK_UNROLL) {
       int ids[WALK_UNROLL];
 #pragma unroll
       for (int u = 0; u < WALK_UNROLL; ++u) {
         const int64_t p = wp0 + c0 + u * 32 + lane;
-        ids[u] = (c0 + u * 32 < sub && p < a.P) ? __ldg(a.topk + p) : -1;
+        ids[u] = (c0 + u * 32 + lane < sub && p < a.P) ? __ldg(a.topk + p) : -1;
       }
 #pragma unroll
-      for (int u = 0; u < WALK_UNROLL; ++u) {
-        if (c0 + u * 32 >= sub) break;  // warp-uniform
-        const int e = (ids[u] >= 0 && ids[u] < E) ? ids[u] : -1;
-        const uint32_t peers = warp_match((uint32_t)(e + 1), nbits1);
-        if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-        __syncwarp();
-      }
+      for (int u = 0; u < WALK_UNROLL; ++u)
+        if (ids[u] >= 0 && ids[u] < E) atomicAdd(my + ids[u], 1);
     }
   }
   __syncthreads();
@@ -290,7 +287,8 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
     __syncthreads();
   }
 
-  // ---- 3. planner on the last CTA; align-sort ranks on the tile CTAs
+  // ---- 3. planner on the last CTA; the align-sort's group offsets, padding
+  // and block experts on the tile CTAs
   if (planner) {
     int32_t m = 0;
     for (int e = tid; e < E; e += FUSED_THREADS) m = max(m, s_loads[e]);
@@ -316,11 +314,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
     __syncthreads();
     const int32_t total = block_scan_inplace(s_off, E, warp_sums);
     if (tid == 0) s_off[E] = total;
-    for (int i = tid; i < FUSED_WARPS * E; i += FUSED_THREADS) s_run[i] = s_wb[i] + s_excl[i % E];
     __syncthreads();
+    // the pairs' own ids go out in the layout walk below (same stable rank);
+    // here only what needs no rank: the padding, the block experts, the total
     int32_t* sorted_ids = a.sorted_ids;
-    walk_warp(a.topk, a.P, E, wp0, sub, s_run + warp * E,
-              [&](int64_t p, int e, int32_t g) { sorted_ids[s_off[e] + g] = (int32_t)p; }, &s_bad);
     const int32_t sentinel = (int32_t)a.P;
     for (int e = t; e < E; e += NT)
       for (int32_t i = s_off[e] + s_loads[e] + tid; i < s_off[e + 1]; i += FUSED_THREADS) sorted_ids[i] = sentinel;
@@ -368,9 +365,11 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   int32_t* pos = a.pos;
   int32_t* src = a.src;
   int32_t* pair_slot = a.pair_slot;
+  int32_t* sorted_ids = a.sorted_ids;
   const int64_t P = a.P;
   walk_warp(a.topk, P, E, wp0, sub, s_run + warp * E,
             [&](int64_t p, int e, int32_t g) {
+              if (sorted_ids) sorted_ids[s_off[e] + g] = (int32_t)p;  // align-sort: same rank within the expert
               int32_t row = -1, slot = -1;
               if (g < s_hc[e]) {
                 row = s_hb[e] + g;
