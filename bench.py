@@ -21,11 +21,11 @@ replayed K times, with CUDA events around each replay on the launching stream,
 L2 flushed (a 512 MB write) between replays outside the events, max over ranks.
 The per-op breakdown and the roofline come from an eager pass of the same K
 steps with CUDA events between the ops.  `e2e`: the same steps through the
-public API (EpLayer.run_host, one call per layer) from pinned host buffers:
-each layer's routing, gate weights and hidden rows copied in and its combined
-rows copied out inside the timed region (run_host pipelines the copies in
-token slices over two copy streams; the copies are torch's, around the C-ABI
-kernels).  Under torchrun each rank runs its own independent layers (weak
+public API (layer.run_host_layers, EpLayer.run_host for every layer with the
+layers' copies overlapped) from pinned host buffers: each layer's routing,
+gate weights and hidden rows copied in and its combined rows copied out inside
+the timed region (the copies go in token slices over two copy streams; they
+are torch's, around the C-ABI kernels).  Under torchrun each rank runs its own independent layers (weak
 scaling, no data-path collective).
 
 `cpu_baseline` and --impl reference time the CPU oracle (the plain
@@ -76,6 +76,7 @@ def parse(argv=None):
     ap.add_argument("--hidden", type=int, default=None,
                     help="override H (e.g. a full-size route with small rows, for a profiler capture of the route)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=8, help="token slices of the host-fed pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the backward of dispatch and combine")
     ap.add_argument("--no-quota", action="store_true", help="skip timing the quota-driven planner")
@@ -270,6 +271,7 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     import torch
     import token_dispatch_histogram_b200 as tdh
     import workload as W
+    from token_dispatch_histogram_b200.layer import run_host_layers
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -692,9 +694,9 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
         x_h.copy_(layer.x)  # the generator's rows, as a caller's host batch
         out_h = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
 
-        def host_step():
-            for li, ly in enumerate(layers):
-                ly.run_host(topk_h[li], w_h[li], x_h, out_h, stream, fused=fused)
+        def host_step():  # the layers' copies overlap one another (run_host_layers)
+            run_host_layers(layers, topk_h, w_h, [x_h] * nl, [out_h] * nl, stream, fused=fused,
+                            chunks=args.e2e_chunks)
 
         host_step()
         torch.cuda.synchronize()
@@ -721,8 +723,10 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
         bo = nl * out_h.numel() * 2
         e2e = {"value": job_throughput(world, nl * P, n_e2e, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / n_e2e, "steps": n_e2e,
-               "what": "EpLayer.run_host per layer: torch copies between pinned host buffers and the layer's device "
-                       "buffers around the C-ABI kernels, in token slices on two copy streams"}
+               "chunks": args.e2e_chunks,
+               "what": "run_host_layers: per layer its routing, weights and hidden rows in from pinned host memory "
+                       "and its combined rows out (torch copies around the C-ABI kernels), in token slices on two "
+                       "copy streams, the next layer's inbound copies overlapping this layer's outbound ones"}
         del topk_h, w_h, x_h, out_h
 
     # ---- roofline of the dominant kernel and the per-op breakdown (bytes summed over layers)

@@ -61,3 +61,41 @@ def test_overlapped_step_matches_the_sequential_one():
     assert lay.status() == 0
     assert int(lay.plan_view("n_rep", 1).item()) > 0
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("chunks", [1, 5, 8])
+def test_run_host_layers_matches_each_layer(chunks):
+    """Three layers sharing their row buffers, fed from the host with the
+    layers' copies overlapped (run_host_layers): each layer's combined rows
+    equal the oracle's for that layer's routing, whether every layer has its
+    own output buffer or all share one (which then holds the last layer's)."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    from token_dispatch_histogram_b200.layer import run_host_layers
+    R, S, K, E, H, bm = 8, 384, 6, 64, 512, 64
+    T = R * S
+    layers = []
+    for _ in range(3):
+        layers.append(tdh.EpLayer(R, S, K, E, H, bm, device="cuda", share=layers[0] if layers else None))
+    routes = [W.routing_from(T, E, K, seed=20 + l, bias_e=W.bias(2, l)) for l in range(3)]
+    xs = [W.hidden(T, H, seed=30 + l) for l in range(3)]
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    topk_hs = [pin(tk) for tk, _ in routes]
+    w_hs = [pin(w) for _, w in routes]
+    x_hs = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs]
+    refs = []
+    for (tk, w), x in zip(routes, xs):
+        loads, _, _ = O.route_stats(tk, E)
+        pl = O.plan(loads, R, S, K, E)
+        lo = O.layout(tk, pl, R, S, E)
+        refs.append(O.combine(O.dispatch(x, lo["pos"], K, T * K), w, lo["pos"], K))
+    own = [torch.zeros((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    run_host_layers(layers, topk_hs, w_hs, x_hs, own, grads=False, chunks=chunks)
+    torch.cuda.synchronize()
+    assert all(ly.status() == 0 for ly in layers)
+    for got, ref in zip(own, refs):
+        np.testing.assert_array_equal(got.view(torch.int16).numpy().view(np.uint16), ref)
+    shared = torch.zeros((T, H), dtype=torch.bfloat16).pin_memory()
+    run_host_layers(layers, topk_hs, w_hs, x_hs, [shared] * 3, grads=False, chunks=chunks)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(shared.view(torch.int16).numpy().view(np.uint16), refs[-1])

@@ -366,8 +366,13 @@ def _nccl_one_rank(port, q):
         rk.dispatch()
         rk.combine()
         torch.cuda.synchronize()
+        # the handle records are host bytes: through NCCL they are staged on the GPU and come back to the host
+        from token_dispatch_histogram_b200.ranks import all_gather_rows
+        recs = torch.arange(2 * 88, dtype=torch.int32).to(torch.uint8).view(2, 88)
+        back = all_gather_rows(recs)
         q.put(dict(status=rk.status(), counts=rk.counts.cpu().numpy(), pos=rk.pos_local.cpu().numpy(),
-                   out=rk.out_local.view(torch.int16).cpu().numpy().view(np.uint16)))
+                   out=rk.out_local.view(torch.int16).cpu().numpy().view(np.uint16),
+                   recs_ok=bool(back.device.type == "cpu" and torch.equal(back, recs))))
     finally:
         dist.destroy_process_group()
 
@@ -392,6 +397,7 @@ def test_rank_local_route_through_nccl():
     pl = O.plan(loads, 1, S, K, E)
     lo = O.layout(topk, pl, 1, S, E)
     assert res["status"] == 0
+    assert res["recs_ok"]
     np.testing.assert_array_equal(res["counts"][0], loads)
     np.testing.assert_array_equal(res["pos"], lo["pos"])
     buf = O.dispatch(x, lo["pos"], K, S * K)

@@ -8,8 +8,8 @@
 // One kernel, one pass over topk_ids:
 //  - each CTA takes a tile of consecutive flattened pairs (tile index from an
 //    atomic ticket, so a CTA only ever waits on tiles that started earlier),
-//  - builds the tile's histogram in shared memory, one shared-memory add per
-//    distinct expert per warp (warp_match aggregation: one ballot per key bit),
+//  - builds the tile's histogram in shared memory (integer atomics: a sum, so
+//    the order they are served in does not matter),
 //  - publishes it and resolves its exclusive prefix over earlier tiles with a
 //    decoupled look-back (Merrill & Garland, "Single-pass Parallel Prefix Scan
 //    with Decoupled Look-back", 2016), one 64-bit {flag, value} word per
@@ -46,19 +46,15 @@ __global__ void __launch_bounds__(HIST_THREADS)
   const int64_t p0 = (int64_t)t * tile;
   const int64_t p1 = min(P, p0 + tile);
 
-  const int nbits = key_bits(E + 1);
   for (int64_t base = p0; base < p1; base += blockDim.x) {
     const int64_t p = base + threadIdx.x;
-    int e = -1;
     if (p < p1) {
-      e = __ldg(topk + p);
-      if (e < 0 || e >= E) {
-        e = -1;
+      const int e = __ldg(topk + p);
+      if (e >= 0 && e < E)
+        atomicAdd(&s_hist[e], 1);  // a sum: the order the lanes are served in does not matter
+      else
         s_bad = 1;
-      }
     }
-    const uint32_t peers = warp_match((uint32_t)(e + 1), nbits);
-    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[e], __popc(peers));
   }
   __syncthreads();
   if (threadIdx.x == 0 && s_bad) flag(dev_status, EP_DEV_BAD_EXPERT_ID);

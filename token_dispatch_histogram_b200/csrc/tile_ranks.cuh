@@ -3,7 +3,9 @@
 // expert = (pairs of that expert before the tile) + (pairs of it in earlier
 // warps of the tile) + (earlier pairs of it in this warp's sub-tile).  The last
 // term comes from a warp match over 32 consecutive pairs (one ballot per key
-// bit) plus a per-warp running counter.  No atomics feed the ranks.
+// bit) plus a per-warp running counter.  The per-warp counts behind the second
+// term are summed with shared-memory integer atomics (a sum, so the order the
+// lanes are served in does not matter); no atomic feeds a rank directly.
 #pragma once
 
 #include "common.cuh"
@@ -37,13 +39,10 @@ __device__ __forceinline__ void tile_ranks_prepare(const int32_t* __restrict__ t
   __syncthreads();
 
   const int sub = tile / SCAT_WARPS;  // pairs per warp, a multiple of 32
-  const int nbits = key_bits(E + 2);  // keys e + 2: -2 (invalid id), -1 (past the end), experts
   int32_t* my = s_whist + warp * E;
-  for (int c = 0; c < sub; c += 32) {
+  for (int c = 0; c < sub; c += 32) {  // counts only: integer atomics (order-free) into the warp's own row
     const int e = s_ids[warp * sub + c + lane];
-    const uint32_t peers = warp_match((uint32_t)(e + 2), nbits);
-    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-    __syncwarp();
+    if (e >= 0) atomicAdd(my + e, 1);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {

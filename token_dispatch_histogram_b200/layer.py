@@ -168,10 +168,7 @@ class EpLayer:
                 self.step(main, grads, fused)
                 out_h.copy_(self.out, non_blocking=True)
             return
-        if not hasattr(self, "_h2d"):
-            self._h2d = torch.cuda.Stream(self.device)
-            self._d2h = torch.cuda.Stream(self.device)
-        h2d, d2h = self._h2d, self._d2h
+        h2d, d2h = self._copy_streams()
         h2d.wait_stream(main)  # buffers are free once the caller's earlier work is done
         d2h.wait_stream(main)
         with torch.cuda.stream(h2d):
@@ -204,7 +201,80 @@ class EpLayer:
     def status(self, stream=None):
         return ep_status_read(self.dev_status, stream)
 
+    def _copy_streams(self):
+        if not hasattr(self, "_h2d"):
+            self._h2d = torch.cuda.Stream(self.device)
+            self._d2h = torch.cuda.Stream(self.device)
+        return self._h2d, self._d2h
+
     # --- plan views -------------------------------------------------------
     def plan_view(self, name, count):
         off = self.plan_layout[name]
         return self.plan[off:off + count]
+
+
+def run_host_layers(layers, topk_hs, w_hs, x_hs, out_hs, stream=None, grads=True, fused=True, chunks=8):
+    """Several layers' host-fed passes (each as EpLayer.run_host: its routing,
+    gate weights and hidden rows in from pinned host memory, its combined rows
+    out), with the layers' copies overlapping one another.
+
+    The layers may share their row buffers (EpLayer(share=...)): then layer
+    l+1's slice j of hidden rows may arrive as soon as layer l has dispatched
+    its slice j, and layer l+1 may combine slice j as soon as layer l's slice j
+    has left for the host, so layer l+1's inbound copies run while layer l's
+    outbound copies drain (the host link is full duplex).  Within a layer the
+    slices pipeline exactly as in run_host.  Results: out_hs[l] holds layer
+    l's combined rows (the same tensor may be given for every layer; it then
+    ends with the last layer's).  The caller's stream waits for every copy."""
+    n = len(layers)
+    if not (len(topk_hs) == len(w_hs) == len(x_hs) == len(out_hs) == n):
+        raise ValueError("one routing, weight, hidden and output buffer per layer")
+    if n == 0:
+        return
+    first = layers[0]
+    main = stream if stream is not None else torch.cuda.current_stream(first.device)
+    h2d, d2h = first._copy_streams()
+    h2d.wait_stream(main)
+    d2h.wait_stream(main)
+    prev = None  # (x, out, [dispatched events], [sent events]) of the layer before
+    for ly, topk_h, w_h, x_h, out_h in zip(layers, topk_hs, w_hs, x_hs, out_hs):
+        with torch.cuda.stream(h2d):
+            ly.topk_ids.copy_(topk_h, non_blocking=True)
+            ly.w.copy_(w_h, non_blocking=True)
+            routed = torch.cuda.Event()
+            routed.record(h2d)
+        main.wait_event(routed)
+        ly.route(main, fused)
+        bounds = slice_bounds(ly.T, max(1, min(chunks, ly.T)))
+        K = ly.K
+        same_x = prev is not None and prev[0].data_ptr() == ly.x.data_ptr()
+        same_out = prev is not None and prev[1].data_ptr() == ly.out.data_ptr()
+        dispatched, sent = [], []
+        for j, (t0, t1) in enumerate(zip(bounds[:-1], bounds[1:])):
+            with torch.cuda.stream(h2d):
+                if same_x:
+                    h2d.wait_event(prev[2][j])  # the layer before has read these rows of x
+                ly.x[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(h2d)
+            main.wait_event(arrived)
+            ep_dispatch(ly.x[t0:t1], K, ly.pos[t0 * K:t1 * K], ly.buf, ly.dev_status, main)
+            ev = torch.cuda.Event()
+            ev.record(main)
+            dispatched.append(ev)
+            if same_out:
+                main.wait_event(prev[3][j])  # the layer before's rows of out have left
+            ep_combine(ly.buf, ly.w[t0:t1], ly.pos[t0 * K:t1 * K], ly.out[t0:t1], ly.dev_status, main)
+            combined = torch.cuda.Event()
+            combined.record(main)
+            d2h.wait_event(combined)
+            with torch.cuda.stream(d2h):
+                out_h[t0:t1].copy_(ly.out[t0:t1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(d2h)
+                sent.append(ev)
+        if grads:
+            ly.grad_reduce(False, main)
+        prev = (ly.x, ly.out, dispatched, sent)
+    main.wait_stream(d2h)
+    main.wait_stream(h2d)

@@ -39,10 +39,13 @@ from . import (EP_IPC_HANDLE_BYTES, ep_combine_peer, ep_dispatch_peer, ep_ipc_cl
 
 
 def _on_backend(t, group=None):
-    """`t` on the device the group's backend exchanges (CPU for gloo)."""
+    """`t` on the device the group's backend exchanges: CPU for gloo, this
+    process's current GPU for NCCL."""
     backend = dist.get_backend(group)
     if backend == "gloo":
         return t.cpu()
+    if backend == "nccl" and not t.is_cuda:
+        return t.to(torch.device("cuda", torch.cuda.current_device()))
     return t
 
 
@@ -53,7 +56,7 @@ def all_gather_rows(rows, group=None):
     mine = _on_backend(rows.contiguous(), group)
     parts = [torch.empty_like(mine) for _ in range(world)]
     dist.all_gather(parts, mine, group=group)
-    return torch.cat(parts).to(rows.device)
+    return torch.cat(parts).to(rows.device)  # back where the caller's rows live
 
 
 def gather_counts(counts_row, counts, group=None):
