@@ -76,7 +76,7 @@ def parse(argv=None):
     ap.add_argument("--hidden", type=int, default=None,
                     help="override H (e.g. a full-size route with small rows, for a profiler capture of the route)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=8, help="token slices of the host-fed pipeline")
+    ap.add_argument("--e2e-chunks", type=int, default=12, help="token slices of the host-fed pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the backward of dispatch and combine")
     ap.add_argument("--no-quota", action="store_true", help="skip timing the quota-driven planner")
