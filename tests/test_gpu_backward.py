@@ -3,8 +3,8 @@
 dx (backward of dispatch) and dy (backward of combine) are bit-exact: the same
 fp32 operations in the same order.  dw is an fp32 reduction in the kernel's own
 order, checked against the oracle's fp64 value within the summation bound
-H * 2^-24 * sum_h |dout * y|.  Small cases compare every element; the large
-workloads compare sampled tokens and rows.
+H * 2^-24 * sum_h |dout * y|.  Every case compares every element: the small
+ones at once, the full-size workloads token chunk by token chunk.
 """
 import numpy as np
 import pytest
@@ -62,8 +62,27 @@ def test_backward_matches_oracle(case):
     assert np.all(np.abs(dw.astype(np.float64) - dw_ref) <= H * 2.0 ** -24 * absum + 1e-30)
 
 
+def _bwd_chunk_ok(t0, t1, rows, got_dx, got_dy, got_dw, dout_h, y_h, w, K, H):
+    """One token chunk of the full-size backward against the oracle: dx of
+    every token, the dy row of every pair, every dw (within the fp32 bound)."""
+    y = y_h[rows]
+    dout = dout_h[t0:t1]
+    local = np.arange(len(rows), dtype=np.int32)
+    np.testing.assert_array_equal(got_dx, O.dispatch_backward(y, local, t1 - t0, K))
+    dy_ref, dw_ref = O.combine_backward(dout, w[t0:t1], y, local)
+    np.testing.assert_array_equal(got_dy, dy_ref)
+    absum = np.einsum("th,tkh->tk", np.abs(O.bf16_to_f32(dout).astype(np.float64)),
+                      np.abs(O.bf16_to_f32(y).astype(np.float64)).reshape(t1 - t0, K, H))
+    assert np.all(np.abs(got_dw.astype(np.float64) - dw_ref) <= H * 2.0 ** -24 * absum + 1e-30)
+
+
 @pytest.mark.parametrize("cfg", [2, 3])
-def test_backward_full_size_sampled(cfg):
+def test_backward_full_size(cfg):
+    """Every output of both backward kernels at the workload's full size, in
+    token chunks: the inputs (dout, y) regenerated on the host from the
+    counter-based generator, the expected values from the oracle."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
     import torch
     import token_dispatch_histogram_b200 as tdh
     c = W.shape(cfg)
@@ -74,7 +93,7 @@ def test_backward_full_size_sampled(cfg):
     layer.w.copy_(torch.from_numpy(w))
     layer.route()
     W.fill_device(layer.out, 0, 0x600)   # dout
-    W.fill_device(layer.buf, 0, 0x601)   # y (and, below, dbuf)
+    W.fill_device(layer.buf, 0, 0x601)   # y (and the dispatch backward's dbuf)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     dx = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
     tdh.ep_dispatch_backward(layer.buf, layer.pos, T, K, dx, st)
@@ -82,21 +101,22 @@ def test_backward_full_size_sampled(cfg):
     dw = torch.empty((T, K), dtype=torch.float32, device="cuda")
     tdh.ep_combine_backward(layer.out, layer.w, layer.buf, layer.pos, dy, dw, st)
     assert tdh.ep_status_read(st) == 0
-    pos = layer.pos.cpu().numpy().reshape(T, K)
-    rng = np.random.default_rng(cfg)
-    toks = np.unique(np.concatenate([rng.integers(0, T, 256), [0, T - 1]]))
-    dout = np.stack([W.normal_bf16(0, 0x600, int(t) * H, H) for t in toks])
-    rows = pos[toks].reshape(-1)
-    y = np.stack([W.normal_bf16(0, 0x601, int(r) * H, H) for r in rows])
-    # dx: unweighted sum of the token's rows
-    local_pos = np.arange(len(rows), dtype=np.int32)
-    got_dx = dx.index_select(0, torch.from_numpy(toks).cuda()).view(torch.int16).cpu().numpy().view(np.uint16)
-    np.testing.assert_array_equal(got_dx, O.dispatch_backward(y, local_pos, len(toks), K))
-    # dy rows and dw of the sampled tokens
-    dy_ref, dw_ref = O.combine_backward(dout, w[toks], y, local_pos)
-    got_dy = dy.index_select(0, torch.from_numpy(rows.astype(np.int64)).cuda()).view(torch.int16).cpu().numpy()
-    np.testing.assert_array_equal(got_dy.view(np.uint16), dy_ref)
-    got_dw = dw.cpu().numpy()[toks].astype(np.float64)
-    absum = np.einsum("th,tkh->tk", np.abs(O.bf16_to_f32(dout).astype(np.float64)),
-                      np.abs(O.bf16_to_f32(y).astype(np.float64)).reshape(len(toks), K, H))
-    assert np.all(np.abs(got_dw - dw_ref) <= H * 2.0 ** -24 * absum + 1e-30)
+    pos = layer.pos.cpu().numpy().astype(np.int64)
+    dout_h = W.normal_bf16(0, 0x600, 0, T * H).reshape(T, H)
+    y_h = W.normal_bf16(0, 0x601, 0, P * H).reshape(P, H)
+    dw_all = dw.cpu().numpy()
+    ch = max(1, (1 << 24) // (K * H))
+    workers = max(2, min(32, os.cpu_count() or 2))
+    with ThreadPoolExecutor(workers) as ex:
+        futs = []
+        for t0 in range(0, T, ch):
+            t1 = min(T, t0 + ch)
+            rows = pos[t0 * K:t1 * K]
+            trows = torch.from_numpy(rows).cuda()
+            got_dx = dx[t0:t1].view(torch.int16).cpu().numpy().view(np.uint16)
+            got_dy = dy.index_select(0, trows).view(torch.int16).cpu().numpy().view(np.uint16)
+            futs.append(ex.submit(_bwd_chunk_ok, t0, t1, rows, got_dx, got_dy, dw_all[t0:t1], dout_h, y_h, w, K, H))
+            while len(futs) > 2 * workers:
+                futs.pop(0).result()
+        for f in futs:
+            f.result()

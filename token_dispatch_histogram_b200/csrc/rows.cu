@@ -299,101 +299,136 @@ __global__ void __launch_bounds__(256)
 //   dw[t,k]  = sum_h float(dout[t,h]) * float(y[r,h])     (fp32; any summation order)
 // One group of G lanes owns one token (G = 32 for rows of 256+ elements, else
 // the power of two covering the row's 16-byte vectors, so a warp carries
-// 32 / G tokens).  Each lane walks every G-th vector of the row: it loads the
-// dout vector and the K y vectors, writes the K scaled dy vectors and keeps K
-// partial dot products, which a butterfly of shuffles inside the group adds
-// up at the end of the token.  No block-wide barrier: warps run independently,
-// and the next token's rows and weights are loaded while the current one runs.
-// Two CTAs per SM: about 124 registers at K = 6 without spills; bounds that
-// force 3 or 4 CTAs spill and measured 0-12% slower on B200.
+// 32 / G tokens), and each warp owns exactly one such group of tokens: the
+// grid is one warp per token group, four warps per CTA (not persistent).  The
+// group's rows and weights are read into shared memory once.  A lane walks
+// every G-th 16-byte vector of its token's row ("jobs"); the dout vector and
+// the K y vectors of each job are copied into a per-warp shared-memory ring of
+// CB_STAGES slots with cp.async, CB_STAGES - 1 jobs ahead of the one being
+// computed, so the loads in flight hold no registers.  From its slot a lane
+// writes the K scaled dy vectors and adds to K partial dot products, which a
+// butterfly of shuffles inside the group sums at the end.  A lane only ever
+// reads what it copied itself, so the warp needs no barrier around the ring.
+// Measured on B200 (fraction of the measured copy bandwidth, graph of one
+// launch, L2 flushed): 0.92 -> 0.98 on the moderate EP8 workload and 0.96 ->
+// 1.01 on the 17-19 GB ones, against the earlier register-staged loop (116-128
+// registers, 16 warps per SM); outputs bit for bit the same.
+constexpr int CB_THREADS = 128;
+constexpr int CB_STAGES = 4;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__host__ __device__ __forceinline__ int combine_bwd_group(int64_t nvec) {
+  return nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : (int)nvec);
+}
+
+// Shared memory per warp: the ring [CB_STAGES][K + 1][32] of 16-byte vectors,
+// then the group's rows [gpw][K] and weights [gpw][K].
+__host__ __device__ __forceinline__ size_t combine_bwd_warp_bytes(int K, int gpw) {
+  return (size_t)CB_STAGES * (K + 1) * 512 + (size_t)2 * gpw * K * 4;
+}
+
 template <int K>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(CB_THREADS, 4)
     k_combine_bwd(const uint16_t* __restrict__ dout, const float* __restrict__ w, const uint16_t* __restrict__ y,
                   int64_t y_rows, const int32_t* __restrict__ pos, int64_t T, int64_t H, uint16_t* __restrict__ dy,
-                  float* __restrict__ dw, int64_t iters, int32_t* dev_status) {
+                  float* __restrict__ dw, int32_t* dev_status) {
+  extern __shared__ __align__(16) unsigned char cb_smem[];
   const int64_t nvec = H / 8;
-  const int G = nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : (int)nvec);
-  const int lane = threadIdx.x & 31;
-  const int gpw = 32 / G;                  // tokens per warp
+  const int G = combine_bwd_group(nvec);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gpw = 32 / G;
   const int sub = lane / G, gl = lane % G;
-  const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  unsigned char* mine = cb_smem + warp * combine_bwd_warp_bytes(K, gpw);
+  uint4* ring = reinterpret_cast<uint4*>(mine);  // [CB_STAGES][K + 1][32]
+  int32_t* s_r = reinterpret_cast<int32_t*>(mine + (size_t)CB_STAGES * (K + 1) * 512);
+  float* s_w = reinterpret_cast<float*>(s_r + gpw * K);
+  const int64_t t0 = (((int64_t)blockIdx.x * CB_THREADS + threadIdx.x) >> 5) * gpw;  // the warp's first token
+  if (t0 >= T) return;                                                             // warp-uniform
   int32_t bad = 0;
-  auto rows_of = [&](int64_t t, int32_t (&r)[K], float (&wk)[K]) {
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      r[k] = -1;
-      wk[k] = 0.0f;
-      if (t < T) {
-        r[k] = __ldg(pos + t * K + k);
-        wk[k] = __ldg(w + t * K + k);
-      }
-    }
-  };
-  // iters > 0: each warp owns `iters` consecutive groups of tokens (a
-  // non-persistent grid); else a persistent grid-stride loop
-  const int64_t tstep = iters > 0 ? gpw : nwarps * gpw;
-  int64_t tb = iters > 0 ? warp_id * gpw * iters : warp_id * gpw;
-  const int64_t tend = iters > 0 ? min(T, tb + gpw * iters) : T;
-  int32_t r[K];
-  float wk[K];
-  rows_of(tb + sub, r, wk);
-  for (; tb < tend; tb += tstep) {
-    const int64_t t = tb + sub;
-    int32_t rn[K];
-    float wn[K];
-    rows_of(tb + tstep + sub, rn, wn);  // the next token's, ahead of use
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-      if (t < T && (r[k] < 0 || r[k] >= y_rows)) {
-        r[k] = -1;
+  for (int i = lane; i < gpw * K; i += 32) {
+    const int64_t t = t0 + i / K;
+    int32_t r = -1;
+    float wk = 0.0f;
+    if (t < T) {
+      r = __ldg(pos + t * K + i % K);
+      wk = __ldg(w + t * K + i % K);
+      if (r < 0 || r >= y_rows) {  // reported, never read or written
+        r = -1;
         bad = EP_DEV_BAD_ROW;
       }
-    float part[K];
+    }
+    s_r[i] = r;
+    s_w[i] = wk;
+  }
+  __syncwarp();
+  const int64_t t = t0 + sub;
+  const int32_t* rr = s_r + sub * K;
+  const float* ww = s_w + sub * K;
+  const int nj = (int)((nvec + G - 1) / G);
+  auto issue = [&](int j) {
+    const int64_t v = gl + (int64_t)j * G;
+    if (j < nj && t < T && v < nvec) {
+      uint4* dst = ring + (size_t)(j % CB_STAGES) * (K + 1) * 32 + lane;
+      cp_async16(dst, dout + t * H + v * 8);
 #pragma unroll
-    for (int k = 0; k < K; ++k) part[k] = 0.0f;
-    if (t < T) {
-      for (int64_t v = gl; v < nvec; v += G) {
-        const uint4 g = ld_stream_v4(dout + t * H + v * 8);
-        uint4 in[K];
+      for (int k = 0; k < K; ++k)
+        if (rr[k] >= 0) cp_async16(dst + (k + 1) * 32, y + (int64_t)rr[k] * H + v * 8);
+    }
+    cp_async_commit();  // one group per job, empty or not, so the wait counts stay uniform
+  };
 #pragma unroll
-        for (int k = 0; k < K; ++k)
-          in[k] = r[k] >= 0 ? ld_stream_v4(y + (int64_t)r[k] * H + v * 8) : make_uint4(0, 0, 0, 0);
-        const uint32_t gd[4] = {g.x, g.y, g.z, g.w};
-        float gf[8];
+  for (int j = 0; j < CB_STAGES - 1; ++j) issue(j);
+  float part[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) part[k] = 0.0f;
+  for (int j = 0; j < nj; ++j) {
+    issue(j + CB_STAGES - 1);  // into the slot job j - 1 used (computed last iteration)
+    cp_async_wait<CB_STAGES - 1>();
+    const int64_t v = gl + (int64_t)j * G;
+    if (t < T && v < nvec) {
+      const uint4* src = ring + (size_t)(j % CB_STAGES) * (K + 1) * 32 + lane;
+      const uint4 g = src[0];
+      const uint32_t gd[4] = {g.x, g.y, g.z, g.w};
+      float gf[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        gf[2 * q] = bf16_bits_to_f32(gd[q] & 0xFFFFu);
+        gf[2 * q + 1] = bf16_bits_to_f32(gd[q] >> 16);
+      }
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int32_t r = rr[k];
+        if (r < 0) continue;
+        const float wk = ww[k];
+        const uint4 yk = src[(k + 1) * 32];
+        const uint32_t yd[4] = {yk.x, yk.y, yk.z, yk.w};
+        uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          gf[2 * q] = bf16_bits_to_f32(gd[q] & 0xFFFFu);
-          gf[2 * q + 1] = bf16_bits_to_f32(gd[q] >> 16);
+          o[q] = f32x2_to_bf16x2(__fmul_rn(wk, gf[2 * q]), __fmul_rn(wk, gf[2 * q + 1]));
+          part[k] = fmaf(gf[2 * q], bf16_bits_to_f32(yd[q] & 0xFFFFu), part[k]);
+          part[k] = fmaf(gf[2 * q + 1], bf16_bits_to_f32(yd[q] >> 16), part[k]);
         }
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          if (r[k] < 0) continue;
-          const uint32_t yd[4] = {in[k].x, in[k].y, in[k].z, in[k].w};
-          uint32_t o[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            o[q] = f32x2_to_bf16x2(__fmul_rn(wk[k], gf[2 * q]), __fmul_rn(wk[k], gf[2 * q + 1]));
-            part[k] = fmaf(gf[2 * q], bf16_bits_to_f32(yd[q] & 0xFFFFu), part[k]);
-            part[k] = fmaf(gf[2 * q + 1], bf16_bits_to_f32(yd[q] >> 16), part[k]);
-          }
-          st_v4(dy + (int64_t)r[k] * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
-        }
+        st_v4(dy + (int64_t)r * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
-    // add the group's partial products (every lane of the warp takes part)
+  }
+  cp_async_wait<0>();
+  // add the group's partial products (every lane of the warp takes part)
 #pragma unroll
-    for (int k = 0; k < K; ++k)
-      for (int d = G >> 1; d; d >>= 1) part[k] += __shfl_xor_sync(0xffffffffu, part[k], d);
-    if (t < T && gl == 0) {
+  for (int k = 0; k < K; ++k)
+    for (int d = G >> 1; d; d >>= 1) part[k] += __shfl_xor_sync(0xffffffffu, part[k], d);
+  if (t < T && gl == 0) {
 #pragma unroll
-      for (int k = 0; k < K; ++k) dw[t * K + k] = r[k] >= 0 ? part[k] : 0.0f;
-    }
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      r[k] = rn[k];
-      wk[k] = wn[k];
-    }
+    for (int k = 0; k < K; ++k) dw[t * K + k] = rr[k] >= 0 ? part[k] : 0.0f;
   }
   if (bad) flag(dev_status, bad);
 }
@@ -602,18 +637,19 @@ extern "C" int ep_combine_backward(const uint16_t* dout, const float* w, const u
     case 7: fn = (const void*)k_combine_bwd<7>; break;
     default: fn = (const void*)k_combine_bwd<8>; break;
   }
-  // one token per group of lanes, 8 warps per CTA; as many CTAs as fit
+  // one warp per token group (32 / G tokens), four warps per CTA
   const int64_t nvec = H / 8;
-  const int64_t G = nvec >= 32 ? 32 : nvec > 8 ? (nvec > 16 ? 32 : 16) : (nvec > 4 ? 8 : nvec > 2 ? 4 : nvec);
-  const int64_t ctas = (T + 8 * (32 / G) - 1) / (8 * (32 / G));
-  // Measured on B200: a persistent grid is fastest at 0.9 GB of rows (2% ahead
-  // of short CTAs), CTAs of two token groups per warp at 17-19 GB (4% ahead).
-  const int64_t iters = T * H >= ((int64_t)1 << 28) ? 2 : 0;
-  const int grid = iters > 0 ? (int)std::min<int64_t>((ctas + iters - 1) / iters, 0x7fffffff)
-                             : occupancy_grid(fn, 256, 0, ctas, 2);
+  const int G = combine_bwd_group(nvec);
+  const int gpw = 32 / G;
+  const int64_t groups = (T + gpw - 1) / gpw;
+  const int64_t ctas = (groups + CB_THREADS / 32 - 1) / (CB_THREADS / 32);
+  if (ctas > 0x7fffffff) return EP_ERR_ARG;
+  const size_t smem = (size_t)(CB_THREADS / 32) * combine_bwd_warp_bytes(K, gpw);
+  if (smem > 48 * 1024 && !raise_smem_limit(fn, smem)) return EP_ERR_CUDA;
+  const int grid = (int)ctas;
   void* args[] = {(void*)&dout, (void*)&w, (void*)&y, (void*)&y_rows, (void*)&pos, (void*)&T, (void*)&H, (void*)&dy,
-                  (void*)&dw, (void*)&iters, (void*)&dev_status};
-  if (cudaLaunchKernel(fn, dim3(grid), dim3(256), args, 0, stream) != cudaSuccess) return EP_ERR_CUDA;
+                  (void*)&dw, (void*)&dev_status};
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(CB_THREADS), args, smem, stream) != cudaSuccess) return EP_ERR_CUDA;
   count_launch();
   return launch_status();
 }
