@@ -11,22 +11,25 @@ reads the dispatched rows).  Metric: routed (token, k) pairs per second.
 Headline workload (default, --config 4): the fine-grained layer sequence,
 R=64 simulated EP ranks x S=8192 tokens, E=384 experts, top-K=8, H=7168 bf16,
 block_m=128, router bias b_e ~ N(0,1) redrawn for each of 8 consecutive
-layers; a step runs all 8 layers (4,194,304 pairs each, a 60 GB dispatch
-buffer shared by the layers).  It is the largest workload that fits one GPU.
-After it, the same run times the other four workloads (--others) with the same
-method and reports each under `workloads`.
+layers; a step runs all 8 layers (4,194,304 pairs each), chained as in one
+forward pass: layer l+1 dispatches the rows layer l combined (two row buffers
+and a 60 GB dispatch buffer shared by the layers).  It is the largest
+workload that fits one GPU.  After it, the same run times the other four
+workloads (--others) with the same method and reports each under `workloads`.
 
 `value`: device-resident inputs; the step is captured once as a CUDA graph and
 replayed K times, with CUDA events around each replay on the launching stream,
 L2 flushed (a 512 MB write) between replays outside the events, max over ranks.
 The per-op breakdown and the roofline come from an eager pass of the same K
-steps with CUDA events between the ops.  `e2e`: the same steps through the
-public API (layer.run_host_layers, EpLayer.run_host for every layer with the
-layers' copies overlapped) from pinned host buffers: each layer's routing,
-gate weights and hidden rows copied in and its combined rows copied out inside
-the timed region (the copies go in token slices over two copy streams; they
-are torch's, around the C-ABI kernels).  Under torchrun each rank runs its own independent layers (weak
-scaling, no data-path collective).
+steps with CUDA events between the ops.  `e2e`: the same step through the
+public API (layer.run_host_chain) from pinned host buffers: every layer's
+routing and gate weights and the batch's hidden rows copied in, the last
+layer's combined rows copied out, inside the timed region (in token slices
+over two copy streams, overlapping the first and the last layer; the copies
+are torch's, around the C-ABI kernels).  `e2e_rows_per_layer`: every layer's
+hidden rows in and combined rows out (layer.run_host_layers).  Under torchrun
+each rank runs its own independent layers (weak scaling, no data-path
+collective); --rank-local times the rank-local form instead.
 
 `cpu_baseline` and --impl reference time the CPU oracle (the plain
 single-threaded definition of the same path) on one host core, on a bounded
@@ -122,7 +125,8 @@ def config_obj(c):
     return {"workload": workload_desc(c), "layers": c["layers"], "R": c["R"], "S": c["S"], "E": c["E"], "K": c["K"],
             "H": c["H"], "tokens_per_layer": c["T"], "pairs_per_layer": c["P"], "pairs_per_step": c["P"] * c["layers"],
             "block_m": c["block_m"], "step": "per layer: route(" + "+".join(ROUTE_PARTS) + ")+dispatch+combine"
-            + ("+grad_reduce" if c["grad_n"] else "")}
+            + ("+grad_reduce" if c["grad_n"] else "")
+            + ("; layer l+1 dispatches the rows layer l combined" if c["layers"] > 1 else "")}
 
 
 def algorithmic_bytes(c, n_rep, n_chunks):
@@ -271,7 +275,7 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     import torch
     import token_dispatch_histogram_b200 as tdh
     import workload as W
-    from token_dispatch_histogram_b200.layer import run_host_layers
+    from token_dispatch_histogram_b200.layer import chain_buffers, run_host_chain, run_host_layers
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -286,6 +290,8 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     for i in range(nl):  # consecutive layers share the large buffers
         layers.append(tdh.EpLayer(R, S, K, E, H, c["block_m"], device=dev, grad_n=c["grad_n"] or 0, grad_dtype=gdt,
                                   share=layers[0] if layers else None))
+    # as in one forward pass, layer l+1 reads the rows layer l combined (two row buffers, nothing copied)
+    chain_buffers(layers)
     layer = layers[0]
 
     # inputs: host-generated routing (per layer); hidden rows and gradients
@@ -683,50 +689,62 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
                                   "max_rank_load_if_pairs_stay_home_over_SK": worst if nl > 1 else worst[0]}
         del pf_slot, pf_rem, pf_load
 
-    # ---- end to end through the public API, pinned host buffers: one
-    # run_host call per layer (its routing, gate weights and hidden rows in,
-    # its combined rows out)
+    # ---- end to end through the public API, pinned host buffers: the batch's
+    # hidden rows and every layer's routing in, the last layer's combined rows
+    # out (run_host_chain); and, for several layers, every layer's rows in and
+    # out (run_host_layers)
     e2e = None
+    e2e_rows = None
     if not args.no_e2e:
         topk_h = [torch.from_numpy(tk).pin_memory() for tk, _ in routes]
         w_h = [torch.from_numpy(ww).pin_memory() for _, ww in routes]
         x_h = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
+        W.fill_device(layer.x, seed, W.STREAM_X)
         x_h.copy_(layer.x)  # the generator's rows, as a caller's host batch
         out_h = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
+        route_bytes = sum(t.numel() * 4 for t in topk_h) + sum(t.numel() * 4 for t in w_h)
 
-        def host_step():  # the layers' copies overlap one another (run_host_layers)
-            run_host_layers(layers, topk_h, w_h, [x_h] * nl, [out_h] * nl, stream, fused=fused,
-                            chunks=args.e2e_chunks)
+        def timed_host(host_step, budget_ms):
+            host_step()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            host_step()
+            torch.cuda.synchronize()
+            n = side_steps(args.steps, (time.perf_counter() - t0) * 1e3, budget_ms)
+            for _ in range(max(0, min(2, args.warmup) - 1)):
+                host_step()
+            torch.cuda.synchronize()
+            barrier()
+            starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+            ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+            for i in range(n):
+                flush.fill_(i & 0xFF)
+                starts[i].record(stream)
+                host_step()
+                ends[i].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            check("in the end-to-end pass")
+            return max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev), n
 
-        host_step()
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        host_step()
-        torch.cuda.synchronize()
-        n_e2e = side_steps(args.steps, (time.perf_counter() - t0) * 1e3, 30000.0)
-        for _ in range(max(0, min(2, args.warmup) - 1)):
-            host_step()
-        torch.cuda.synchronize()
-        barrier()
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
-        for i in range(n_e2e):
-            flush.fill_(i & 0xFF)
-            starts[i].record(stream)
-            host_step()
-            ends[i].record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        check("in the end-to-end pass")
-        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
-        bi = sum(t.numel() * 4 for t in topk_h) + sum(t.numel() * 4 for t in w_h) + nl * x_h.numel() * 2
-        bo = nl * out_h.numel() * 2
-        e2e = {"value": job_throughput(world, nl * P, n_e2e, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": bi,
-               "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / n_e2e, "steps": n_e2e,
-               "chunks": args.e2e_chunks,
-               "what": "run_host_layers: per layer its routing, weights and hidden rows in from pinned host memory "
-                       "and its combined rows out (torch copies around the C-ABI kernels), in token slices on two "
-                       "copy streams, the next layer's inbound copies overlapping this layer's outbound ones"}
+        ms, n = timed_host(lambda: run_host_chain(layers, topk_h, w_h, x_h, out_h, stream, fused=fused,
+                                                  chunks=args.e2e_chunks), 30000.0)
+        e2e = {"value": job_throughput(world, nl * P, n, ms), "unit": UNIT,
+               "h2d_bytes_per_step": route_bytes + x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+               "ms_per_step": ms / n, "steps": n, "chunks": args.e2e_chunks,
+               "what": "run_host_chain: every layer's routing and weights and the batch's hidden rows in from pinned "
+                       "host memory, the layers in sequence (each reads the rows the one before combined), the last "
+                       "layer's combined rows out; torch copies around the C-ABI kernels, in token slices on two copy "
+                       "streams overlapping the first and the last layer"}
+        if nl > 1:
+            ms, n = timed_host(lambda: run_host_layers(layers, topk_h, w_h, [x_h] * nl, [out_h] * nl, stream,
+                                                       fused=fused, chunks=args.e2e_chunks), 20000.0)
+            e2e_rows = {"value": job_throughput(world, nl * P, n, ms), "unit": UNIT,
+                        "h2d_bytes_per_step": route_bytes + nl * x_h.numel() * 2,
+                        "d2h_bytes_per_step": nl * out_h.numel() * 2, "ms_per_step": ms / n, "steps": n,
+                        "what": "run_host_layers: every layer's hidden rows in from and its combined rows out to "
+                                "pinned host memory, the next layer's inbound copies overlapping this layer's "
+                                "outbound ones"}
         del topk_h, w_h, x_h, out_h
 
     # ---- roofline of the dominant kernel and the per-op breakdown (bytes summed over layers)
@@ -766,6 +784,7 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
         "l2": L2_NOTE,
         "roofline": roofline,
         "e2e": e2e,
+        "e2e_rows_per_layer": e2e_rows,
         "gpu_launches": graph["launches"] if graph else int(launches),
         "clocks": graph["clocks"] if graph else clk,
         "timing": ("one captured CUDA graph per step, replayed; CUDA events around each replay"

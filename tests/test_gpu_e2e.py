@@ -99,3 +99,49 @@ def test_run_host_layers_matches_each_layer(chunks):
     run_host_layers(layers, topk_hs, w_hs, x_hs, [shared] * 3, grads=False, chunks=chunks)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(shared.view(torch.int16).numpy().view(np.uint16), refs[-1])
+
+
+@pytest.mark.parametrize("chunks", [1, 5, 8])
+@pytest.mark.parametrize("nl", [1, 2, 3])
+def test_run_host_chain_matches_the_oracle_chain(nl, chunks):
+    """Layers chained on two row buffers (layer l+1 dispatches the rows layer l
+    combined), fed from the host (run_host_chain): the batch's hidden rows in,
+    the last layer's combined rows out, equal to the oracle's chain of
+    dispatch and combine through every layer's own routing; and equal to the
+    same chain run on device-resident inputs."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    from token_dispatch_histogram_b200.layer import chain_buffers, run_host_chain
+    R, S, K, E, H, bm = 8, 384, 6, 64, 512, 64
+    T = R * S
+    layers = []
+    for _ in range(nl):
+        layers.append(tdh.EpLayer(R, S, K, E, H, bm, device="cuda", share=layers[0] if layers else None))
+    chain_buffers(layers)
+    assert nl == 1 or layers[1].x.data_ptr() == layers[0].out.data_ptr()
+    routes = [W.routing_from(T, E, K, seed=40 + l, bias_e=W.bias(2, l)) for l in range(nl)]
+    x = W.hidden(T, H, seed=50)
+    want = x
+    for tk, w in routes:
+        loads, _, _ = O.route_stats(tk, E)
+        pl = O.plan(loads, R, S, K, E)
+        lo = O.layout(tk, pl, R, S, E)
+        want = O.combine(O.dispatch(want, lo["pos"], K, T * K), w, lo["pos"], K)
+    topk_hs = [torch.from_numpy(tk).pin_memory() for tk, _ in routes]
+    w_hs = [torch.from_numpy(w).pin_memory() for _, w in routes]
+    x_h = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_h = torch.zeros((T, H), dtype=torch.bfloat16).pin_memory()
+    run_host_chain(layers, topk_hs, w_hs, x_h, out_h, grads=False, chunks=chunks)
+    torch.cuda.synchronize()
+    assert all(ly.status() == 0 for ly in layers)
+    np.testing.assert_array_equal(out_h.view(torch.int16).numpy().view(np.uint16), want)
+    # the same chain on the device
+    layers[0].x.copy_(x_h)
+    for ly, tk in zip(layers, topk_hs):
+        ly.topk_ids.copy_(tk)
+    for ly, w in zip(layers, w_hs):
+        ly.w.copy_(w)
+    for ly in layers:
+        ly.step(grads=False)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(layers[-1].out.view(torch.int16).cpu().numpy().view(np.uint16), want)

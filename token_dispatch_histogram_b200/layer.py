@@ -247,13 +247,17 @@ def run_host_layers(layers, topk_hs, w_hs, x_hs, out_hs, stream=None, grads=True
         ly.route(main, fused)
         bounds = slice_bounds(ly.T, max(1, min(chunks, ly.T)))
         K = ly.K
-        same_x = prev is not None and prev[0].data_ptr() == ly.x.data_ptr()
-        same_out = prev is not None and prev[1].data_ptr() == ly.out.data_ptr()
+        ptr = (lambda t: t.data_ptr())
+        same_x = prev is not None and ptr(prev[0]) == ptr(ly.x)
+        x_is_prev_out = prev is not None and ptr(prev[1]) == ptr(ly.x)  # chained layers (chain_buffers)
+        same_out = prev is not None and ptr(prev[1]) == ptr(ly.out)
         dispatched, sent = [], []
         for j, (t0, t1) in enumerate(zip(bounds[:-1], bounds[1:])):
             with torch.cuda.stream(h2d):
                 if same_x:
                     h2d.wait_event(prev[2][j])  # the layer before has read these rows of x
+                if x_is_prev_out:
+                    h2d.wait_event(prev[3][j])  # the layer before's rows here have left for the host
                 ly.x[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
                 arrived = torch.cuda.Event()
                 arrived.record(h2d)
@@ -276,5 +280,87 @@ def run_host_layers(layers, topk_hs, w_hs, x_hs, out_hs, stream=None, grads=True
         if grads:
             ly.grad_reduce(False, main)
         prev = (ly.x, ly.out, dispatched, sent)
+    main.wait_stream(d2h)
+    main.wait_stream(h2d)
+
+
+def chain_buffers(layers):
+    """Make consecutive layers a chain on two row buffers: layer l reads its
+    hidden rows from the buffer layer l-1 combined into (layer 0 from the first
+    one), as the MoE layers of one forward pass do.  The layers must share
+    their row buffers (EpLayer(share=...)); nothing is copied."""
+    if not layers:
+        return
+    a, b = layers[0].x, layers[0].out
+    for i, ly in enumerate(layers):
+        if ly.x.data_ptr() not in (a.data_ptr(), b.data_ptr()) or ly.out.data_ptr() not in (a.data_ptr(), b.data_ptr()):
+            raise ValueError("chained layers must share their row buffers")
+        ly.x, ly.out = (a, b) if i % 2 == 0 else (b, a)
+
+
+def run_host_chain(layers, topk_hs, w_hs, x_h, out_h, stream=None, grads=True, fused=True, chunks=8):
+    """A chain of layers (chain_buffers) fed from pinned host memory: every
+    layer's routing and gate weights and the batch's hidden rows in, the last
+    layer's combined rows out.
+
+    The hidden rows arrive in token slices and the first layer dispatches and
+    combines each slice as it lands; the middle layers run on the device; the
+    last layer combines slice by slice and each slice leaves as soon as it is
+    combined.  Routing for the later layers is copied behind the first layer's
+    rows on the same copy stream.  With one layer this is EpLayer.run_host.
+    The caller's stream waits for the last copy out."""
+    n = len(layers)
+    if not (len(topk_hs) == len(w_hs) == n) or n == 0:
+        raise ValueError("one routing and weight buffer per layer")
+    first, last = layers[0], layers[-1]
+    main = stream if stream is not None else torch.cuda.current_stream(first.device)
+    h2d, d2h = first._copy_streams()
+    h2d.wait_stream(main)
+    d2h.wait_stream(main)
+    T, K = first.T, first.K
+    bounds = slice_bounds(T, max(1, min(chunks, T)))
+    spans = list(zip(bounds[:-1], bounds[1:]))
+    routed = []
+    with torch.cuda.stream(h2d):
+        first.topk_ids.copy_(topk_hs[0], non_blocking=True)
+        first.w.copy_(w_hs[0], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(h2d)
+        routed.append(ev)
+    arrived = []
+    for t0, t1 in spans:
+        with torch.cuda.stream(h2d):
+            first.x[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(h2d)
+            arrived.append(ev)
+    with torch.cuda.stream(h2d):
+        for ly, tk, w in zip(layers[1:], topk_hs[1:], w_hs[1:]):
+            ly.topk_ids.copy_(tk, non_blocking=True)
+            ly.w.copy_(w, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(h2d)
+            routed.append(ev)
+    for li, ly in enumerate(layers):
+        main.wait_event(routed[li])
+        ly.route(main, fused)
+        if li == 0 or li == n - 1:
+            # a token slice's combine reads only the rows its own dispatch wrote
+            for j, (t0, t1) in enumerate(spans):
+                if li == 0:
+                    main.wait_event(arrived[j])
+                ep_dispatch(ly.x[t0:t1], K, ly.pos[t0 * K:t1 * K], ly.buf, ly.dev_status, main)
+                ep_combine(ly.buf, ly.w[t0:t1], ly.pos[t0 * K:t1 * K], ly.out[t0:t1], ly.dev_status, main)
+                if li == n - 1:
+                    combined = torch.cuda.Event()
+                    combined.record(main)
+                    d2h.wait_event(combined)
+                    with torch.cuda.stream(d2h):
+                        out_h[t0:t1].copy_(ly.out[t0:t1], non_blocking=True)
+        else:
+            ly.dispatch(main)
+            ly.combine(main)
+        if grads:
+            ly.grad_reduce(False, main)
     main.wait_stream(d2h)
     main.wait_stream(h2d)
