@@ -122,3 +122,21 @@ def test_side_measurement_replays():
     assert bench.side_steps(20, 0.4) == 20          # short steps: all of them
     assert bench.side_steps(20, 163.0) == 15        # 2.5 s of replays
     assert bench.side_steps(20, 5000.0) == 3        # at least three
+
+
+def test_reference_arm_runs_on_the_host():
+    """bench.py --impl reference (the CPU oracle on a sample of the workload)
+    runs on a machine without a GPU and prints one JSON line whose config is
+    the one our arm prints for the same workload."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "1",
+                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    import bench
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["value"] > 0
+    assert line["config"] == bench.config_obj(bench.workload_shape(1))
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
