@@ -753,7 +753,9 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     peak, peak_kind = peaks()
     mean_ms = {op: per_op[op] / args.steps for op in OPS}  # per step (all layers)
     dom = max(("dispatch", "combine", "grad_reduce"), key=lambda op: mean_ms[op])
-    kernel_of = {"dispatch": "k_dispatch", "combine": "k_combine", "grad_reduce": "k_grad_reduce"}
+    # the library's combine for problems of 2^28 row elements and more (K <= 8) is its shared-memory ring kernel
+    kernel_of = {"dispatch": "k_dispatch", "combine": "k_combine_ring" if T * H >= (1 << 28) and K <= 8 else "k_combine",
+                 "grad_reduce": "k_grad_reduce"}
     achieved = ab[dom] / (mean_ms[dom] / 1e3) / 1e9 if mean_ms[dom] else 0.0
     tr = traffic_record(kernel_of[dom], c)
     roofline = {"bound": "hbm", "kernel": kernel_of[dom], "achieved": round(achieved, 1), "peak": peak,

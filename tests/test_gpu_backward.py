@@ -46,7 +46,9 @@ def _run(topk, w, R, S, E, H, seed, rows_extra=0):
 
 
 @pytest.mark.parametrize("case", [(4, 64, 2, 16, 128), (8, 256, 6, 64, 2048), (4, 97, 8, 32, 7168),
-                                  (2, 50, 1, 4, 64), (3, 33, 5, 9, 24), (16, 64, 8, 256, 4096)],
+                                  (2, 50, 1, 4, 64), (3, 33, 5, 9, 24), (16, 64, 8, 256, 4096),
+                                  # odd K with one token per warp: the per-warp shared-memory regions' alignment
+                                  (4, 100, 3, 16, 2048), (4, 61, 5, 16, 1024), (2, 90, 7, 8, 520)],
                          ids=lambda c: "R{}_S{}_K{}_E{}_H{}".format(*c))
 def test_backward_matches_oracle(case):
     R, S, K, E, H = case
