@@ -389,8 +389,11 @@ EP_API int ep_expert_scale(const uint16_t* buf, int64_t rows, int64_t H, const i
  * a6. Combine.  out[t] = bf16_rn( sum_{k=0..K-1} w[t,k] * float(y[pos[t*K+k]]) ),
  * accumulated in fp32 in k order from 0, each product and sum rounded
  * separately (no fused multiply-add), one rounding to bf16 at the end.
- *   y [y_rows, H] bf16; w [T, K] fp32; pos [P] int32; out [T, H] bf16 out.
+ *   y [y_rows, H] bf16; w [T, K] fp32 (NULL: unit weights); pos [P] int32; out [T, H] bf16 out.
  *   Pairs whose pos is outside [0, y_rows) contribute nothing and are flagged.
+ *   From T*H >= 2^28 with K <= 8 the rows are read through a per-warp
+ *   shared-memory ring (cp.async); below, each thread loads its K vectors into
+ *   registers.  The two give the same bits.
  */
 EP_API int ep_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* pos, int64_t T, int K, int64_t H,
                uint16_t* out, int32_t* dev_status, cudaStream_t stream);
