@@ -710,7 +710,8 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
             t0 = time.perf_counter()
             host_step()
             torch.cuda.synchronize()
-            n = side_steps(args.steps, (time.perf_counter() - t0) * 1e3, budget_ms)
+            first_ms = max_over_ranks((time.perf_counter() - t0) * 1e3, world, dev)  # every rank takes the same count
+            n = side_steps(args.steps, first_ms, budget_ms)
             for _ in range(max(0, min(2, args.warmup) - 1)):
                 host_step()
             torch.cuda.synchronize()
