@@ -172,15 +172,17 @@ class RankLocalJob:
                 rk.set_grad_peers(gpeers)
 
     def route(self, stream=None):
-        for rk in self.ranks:
-            rk.count(stream)
-        rows = torch.stack([rk.counts_row for rk in self.ranks])
-        if self.world > 1:
-            rows = all_gather_rows(rows, self.group)
-        self.counts.copy_(rows)
-        for rk in self.ranks:
-            rk.counts.copy_(self.counts)
-            rk.plan_and_layout(stream)
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(st):  # the row copies in order with the kernels
+            for rk in self.ranks:
+                rk.count(st)
+            rows = torch.stack([rk.counts_row for rk in self.ranks])
+            if self.world > 1:
+                rows = all_gather_rows(rows, self.group)
+            self.counts.copy_(rows)
+            for rk in self.ranks:
+                rk.counts.copy_(self.counts)
+                rk.plan_and_layout(st)
 
     def dispatch(self, stream=None):
         for rk in self.ranks:
