@@ -71,6 +71,7 @@ struct FusedArgs {
   int64_t expert_ids_cap;
   int32_t* ntpp;
   int32_t* dev_status;
+  int stage;            // tile CTAs stage their pairs in shared memory; src and sorted ids go out in runs
   // fused dispatch (DISPATCH = true only)
   const uint8_t* x;     // [T, row_bytes] token rows
   uint8_t* buf;         // [buf_rows, row_bytes]
@@ -83,6 +84,41 @@ struct FusedArgs {
 };
 
 constexpr int WALK_UNROLL = 8;  // tile loads each lane keeps in flight during a walk
+constexpr int SWEEP_RUN = 256;  // entries of an expert's run its own warp writes; the rest, all warps
+
+// A pair's layout row from its expert e and stable rank g within e (the plan
+// in shared memory): the home copy takes ranks [0, home_count), then the
+// expert's replicas in order, replica m ranks [rep_begin, rep_begin +
+// rep_count).  slot = e (home) or E + m; -1 when g lies outside every copy.
+struct RowMap {
+  const int32_t *hc, *hb, *cf, *cc, *rb, *rc, *rbase;
+  int n_rep, E;
+  __device__ __forceinline__ int32_t row(int e, int32_t g, int32_t* slot) const {
+    if (g < hc[e]) {
+      *slot = e;
+      return hb[e] + g;
+    }
+    if (cc[e] > 0) {
+      int lo = cf[e], hi = cf[e] + cc[e] - 1;  // last replica with rep_begin <= g
+      if (lo >= 0 && hi < n_rep) {
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (rb[mid] <= g)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        const int32_t off = g - rb[lo];
+        if (off >= 0 && off < rc[lo]) {
+          *slot = E + lo;
+          return rbase[lo] + off;
+        }
+      }
+    }
+    *slot = -1;
+    return -1;
+  }
+};
 
 // Walk this warp's part of the tile in flattened order; `run` is the warp's
 // running per-expert count (initialised to the rank of its first pair).  Ids
@@ -224,8 +260,15 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   int32_t* s_rb = s_cc + E;                    // [cap] rep_begin
   int32_t* s_rc = s_rb + cap;                  // [cap] rep_count
   int32_t* s_rbase = s_rc + cap;               // [cap] rep_base
+  // staged sweep only: tile count per expert, its run's base in the stage
+  // (less the tile prefix), experts with runs longer than SWEEP_RUN, and the
+  // tile's pairs (offsets from the tile's first pair) in (expert, rank) order
+  int32_t* s_tc = s_rbase + cap;               // [E]
+  int32_t* s_tb = s_tc + E;                    // [E]
+  int32_t* s_long = s_tb + E;                  // [E]
+  uint16_t* s_stage = reinterpret_cast<uint16_t*>(s_long + E);  // [tile]
   __shared__ int32_t warp_sums[32];
-  __shared__ int s_bad, s_badrow;
+  __shared__ int s_bad, s_badrow, s_nlong;
   __shared__ int32_t s_max[FUSED_WARPS];
   const int64_t p0 = (int64_t)t * tile;
   const int64_t wp0 = p0 + (int64_t)warp * sub;
@@ -263,6 +306,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
         run += c;
       }
       a.counts[(int64_t)e * NT + t] = run;
+      if (a.stage) s_tc[e] = run;
       if (run) atomicAdd(a.tot + e, run);
     }
   }
@@ -343,6 +387,18 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
     if (t == 0 && tid == 0) *a.ntpp = total;  // tile 0 always exists when P > 0
     __syncthreads();
   }
+  if (a.stage && has_tile) {
+    // where each expert's run starts in the stage: an exclusive scan of the
+    // tile counts, less the tile prefix (so a pair of rank g sits at s_tb[e] + g)
+    for (int e = tid; e < E; e += FUSED_THREADS) s_tb[e] = s_tc[e];
+    if (tid == 0) s_nlong = 0;
+    __syncthreads();
+    block_scan_inplace(s_tb, E, warp_sums);
+    for (int e = tid; e < E; e += FUSED_THREADS) {
+      s_tb[e] -= s_excl[e];
+      if (s_tc[e] > SWEEP_RUN) s_long[atomicAdd(&s_nlong, 1)] = e;  // list order is free: writes are disjoint
+    }
+  }
 
   // ---- 4. layout ranks once the plan is out
   if (!has_tile) return;
@@ -367,30 +423,18 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   int32_t* pair_slot = a.pair_slot;
   int32_t* sorted_ids = a.sorted_ids;
   const int64_t P = a.P;
+  const RowMap rm{s_hc, s_hb, s_cf, s_cc, s_rb, s_rc, s_rbase, n_rep, E};
+  const bool stage = a.stage != 0;
+  const int32_t p0_32 = (int32_t)p0;  // P < 2^31
   walk_warp(a.topk, P, E, wp0, sub, s_run + warp * E,
             [&](int64_t p, int e, int32_t g) {
-              if (sorted_ids) sorted_ids[s_off[e] + g] = (int32_t)p;  // align-sort: same rank within the expert
-              int32_t row = -1, slot = -1;
-              if (g < s_hc[e]) {
-                row = s_hb[e] + g;
-                slot = e;
-              } else if (s_cc[e] > 0) {
-                int lo = s_cf[e], hi = s_cf[e] + s_cc[e] - 1;  // last replica with rep_begin <= g
-                if (lo >= 0 && hi < n_rep) {
-                  while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (s_rb[mid] <= g)
-                      lo = mid;
-                    else
-                      hi = mid - 1;
-                  }
-                  const int32_t off = g - s_rb[lo];
-                  if (off >= 0 && off < s_rc[lo]) {
-                    row = s_rbase[lo] + off;
-                    slot = E + lo;
-                  }
-                }
-              }
+              if (stage) {  // sorted id and src: the sweep below (q < tile by the count pass; checked)
+                const int32_t q = s_tb[e] + g;
+                if ((uint32_t)q < (uint32_t)a.tile) s_stage[q] = (uint16_t)((int32_t)p - p0_32);
+              } else if (sorted_ids)
+                sorted_ids[s_off[e] + g] = (int32_t)p;  // align-sort: same rank within the expert
+              int32_t slot;
+              const int32_t row = rm.row(e, g, &slot);
               if (row < 0 || row >= P) {
                 s_badrow = 1;
                 pos[p] = -1;
@@ -398,7 +442,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
                 return;
               }
               pos[p] = row;
-              src[row] = (int32_t)p;
+              if (!stage) src[row] = (int32_t)p;
               if (pair_slot) pair_slot[p] = slot;
             },
             &s_bad);
@@ -414,6 +458,32 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
       }
     }
   }
+  if (stage) {
+    // the staged sweep: each expert's run of this tile holds consecutive
+    // ranks, so its align-sort ids and (within one copy) its src rows are
+    // consecutive words; a warp writes its own experts' runs up to SWEEP_RUN
+    // entries, then all warps write the rest of the longer runs
+    auto put = [&](int e, int32_t i, int32_t qbase, int32_t g0, int32_t so) {
+      const int32_t p = p0_32 + (int32_t)s_stage[qbase + i];
+      const int32_t g = g0 + i;
+      if (sorted_ids) sorted_ids[so + g] = p;
+      int32_t slot;
+      const int32_t row = rm.row(e, g, &slot);
+      if (row >= 0 && row < P) src[row] = p;
+    };
+    for (int e = warp; e < E; e += FUSED_WARPS) {
+      const int32_t n = min(s_tc[e], SWEEP_RUN);
+      const int32_t g0 = s_excl[e], qbase = s_tb[e] + g0, so = sorted_ids ? s_off[e] : 0;
+      for (int32_t i = lane; i < n; i += 32) put(e, i, qbase, g0, so);
+    }
+    const int nlong = s_nlong;
+    for (int j = 0; j < nlong; ++j) {
+      const int e = s_long[j];
+      const int32_t n = s_tc[e];
+      const int32_t g0 = s_excl[e], qbase = s_tb[e] + g0, so = sorted_ids ? s_off[e] : 0;
+      for (int32_t i = SWEEP_RUN + tid; i < n; i += FUSED_THREADS) put(e, i, qbase, g0, so);
+    }
+  }
   if (tid == 0) {
     if (s_bad) flag(a.dev_status, EP_DEV_BAD_EXPERT_ID);
     if (s_badrow) flag(a.dev_status, EP_DEV_BAD_ROW);
@@ -424,10 +494,12 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_route_fused(FusedArgs a) {
   }
 }
 
-size_t fused_smem_bytes(int E, int R) {
+// stage_tile > 0: with the staged sweep's tables and a tile of that many pairs
+size_t fused_smem_bytes(int E, int R, int64_t stage_tile = 0) {
   const int cap = E + R - 1;
-  const size_t words = (size_t)FUSED_WARPS * E + std::max(FUSED_WARPS * E, plan_work_words(E, R)) + 3 * (size_t)E +
-                       1 + 4 * (size_t)E + 3 * (size_t)cap;
+  size_t words = (size_t)FUSED_WARPS * E + std::max(FUSED_WARPS * E, plan_work_words(E, R)) + 3 * (size_t)E +
+                 1 + 4 * (size_t)E + 3 * (size_t)cap;
+  if (stage_tile > 0) words += 3 * (size_t)E + ((size_t)stage_tile + 1) / 2;
   return words * sizeof(int32_t);
 }
 
@@ -457,6 +529,14 @@ static CopyShape copy_shape(uint32_t row_bytes, int K, int per_sm) {
   c.bytes = (size_t)c.warps * c.stages * (stride_b + 8 + 4 * (size_t)K);
   return c;
 }
+
+// Smallest tile that stages its pairs.  Measured on B200 with the L2 flushed
+// before each route (as in a step, where dispatch and combine stream far more
+// than the L2 between routes): tiles of 14,336 pairs (4.2M pairs, E = 384)
+// 104.4 -> 90.1 us per route; tiles of 7,168 (2.1M pairs, E = 256) 53.4 ->
+// 57.2 us and of 3,584 (1M pairs) 34.8 -> 43.1 us, the sweep costing more
+// than the scattered stores it replaces.
+constexpr int64_t STAGE_MIN_TILE = 12288;
 
 // ep_route_fused, and with x != nullptr the dispatch of x into buf in the
 // same launch (ep_route_dispatch_fused).
@@ -518,13 +598,24 @@ static int route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, 
     const int64_t t1 = ((P + num_sms() - 2) / (num_sms() - 1) + 511) / 512 * 512;
     if (t1 <= 2048 && resident_ok(1, smem_for(1))) per_sm = 1;
   }
-  const size_t smem = per_sm ? smem_for(per_sm) : 0;
+  size_t smem = per_sm ? smem_for(per_sm) : 0;
   const int64_t resident = (int64_t)num_sms() * per_sm;
   int64_t tile = 0, ntiles = 0;
   if (resident > 1) {  // one CTA per tile plus the planner CTA
     tile = (P + resident - 2) / (resident - 1);
     tile = std::max<int64_t>(512, (tile + 511) / 512 * 512);
     ntiles = (P + tile - 1) / tile;
+  }
+  // Large tiles stage their pairs in shared memory (16-bit offsets) when that
+  // still leaves the grid resident: the walk's scattered 4-byte stores of src
+  // and the align-sort ids become runs of consecutive words.
+  bool stage = false;
+  if (!dispatch && per_sm > 0 && tile >= STAGE_MIN_TILE && tile <= 65536) {
+    const size_t ss = (fused_smem_bytes(E, R, tile) + 127) & ~(size_t)127;
+    if (resident_ok(per_sm, ss)) {
+      stage = true;
+      smem = ss;
+    }
   }
   // the [E][tiles] counts must fit below T_e (the separate path's regions are unused here)
   const bool fits = resident > 1 && ntiles + 1 <= resident && tile <= (1 << 20) &&
@@ -567,6 +658,7 @@ static int route_fused(const int32_t* topk_ids, int64_t T, int K, int E, int R, 
   args.expert_ids_cap = expert_ids_cap;
   args.ntpp = num_tokens_post_pad;
   args.dev_status = dev_status;
+  args.stage = stage ? 1 : 0;
   if (dispatch) {
     const CopyShape c = copy_shape(row_bytes, K, per_sm);
     args.x = reinterpret_cast<const uint8_t*>(x);
