@@ -21,12 +21,14 @@ workloads (--others) with the same method and reports each under `workloads`.
 replayed K times, with CUDA events around each replay on the launching stream,
 L2 flushed (a 512 MB write) between replays outside the events, max over ranks.
 The per-op breakdown and the roofline come from an eager pass of the same K
-steps with CUDA events between the ops.  `e2e`: the same step through the
-public API (layer.run_host_chain) from pinned host buffers: every layer's
-routing and gate weights and the batch's hidden rows copied in, the last
-layer's combined rows copied out, inside the timed region (in token slices
-over two copy streams, overlapping the first and the last layer; the copies
-are torch's, around the C-ABI kernels).  `e2e_rows_per_layer`: every layer's
+steps with CUDA events between the ops.  `e2e`: the same steps through the
+public API (layer.run_host_batches) from pinned host buffers: every batch's
+routing and gate weights for every layer and its hidden rows copied in, the
+last layer's combined rows copied out, all inside one timed region, batch b+1's
+inbound copies running while batch b's layers run and its outbound copies
+drain (in token slices over two copy streams; the copies are torch's, around
+the C-ABI kernels); `e2e.one_batch_at_a_time`: each batch alone
+(layer.run_host_chain), timed step by step.  `e2e_rows_per_layer`: every layer's
 hidden rows in and combined rows out (layer.run_host_layers).  Under torchrun
 each rank runs its own independent layers (weak scaling, no data-path
 collective); --rank-local times the rank-local form instead.
@@ -79,7 +81,11 @@ def parse(argv=None):
     ap.add_argument("--hidden", type=int, default=None,
                     help="override H (e.g. a full-size route with small rows, for a profiler capture of the route)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=12, help="token slices of the host-fed pipeline")
+    ap.add_argument("--e2e-chunks", type=int, default=12, help="token slices of the host-fed pipeline, one batch at a time")
+    ap.add_argument("--e2e-batch-chunks", type=int, default=4,
+                    help="token slices per batch with batches in flight (measured on B200: moderate EP8 3.03 ms per "
+                         "batch with 2 slices, 3.05 with 4, 3.19 with 12; the fine-grained workload 200-201 ms for "
+                         "4 to 24)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the backward of dispatch and combine")
     ap.add_argument("--no-quota", action="store_true", help="skip timing the quota-driven planner")
@@ -275,7 +281,7 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     import torch
     import token_dispatch_histogram_b200 as tdh
     import workload as W
-    from token_dispatch_histogram_b200.layer import chain_buffers, run_host_chain, run_host_layers
+    from token_dispatch_histogram_b200.layer import chain_buffers, run_host_batches, run_host_chain, run_host_layers
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -691,8 +697,9 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
 
     # ---- end to end through the public API, pinned host buffers: the batch's
     # hidden rows and every layer's routing in, the last layer's combined rows
-    # out (run_host_chain); and, for several layers, every layer's rows in and
-    # out (run_host_layers)
+    # out -- batches in flight (run_host_batches) and one batch at a time
+    # (run_host_chain); and, for several layers, every layer's rows in and out
+    # (run_host_layers)
     e2e = None
     e2e_rows = None
     if not args.no_e2e:
@@ -730,13 +737,83 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
 
         ms, n = timed_host(lambda: run_host_chain(layers, topk_h, w_h, x_h, out_h, stream, fused=fused,
                                                   chunks=args.e2e_chunks), 30000.0)
-        e2e = {"value": job_throughput(world, nl * P, n, ms), "unit": UNIT,
-               "h2d_bytes_per_step": route_bytes + x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
-               "ms_per_step": ms / n, "steps": n, "chunks": args.e2e_chunks,
-               "what": "run_host_chain: every layer's routing and weights and the batch's hidden rows in from pinned "
-                       "host memory, the layers in sequence (each reads the rows the one before combined), the last "
-                       "layer's combined rows out; torch copies around the C-ABI kernels, in token slices on two copy "
-                       "streams overlapping the first and the last layer"}
+        alone = {"value": job_throughput(world, nl * P, n, ms), "unit": UNIT,
+                 "h2d_bytes_per_step": route_bytes + x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+                 "ms_per_step": ms / n, "steps": n, "chunks": args.e2e_chunks,
+                 "what": "run_host_chain, one batch at a time (each timed alone, L2 flushed before it): every layer's "
+                         "routing and weights and the batch's hidden rows in from pinned host memory, the layers in "
+                         "sequence (each reads the rows the one before combined), the last layer's combined rows "
+                         "out; torch copies around the C-ABI kernels, in token slices on two copy streams "
+                         "overlapping the first and the last layer"}
+        e2e = alone
+        # the host link alone, for the same bytes: the batch's hidden rows in and the combined rows out as whole
+        # copies, each direction alone and both at once (the floor any host-fed step on this machine has)
+        h2d_s, d2h_s = layer._copy_streams()
+
+        def link_ms(inbound, outbound, reps=3):
+            best = None
+            for _ in range(reps):
+                torch.cuda.synchronize()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                h2d_s.wait_stream(stream)
+                d2h_s.wait_stream(stream)
+                if inbound:
+                    with torch.cuda.stream(h2d_s):
+                        layer.x.copy_(x_h, non_blocking=True)
+                if outbound:
+                    with torch.cuda.stream(d2h_s):
+                        out_h.copy_(layer.out, non_blocking=True)
+                stream.wait_stream(h2d_s)
+                stream.wait_stream(d2h_s)
+                b.record(stream)
+                torch.cuda.synchronize()
+                t = a.elapsed_time(b)
+                best = t if best is None else min(best, t)
+            return max_over_ranks(best, world, dev)
+
+        host_link = {"rows_in_ms": round(link_ms(True, False), 4), "rows_out_ms": round(link_ms(False, True), 4),
+                     "both_ms": round(link_ms(True, True), 4), "bytes_each_way": x_h.numel() * 2,
+                     "what": "the batch's hidden rows copied in and the combined rows copied out as one whole copy "
+                             "each (pinned host memory), each direction alone and both at once; best of 3"}
+        alone["host_link"] = host_link
+        # batches in flight: batch b+1's rows come in while batch b's layers run and its rows go out
+        # (run_host_batches with stage buffers apart from the chain's row buffers)
+        if 2 * x_h.numel() * 2 + (2 << 30) <= torch.cuda.mem_get_info(dev)[0]:
+            x_stage = torch.empty_like(layer.x)
+            out_stage = torch.empty_like(layer.x)
+            nb = side_steps(args.steps, alone["ms_per_step"], 30000.0)
+
+            def batches(k):
+                run_host_batches(layers, [(topk_h, w_h, x_h, out_h)] * k, x_stage, out_stage, stream, fused=fused,
+                                 chunks=args.e2e_batch_chunks)
+
+            batches(2)
+            torch.cuda.synchronize()
+            barrier()
+            flush.fill_(0)
+            b0 = torch.cuda.Event(enable_timing=True)
+            b1 = torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            batches(nb)
+            b1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            check("in the batched end-to-end pass")
+            ms_b = max_over_ranks(b0.elapsed_time(b1), world, dev)
+            e2e = {"value": job_throughput(world, nl * P, nb, ms_b), "unit": UNIT,
+                   "h2d_bytes_per_step": alone["h2d_bytes_per_step"], "d2h_bytes_per_step": alone["d2h_bytes_per_step"],
+                   "ms_per_step": ms_b / nb, "steps": nb, "chunks": args.e2e_batch_chunks,
+                   "what": f"run_host_batches: {nb} batches (steps) in one timed region, each batch's routing and "
+                           "weights for every layer and its hidden rows in from pinned host memory and the last "
+                           "layer's combined rows out, every copy inside the region; batch b+1's inbound copies "
+                           "run while batch b's layers run and its outbound copies drain (stage buffers apart from "
+                           "the chain's row buffers); torch copies around the C-ABI kernels, in token slices on "
+                           "two copy streams; L2 flushed once before the region, not between the batches (each "
+                           "batch's rows are larger than the L2 on every workload but the tiny one)",
+                   "host_link": host_link, "one_batch_at_a_time": alone}
+            del x_stage, out_stage
         if nl > 1:
             ms, n = timed_host(lambda: run_host_layers(layers, topk_h, w_h, [x_h] * nl, [out_h] * nl, stream,
                                                        fused=fused, chunks=args.e2e_chunks), 20000.0)

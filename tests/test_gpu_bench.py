@@ -34,6 +34,8 @@ def test_bench_line_has_every_field():
     assert abs(r["frac"] - r["achieved"] / r["peak"]) <= 1e-4 + 1e-3 * r["frac"]  # both rounded in the line
     e = line["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert e["value"] == pytest.approx(P / (e["ms_per_step"] / 1e3), rel=1e-6)
+    assert "run_host_batches" in e["what"] and e["one_batch_at_a_time"]["value"] > 0  # batches in flight, and alone
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
 
 

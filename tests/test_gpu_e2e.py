@@ -101,6 +101,19 @@ def test_run_host_layers_matches_each_layer(chunks):
     np.testing.assert_array_equal(shared.view(torch.int16).numpy().view(np.uint16), refs[-1])
 
 
+def _oracle_chain(routes, x, R, S, K, E):
+    """The oracle's forward chain: each layer dispatches the rows the one
+    before combined, through its own routing."""
+    T = x.shape[0]
+    want = x
+    for tk, w in routes:
+        loads, _, _ = O.route_stats(tk, E)
+        pl = O.plan(loads, R, S, K, E)
+        lo = O.layout(tk, pl, R, S, E)
+        want = O.combine(O.dispatch(want, lo["pos"], K, T * K), w, lo["pos"], K)
+    return want
+
+
 @pytest.mark.parametrize("chunks", [1, 5, 8])
 @pytest.mark.parametrize("nl", [1, 2, 3])
 def test_run_host_chain_matches_the_oracle_chain(nl, chunks):
@@ -121,12 +134,7 @@ def test_run_host_chain_matches_the_oracle_chain(nl, chunks):
     assert nl == 1 or layers[1].x.data_ptr() == layers[0].out.data_ptr()
     routes = [W.routing_from(T, E, K, seed=40 + l, bias_e=W.bias(2, l)) for l in range(nl)]
     x = W.hidden(T, H, seed=50)
-    want = x
-    for tk, w in routes:
-        loads, _, _ = O.route_stats(tk, E)
-        pl = O.plan(loads, R, S, K, E)
-        lo = O.layout(tk, pl, R, S, E)
-        want = O.combine(O.dispatch(want, lo["pos"], K, T * K), w, lo["pos"], K)
+    want = _oracle_chain(routes, x, R, S, K, E)
     topk_hs = [torch.from_numpy(tk).pin_memory() for tk, _ in routes]
     w_hs = [torch.from_numpy(w).pin_memory() for _, w in routes]
     x_h = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -145,3 +153,39 @@ def test_run_host_chain_matches_the_oracle_chain(nl, chunks):
         ly.step(grads=False)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(layers[-1].out.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+@pytest.mark.parametrize("staged", [True, False], ids=["stage_buffers", "chain_buffers"])
+@pytest.mark.parametrize("nl", [1, 2, 3])
+def test_run_host_batches_matches_the_oracle_chain(nl, staged):
+    """Three batches in flight through a chain of layers (run_host_batches),
+    each with its own routing per layer and its own hidden rows: every batch's
+    combined rows, copied to its own host buffer, equal the oracle's chain for
+    that batch.  With separate stage buffers batch b+1's rows arrive while
+    batch b's layers still run; with the defaults (the chain's own buffers)
+    the batches wait for one another."""
+    import torch
+    import token_dispatch_histogram_b200 as tdh
+    from token_dispatch_histogram_b200.layer import chain_buffers, run_host_batches
+    R, S, K, E, H, bm = 8, 384, 6, 64, 512, 64
+    T = R * S
+    layers = []
+    for _ in range(nl):
+        layers.append(tdh.EpLayer(R, S, K, E, H, bm, device="cuda", share=layers[0] if layers else None))
+    chain_buffers(layers)
+    batches, wants = [], []
+    for b in range(3):
+        routes = [W.routing_from(T, E, K, seed=100 * b + l, bias_e=W.bias(2, l + b)) for l in range(nl)]
+        x = W.hidden(T, H, seed=60 + b)
+        wants.append(_oracle_chain(routes, x, R, S, K, E))
+        batches.append(([torch.from_numpy(tk).pin_memory() for tk, _ in routes],
+                        [torch.from_numpy(w).pin_memory() for _, w in routes],
+                        torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                        torch.zeros((T, H), dtype=torch.bfloat16).pin_memory()))
+    xs = torch.empty_like(layers[0].x) if staged else None
+    os_ = torch.empty_like(layers[0].x) if staged else None
+    run_host_batches(layers, batches, xs, os_, grads=False, chunks=5)
+    torch.cuda.synchronize()
+    assert all(ly.status() == 0 for ly in layers)
+    for (_, _, _, out_h), want in zip(batches, wants):
+        np.testing.assert_array_equal(out_h.view(torch.int16).numpy().view(np.uint16), want)

@@ -308,11 +308,57 @@ def run_host_chain(layers, topk_hs, w_hs, x_h, out_h, stream=None, grads=True, f
     last layer combines slice by slice and each slice leaves as soon as it is
     combined.  Routing for the later layers is copied behind the first layer's
     rows on the same copy stream.  With one layer this is EpLayer.run_host.
-    The caller's stream waits for the last copy out."""
+    The caller's stream waits for the last copy out.  (run_host_batches with
+    one batch, the rows arriving in the first layer's x and leaving from the
+    last layer's out.)"""
+    run_host_batches(layers, [(topk_hs, w_hs, x_h, out_h)], None, None, stream, grads, fused, chunks)
+
+
+def _record(stream):
+    ev = torch.cuda.Event()
+    ev.record(stream)
+    return ev
+
+
+def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None, grads=True, fused=True, chunks=8):
+    """A chain of layers (chain_buffers) over a sequence of batches fed from
+    pinned host memory, the batches overlapping on the host link.
+
+    batches: (topk_hs, w_hs, x_h, out_h) per batch -- every layer's routing
+    and gate weights, the batch's hidden rows, and the host buffer for the last
+    layer's combined rows.  Each batch runs as in run_host_chain: its rows
+    arrive in token slices that the first layer dispatches and combines as
+    they land, the middle layers run on the device, and the last layer's
+    slices leave as soon as they are combined.
+
+    x_stage and out_stage are the device buffers [T, H] the first layer
+    dispatches from and the last layer combines into (default: the first
+    layer's x and the last layer's out).  Given apart from the chain's two row
+    buffers, batch b+1's rows come in while batch b's later layers still run
+    and batch b's rows go out while batch b+1's layers run: the inbound copies
+    wait only for batch b's first layer to have read x_stage, and the last
+    layer of batch b+1 waits for batch b's rows to have left out_stage.  A
+    layer's routing and gate weights for batch b+1 arrive once that layer has
+    finished batch b.  With the defaults every such wait falls on the last
+    layer that uses the buffer, so the batches run one after another.  The
+    caller's stream waits for every copy."""
     n = len(layers)
-    if not (len(topk_hs) == len(w_hs) == n) or n == 0:
-        raise ValueError("one routing and weight buffer per layer")
+    if n == 0:
+        raise ValueError("no layers")
     first, last = layers[0], layers[-1]
+    x_stage = first.x if x_stage is None else x_stage
+    out_stage = last.out if out_stage is None else out_stage
+    for t in (x_stage, out_stage):
+        if t.shape != first.x.shape or t.dtype != first.x.dtype or t.device != first.x.device:
+            raise ValueError("x_stage and out_stage must be [T, H] bf16 buffers on the layers' device")
+    ptr = (lambda t: t.data_ptr())
+    # the last layer of a batch that reads or writes x_stage's storage (layer 0
+    # reads it), and the first that writes out_stage's; when the two are one
+    # buffer (a chain of an even number of layers, by default), the inbound
+    # rows also wait for the batch before's rows to have left
+    x_waits_sent = ptr(x_stage) == ptr(out_stage)
+    x_last_use = max([0] + [l for l, ly in enumerate(layers) if ptr(x_stage) in (ptr(ly.x), ptr(ly.out))])
+    out_first_write = min([n - 1] + [l for l, ly in enumerate(layers) if ptr(ly.out) == ptr(out_stage)])
     main = stream if stream is not None else torch.cuda.current_stream(first.device)
     h2d, d2h = first._copy_streams()
     h2d.wait_stream(main)
@@ -320,47 +366,55 @@ def run_host_chain(layers, topk_hs, w_hs, x_h, out_h, stream=None, grads=True, f
     T, K = first.T, first.K
     bounds = slice_bounds(T, max(1, min(chunks, T)))
     spans = list(zip(bounds[:-1], bounds[1:]))
-    routed = []
-    with torch.cuda.stream(h2d):
-        first.topk_ids.copy_(topk_hs[0], non_blocking=True)
-        first.w.copy_(w_hs[0], non_blocking=True)
-        ev = torch.cuda.Event()
-        ev.record(h2d)
-        routed.append(ev)
-    arrived = []
-    for t0, t1 in spans:
+    layer_done = [None] * n  # main finished layer l of the batch before (its routing buffers are free)
+    sent = None              # the batch before's rows have all left out_stage
+    for topk_hs, w_hs, x_h, out_h in batches:
+        if not (len(topk_hs) == len(w_hs) == n):
+            raise ValueError("one routing and weight buffer per layer")
+        routed, arrived = [None] * n, []
         with torch.cuda.stream(h2d):
-            first.x[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(h2d)
-            arrived.append(ev)
-    with torch.cuda.stream(h2d):
-        for ly, tk, w in zip(layers[1:], topk_hs[1:], w_hs[1:]):
-            ly.topk_ids.copy_(tk, non_blocking=True)
-            ly.w.copy_(w, non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(h2d)
-            routed.append(ev)
-    for li, ly in enumerate(layers):
-        main.wait_event(routed[li])
-        ly.route(main, fused)
-        if li == 0 or li == n - 1:
-            # a token slice's combine reads only the rows its own dispatch wrote
-            for j, (t0, t1) in enumerate(spans):
-                if li == 0:
-                    main.wait_event(arrived[j])
-                ep_dispatch(ly.x[t0:t1], K, ly.pos[t0 * K:t1 * K], ly.buf, ly.dev_status, main)
-                ep_combine(ly.buf, ly.w[t0:t1], ly.pos[t0 * K:t1 * K], ly.out[t0:t1], ly.dev_status, main)
-                if li == n - 1:
-                    combined = torch.cuda.Event()
-                    combined.record(main)
-                    d2h.wait_event(combined)
-                    with torch.cuda.stream(d2h):
-                        out_h[t0:t1].copy_(ly.out[t0:t1], non_blocking=True)
-        else:
-            ly.dispatch(main)
-            ly.combine(main)
-        if grads:
-            ly.grad_reduce(False, main)
+            if layer_done[0] is not None:
+                h2d.wait_event(layer_done[0])
+            first.topk_ids.copy_(topk_hs[0], non_blocking=True)
+            first.w.copy_(w_hs[0], non_blocking=True)
+            routed[0] = _record(h2d)
+            if layer_done[x_last_use] is not None:
+                h2d.wait_event(layer_done[x_last_use])
+            if x_waits_sent and sent is not None:
+                h2d.wait_event(sent)
+            for t0, t1 in spans:
+                x_stage[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
+                arrived.append(_record(h2d))
+            for l in range(1, n):
+                if layer_done[l] is not None:
+                    h2d.wait_event(layer_done[l])
+                layers[l].topk_ids.copy_(topk_hs[l], non_blocking=True)
+                layers[l].w.copy_(w_hs[l], non_blocking=True)
+                routed[l] = _record(h2d)
+        for l, ly in enumerate(layers):
+            main.wait_event(routed[l])
+            ly.route(main, fused)
+            if l == out_first_write and sent is not None:
+                main.wait_event(sent)
+            if l == 0 or l == n - 1:
+                # a token slice's combine reads only the rows its own dispatch wrote
+                rows_in = x_stage if l == 0 else ly.x
+                rows_out = out_stage if l == n - 1 else ly.out
+                for j, (t0, t1) in enumerate(spans):
+                    if l == 0:
+                        main.wait_event(arrived[j])
+                    ep_dispatch(rows_in[t0:t1], K, ly.pos[t0 * K:t1 * K], ly.buf, ly.dev_status, main)
+                    ep_combine(ly.buf, ly.w[t0:t1], ly.pos[t0 * K:t1 * K], rows_out[t0:t1], ly.dev_status, main)
+                    if l == n - 1:
+                        d2h.wait_event(_record(main))
+                        with torch.cuda.stream(d2h):
+                            out_h[t0:t1].copy_(rows_out[t0:t1], non_blocking=True)
+            else:
+                ly.dispatch(main)
+                ly.combine(main)
+            layer_done[l] = _record(main)
+            if grads:
+                ly.grad_reduce(False, main)
+        sent = _record(d2h)
     main.wait_stream(d2h)
     main.wait_stream(h2d)
