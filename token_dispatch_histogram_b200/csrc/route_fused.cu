@@ -22,6 +22,9 @@
 // A pair's stable rank within its expert = (its tile's prefix) + (earlier warps
 // of the tile) + (earlier chunks of its warp) + popc(peers & lanemask_lt):
 // integer adds only, so nothing depends on scheduling.  Every wait is bounded.
+// Large tiles (STAGE_MIN_TILE pairs and more) stage the walk's pairs in shared
+// memory in (expert, rank) order and write the align-sort ids and src from a
+// sweep over the experts' runs, as consecutive words instead of scattered ones.
 //
 // Fused layout + dispatch (ep_route_dispatch_fused, DISPATCH = true): once a
 // tile CTA has written its pairs' rows (step 4), it copies the hidden rows of
