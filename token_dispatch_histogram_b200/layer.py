@@ -320,6 +320,14 @@ def _record(stream):
     return ev
 
 
+def _routing_stage(ly):
+    """Device copies of a layer's routing and gate weights that the next
+    batch's may land in while this batch still reads the layer's own."""
+    if not hasattr(ly, "_rt_stage"):
+        ly._rt_stage = (torch.empty_like(ly.topk_ids), torch.empty_like(ly.w))
+    return ly._rt_stage
+
+
 def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None, grads=True, fused=True, chunks=8):
     """A chain of layers (chain_buffers) over a sequence of batches fed from
     pinned host memory, the batches overlapping on the host link.
@@ -336,12 +344,15 @@ def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None,
     layer's x and the last layer's out).  Given apart from the chain's two row
     buffers, batch b+1's rows come in while batch b's later layers still run
     and batch b's rows go out while batch b+1's layers run: the inbound copies
-    wait only for batch b's first layer to have read x_stage, and the last
-    layer of batch b+1 waits for batch b's rows to have left out_stage.  A
-    layer's routing and gate weights for batch b+1 arrive once that layer has
-    finished batch b.  With the defaults every such wait falls on the last
-    layer that uses the buffer, so the batches run one after another.  The
-    caller's stream waits for every copy."""
+    wait for batch b's first layer to have read x_stage (with one layer, slice
+    j waits only for batch b's slice j to have been dispatched), and the last
+    layer of batch b+1 writes slice j of out_stage once batch b's slice j has
+    left.  With several batches a layer's routing and gate weights for batch
+    b+1 arrive in a device copy of their own and move into the layer's buffers
+    on the compute stream, so they never wait for batch b.  With the default
+    buffers every wait falls on the last layer that uses the buffer, so the
+    batches run one after another.  The caller's stream waits for every copy."""
+    batches = list(batches)
     n = len(layers)
     if n == 0:
         raise ValueError("no layers")
@@ -359,6 +370,13 @@ def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None,
     x_waits_sent = ptr(x_stage) == ptr(out_stage)
     x_last_use = max([0] + [l for l, ly in enumerate(layers) if ptr(x_stage) in (ptr(ly.x), ptr(ly.out))])
     out_first_write = min([n - 1] + [l for l, ly in enumerate(layers) if ptr(ly.out) == ptr(out_stage)])
+    # slice by slice where only the one layer's slices use the stage buffers:
+    # on a chain the next batch's rows would keep the inbound direction busy
+    # the whole time and slow the outbound copies the last layer waits for
+    # (measured on B200), so there they wait for the whole first layer
+    x_by_slice = n == 1 and x_last_use == 0 and not x_waits_sent
+    out_by_slice = out_first_write == n - 1 and not x_waits_sent
+    staged_routing = len(batches) > 1
     main = stream if stream is not None else torch.cuda.current_stream(first.device)
     h2d, d2h = first._copy_streams()
     h2d.wait_stream(main)
@@ -366,35 +384,54 @@ def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None,
     T, K = first.T, first.K
     bounds = slice_bounds(T, max(1, min(chunks, T)))
     spans = list(zip(bounds[:-1], bounds[1:]))
-    layer_done = [None] * n  # main finished layer l of the batch before (its routing buffers are free)
-    sent = None              # the batch before's rows have all left out_stage
+    layer_done = [None] * n          # main finished layer l of the batch before
+    rt_taken = [None] * n            # main moved the batch before's staged routing of layer l into the layer
+    dispatched = [None] * len(spans)  # the batch before's first layer dispatched slice j (its rows are free)
+    left = [None] * len(spans)       # the batch before's slice j has left out_stage
+    sent = None                      # the batch before's rows have all left out_stage
+
+    def routing_in(l, topk_h, w_h):
+        ly = layers[l]
+        if staged_routing:
+            if rt_taken[l] is not None:
+                h2d.wait_event(rt_taken[l])
+            st_t, st_w = _routing_stage(ly)
+        else:
+            if layer_done[l] is not None:
+                h2d.wait_event(layer_done[l])
+            st_t, st_w = ly.topk_ids, ly.w
+        st_t.copy_(topk_h, non_blocking=True)
+        st_w.copy_(w_h, non_blocking=True)
+        return _record(h2d)
+
     for topk_hs, w_hs, x_h, out_h in batches:
         if not (len(topk_hs) == len(w_hs) == n):
             raise ValueError("one routing and weight buffer per layer")
         routed, arrived = [None] * n, []
         with torch.cuda.stream(h2d):
-            if layer_done[0] is not None:
-                h2d.wait_event(layer_done[0])
-            first.topk_ids.copy_(topk_hs[0], non_blocking=True)
-            first.w.copy_(w_hs[0], non_blocking=True)
-            routed[0] = _record(h2d)
-            if layer_done[x_last_use] is not None:
-                h2d.wait_event(layer_done[x_last_use])
-            if x_waits_sent and sent is not None:
-                h2d.wait_event(sent)
-            for t0, t1 in spans:
+            routed[0] = routing_in(0, topk_hs[0], w_hs[0])
+            if not x_by_slice:
+                if layer_done[x_last_use] is not None:
+                    h2d.wait_event(layer_done[x_last_use])
+                if x_waits_sent and sent is not None:
+                    h2d.wait_event(sent)
+            for j, (t0, t1) in enumerate(spans):
+                if x_by_slice and dispatched[j] is not None:
+                    h2d.wait_event(dispatched[j])
                 x_stage[t0:t1].copy_(x_h[t0:t1], non_blocking=True)
                 arrived.append(_record(h2d))
             for l in range(1, n):
-                if layer_done[l] is not None:
-                    h2d.wait_event(layer_done[l])
-                layers[l].topk_ids.copy_(topk_hs[l], non_blocking=True)
-                layers[l].w.copy_(w_hs[l], non_blocking=True)
-                routed[l] = _record(h2d)
+                routed[l] = routing_in(l, topk_hs[l], w_hs[l])
         for l, ly in enumerate(layers):
             main.wait_event(routed[l])
+            if staged_routing:
+                st_t, st_w = _routing_stage(ly)
+                with torch.cuda.stream(main):
+                    ly.topk_ids.copy_(st_t, non_blocking=True)
+                    ly.w.copy_(st_w, non_blocking=True)
+                rt_taken[l] = _record(main)
             ly.route(main, fused)
-            if l == out_first_write and sent is not None:
+            if l == out_first_write and sent is not None and not out_by_slice:
                 main.wait_event(sent)
             if l == 0 or l == n - 1:
                 # a token slice's combine reads only the rows its own dispatch wrote
@@ -404,11 +441,16 @@ def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None,
                     if l == 0:
                         main.wait_event(arrived[j])
                     ep_dispatch(rows_in[t0:t1], K, ly.pos[t0 * K:t1 * K], ly.buf, ly.dev_status, main)
+                    if l == 0:
+                        dispatched[j] = _record(main)
+                    if l == n - 1 and out_by_slice and left[j] is not None:
+                        main.wait_event(left[j])
                     ep_combine(ly.buf, ly.w[t0:t1], ly.pos[t0 * K:t1 * K], rows_out[t0:t1], ly.dev_status, main)
                     if l == n - 1:
                         d2h.wait_event(_record(main))
                         with torch.cuda.stream(d2h):
                             out_h[t0:t1].copy_(rows_out[t0:t1], non_blocking=True)
+                            left[j] = _record(d2h)
             else:
                 ly.dispatch(main)
                 ly.combine(main)
