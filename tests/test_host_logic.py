@@ -1,5 +1,5 @@
 """Host-side logic of the layer and the benchmark, on CPU: the host-fed
-pipeline's token slices, the algorithmic byte counts behind every roofline
+pipeline's token slices and the waits between host-fed batches, the algorithmic byte counts behind every roofline
 fraction, the clock sampler's parsing, and the rule that a committed DRAM
 traffic figure is used only for the source it was captured on."""
 import hashlib
@@ -20,6 +20,39 @@ def test_slice_bounds_cover_the_tokens_in_order():
     b = slice_bounds(22 * 1000, 8)
     sizes = [y - x for x, y in zip(b, b[1:])]
     assert sizes == [1000, 2000, 4000, 4000, 4000, 4000, 2000, 1000]
+
+
+def test_batch_gating_follows_the_buffers():
+    """The waits between host-fed batches, from which storage each buffer is
+    (A, B: the chain's two row buffers; C, D: stage buffers of their own)."""
+    from token_dispatch_histogram_b200.layer import batch_gating
+    A, B, C, D = 1, 2, 3, 4
+    # one layer with stage buffers apart, or its own x and out: slice by slice both ways
+    for xs, os_ in ((C, D), (A, B)):
+        g = batch_gating([(A, B)], xs, os_)
+        assert g == {"x_last_use": 0, "out_first_write": 0, "x_waits_sent": False, "x_by_slice": True,
+                     "out_by_slice": True}
+    # one layer whose stage buffers are one storage: everything waits for the rows to have left
+    g = batch_gating([(A, B)], C, C)
+    assert g["x_waits_sent"] and not g["x_by_slice"] and not g["out_by_slice"]
+    # a chain of two on its own buffers: x_stage = layer 0's x = A = layer 1's out = out_stage
+    g = batch_gating([(A, B), (B, A)], A, A)
+    assert g["x_waits_sent"] and g["x_last_use"] == 1 and g["out_first_write"] == 1
+    assert not g["x_by_slice"] and not g["out_by_slice"]
+    # a chain of three on its own buffers: A is used up to the last layer, B is written from layer 0 on
+    g = batch_gating([(A, B), (B, A), (A, B)], A, B)
+    assert not g["x_waits_sent"] and g["x_last_use"] == 2 and g["out_first_write"] == 0
+    assert not g["x_by_slice"] and not g["out_by_slice"]
+    # eight chained layers with stage buffers apart: rows in after the first layer, out slice by slice
+    chain = [(A, B) if l % 2 == 0 else (B, A) for l in range(8)]
+    g = batch_gating(chain, C, D)
+    assert g == {"x_last_use": 0, "out_first_write": 7, "x_waits_sent": False, "x_by_slice": False,
+                 "out_by_slice": True}
+    # a stage buffer that is one of the chain's: waits for the last layer using it
+    g = batch_gating(chain, B, D)
+    assert g["x_last_use"] == 7 and not g["x_by_slice"]
+    with pytest.raises(ValueError):
+        batch_gating([], C, D)
 
 
 def test_algorithmic_bytes_of_the_moderate_workload():

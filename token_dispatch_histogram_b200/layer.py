@@ -328,6 +328,31 @@ def _routing_stage(ly):
     return ly._rt_stage
 
 
+def batch_gating(layer_bufs, x_stage, out_stage):
+    """The waits run_host_batches takes between batch b and batch b+1, from
+    which storage each buffer is.  layer_bufs: (x, out) storage identities of
+    every layer, in order; x_stage, out_stage: those of the stage buffers.
+
+    x_last_use: the last layer of a batch that reads or writes x_stage's
+    storage (layer 0 reads it); out_first_write: the first layer that writes
+    out_stage's storage; x_waits_sent: x_stage is out_stage's storage, so the
+    next rows also wait for the rows before to have left; x_by_slice: the next
+    batch's slice j may come in once this batch's slice j is dispatched (one
+    layer only: on a chain the rows wait for the whole first layer, which
+    measured faster); out_by_slice: the last layer's slice j may be combined
+    once the batch before's slice j has left (no other layer writes
+    out_stage's storage)."""
+    n = len(layer_bufs)
+    if n == 0:
+        raise ValueError("no layers")
+    x_waits_sent = x_stage == out_stage
+    x_last_use = max([0] + [l for l, (x, o) in enumerate(layer_bufs) if x_stage in (x, o)])
+    out_first_write = min([n - 1] + [l for l, (x, o) in enumerate(layer_bufs) if o == out_stage])
+    return {"x_last_use": x_last_use, "out_first_write": out_first_write, "x_waits_sent": x_waits_sent,
+            "x_by_slice": n == 1 and x_last_use == 0 and not x_waits_sent,
+            "out_by_slice": out_first_write == n - 1 and not x_waits_sent}
+
+
 def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None, grads=True, fused=True, chunks=8):
     """A chain of layers (chain_buffers) over a sequence of batches fed from
     pinned host memory, the batches overlapping on the host link.
@@ -363,19 +388,9 @@ def run_host_batches(layers, batches, x_stage=None, out_stage=None, stream=None,
         if t.shape != first.x.shape or t.dtype != first.x.dtype or t.device != first.x.device:
             raise ValueError("x_stage and out_stage must be [T, H] bf16 buffers on the layers' device")
     ptr = (lambda t: t.data_ptr())
-    # the last layer of a batch that reads or writes x_stage's storage (layer 0
-    # reads it), and the first that writes out_stage's; when the two are one
-    # buffer (a chain of an even number of layers, by default), the inbound
-    # rows also wait for the batch before's rows to have left
-    x_waits_sent = ptr(x_stage) == ptr(out_stage)
-    x_last_use = max([0] + [l for l, ly in enumerate(layers) if ptr(x_stage) in (ptr(ly.x), ptr(ly.out))])
-    out_first_write = min([n - 1] + [l for l, ly in enumerate(layers) if ptr(ly.out) == ptr(out_stage)])
-    # slice by slice where only the one layer's slices use the stage buffers:
-    # on a chain the next batch's rows would keep the inbound direction busy
-    # the whole time and slow the outbound copies the last layer waits for
-    # (measured on B200), so there they wait for the whole first layer
-    x_by_slice = n == 1 and x_last_use == 0 and not x_waits_sent
-    out_by_slice = out_first_write == n - 1 and not x_waits_sent
+    g = batch_gating([(ptr(ly.x), ptr(ly.out)) for ly in layers], ptr(x_stage), ptr(out_stage))
+    x_waits_sent, x_last_use, out_first_write = g["x_waits_sent"], g["x_last_use"], g["out_first_write"]
+    x_by_slice, out_by_slice = g["x_by_slice"], g["out_by_slice"]
     staged_routing = len(batches) > 1
     main = stream if stream is not None else torch.cuda.current_stream(first.device)
     h2d, d2h = first._copy_streams()
