@@ -232,6 +232,12 @@ def max_over_ranks(value_ms, world, device):
     return float(t.item())
 
 
+def all_ranks_ok(ok, world, device):
+    """True on every rank when every rank's `ok` is true (one max over ranks),
+    so that all ranks take an optional pass together or none does."""
+    return max_over_ranks(0.0 if ok else 1.0, world, device) == 0.0
+
+
 def job_throughput(world, pairs_per_step, steps, job_ms):
     """Whole-job pairs/s: all ranks' pairs over the slowest rank's time."""
     return world * pairs_per_step * steps / (job_ms / 1e3)
@@ -702,13 +708,26 @@ def run_workload(args, cfg, rank, world, local_rank, full=True):
     # (run_host_layers)
     e2e = None
     e2e_rows = None
+    pinned = None
     if not args.no_e2e:
-        topk_h = [torch.from_numpy(tk).pin_memory() for tk, _ in routes]
-        w_h = [torch.from_numpy(ww).pin_memory() for _, ww in routes]
-        x_h = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
+        # every rank pins its own batch (15 GB on the fine-grained workload); the ranks take the end-to-end pass
+        # together or not at all, so that none waits at a barrier for a rank that could not pin its buffers
+        try:
+            pinned = ([torch.from_numpy(tk).pin_memory() for tk, _ in routes],
+                      [torch.from_numpy(ww).pin_memory() for _, ww in routes],
+                      torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True),
+                      torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True))
+        except RuntimeError as exc:
+            print(f"pinned host buffers for the end-to-end pass: {str(exc).splitlines()[0][:200]}", file=sys.stderr)
+            pinned = None
+        if not all_ranks_ok(pinned is not None, world, dev):
+            pinned = None
+            e2e = {"unavailable": "the pinned host buffers of the end-to-end pass could not be allocated on every rank"}
+    if pinned is not None:
+        topk_h, w_h, x_h, out_h = pinned
+        del pinned
         W.fill_device(layer.x, seed, W.STREAM_X)
         x_h.copy_(layer.x)  # the generator's rows, as a caller's host batch
-        out_h = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
         route_bytes = sum(t.numel() * 4 for t in topk_h) + sum(t.numel() * 4 for t in w_h)
 
         def timed_host(host_step, budget_ms):

@@ -50,6 +50,38 @@ def test_two_ranks_gloo():
     assert all(r[3] == pytest.approx(2 * 196608 * 20 / 0.015) for r in res)
 
 
+def _agree_worker(rank, world, port, fail_rank, q):
+    import datetime
+    import sys
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        q.put((rank, bench.all_ranks_ok(rank != fail_rank, world, "cpu")))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("fail_rank", [None, 0, 1])
+def test_optional_pass_is_all_or_none(fail_rank):
+    """The end-to-end pass's pinned buffers: when one rank cannot allocate
+    them, every rank skips the pass (none waits at a barrier for it)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_agree_worker, args=(r, 2, port, fail_rank, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [ok for _, ok in res] == [fail_rank is None] * 2
+
+
 def _gather_worker(rank, world, port, q):
     """One rank of the rank-local form's exchange: its own expert counts, the
     all-gather into [R, E] (gather_counts, gloo), and the list offsets a rank
